@@ -1,0 +1,314 @@
+"""Float64 CPU oracle for causal grouped-query attention with RoPE'd Q and K.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path imports, calls or links
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may use it. It
+shares no code with the CUDA library and imports nothing from it.
+
+What it computes is the plain definition, in the pages' own order of steps
+("Attention from Scratch", section "Attention, the math: Grouped-Query
+Attention with RoPE'd Q/K", the six-step walk-through of
+``GroupedQueryAttention.forward``), with the projections left out because the
+inputs are already per-head Q, K, V:
+
+  2. Rotate   -- RoPE on Q and K, never on V ("Embeddings & the Residual
+                 Stream", section "Positional information: RoPE, not a learned
+                 table": inv_freq[i] = theta^(-2i/d), angle = pos*inv_freq[i],
+                 table duplicated as cat([f, f]) and x*cos + rotate_half(x)*sin
+                 with rotate_half(x1, x2) = (-x2, x1), i.e. feature i is
+                 paired with feature i + d/2).
+  3. Share    -- each KV head serves G = n_q/n_kv consecutive query heads
+                 (repeat_interleave along the head axis, not repeat).
+  4. Score    -- q @ k^T / sqrt(head_dim).
+  5. Mask     -- entries above the diagonal set to -inf (causal), then a
+                 max-shifted softmax over keys ("Attention from Scratch",
+                 section "The compute thread": reduce_max, subtract, exp,
+                 reduce_sum, divide).
+  6. Gather   -- weights @ v.
+
+plus the natural-log log-sum-exp of each row's scaled, masked scores (not on
+the pages; it is the normaliser a backward pass needs).
+
+Packed batches: ``cu_seqlens`` holds prefix sums of the sequence lengths; each
+sequence is attended to on its own (no token sees another sequence) and its
+positions default to 0..L-1 ("Kohaku-TT" page, Highlights: flash attention with
+packed variable-length batches).
+
+Precision. Everything is float64. One quantisation is part of the method and
+is modelled on purpose: the rotated Q and K are tensors of the input dtype
+(the RoPE page's ``apply_rope`` returns ``x.dtype``; for bf16 inputs that is
+bf16, which is also what the tensor-core operands are). With
+``operand_rounding=True`` the rotation uses the fp32 cos/sin table the RoPE
+page builds (here: the float64 cos/sin of the float64 angle, rounded once to
+fp32), evaluates x*cos - y*sin in float64 and rounds that once to bf16 (round
+to nearest, ties to even). With ``operand_rounding=False`` the rotation is
+exact float64 and nothing is rounded; the RoPE pins use that form.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+__all__ = [
+    "round_to_bf16",
+    "rope_inv_freq",
+    "rope_cos_sin",
+    "rotate_half",
+    "apply_rope",
+    "share_kv_heads",
+    "score",
+    "causal_mask",
+    "softmax_with_lse",
+    "gather",
+    "gqa_rope_attention",
+    "brute_force_attention",
+]
+
+
+# ---------------------------------------------------------------------------
+# Rounding
+# ---------------------------------------------------------------------------
+
+_BF16_MAX_FINITE_NEXT = 2.0 ** 128  # first magnitude that rounds to inf
+
+
+def round_to_bf16(x) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 value (ties to even) in a
+    single rounding, returned as float64.
+
+    bfloat16 has 8 significant bits, exponent range as fp32: normal numbers
+    down to 2^-126, subnormals with a fixed quantum of 2^-133.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)  # x = m * 2^e with 0.5 <= |m| < 1
+    normal = e >= -125  # |x| >= 2^-126
+    with np.errstate(over="ignore", invalid="ignore"):
+        qn = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
+        qs = np.ldexp(np.rint(np.ldexp(x, 133)), -133)
+    q = np.where(normal, qn, qs)
+    q = np.where(np.abs(q) >= _BF16_MAX_FINITE_NEXT, np.copysign(np.inf, x), q)
+    q = np.where(np.isnan(x), np.nan, q)
+    q = np.where(np.isinf(x), x, q)
+    return q
+
+
+def _round_to_fp32(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# RoPE ("Embeddings & the Residual Stream", section "Positional information:
+# RoPE, not a learned table")
+# ---------------------------------------------------------------------------
+
+def rope_inv_freq(head_dim: int, theta: float) -> np.ndarray:
+    """inv_freq[i] = theta^(-2i/head_dim) for i in [0, head_dim/2)."""
+    if head_dim % 2:
+        raise ValueError("RoPE needs an even head_dim")
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    return np.power(float(theta), -(2.0 * i) / float(head_dim))
+
+
+def rope_cos_sin(positions, head_dim: int, theta: float, table_fp32: bool = False) -> Tuple[np.ndarray, np.ndarray]:
+    """cos/sin tables of shape [T, head_dim]: angle(pos, i) = pos * inv_freq[i],
+    duplicated across the two halves (cat([f, f])) to line up with
+    rotate_half. ``table_fp32`` rounds each entry to fp32, as the page's
+    table is an fp32 tensor."""
+    pos = np.asarray(positions, dtype=np.float64).reshape(-1)
+    freqs = np.outer(pos, rope_inv_freq(head_dim, theta))  # [T, d/2]
+    emb = np.concatenate([freqs, freqs], axis=-1)  # [T, d]
+    c, s = np.cos(emb), np.sin(emb)
+    if table_fp32:
+        c, s = _round_to_fp32(c), _round_to_fp32(s)
+    return c, s
+
+
+def rotate_half(x: np.ndarray) -> np.ndarray:
+    """(x1, x2) -> (-x2, x1) on the two halves of the last axis."""
+    h = x.shape[-1] // 2
+    return np.concatenate([-x[..., h:], x[..., :h]], axis=-1)
+
+
+def apply_rope(x: np.ndarray, positions, theta: float, operand_rounding: bool = False) -> np.ndarray:
+    """x: [T, H, d] (token-major). Returns x*cos + rotate_half(x)*sin with the
+    cos/sin row of each token's position broadcast over heads."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    c, s = rope_cos_sin(positions, d, theta, table_fp32=operand_rounding)
+    c = c[:, None, :]
+    s = s[:, None, :]
+    if not operand_rounding:
+        return x * c + rotate_half(x) * s
+    # Each product below is exact in float64 (8-bit by 24-bit significands);
+    # the sum is rounded once to float64, then once to bf16.
+    y = x * c + rotate_half(x) * s
+    return round_to_bf16(y)
+
+
+# ---------------------------------------------------------------------------
+# GQA sharing ("Attention from Scratch": repeat_interleave keeps the query
+# heads of one group adjacent)
+# ---------------------------------------------------------------------------
+
+def share_kv_heads(kv: np.ndarray, group_size: int, axis: int = 1) -> np.ndarray:
+    """Repeat each KV head ``group_size`` times in place (repeat_interleave):
+    query head h reads KV head h // group_size."""
+    return np.repeat(kv, group_size, axis=axis)
+
+
+# ---------------------------------------------------------------------------
+# Attention steps ("Attention from Scratch", section "Attention, the math")
+# ---------------------------------------------------------------------------
+
+def score(qh: np.ndarray, kh: np.ndarray) -> np.ndarray:
+    """Step 4: q @ k^T / sqrt(head_dim) for head-major [H, Tq, d], [H, Tk, d]."""
+    d = qh.shape[-1]
+    return np.matmul(qh, np.swapaxes(kh, -1, -2)) / math.sqrt(d)
+
+
+def causal_mask(scores: np.ndarray, query_idx: np.ndarray, key_idx: np.ndarray) -> np.ndarray:
+    """Step 5a: key j is visible to query i iff j <= i (indices inside the
+    sequence); the rest is filled with -inf."""
+    visible = key_idx[None, :] <= query_idx[:, None]
+    return np.where(visible[None, :, :], scores, -np.inf)
+
+
+def softmax_with_lse(scores: np.ndarray):
+    """Step 5b: max-shifted softmax over the key axis ("The compute thread":
+    reduce_max, subtract, exp, reduce_sum, divide) and the natural-log
+    log-sum-exp m + ln(sum exp(s - m)) of each row."""
+    m = np.max(scores, axis=-1, keepdims=True)
+    e = np.exp(scores - m)
+    z = np.sum(e, axis=-1, keepdims=True)
+    return e / z, (m + np.log(z))[..., 0]
+
+
+def gather(weights: np.ndarray, vh: np.ndarray) -> np.ndarray:
+    """Step 6: weights @ v."""
+    return np.matmul(weights, vh)
+
+
+# ---------------------------------------------------------------------------
+# Forward
+# ---------------------------------------------------------------------------
+
+def _check_args(q, k, v, cu_seqlens, n_q_heads, n_kv_heads):
+    if q.ndim != 3 or k.ndim != 3 or v.ndim != 3:
+        raise ValueError("q, k, v must be [N, heads, d]")
+    N, hq, d = q.shape
+    if hq != n_q_heads or k.shape != (N, n_kv_heads, d) or v.shape != (N, n_kv_heads, d):
+        raise ValueError("shape mismatch")
+    if n_q_heads % n_kv_heads:
+        raise ValueError("n_q_heads must be a multiple of n_kv_heads")
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    if cu[0] != 0 or cu[-1] != N or np.any(np.diff(cu) < 0):
+        raise ValueError("bad cu_seqlens")
+    return N, d, cu
+
+
+def gqa_rope_attention(q, k, v, cu_seqlens, n_q_heads: int, n_kv_heads: int, rope_theta: float,
+                       positions=None, causal: bool = True, operand_rounding: bool = True,
+                       query_rows: Optional[Sequence[int]] = None, row_block: int = 1024):
+    """Reference forward.
+
+    q: [N, n_q, d], k, v: [N, n_kv, d] (any float dtype; used as float64).
+    cu_seqlens: [num_seqs+1] prefix sums. positions: [N] ints or None (then
+    the index inside each sequence). Returns (out [N, n_q, d] float64,
+    lse [n_q, N] float64). If ``query_rows`` (global token indices) is given,
+    only those rows are computed; the others are NaN.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    N, d, cu = _check_args(q, k, v, cu_seqlens, n_q_heads, n_kv_heads)
+    G = n_q_heads // n_kv_heads
+    if positions is None:
+        pos = np.concatenate([np.arange(cu[i + 1] - cu[i]) for i in range(len(cu) - 1)] + [np.zeros(0)])
+    else:
+        pos = np.asarray(positions, dtype=np.int64).reshape(-1)
+    out = np.full((N, n_q_heads, d), np.nan)
+    lse = np.full((n_q_heads, N), np.nan)
+    want = None
+    if query_rows is not None:
+        want = np.zeros(N, dtype=bool)
+        want[np.asarray(query_rows, dtype=np.int64)] = True
+
+    for si in range(len(cu) - 1):
+        a, b = int(cu[si]), int(cu[si + 1])
+        L = b - a
+        if L == 0:
+            continue
+        rows = np.arange(L) if want is None else np.nonzero(want[a:b])[0]
+        if rows.size == 0:
+            continue
+        # 2. Rotate Q and K (never V) by each token's position.
+        qr = apply_rope(q[a:b], pos[a:b], rope_theta, operand_rounding)  # [L, n_q, d]
+        kr = apply_rope(k[a:b], pos[a:b], rope_theta, operand_rounding)  # [L, n_kv, d]
+        # 3. Share each KV head across its group of query heads.
+        ks = share_kv_heads(kr, G, axis=1)  # [L, n_q, d]
+        vs = share_kv_heads(v[a:b], G, axis=1)
+        # head-major views [H, L, d]
+        qh = np.transpose(qr, (1, 0, 2))
+        kh = np.transpose(ks, (1, 0, 2))
+        vh = np.transpose(vs, (1, 0, 2))
+        for r0 in range(0, rows.size, row_block):
+            rsel = rows[r0:r0 + row_block]
+            kmax = int(rsel.max()) + 1 if causal else L
+            scores = score(qh[:, rsel, :], kh[:, :kmax, :])  # 4. Score
+            if causal:
+                scores = causal_mask(scores, rsel, np.arange(kmax))  # 5. Mask
+            w, row_lse = softmax_with_lse(scores)  # 5. Softmax
+            o = gather(w, vh[:, :kmax, :])  # 6. Gather, [H, rows, d]
+            out[a + rsel, :, :] = np.transpose(o, (1, 0, 2))
+            lse[:, a + rsel] = row_lse
+    return out, lse
+
+
+def brute_force_attention(q, k, v, cu_seqlens, n_q_heads: int, n_kv_heads: int, rope_theta: float,
+                          positions=None, causal: bool = True):
+    """Pure-Python loops with math.cos/sin/exp, no rounding of the rotated
+    operands. For tiny inputs only (T <= ~16, d <= ~8)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    N, hq, d = q.shape
+    G = n_q_heads // n_kv_heads
+    half = d // 2
+    cu = [int(x) for x in cu_seqlens]
+    out = [[[0.0] * d for _ in range(hq)] for _ in range(N)]
+    lse = [[0.0] * N for _ in range(hq)]
+
+    def rot(vec, p):
+        r = [0.0] * d
+        for i in range(half):
+            ang = p * rope_theta ** (-(2.0 * i) / d)
+            c, s = math.cos(ang), math.sin(ang)
+            r[i] = vec[i] * c - vec[i + half] * s
+            r[i + half] = vec[i + half] * c + vec[i] * s
+        return r
+
+    for si in range(len(cu) - 1):
+        a, b = cu[si], cu[si + 1]
+        for h in range(hq):
+            g = h // G
+            for i in range(a, b):
+                pi = (i - a) if positions is None else int(positions[i])
+                qi = rot(list(q[i, h]), pi)
+                sc = []
+                js = []
+                for j in range(a, b):
+                    if causal and (j - a) > (i - a):
+                        continue
+                    pj = (j - a) if positions is None else int(positions[j])
+                    kj = rot(list(k[j, g]), pj)
+                    sc.append(sum(qi[t] * kj[t] for t in range(d)) / math.sqrt(d))
+                    js.append(j)
+                mx = max(sc)
+                ex = [math.exp(s - mx) for s in sc]
+                z = sum(ex)
+                for t in range(d):
+                    out[i][h][t] = sum(ex[n] * v[js[n], g, t] for n in range(len(js))) / z
+                lse[h][i] = mx + math.log(z)
+    return np.array(out, dtype=np.float64).reshape(N, hq, d), np.array(lse, dtype=np.float64).reshape(hq, N)

@@ -1,0 +1,170 @@
+"""Seeded synthetic inputs for causal GQA + RoPE attention.
+
+This module is shared by the tests, the benchmark and the float64 oracle's
+checks. It only draws random numbers and lays them out; it holds none of the
+attention or RoPE arithmetic. Every array it returns is a plain NumPy array, so
+nothing here touches a GPU.
+
+The five named workloads follow the shapes used throughout the pages' model
+family (the "Attention from Scratch" page's GQA module with n_head query heads
+sharing n_kv_groups key/value heads; the "Embeddings & the Residual Stream"
+page's RoPE with theta = 500000 for the nano config) scaled to Llama-3-8B /
+Qwen2.5-0.5B head layouts:
+
+  tiny      B=1,  T=128,  n_q=4,  n_kv=2, d=32,  theta=1e4, fp32 I/O
+  nano      B=16, T=512,  n_q=6,  n_kv=2, d=64,  theta=1e4
+  qwen05b   B=4,  T=2048, n_q=14, n_kv=2, d=64,  theta=1e6, K scaled by 0.5
+  llama8b   B=1,  T=8192, n_q=32, n_kv=8, d=128, theta=5e5
+  varlen    16384 packed tokens, lengths ~ U{64..4096} (seed 0, last one
+            truncated), n_q=32, n_kv=8, d=128, theta=5e5
+
+Recipe: ``numpy.random.default_rng(seed)`` draws ``standard_normal`` float32
+arrays in the order q, k, v; values are then rounded to bfloat16 (round to
+nearest even, done by ``torch.Tensor.to(torch.bfloat16)``) because the kernel's
+tensor-core operands are bf16. The tiny workload keeps fp32 buffers that hold
+those bf16-representable values. Positions restart at 0 for every sequence.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional
+
+import numpy as np
+
+__all__ = [
+    "Workload",
+    "WORKLOADS",
+    "varlen_lengths",
+    "make_inputs",
+    "make_custom",
+    "to_bf16_values",
+]
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    seq_lens: tuple
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    rope_theta: float
+    causal: bool = True
+    io_dtype: str = "bf16"  # "bf16" or "fp32"
+    k_scale: float = 1.0
+    seed: int = 0
+    description: str = ""
+
+    @property
+    def total_tokens(self) -> int:
+        return int(sum(self.seq_lens))
+
+    @property
+    def num_seqs(self) -> int:
+        return len(self.seq_lens)
+
+    @property
+    def group_size(self) -> int:
+        return self.n_q_heads // self.n_kv_heads
+
+    def flops(self) -> float:
+        """Metric convention: 4*Tq*Tk*d per query head, halved when causal.
+
+        For a packed batch this is summed per sequence: sum_i 4*L_i^2*d*n_q/2.
+        """
+        tot = 0.0
+        for L in self.seq_lens:
+            f = 4.0 * L * L * self.head_dim * self.n_q_heads
+            tot += f / 2.0 if self.causal else f
+        return tot
+
+    def io_bytes(self) -> int:
+        """Algorithmic HBM bytes: read q, k, v once; write out once, lse once."""
+        el = 4 if self.io_dtype == "fp32" else 2
+        n = self.total_tokens
+        d = self.head_dim
+        qo = 2 * n * self.n_q_heads * d * el
+        kv = 2 * n * self.n_kv_heads * d * el
+        lse = n * self.n_q_heads * 4
+        pos = n * 4
+        return qo + kv + lse + pos
+
+
+def varlen_lengths(total: int = 16384, lo: int = 64, hi: int = 4096, seed: int = 0) -> List[int]:
+    """Sequence lengths drawn uniformly from lo..hi inclusive until they cover
+    ``total`` tokens; the last one is truncated so the sum is exactly total."""
+    rng = np.random.default_rng(seed)
+    out: List[int] = []
+    s = 0
+    while s < total:
+        x = int(rng.integers(lo, hi, endpoint=True))
+        x = min(x, total - s)
+        out.append(x)
+        s += x
+    return out
+
+
+WORKLOADS: Dict[str, Workload] = {
+    "tiny": Workload("tiny", (128,), 4, 2, 32, 1e4, io_dtype="fp32", seed=0,
+                     description="B=1 T=128 n_q=4 n_kv=2 d=32 theta=1e4 fp32 I/O causal"),
+    "nano": Workload("nano", (512,) * 16, 6, 2, 64, 1e4, seed=1,
+                     description="B=16 T=512 n_q=6 n_kv=2 d=64 theta=1e4 bf16 causal"),
+    "qwen05b": Workload("qwen05b", (2048,) * 4, 14, 2, 64, 1e6, k_scale=0.5, seed=2,
+                        description="B=4 T=2048 n_q=14 n_kv=2 d=64 theta=1e6 K*0.5 bf16 causal"),
+    "llama8b": Workload("llama8b", (8192,), 32, 8, 128, 5e5, seed=3,
+                        description="B=1 T=8192 n_q=32 n_kv=8 d=128 theta=5e5 bf16 causal"),
+    "varlen": Workload("varlen", tuple(varlen_lengths()), 32, 8, 128, 5e5, seed=4,
+                       description="packed 16384 tokens, L~U{64..4096} seed 0, n_q=32 n_kv=8 d=128 theta=5e5 causal"),
+}
+
+
+def to_bf16_values(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bfloat16 (ties to even) and return
+    them as float32. Uses torch's conversion; this is input preparation, not
+    part of the method."""
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.bfloat16).to(torch.float32).numpy()
+
+
+@dataclass
+class Inputs:
+    workload: Workload
+    q: np.ndarray  # [N, n_q, d] float32 holding bf16-representable values
+    k: np.ndarray  # [N, n_kv, d]
+    v: np.ndarray  # [N, n_kv, d]
+    cu_seqlens: np.ndarray  # [num_seqs+1] int32
+    positions: np.ndarray  # [N] int32, restarting at 0 per sequence
+    extra: dict = field(default_factory=dict)
+
+
+def _cu_and_positions(seq_lens):
+    cu = np.zeros(len(seq_lens) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(np.asarray(seq_lens, dtype=np.int64)).astype(np.int32)
+    pos = np.concatenate([np.arange(L, dtype=np.int32) for L in seq_lens]) if len(seq_lens) else np.zeros(0, np.int32)
+    if pos.size == 0:
+        pos = np.zeros(0, dtype=np.int32)
+    return cu, pos
+
+
+def make_custom(seq_lens, n_q_heads: int, n_kv_heads: int, head_dim: int, rope_theta: float = 1e4,
+                causal: bool = True, seed: int = 0, k_scale: float = 1.0, io_dtype: str = "bf16",
+                name: str = "custom") -> Inputs:
+    w = Workload(name, tuple(int(x) for x in seq_lens), n_q_heads, n_kv_heads, head_dim, float(rope_theta),
+                 causal=causal, io_dtype=io_dtype, k_scale=k_scale, seed=seed)
+    return make_inputs(w)
+
+
+def make_inputs(w: Workload, seed: Optional[int] = None) -> Inputs:
+    rng = np.random.default_rng(w.seed if seed is None else seed)
+    n = w.total_tokens
+    d = w.head_dim
+    q = rng.standard_normal((n, w.n_q_heads, d), dtype=np.float32)
+    k = rng.standard_normal((n, w.n_kv_heads, d), dtype=np.float32)
+    v = rng.standard_normal((n, w.n_kv_heads, d), dtype=np.float32)
+    if w.k_scale != 1.0:
+        k = (k * np.float32(w.k_scale)).astype(np.float32)
+    q, k, v = to_bf16_values(q), to_bf16_values(k), to_bf16_values(v)
+    cu, pos = _cu_and_positions(w.seq_lens)
+    return Inputs(w, q, k, v, cu, pos)
