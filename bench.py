@@ -1,0 +1,337 @@
+#!/usr/bin/env python
+"""Benchmark of the fused causal GQA + RoPE attention forward on B200.
+
+One step = one call of the public C-ABI entry point (prologue kernel +
+attention kernel) over one batch of synthetic, seeded inputs already resident
+in HBM. Default workload: Llama-3-8B-shaped causal prefill (B=1, T=8192,
+32 query / 8 KV heads, d=128, theta=5e5, bf16). Metric: TFLOP/s counting
+4*T*T*d per query head, halved for causal.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   (the float64 CPU oracle, timed)
+
+Under torchrun each rank runs its own replica of the workload (independent
+problems, weak scaling); the elapsed time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal GQA+RoPE attention fwd TFLOP/s on 1 B200; % of dense-BF16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import shutil
+        import tempfile
+        if not shutil.which("nvidia-smi"):
+            return
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        self.fh = open(self.path, "w")
+        self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits", "-lms", "200"],
+                                     stdout=self.fh, stderr=subprocess.DEVNULL)
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle timing
+def cpu_baseline(workload, budget_s: float = 15.0, seed_rows: int = 0):
+    """Times the float64 oracle, as it stands, on a bounded sample of query
+    rows of the workload; returns (TFLOP/s by the metric's convention, info)."""
+    import oracle.gqa_oracle as orc
+    from transformer_attention_gqa_b200 import workloads as wl
+
+    inp = wl.make_inputs(workload)
+    w = workload
+    cu = inp.cu_seqlens
+    rng = np.random.default_rng(seed_rows)
+    # grow the sample until the budget is used
+    n_rows = 8
+    spent, flops, rows_done = 0.0, 0.0, 0
+    while spent < budget_s:
+        rows = np.sort(rng.integers(0, w.total_tokens, n_rows))
+        t0 = time.perf_counter()
+        orc.gqa_rope_attention(inp.q, inp.k, inp.v, cu, w.n_q_heads, w.n_kv_heads, w.rope_theta,
+                               causal=w.causal, query_rows=rows)
+        dt = time.perf_counter() - t0
+        seq = np.searchsorted(cu, rows, side="right") - 1
+        tok = rows - cu[seq]
+        L = cu[seq + 1] - cu[seq]
+        keys = (tok + 1) if w.causal else L
+        # metric convention: 4*Tq*Tk*d per head halved for causal == 4*d per (row, visible key)
+        flops += float(np.sum(4.0 * keys * w.head_dim * w.n_q_heads))
+        spent += dt
+        rows_done += n_rows
+        n_rows = min(n_rows * 2, 4096)
+    cores = len(os.sched_getaffinity(0))
+    threads = None
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((x.get("num_threads", 0) for x in threadpool_info()), default=None)
+    except Exception:
+        pass
+    info = {"value": flops / spent / 1e12, "unit": UNIT, "cores": threads or cores, "kind": "oracle",
+            "sample": f"{rows_done} random query rows x {w.n_q_heads} heads of {w.name}, float64 NumPy, "
+                      f"{spent:.1f} s", "host_cores": cores}
+    return info
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import transformer_attention_gqa_b200 as g
+    from transformer_attention_gqa_b200 import _abi, workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = wl.WORKLOADS[args.workload]
+    inp = wl.make_inputs(w)
+    dt = torch.float32 if w.io_dtype == "fp32" else torch.bfloat16
+    q = torch.from_numpy(inp.q).to(dt).to(dev)
+    k = torch.from_numpy(inp.k).to(dt).to(dev)
+    v = torch.from_numpy(inp.v).to(dt).to(dev)
+    cu = torch.from_numpy(inp.cu_seqlens).to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.n_q_heads, w.total_tokens), dtype=torch.float32, device=dev)
+    ws = g.Workspace(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        g.gqa_rope_attn_fwd(q, k, v, cu, w.rope_theta, causal=w.causal, out=out, lse=lse, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert g.get_device_status() == 0
+    launches_per_step = _abi.last_launch_count()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()  # L2 flush, outside the per-step events
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    wall = time.perf_counter() - t_wall
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+
+    # per-kernel durations (second pass, same stream, events recorded by the library)
+    kern = []
+    for i in range(max(3, min(args.steps, 10))):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        flush.zero_()
+        _abi.set_profile_events(e[0].cuda_event, e[1].cuda_event, e[2].cuda_event)
+        step()
+        kern.append(e)
+    torch.cuda.synchronize()
+    prep_ms = statistics.median(a.elapsed_time(b) for a, b, _ in kern)
+    attn_ms = statistics.median(b.elapsed_time(c) for _, b, c in kern)
+    clk = clocks.stop()
+
+    # end to end through the public API with host buffers
+    qh = torch.from_numpy(inp.q).to(dt).pin_memory()
+    kh = torch.from_numpy(inp.k).to(dt).pin_memory()
+    vh = torch.from_numpy(inp.v).to(dt).pin_memory()
+    cuh = torch.from_numpy(inp.cu_seqlens).pin_memory()
+    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, cuh))
+    d2h = outh.numel() * outh.element_size() + lseh.numel() * lseh.element_size()
+
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        cu.copy_(cuh, non_blocking=True)
+        step()
+        outh.copy_(out, non_blocking=True)
+        lseh.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    assert g.get_device_status() == 0
+
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms, e2e_ms, attn_ms, prep_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms, attn_ms, prep_ms = t.tolist()
+
+    flops = w.flops()
+    ms_per_step = total_ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "shape": w.description, "total_tokens": w.total_tokens,
+                   "num_seqs": w.num_seqs, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+                   "head_dim": w.head_dim, "rope_theta": w.rope_theta, "causal": w.causal,
+                   "flops_per_step": flops, "parallelism": f"replicas x{world}",
+                   "l2": "256 MiB written before every timed step, outside the step's events"},
+        "pct_of_peak": round(100.0 * value / world / peak, 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{src} bf16_tflops (burst)", "kernel": "gqa_attn_fwd_kernel",
+                     "kernel_ms": round(attn_ms, 4), "prologue_ms": round(prep_ms, 4)},
+        "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches_per_step * args.steps,
+        "wall_s": round(wall, 4),
+    }
+    if clk:
+        res["clocks"] = clk
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from transformer_attention_gqa_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        per_step = []
+        for _ in range(args.warmup):
+            cpu_baseline(w, budget_s=0.5)
+        info = None
+        for _ in range(args.steps):
+            info = cpu_baseline(w, budget_s=max(1.0, 60.0 / max(args.steps, 1)))
+            per_step.append(info["value"])
+        val = statistics.median(per_step)
+        res = {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": UNIT, "n_gpus": world,
+               "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+               "config": {"workload": w.name, "shape": w.description},
+               "cpu_baseline": {"value": round(val, 6), "unit": UNIT, "cores": info["cores"], "kind": "oracle",
+                                "sample": info["sample"]},
+               "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(res))
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,149 @@
+/*
+ * gqa_rope_attn.h -- C ABI of the B200 (sm_100a) fused causal grouped-query
+ * attention with rotary position embeddings.
+ *
+ * The operation (per sequence s of a packed batch, per query head h, with
+ * G = n_q_heads / n_kv_heads and kv = h / G):
+ *
+ *   out[t, h, :] = softmax_j( rope(q[t, h]) . rope(k[j, kv]) / sqrt(d) ) v[j, kv]
+ *   lse[h, t]    = ln sum_j exp( rope(q[t, h]) . rope(k[j, kv]) / sqrt(d) )
+ *
+ * over keys j of the same sequence with j <= t (causal) or all j of the
+ * sequence (causal = 0). Sources:
+ *   - "Attention from Scratch", section "Attention, the math: Grouped-Query
+ *     Attention with RoPE'd Q/K": rotate Q and K (never V), share each KV
+ *     head over a group of consecutive query heads (repeat_interleave),
+ *     score q.k^T / sqrt(head_dim), fill the future with -inf, softmax,
+ *     weights @ v.
+ *   - "Embeddings & the Residual Stream", section "Positional information:
+ *     RoPE, not a learned table": inv_freq[i] = theta^(-2i/d), angle =
+ *     position * inv_freq[i], x*cos + rotate_half(x)*sin, i.e. feature i is
+ *     rotated together with feature i + d/2.
+ *   - "Kohaku-TT", Highlights: flash attention over packed variable-length
+ *     batches (cu_seqlens prefix sums).
+ *   The log-sum-exp output is not on the pages; it is the natural-log
+ *   normaliser of each row's scaled, masked scores.
+ *
+ * Precision: q, k, v, out are bf16 (or fp32 with dtype GQA_DTYPE_FP32; then
+ * q, k, v are rounded to bf16 on load and out is written as fp32). cos/sin
+ * are the fp32 values of the float64 angle's cos/sin; the rotated q and k are
+ * rounded once, to nearest even, to bf16 (the tensor-core operands). Scores
+ * and the output accumulate in fp32; the softmax weights enter P.V as bf16.
+ * lse is fp32.
+ *
+ * Memory layout ("THD", all row-major, contiguous, device memory):
+ *   q          [total_tokens, n_q_heads,  head_dim]
+ *   k, v       [total_tokens, n_kv_heads, head_dim]
+ *   out        [total_tokens, n_q_heads,  head_dim]
+ *   lse        [n_q_heads, total_tokens]  fp32
+ *   positions  [total_tokens] int32
+ *   cu_seqlens [num_seqs + 1] int32, cu[0] = 0, nondecreasing,
+ *              cu[num_seqs] = total_tokens
+ * A fixed batch [B, T, ...] is the same memory with cu = {0, T, 2T, ..., BT}.
+ *
+ * Ownership: the caller allocates and owns every buffer, the workspace
+ * included. The library keeps only a cache of TMA descriptors (per device)
+ * and a device status word. It allocates nothing per call and never
+ * synchronises inside gqa_rope_attn_fwd.
+ */
+#ifndef GQA_ROPE_ATTN_H_
+#define GQA_ROPE_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GQA_ROPE_ATTN_ABI_VERSION 1
+
+/* Element type of q, k, v and out. */
+typedef enum gqa_dtype_e {
+  GQA_DTYPE_BF16 = 0,
+  GQA_DTYPE_FP32 = 1
+} gqa_dtype_t;
+
+/* Status codes. Host-detected errors are returned by the call itself before
+ * any CUDA work is queued; device-detected ones are read later with
+ * gqa_rope_attn_get_device_status. */
+enum {
+  GQA_OK = 0,
+  GQA_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size or flag   */
+  GQA_ERR_UNSUPPORTED = 2, /* head_dim not in {32,64,128}, group > 128, ... */
+  GQA_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed          */
+  GQA_ERR_BAD_SEQLENS = 4, /* device: cu_seqlens not a valid prefix sum     */
+  GQA_ERR_TIMEOUT = 5,     /* device: a bounded wait in the kernel ran out  */
+  GQA_ERR_WORKSPACE = 6    /* workspace missing, too small or misaligned    */
+};
+
+/* Bytes of scratch the caller must pass to gqa_rope_attn_fwd for this shape
+ * (the RoPE'd K in head-major layout, the cos/sin table, the tile schedule
+ * and, for fp32 inputs, bf16 copies of q and v). Returns 0 for invalid
+ * arguments. Pure host arithmetic: no CUDA call. */
+size_t gqa_rope_attn_workspace_size(int num_seqs, int total_tokens, int n_q_heads,
+                                    int n_kv_heads, int head_dim, int dtype);
+
+/* The fused forward.
+ *
+ * q, k, v      device pointers, layout above, 16-byte aligned.
+ * positions    device int32 [total_tokens] giving each token's RoPE
+ *              position, or NULL for the index inside its sequence. The
+ *              causal mask always uses the index inside the sequence.
+ * rope_theta   RoPE base, finite and > 0.
+ * cu_seqlens   device int32 [num_seqs + 1]. Checked on the device: a bad
+ *              array makes the call write nothing and sets
+ *              GQA_ERR_BAD_SEQLENS in the device status word.
+ * num_seqs     >= 1 (or 0 with total_tokens == 0).
+ * total_tokens >= 0; 0 is a no-op returning GQA_OK.
+ * n_q_heads, n_kv_heads  >= 1, n_q_heads % n_kv_heads == 0,
+ *              n_q_heads / n_kv_heads <= 128.
+ * head_dim     32, 64 or 128.
+ * causal       1: key j visible to query t iff j <= t inside the sequence;
+ *              0: every key of the sequence is visible.
+ * dtype        GQA_DTYPE_BF16 or GQA_DTYPE_FP32 (for q, k, v and out).
+ * out          device pointer, written for every token of every sequence.
+ * lse          device fp32 [n_q_heads, total_tokens] or NULL.
+ * workspace    device scratch of at least gqa_rope_attn_workspace_size()
+ *              bytes, 256-byte aligned; contents need not be initialised;
+ *              it must not be shared by calls that may overlap on the GPU.
+ * stream       a cudaStream_t (passed as void*), NULL for the default
+ *              stream. Work is queued on it; the call does not wait.
+ *
+ * Returns GQA_OK or an error code; on an error nothing has been queued.
+ */
+int gqa_rope_attn_fwd(const void* q, const void* k, const void* v, const int32_t* positions,
+                      double rope_theta, const int32_t* cu_seqlens, int num_seqs,
+                      int total_tokens, int n_q_heads, int n_kv_heads, int head_dim,
+                      int causal, int dtype, void* out, float* lse, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/* Waits for `stream` (a cudaStream_t as void*, NULL for the default stream),
+ * then returns and clears the current device's status word: GQA_OK, or the
+ * first device-detected error (GQA_ERR_BAD_SEQLENS, GQA_ERR_TIMEOUT) since
+ * the last read. Returns GQA_ERR_CUDA if the synchronisation fails. */
+int gqa_rope_attn_get_device_status(void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* gqa_rope_attn_strerror(int status);
+
+/* GQA_ROPE_ATTN_ABI_VERSION of the loaded library. */
+int gqa_rope_attn_abi_version(void);
+
+/* Number of kernel launches the last successful gqa_rope_attn_fwd queued on
+ * the calling thread (0 for a no-op). */
+int gqa_rope_attn_last_launch_count(void);
+
+/* Measurement aid. Arms the calling thread's next gqa_rope_attn_fwd call to
+ * record three CUDA events (cudaEvent_t passed as void*, any may be NULL) on
+ * its stream: before the prologue kernel, between the prologue and the
+ * attention kernel, and after the attention kernel, so that each kernel's
+ * duration can be read with cudaEventElapsedTime. The arming is consumed by
+ * that one call (also when it fails). The caller owns the events. */
+void gqa_rope_attn_set_profile_events(void* ev_start, void* ev_mid, void* ev_end);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_ROPE_ATTN_H_ */

@@ -1,0 +1,106 @@
+"""CPU-only checks of the C ABI: the library loads, exports every function
+include/gqa_rope_attn.h declares, and rejects bad arguments on the host
+before any CUDA call (no GPU is touched here)."""
+import os
+import re
+import subprocess
+
+import pytest
+
+from transformer_attention_gqa_b200 import _abi
+from transformer_attention_gqa_b200.build import LIB, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build()
+    _abi.load()
+
+
+def declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for fn in sorted(os.listdir(inc)):
+        if fn.endswith(".h"):
+            text = open(os.path.join(inc, fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(gqa_rope_attn_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_function():
+    decl = declared_functions()
+    assert "gqa_rope_attn_fwd" in decl and len(decl) >= 5
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (gqa_rope_attn_\w+)", out))
+    assert set(decl) <= exported, set(decl) - exported
+    lib = _abi.load()
+    for name in decl:
+        assert hasattr(lib, name)
+    assert set(_abi.EXPORTED) == set(decl)
+
+
+def test_abi_version_and_strerror():
+    assert _abi.abi_version() == 1
+    for code in range(7):
+        assert isinstance(_abi.strerror(code), str) and _abi.strerror(code)
+    assert _abi.strerror(99) == "unknown status"
+
+
+def test_workspace_size():
+    ws = _abi.workspace_size(1, 8192, 32, 8, 128)
+    # at least the RoPE'd K (n_kv * N * d * 2) and the cos/sin table (N * d/2 * 8)
+    assert ws >= 8 * 8192 * 128 * 2 + 8192 * 64 * 8
+    assert ws % 256 == 0
+    assert _abi.workspace_size(1, 8192, 32, 8, 128, _abi.GQA_DTYPE_FP32) > ws
+    assert _abi.workspace_size(1, 8192, 32, 8, 96) == 0
+    assert _abi.workspace_size(1, 8192, 30, 8, 128) == 0
+    assert _abi.workspace_size(1, 8192, 256, 1, 128) == 0  # group of 256 heads
+    assert _abi.workspace_size(-1, 8192, 32, 8, 128) == 0
+    assert _abi.workspace_size(2, 100, 4, 2, 64) < _abi.workspace_size(2, 200, 4, 2, 64)
+
+
+A = 4096  # fake, 256-byte aligned "device" addresses; never dereferenced by these checks
+
+
+def call(**kw):
+    args = dict(q=A, k=A, v=A, positions=0, rope_theta=1e4, cu_seqlens=A, num_seqs=1, total_tokens=128,
+                n_q_heads=4, n_kv_heads=2, head_dim=64, causal=1, dtype=0, out=A, lse=0, workspace=0,
+                workspace_bytes=0, stream=None)
+    args.update(kw)
+    return _abi.gqa_rope_attn_fwd(**args)
+
+
+def test_host_rejections_before_any_cuda_call():
+    E = _abi
+    assert call(total_tokens=0) == E.GQA_OK  # no-op
+    assert call(total_tokens=-1) == E.GQA_ERR_INVALID_ARG
+    assert call(n_q_heads=6, n_kv_heads=4) == E.GQA_ERR_INVALID_ARG
+    assert call(n_kv_heads=0) == E.GQA_ERR_INVALID_ARG
+    assert call(causal=2) == E.GQA_ERR_INVALID_ARG
+    assert call(dtype=7) == E.GQA_ERR_INVALID_ARG
+    assert call(rope_theta=0.0) == E.GQA_ERR_INVALID_ARG
+    assert call(rope_theta=float("nan")) == E.GQA_ERR_INVALID_ARG
+    assert call(head_dim=96) == E.GQA_ERR_UNSUPPORTED
+    assert call(n_q_heads=256, n_kv_heads=1) == E.GQA_ERR_UNSUPPORTED
+    assert call(num_seqs=0) == E.GQA_ERR_INVALID_ARG
+    assert call(q=0) == E.GQA_ERR_INVALID_ARG
+    assert call(out=0) == E.GQA_ERR_INVALID_ARG
+    assert call(cu_seqlens=0) == E.GQA_ERR_INVALID_ARG
+    assert call(k=A + 8) == E.GQA_ERR_INVALID_ARG  # misaligned
+    assert call(lse=A + 2) == E.GQA_ERR_INVALID_ARG
+    # every argument fine but the workspace
+    assert call() == E.GQA_ERR_WORKSPACE
+    need = _abi.workspace_size(1, 128, 4, 2, 64)
+    assert call(workspace=A, workspace_bytes=need - 1) == E.GQA_ERR_WORKSPACE
+    assert call(workspace=A + 16, workspace_bytes=need) == E.GQA_ERR_WORKSPACE
+    assert _abi.last_launch_count() == 0
+
+
+def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_abi, "_lib", None)
+    with pytest.raises(ImportError):
+        _abi.load()

@@ -1,0 +1,119 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+the same seeded, bf16-rounded inputs. Small workloads are compared element
+by element in full; the Llama-3-8B-shaped and packed variable-length
+workloads run at full size in the benchmark's launch configuration and are
+compared on sampled rows the oracle computes one by one."""
+import numpy as np
+import pytest
+
+from tests.conftest import gpu_available
+from tests import gpu_helpers as H
+from transformer_attention_gqa_b200 import workloads as wl
+
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not gpu_available(), reason="needs a CUDA device")]
+
+
+@pytest.mark.parametrize("name", ["tiny", "nano", "qwen05b"])
+def test_named_workload_full(name):
+    inp = wl.make_inputs(wl.WORKLOADS[name])
+    out, lse = H.run_gpu(inp)
+    ref_out, ref_lse = H.oracle(inp)
+    H.compare(out, lse, ref_out, ref_lse, what=name)
+    # outputs also stay within the bar of the unrounded (exact RoPE) oracle
+    ex_out, _ = H.oracle(inp, operand_rounding=False)
+    H.compare(out, None, ex_out, None, what=name + " vs exact RoPE")
+
+
+@pytest.mark.parametrize("name", ["llama8b", "varlen"])
+def test_named_workload_sampled_rows(name):
+    inp = wl.make_inputs(wl.WORKLOADS[name])
+    out, lse = H.run_gpu(inp)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+    rows = H.sample_rows(inp.cu_seqlens, per_seq=16 if name == "varlen" else 48)
+    ref_out, ref_lse = H.oracle(inp, rows=rows)
+    H.compare(out, lse, ref_out, ref_lse, rows=rows, what=name)
+
+
+CASES = [
+    # (seq_lens, n_q, n_kv, d, theta, causal)
+    ([1], 4, 2, 64, 1e4, True),
+    ([1, 1, 1], 8, 8, 128, 5e5, True),
+    ([33], 4, 1, 32, 1e4, True),
+    ([127, 129], 6, 2, 64, 1e4, True),
+    ([300, 0, 45], 14, 2, 64, 1e6, True),
+    ([0, 257], 32, 8, 128, 5e5, True),
+    ([200], 3, 1, 128, 1e4, True),
+    ([131, 64], 16, 2, 128, 5e5, True),
+    ([90], 7, 7, 64, 1e4, True),
+    ([513], 128, 1, 32, 1e4, True),
+    ([100, 260], 8, 2, 64, 1e4, False),
+    ([1, 130], 4, 4, 128, 5e5, False),
+    ([77, 1000, 5], 24, 3, 128, 5e5, True),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"L{c[0]}-q{c[1]}-kv{c[2]}-d{c[3]}-c{int(c[5])}" for c in CASES])
+def test_edge_shapes(case):
+    lens, nq, nkv, d, theta, causal = case
+    inp = wl.make_custom(lens, nq, nkv, d, theta, causal=causal, seed=sum(lens) + nq)
+    out, lse = H.run_gpu(inp)
+    ref_out, ref_lse = H.oracle(inp)
+    H.compare(out, lse, ref_out, ref_lse, what=str(case))
+
+
+def test_explicit_positions_and_fp32_io():
+    inp = wl.make_custom([70, 190], 8, 2, 64, 1e4, seed=5)
+    pos = np.random.default_rng(3).integers(0, 20000, inp.workload.total_tokens).astype(np.int32)
+    out, lse = H.run_gpu(inp, positions=pos)
+    ref_out, ref_lse = H.oracle(inp, positions=pos)
+    H.compare(out, lse, ref_out, ref_lse, what="positions")
+    inp32 = wl.make_custom([150], 4, 2, 128, 5e5, io_dtype="fp32", seed=6)
+    out, lse = H.run_gpu(inp32)
+    ref_out, ref_lse = H.oracle(inp32)
+    H.compare(out, lse, ref_out, ref_lse, what="fp32 io")
+
+
+def test_without_lse_and_deterministic():
+    inp = wl.make_custom([400, 96], 8, 2, 128, 5e5, seed=7)
+    o1, _ = H.run_gpu(inp, need_lse=False)
+    o2, l2 = H.run_gpu(inp)
+    assert np.array_equal(o1, o2)
+    ref_out, ref_lse = H.oracle(inp)
+    H.compare(o2, l2, ref_out, ref_lse, what="no-lse")
+
+
+def test_no_write_outside_outputs():
+    import torch
+    import transformer_attention_gqa_b200 as g
+
+    inp = wl.make_custom([65, 30], 6, 2, 64, 1e4, seed=8)
+    q, k, v, cu, _ = H.to_device(inp)
+    N, nq, d = q.shape
+    canary = 12345.0
+    big = torch.full((N + 64, nq, d), canary, dtype=torch.bfloat16, device="cuda")
+    out = big[:N]
+    lse_big = torch.full((nq * N + 256,), canary, dtype=torch.float32, device="cuda")
+    lse = lse_big[: nq * N].view(nq, N)
+    g.gqa_rope_attn_fwd(q, k, v, cu, 1e4, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert g.get_device_status() == 0
+    assert torch.all(big[N:] == canary)
+    assert torch.all(lse_big[nq * N:] == canary)
+    ref_out, ref_lse = H.oracle(inp)
+    H.compare(out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64), ref_out, ref_lse)
+
+
+def test_bad_cu_seqlens_sets_status_and_writes_nothing():
+    import torch
+    import transformer_attention_gqa_b200 as g
+
+    inp = wl.make_custom([64, 64], 4, 2, 64, 1e4, seed=9)
+    q, k, v, _, _ = H.to_device(inp)
+    for bad in ([0, 100, 64, 128], [0, 64, 100], [3, 64, 128]):
+        cu = torch.tensor(bad, dtype=torch.int32, device="cuda")
+        out = torch.zeros_like(q)
+        g.gqa_rope_attn_fwd(q, k, v, cu, 1e4, out=out)
+        torch.cuda.synchronize()
+        assert g.get_device_status() == 4
+        assert g.get_device_status() == 0  # cleared by the read
+        assert torch.all(out == 0)

@@ -1,0 +1,525 @@
+// Fused causal GQA + RoPE attention forward for sm_100a.
+//
+// What it computes ("Attention from Scratch", section "Attention, the math:
+// Grouped-Query Attention with RoPE'd Q/K"): for every query head h of KV
+// group kv = h / G, softmax(rope(q) . rope(k)^T / sqrt(d) + causal mask) . v,
+// plus the natural-log log-sum-exp of every row. The score matrix never
+// leaves the SM ("Coming from CUDA: FlashAttention"): each KV tile's scores
+// are produced in tensor memory, turned into probabilities by an online
+// (running max / running sum) softmax and consumed by the P.V product.
+//
+// One persistent CTA per SM walks a static, longest-first list of work
+// items (sequence, q-tile, KV head). A q-tile packs tq = 128 / G tokens
+// times the G query heads of one KV head into 128 MMA rows, so every K/V
+// tile loaded by TMA is used by all G heads at once.
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q tile and K tiles (K is RoPE'd already)
+//   warp 1      TMEM allocator and the single MMA-issuing thread
+//   warp 2      TMA producer: V tiles
+//   warp 3      idle
+//   warps 4-7   softmax: one thread per row (TMEM lane), S -> P, running
+//               max/sum, O rescale, epilogue (O / l, LSE)
+//   warps 8-11  Q rotation: RoPE applied in shared memory to each Q tile
+//               after its TMA load, before the first S MMA reads it
+//
+// Tensor memory (512 columns x 128 lanes of 32 bit):
+//   [0,128) [128,256) [256,384): three S buffers; the bf16 P of a tile
+//   overwrites the first 64 columns of its own S buffer; [384, 384+d): O.
+// MMAs: S = Q K^T   kind::f16, A = Q (smem, K-major), B = K (smem, K-major),
+//                   M = 128, N = 128, fp32 accumulate, d/16 steps;
+//       O += P V    A = P (tmem), B = V (smem, MN-major), M = 128, N = d,
+//                   8 steps of 16 keys.
+#pragma once
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace gqa {
+
+
+template <int D>
+struct AttnCfg {
+  static constexpr int BOXC = D >= 64 ? 64 : 32;   // columns per TMA box
+  static constexpr int NBOX = D / BOXC;            // boxes per row of a tile
+  static constexpr int ROWB = BOXC * 2;            // bytes per box row (swizzle span)
+  static constexpr int SWZ_MASK = ROWB == 128 ? 7 : 3;
+  static constexpr uint64_t UMMA_LAYOUT = ROWB == 128 ? 2 : 4;  // SWIZZLE_128B / SWIZZLE_64B
+  static constexpr int SBO = 8 * ROWB;             // bytes between 8-row core-matrix groups
+  static constexpr int Q_BOX_BYTES = BM * ROWB;
+  static constexpr int KV_BOX_BYTES = BN * ROWB;
+  static constexpr int Q_BYTES = NBOX * Q_BOX_BYTES;
+  static constexpr int KV_BYTES = NBOX * KV_BOX_BYTES;
+  static constexpr int KST = D == 128 ? 2 : (D == 64 ? 3 : 4);
+  static constexpr int VST = KST;
+  static constexpr int OFF_K = 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t O_COL = 384;
+  static constexpr int KSTEPS_S = D / 16;
+  static constexpr int KSTEPS_PV = BN / 16;
+  static constexpr int STEPS_PER_BOX = BOXC / 16;
+  // instruction descriptors: bf16 x bf16 -> fp32, M = 128
+  static constexpr uint32_t IDESC_S =
+      (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  static constexpr uint32_t IDESC_O = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                                      ((uint32_t)(D >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(O_COL + D <= TMEM_COLS, "tensor memory budget");
+};
+
+// Shared-memory matrix descriptor (tcgen05): start, leading/stride byte
+// offsets (in 16-byte units), fixed version field 1, swizzle layout type.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint64_t layout) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (layout << 61);
+}
+
+struct Barriers {
+  uint64_t q_loaded[2], q_ready[2], q_empty[2];
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t s_full[NUM_S_BUF], p_full[NUM_S_BUF], pv_done[NUM_S_BUF];
+  uint64_t o_free, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct WorkItem {
+  int seq_start, L, t0, nkv, kvh;
+};
+
+__device__ __forceinline__ WorkItem decode_item(const AttnParams& p, int w) {
+  WorkItem it;
+  const int pair = w / p.nkv;
+  it.kvh = w - pair * p.nkv;
+  const int2 sl = p.pairs[pair];
+  it.seq_start = __ldg(p.cu + sl.x);
+  it.L = __ldg(p.cu + sl.x + 1) - it.seq_start;
+  it.t0 = sl.y * p.tq;
+  const int t_end = p.causal ? min(it.t0 + p.tq, it.L) : it.L;
+  it.nkv = (t_end + BN - 1) / BN;
+  return it;
+}
+
+// Bounded wait on an mbarrier phase. Returns false if the CTA is aborting or
+// the wait exceeded WAIT_TIMEOUT_NS (then the abort flag and the device
+// status word are set).
+__device__ __forceinline__ bool bwait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (ptx::globaltimer() - t0 > WAIT_TIMEOUT_NS) {
+      *abort_flag = 1;
+      atomicCAS(&g_status, 0, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag (used to drain in-flight copies).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if (ptx::globaltimer() - t0 > WAIT_TIMEOUT_NS) {
+      atomicCAS(&g_status, 0, kStatusTimeout);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t swz(uint32_t lin, int mask) { return lin ^ (((lin >> 7) & mask) << 4); }
+
+template <int D, bool OUT_FP32>
+__global__ void __launch_bounds__(ATTN_THREADS, 1)
+    gqa_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using C = AttnCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + C::OFF_BAR);
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  volatile int* abort_flag = &bars->abort_flag;
+
+  auto B = [&](uint64_t& b) { return ptx::smem_u32(&b); };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(B(bars->q_loaded[i]), 1);
+      ptx::mbar_init(B(bars->q_ready[i]), 128);
+      ptx::mbar_init(B(bars->q_empty[i]), 1);
+    }
+    for (int i = 0; i < C::KST; ++i) {
+      ptx::mbar_init(B(bars->k_full[i]), 1);
+      ptx::mbar_init(B(bars->k_empty[i]), 1);
+    }
+    for (int i = 0; i < C::VST; ++i) {
+      ptx::mbar_init(B(bars->v_full[i]), 1);
+      ptx::mbar_init(B(bars->v_empty[i]), 1);
+    }
+    for (int i = 0; i < NUM_S_BUF; ++i) {
+      ptx::mbar_init(B(bars->s_full[i]), 1);
+      ptx::mbar_init(B(bars->p_full[i]), 128);
+      ptx::mbar_init(B(bars->pv_done[i]), 1);
+    }
+    ptx::mbar_init(B(bars->o_free), 128);
+    ptx::mbar_init(B(bars->drain), 1);
+    bars->abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmQ);
+    ptx::prefetch_tmap(&tmK);
+    ptx::prefetch_tmap(&tmV);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(&bars->tmem_base), C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  // Everything below reads what the prologue kernel wrote.
+  ptx::griddep_wait();
+  const int n_items = __ldg(p.header) * p.nkv;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ Q/K producer
+    if (lane == 0) {
+      int q_uses[2] = {0, 0};
+      int k_uses[C::KST];
+      for (int i = 0; i < C::KST; ++i) k_uses[i] = 0;
+      uint32_t g = 0;
+      int it = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
+        const WorkItem wi = decode_item(p, w);
+        const int qb = it & 1;
+        if (!(ok = bwait(B(bars->q_empty[qb]), ((it >> 1) & 1) ^ 1, abort_flag))) break;
+        ptx::mbar_arrive_expect_tx(B(bars->q_loaded[qb]), (uint32_t)(D * 2 * p.G * p.tq));
+        for (int b = 0; b < C::NBOX; ++b)
+          ptx::tma_load_3d(sbase + qb * C::Q_BYTES + b * C::Q_BOX_BYTES, &tmQ, B(bars->q_loaded[qb]),
+                           b * C::BOXC, wi.kvh * p.G, wi.seq_start + wi.t0);
+        ++q_uses[qb];
+        for (int j = 0; j < wi.nkv; ++j, ++g) {
+          const int ks = g % C::KST;
+          if (!(ok = bwait(B(bars->k_empty[ks]), ((g / C::KST) & 1) ^ 1, abort_flag))) break;
+          ptx::mbar_arrive_expect_tx(B(bars->k_full[ks]), (uint32_t)C::KV_BYTES);
+          for (int b = 0; b < C::NBOX; ++b)
+            ptx::tma_load_3d(sbase + C::OFF_K + ks * C::KV_BYTES + b * C::KV_BOX_BYTES, &tmK,
+                             B(bars->k_full[ks]), b * C::BOXC, wi.seq_start + j * BN, wi.kvh);
+          ++k_uses[ks];
+        }
+      }
+      if (!ok) {  // let every copy already issued land before the CTA exits
+        for (int i = 0; i < 2; ++i)
+          if (q_uses[i]) drain_wait(B(bars->q_loaded[i]), (q_uses[i] - 1) & 1);
+        for (int i = 0; i < C::KST; ++i)
+          if (k_uses[i]) drain_wait(B(bars->k_full[i]), (k_uses[i] - 1) & 1);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ V producer
+    if (lane == 0) {
+      int v_uses[C::VST];
+      for (int i = 0; i < C::VST; ++i) v_uses[i] = 0;
+      uint32_t g = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+        const WorkItem wi = decode_item(p, w);
+        for (int j = 0; j < wi.nkv; ++j, ++g) {
+          const int vs = g % C::VST;
+          if (!(ok = bwait(B(bars->v_empty[vs]), ((g / C::VST) & 1) ^ 1, abort_flag))) break;
+          ptx::mbar_arrive_expect_tx(B(bars->v_full[vs]), (uint32_t)C::KV_BYTES);
+          for (int b = 0; b < C::NBOX; ++b)
+            ptx::tma_load_3d(sbase + C::OFF_V + vs * C::KV_BYTES + b * C::KV_BOX_BYTES, &tmV,
+                             B(bars->v_full[vs]), b * C::BOXC, wi.kvh, wi.seq_start + j * BN);
+          ++v_uses[vs];
+        }
+      }
+      if (!ok) {
+        for (int i = 0; i < C::VST; ++i)
+          if (v_uses[i]) drain_wait(B(bars->v_full[i]), (v_uses[i] - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t g = 0;
+      int it = 0;
+      bool ok = true;
+      // S(gg) = Q K(gg)^T into S buffer gg % 3
+      auto issue_s = [&](uint32_t gg, int qb) -> bool {
+        const int b = gg % NUM_S_BUF;
+        if (gg >= NUM_S_BUF)  // PV(gg - 3) read P from this buffer
+          if (!bwait(B(bars->pv_done[b]), ((gg / NUM_S_BUF) - 1) & 1, abort_flag)) return false;
+        const int ks = gg % C::KST;
+        if (!bwait(B(bars->k_full[ks]), (gg / C::KST) & 1, abort_flag)) return false;
+        ptx::tc_fence_after();
+        const uint32_t qaddr = sbase + qb * C::Q_BYTES;
+        const uint32_t kaddr = sbase + C::OFF_K + ks * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < C::KSTEPS_S; ++kk) {
+          const uint32_t off_q = (kk / C::STEPS_PER_BOX) * C::Q_BOX_BYTES + (kk % C::STEPS_PER_BOX) * 32;
+          const uint32_t off_k = (kk / C::STEPS_PER_BOX) * C::KV_BOX_BYTES + (kk % C::STEPS_PER_BOX) * 32;
+          ptx::mma_ss(tmem + b * 128, umma_desc(qaddr + off_q, 16, C::SBO, C::UMMA_LAYOUT),
+                      umma_desc(kaddr + off_k, 16, C::SBO, C::UMMA_LAYOUT), C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(B(bars->s_full[b]));
+        ptx::mma_commit(B(bars->k_empty[ks]));
+        return true;
+      };
+      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
+        const WorkItem wi = decode_item(p, w);
+        const int qb = it & 1;
+        if (!(ok = bwait(B(bars->q_ready[qb]), (it >> 1) & 1, abort_flag))) break;
+        ptx::tc_fence_after();
+        const int npre = wi.nkv < 2 ? wi.nkv : 2;
+        for (int jj = 0; ok && jj < npre; ++jj) ok = issue_s(g + jj, qb);
+        for (int j = 0; ok && j < wi.nkv; ++j) {
+          const uint32_t gg = g + j;
+          const int b = gg % NUM_S_BUF;
+          const int vs = gg % C::VST;
+          if (!(ok = bwait(B(bars->p_full[b]), (gg / NUM_S_BUF) & 1, abort_flag))) break;
+          if (!(ok = bwait(B(bars->v_full[vs]), (gg / C::VST) & 1, abort_flag))) break;
+          if (j == 0 && !(ok = bwait(B(bars->o_free), (it & 1) ^ 1, abort_flag))) break;
+          ptx::tc_fence_after();
+          const uint32_t vaddr = sbase + C::OFF_V + vs * C::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < C::KSTEPS_PV; ++kk) {
+            ptx::mma_ts(tmem + C::O_COL, tmem + b * 128 + kk * 8,
+                        umma_desc(vaddr + kk * 16 * C::ROWB, C::KV_BOX_BYTES, C::SBO, C::UMMA_LAYOUT),
+                        C::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          ptx::mma_commit(B(bars->pv_done[b]));
+          ptx::mma_commit(B(bars->v_empty[vs]));
+          if (j == wi.nkv - 1) ptx::mma_commit(B(bars->q_empty[qb]));
+          if (j + 2 < wi.nkv) ok = issue_s(gg + 2, qb);
+        }
+        g += wi.nkv;
+      }
+      // all tensor-core work of this CTA has finished before TMEM is freed
+      ptx::mma_commit(B(bars->drain));
+      drain_wait(B(bars->drain), 0);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ softmax
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // row of the tile == TMEM lane
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const int G = p.G;
+    const int tok_off = r / G;
+    const int hin = r - tok_off * G;
+    const bool row_in_tile = r < p.tq * G;
+    const float sl2 = p.scale_log2;
+    uint32_t g = 0;
+    int it = 0;
+    bool ok = true;
+    uint32_t sr[128];
+    for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
+      const WorkItem wi = decode_item(p, w);
+      const int tok = wi.t0 + tok_off;  // index inside the sequence
+      const int last_key = p.causal ? tok : wi.L - 1;
+      float m = -INFINITY;
+      float l = 0.f;
+      for (int j = 0; j < wi.nkv; ++j) {
+        const uint32_t gg = g + j;
+        const int b = gg % NUM_S_BUF;
+        ok = __all_sync(0xffffffffu, bwait(B(bars->s_full[b]), (gg / NUM_S_BUF) & 1, abort_flag));
+        if (!ok) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(trow + b * 128 + c * 32, sr + c * 32);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::reg_fence32(sr + c * 32);
+        const int lim = last_key - j * BN;  // columns > lim are masked
+        if (lim < BN - 1) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c > lim) sr[c] = __float_as_uint(-INFINITY);
+        }
+        float mx = __uint_as_float(sr[0]);
+#pragma unroll
+        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+        float alpha = 1.f;
+        bool need = false;
+        if (j == 0) {
+          m = mx;
+        } else if (mx > m + p.rescale_thr) {
+          alpha = ptx::ex2((m - mx) * sl2);
+          m = mx;
+          need = true;
+        }
+        const float neg = -m * sl2;
+        float lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[c]), sl2, neg));
+          const float p1 = ptx::ex2(fmaf(__uint_as_float(sr[c + 1]), sl2, neg));
+          lsum += p0 + p1;
+          const __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
+          sr[c >> 1] = *reinterpret_cast<const uint32_t*>(&pk);
+        }
+        l = l * alpha + lsum;
+        ptx::tmem_st32(trow + b * 128, sr);
+        ptx::tmem_st32(trow + b * 128 + 32, sr + 32);
+        if (__any_sync(0xffffffffu, need)) {
+          // O holds the sum up to the previous tile: wait for PV(gg-1), then scale.
+          const uint32_t gp = gg - 1;
+          ok = __all_sync(0xffffffffu,
+                          bwait(B(bars->pv_done[gp % NUM_S_BUF]), (gp / NUM_S_BUF) & 1, abort_flag));
+          if (!ok) break;
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t* o = sr + 64;
+            ptx::tmem_ld32(trow + C::O_COL + c * 32, o);
+            ptx::tmem_wait_ld();
+            ptx::reg_fence32(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            ptx::tmem_st32(trow + C::O_COL + c * 32, o);
+          }
+        }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(B(bars->p_full[b]));
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l and LSE
+      const uint32_t gl = g + wi.nkv - 1;
+      ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[gl % NUM_S_BUF]), (gl / NUM_S_BUF) & 1, abort_flag));
+      if (!ok) break;
+      ptx::tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(trow + C::O_COL + c * 32, sr + c * 32);
+      ptx::tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) ptx::reg_fence32(sr + c * 32);
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(B(bars->o_free));
+      if (row_in_tile && tok < wi.L) {
+        const float inv_l = 1.f / l;
+        const int h = wi.kvh * G + hin;
+        const size_t row = (size_t)(wi.seq_start + tok) * p.nq + h;
+        if constexpr (OUT_FP32) {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + row * D);
+#pragma unroll
+          for (int c = 0; c < D; c += 4)
+            dst[c / 4] = make_float4(__uint_as_float(sr[c]) * inv_l, __uint_as_float(sr[c + 1]) * inv_l,
+                                     __uint_as_float(sr[c + 2]) * inv_l, __uint_as_float(sr[c + 3]) * inv_l);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + row * D);
+#pragma unroll
+          for (int c = 0; c < D; c += 8) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(sr[c + 2 * e]) * inv_l,
+                                                             __uint_as_float(sr[c + 2 * e + 1]) * inv_l);
+              pk[e] = *reinterpret_cast<const uint32_t*>(&v);
+            }
+            dst[c / 8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+        if (p.lse) p.lse[(size_t)h * p.N + wi.seq_start + tok] = (m * sl2 + __log2f(l)) * 0.69314718055994531f;
+      }
+      g += wi.nkv;
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ Q rotation
+    const int tid = threadIdx.x - 256;
+    const int G = p.G;
+    const int rows = p.tq * G;
+    constexpr int NCH = D / 16;  // 16-byte chunks in the first half of a row
+    constexpr int HALF = D / 2;
+    // padding rows (never written by TMA) are zero in both Q buffers
+    for (int i = tid; i < 2 * C::NBOX * (BM - rows) * (C::ROWB / 16); i += 128) {
+      const int per_buf = C::NBOX * (BM - rows) * (C::ROWB / 16);
+      const int qb = i / per_buf;
+      int rem = i - qb * per_buf;
+      const int bx = rem / ((BM - rows) * (C::ROWB / 16));
+      rem -= bx * (BM - rows) * (C::ROWB / 16);
+      const int row = rows + rem / (C::ROWB / 16);
+      const int ch = rem % (C::ROWB / 16);
+      uint4* dst = reinterpret_cast<uint4*>(smem + qb * C::Q_BYTES + bx * C::Q_BOX_BYTES +
+                                            swz(row * C::ROWB + ch * 16, C::SWZ_MASK));
+      *dst = make_uint4(0, 0, 0, 0);
+    }
+    int it = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
+      const WorkItem wi = decode_item(p, w);
+      const int qb = it & 1;
+      ok = __all_sync(0xffffffffu, bwait(B(bars->q_loaded[qb]), (it >> 1) & 1, abort_flag));
+      if (!ok) break;
+      uint8_t* qbuf = smem + qb * C::Q_BYTES;
+      const int items = p.tq * NCH;
+      for (int item = tid; item < items; item += 128) {
+        const int tt = item / NCH;
+        const int ch = item - tt * NCH;
+        const int tok = wi.t0 + tt;
+        if (tok >= wi.L) continue;
+        const float4* tab = reinterpret_cast<const float4*>(p.table + (size_t)(wi.seq_start + tok) * HALF + ch * 8);
+        float cs[8], sn[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 t4 = __ldg(tab + e);
+          cs[2 * e] = t4.x;
+          sn[2 * e] = t4.y;
+          cs[2 * e + 1] = t4.z;
+          sn[2 * e + 1] = t4.w;
+        }
+        const int col_lo = ch * 8, col_hi = ch * 8 + HALF;
+        const int bx_lo = col_lo / C::BOXC, bx_hi = col_hi / C::BOXC;
+        for (int hh = 0; hh < G; ++hh) {
+          const int row = tt * G + hh;
+          uint4* plo = reinterpret_cast<uint4*>(
+              qbuf + bx_lo * C::Q_BOX_BYTES + swz(row * C::ROWB + (col_lo % C::BOXC) * 2, C::SWZ_MASK));
+          uint4* phi = reinterpret_cast<uint4*>(
+              qbuf + bx_hi * C::Q_BOX_BYTES + swz(row * C::ROWB + (col_hi % C::BOXC) * 2, C::SWZ_MASK));
+          uint4 vlo = *plo, vhi = *phi;
+          __nv_bfloat16* xl = reinterpret_cast<__nv_bfloat16*>(&vlo);
+          __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(&vhi);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const double dl = (double)__bfloat162float(xl[e]);
+            const double dh = (double)__bfloat162float(xh[e]);
+            const double dc = (double)cs[e], ds = (double)sn[e];
+            const double rl = fma(dl, dc, -(dh * ds));
+            const double rh = fma(dh, dc, dl * ds);
+            float fl = __double2float_rz(rl);
+            if ((double)fl != rl) fl = __uint_as_float(__float_as_uint(fl) | 1u);
+            float fh = __double2float_rz(rh);
+            if ((double)fh != rh) fh = __uint_as_float(__float_as_uint(fh) | 1u);
+            xl[e] = __float2bfloat16_rn(fl);
+            xh[e] = __float2bfloat16_rn(fh);
+          }
+          *plo = vlo;
+          *phi = vhi;
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive(B(bars->q_ready[qb]));
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace gqa

@@ -1,0 +1,106 @@
+// Shared constants, parameter blocks and workspace layout of the fused
+// causal GQA + RoPE attention forward (sm_100a).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+namespace gqa {
+
+// A query tile packs BM rows = (tq tokens) x (G query heads of one KV group),
+// row r <-> (token t0 + r / G, head kv*G + r % G). One K/V tile of BN keys
+// feeds every head of the group in a single MMA.
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int NUM_S_BUF = 3;        // S/P buffers in tensor memory
+constexpr int ATTN_THREADS = 384;   // 12 warps, roles below
+constexpr int PREP_THREADS = 256;
+constexpr int SCHED_BINS = 2048;    // cost histogram bins of the tile scheduler
+constexpr unsigned long long WAIT_TIMEOUT_NS = 2000000000ull;  // bounded waits: 2 s
+
+// Device status word: first device-detected error since the host last read
+// it. The library is a single translation unit, so it is defined here.
+__device__ int g_status = 0;
+
+// Status codes (same values as the C ABI).
+constexpr int kStatusBadSeqlens = 4;
+constexpr int kStatusTimeout = 5;
+
+__host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// tokens per packed query tile for a group of G heads
+__host__ __device__ constexpr int tokens_per_tile(int G) { return BM / G; }
+
+// Workspace regions (byte offsets from the 256-byte aligned base).
+struct WsLayout {
+  size_t header;   // int[4]: number of (sequence, q-tile) pairs, ...
+  size_t seq_pfx;  // int[num_seqs + 1]: first pair index of each sequence
+  size_t pairs;    // int2[max_pairs]: (sequence, q-tile) in decreasing cost order
+  size_t table;    // float2[N * d/2]: (cos, sin) of each token's angles
+  size_t kws;      // bf16[n_kv][N][d]: RoPE'd K, head-major
+  size_t qws;      // bf16[N][n_q][d]: q rounded to bf16 (fp32 inputs only)
+  size_t vws;      // bf16[N][n_kv][d]: v rounded to bf16 (fp32 inputs only)
+  size_t total;
+  long long max_pairs;
+};
+
+__host__ inline WsLayout ws_layout(int num_seqs, int N, int nq, int nkv, int d, bool fp32_in) {
+  WsLayout w{};
+  const int G = nq / nkv;
+  const int tq = tokens_per_tile(G);
+  w.max_pairs = (long long)(N + tq - 1) / tq + num_seqs;
+  size_t off = 0;
+  w.header = off;
+  off = align_up(off + 16 * sizeof(int), 256);
+  w.seq_pfx = off;
+  off = align_up(off + (size_t)(num_seqs + 1) * sizeof(int), 256);
+  w.pairs = off;
+  off = align_up(off + (size_t)w.max_pairs * 8, 256);
+  w.table = off;
+  off = align_up(off + (size_t)N * (d / 2) * 8, 256);
+  w.kws = off;
+  off = align_up(off + (size_t)nkv * N * d * 2, 256);
+  if (fp32_in) {
+    w.qws = off;
+    off = align_up(off + (size_t)N * nq * d * 2, 256);
+    w.vws = off;
+    off = align_up(off + (size_t)N * nkv * d * 2, 256);
+  } else {
+    w.qws = w.vws = 0;
+  }
+  w.total = off;
+  return w;
+}
+
+struct PrepParams {
+  const void* q;  // fp32 inputs only
+  const void* k;
+  const void* v;  // fp32 inputs only
+  const int* positions;
+  const int* cu;
+  int N, num_seqs, nq, nkv, tq, causal;
+  double theta;
+  int* header;
+  int* seq_pfx;
+  int2* pairs;
+  float2* table;
+  __nv_bfloat16* kws;
+  __nv_bfloat16* qws;
+  __nv_bfloat16* vws;
+};
+
+struct AttnParams {
+  const int* cu;
+  const int* header;
+  const int2* pairs;
+  const float2* table;
+  void* out;
+  float* lse;
+  int N, nq, nkv, G, tq, causal;
+  float scale_log2;     // log2(e) / sqrt(d)
+  float rescale_thr;    // raw-score growth that triggers an O rescale
+};
+
+}  // namespace gqa

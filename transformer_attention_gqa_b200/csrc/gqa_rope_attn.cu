@@ -1,0 +1,338 @@
+// Host side of the C ABI (include/gqa_rope_attn.h): argument checks, TMA
+// descriptor cache, and the two launches of the fused forward (prologue,
+// then the attention kernel chained by programmatic dependent launch).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/gqa_rope_attn.h"
+#include "attn_kernel.cuh"
+#include "common.cuh"
+#include "prep_kernel.cuh"
+
+namespace gqa {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool init = false;
+  int sm_count = 0;
+  bool attr_set[3][2] = {};
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+thread_local int t_last_launches = 0;
+thread_local cudaEvent_t t_prof_ev[3] = {nullptr, nullptr, nullptr};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+struct TmapKey {
+  int device;
+  const void* ptr;
+  uint64_t dims[3];
+  uint64_t strides[2];
+  uint32_t box[3];
+  int swizzle;
+  bool operator==(const TmapKey& o) const { return std::memcmp(this, &o, sizeof(TmapKey)) == 0; }
+};
+
+struct TmapEntry {
+  TmapKey key;
+  CUtensorMap map;
+  uint64_t stamp;
+  bool valid;
+};
+
+constexpr int kCacheSize = 64;
+TmapEntry g_cache[kCacheSize];
+uint64_t g_clock = 0;
+
+// 3-D bf16 tensor map (innermost dimension first), cached by its arguments.
+bool make_tmap(int device, const void* ptr, const uint64_t dims[3], const uint64_t strides[2],
+               const uint32_t box[3], int swizzle_bytes, CUtensorMap* out) {
+  TmapKey key;
+  std::memset(&key, 0, sizeof(key));
+  key.device = device;
+  key.ptr = ptr;
+  for (int i = 0; i < 3; ++i) key.dims[i] = dims[i], key.box[i] = box[i];
+  key.strides[0] = strides[0];
+  key.strides[1] = strides[1];
+  key.swizzle = swizzle_bytes;
+  int victim = 0;
+  uint64_t oldest = ~0ull;
+  for (int i = 0; i < kCacheSize; ++i) {
+    if (g_cache[i].valid && g_cache[i].key == key) {
+      g_cache[i].stamp = ++g_clock;
+      *out = g_cache[i].map;
+      return true;
+    }
+    const uint64_t st = g_cache[i].valid ? g_cache[i].stamp : 0;
+    if (st < oldest) oldest = st, victim = i;
+  }
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t gdim[3] = {dims[0], dims[1], dims[2]};
+  const cuuint64_t gstr[2] = {strides[0], strides[1]};
+  const cuuint32_t bdim[3] = {box[0], box[1], box[2]};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUtensorMap m;
+  const CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), gdim, gstr, bdim, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  g_cache[victim].key = key;
+  g_cache[victim].map = m;
+  g_cache[victim].stamp = ++g_clock;
+  g_cache[victim].valid = true;
+  *out = m;
+  return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int dim_index(int d) { return d == 32 ? 0 : (d == 64 ? 1 : 2); }
+
+template <int D, bool FP32>
+int launch(const void* q, const void* k, const void* v, const int32_t* positions, double theta,
+           const int32_t* cu, int num_seqs, int N, int nq, int nkv, int causal, void* out, float* lse,
+           uint8_t* ws, const WsLayout& lay, cudaStream_t stream, int device, int sm_count) {
+  using C = AttnCfg<D>;
+  const int G = nq / nkv;
+  const int tq = tokens_per_tile(G);
+
+  {  // caller holds g_mu
+    DeviceState& ds = g_dev[device];
+    if (!ds.attr_set[dim_index(D)][FP32 ? 1 : 0]) {
+      if (cudaFuncSetAttribute(gqa_attn_fwd_kernel<D, FP32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_BYTES) != cudaSuccess)
+        return GQA_ERR_CUDA;
+      ds.attr_set[dim_index(D)][FP32 ? 1 : 0] = true;
+    }
+  }
+
+  PrepParams pp{};
+  pp.q = q;
+  pp.k = k;
+  pp.v = v;
+  pp.positions = positions;
+  pp.cu = cu;
+  pp.N = N;
+  pp.num_seqs = num_seqs;
+  pp.nq = nq;
+  pp.nkv = nkv;
+  pp.tq = tq;
+  pp.causal = causal;
+  pp.theta = theta;
+  pp.header = reinterpret_cast<int*>(ws + lay.header);
+  pp.seq_pfx = reinterpret_cast<int*>(ws + lay.seq_pfx);
+  pp.pairs = reinterpret_cast<int2*>(ws + lay.pairs);
+  pp.table = reinterpret_cast<float2*>(ws + lay.table);
+  pp.kws = reinterpret_cast<__nv_bfloat16*>(ws + lay.kws);
+  pp.qws = FP32 ? reinterpret_cast<__nv_bfloat16*>(ws + lay.qws) : nullptr;
+  pp.vws = FP32 ? reinterpret_cast<__nv_bfloat16*>(ws + lay.vws) : nullptr;
+
+  // Tensor maps. Q: [N][nq][d] (caller's, or its bf16 copy); K: RoPE'd,
+  // head-major [nkv][N][d]; V: [N][nkv][d] (caller's, or its bf16 copy).
+  CUtensorMap tmQ, tmK, tmV;
+  const void* qsrc = FP32 ? (const void*)(ws + lay.qws) : q;
+  const void* vsrc = FP32 ? (const void*)(ws + lay.vws) : v;
+  const uint64_t es = 2;
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)nq, (uint64_t)N};
+    const uint64_t str[2] = {(uint64_t)D * es, (uint64_t)nq * D * es};
+    const uint32_t box[3] = {(uint32_t)C::BOXC, (uint32_t)G, (uint32_t)tq};
+    if (!make_tmap(device, qsrc, dims, str, box, C::ROWB, &tmQ)) return GQA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)N, (uint64_t)nkv};
+    const uint64_t str[2] = {(uint64_t)D * es, (uint64_t)N * D * es};
+    const uint32_t box[3] = {(uint32_t)C::BOXC, (uint32_t)BN, 1u};
+    if (!make_tmap(device, ws + lay.kws, dims, str, box, C::ROWB, &tmK)) return GQA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)nkv, (uint64_t)N};
+    const uint64_t str[2] = {(uint64_t)D * es, (uint64_t)nkv * D * es};
+    const uint32_t box[3] = {(uint32_t)C::BOXC, 1u, (uint32_t)BN};
+    if (!make_tmap(device, vsrc, dims, str, box, C::ROWB, &tmV)) return GQA_ERR_CUDA;
+  }
+
+  const long long work = (long long)N * (D / 4);
+  long long nb = (work + PREP_THREADS - 1) / PREP_THREADS;
+  const long long cap = (long long)sm_count * 8;
+  if (nb > cap) nb = cap;
+  if (nb < 1) nb = 1;
+  if (t_prof_ev[0] && cudaEventRecord(t_prof_ev[0], stream) != cudaSuccess) return GQA_ERR_CUDA;
+  gqa_prep_kernel<D, FP32><<<(unsigned)(nb + 1), PREP_THREADS, 0, stream>>>(pp);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+  if (t_prof_ev[1] && cudaEventRecord(t_prof_ev[1], stream) != cudaSuccess) return GQA_ERR_CUDA;
+
+
+  AttnParams ap{};
+  ap.cu = cu;
+  ap.header = pp.header;
+  ap.pairs = pp.pairs;
+  ap.table = pp.table;
+  ap.out = out;
+  ap.lse = lse;
+  ap.N = N;
+  ap.nq = nq;
+  ap.nkv = nkv;
+  ap.G = G;
+  ap.tq = tq;
+  ap.causal = causal;
+  ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  ap.rescale_thr = (float)(8.0 / (1.4426950408889634 / std::sqrt((double)D)));
+
+  const long long max_items = lay.max_pairs * (long long)nkv;
+  const unsigned grid = (unsigned)(max_items < sm_count ? max_items : sm_count);
+
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(ATTN_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gqa_attn_fwd_kernel<D, FP32>, tmQ, tmK, tmV, ap) != cudaSuccess)
+    return GQA_ERR_CUDA;
+  if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;
+  t_last_launches = 2;
+  return GQA_OK;
+}
+
+}  // namespace
+}  // namespace gqa
+
+using namespace gqa;
+
+extern "C" size_t gqa_rope_attn_workspace_size(int num_seqs, int total_tokens, int n_q_heads, int n_kv_heads,
+                                               int head_dim, int dtype) {
+  if (num_seqs < 0 || total_tokens < 0 || n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return 0;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return 0;
+  if (n_q_heads / n_kv_heads > BM) return 0;
+  if (dtype != GQA_DTYPE_BF16 && dtype != GQA_DTYPE_FP32) return 0;
+  return ws_layout(num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim, dtype == GQA_DTYPE_FP32).total;
+}
+
+extern "C" int gqa_rope_attn_fwd(const void* q, const void* k, const void* v, const int32_t* positions,
+                                 double rope_theta, const int32_t* cu_seqlens, int num_seqs, int total_tokens,
+                                 int n_q_heads, int n_kv_heads, int head_dim, int causal, int dtype, void* out,
+                                 float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  t_last_launches = 0;
+  struct Disarm {
+    ~Disarm() { t_prof_ev[0] = t_prof_ev[1] = t_prof_ev[2] = nullptr; }
+  } disarm;
+  // ---- checks that need no CUDA call
+  if (total_tokens < 0 || num_seqs < 0) return GQA_ERR_INVALID_ARG;
+  if (n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return GQA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return GQA_ERR_INVALID_ARG;
+  if (dtype != GQA_DTYPE_BF16 && dtype != GQA_DTYPE_FP32) return GQA_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.0) || !std::isfinite(rope_theta)) return GQA_ERR_INVALID_ARG;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED;
+  if (n_q_heads / n_kv_heads > BM) return GQA_ERR_UNSUPPORTED;
+  if ((long long)total_tokens * n_q_heads * head_dim > (1ll << 40)) return GQA_ERR_UNSUPPORTED;
+  if (total_tokens == 0) return GQA_OK;
+  if (num_seqs < 1) return GQA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !cu_seqlens) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GQA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(positions) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return GQA_ERR_INVALID_ARG;
+  const bool fp32 = dtype == GQA_DTYPE_FP32;
+  const WsLayout lay = ws_layout(num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim, fp32);
+  if (!workspace || workspace_bytes < lay.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return GQA_ERR_WORKSPACE;
+
+  // ---- device state
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices) return GQA_ERR_CUDA;
+  int sm_count = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState& ds = g_dev[device];
+    if (!ds.init) {
+      int major = 0;
+      if (cudaDeviceGetAttribute(&ds.sm_count, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+          cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess)
+        return GQA_ERR_CUDA;
+      if (major != 10) return GQA_ERR_UNSUPPORTED;
+      ds.init = true;
+    }
+    sm_count = ds.sm_count;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int rc;
+  std::lock_guard<std::mutex> lk(g_mu);  // descriptor cache
+  switch (head_dim * 2 + (fp32 ? 1 : 0)) {
+    case 64: rc = launch<32, false>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count); break;
+    case 65: rc = launch<32, true>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count); break;
+    case 128: rc = launch<64, false>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count); break;
+    case 129: rc = launch<64, true>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count); break;
+    case 256: rc = launch<128, false>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count); break;
+    default: rc = launch<128, true>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count); break;
+  }
+  return rc;
+}
+
+extern "C" int gqa_rope_attn_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GQA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+  }
+  return v;
+}
+
+extern "C" const char* gqa_rope_attn_strerror(int status) {
+  switch (status) {
+    case GQA_OK: return "ok";
+    case GQA_ERR_INVALID_ARG: return "invalid argument";
+    case GQA_ERR_UNSUPPORTED: return "unsupported shape or device";
+    case GQA_ERR_CUDA: return "CUDA error";
+    case GQA_ERR_BAD_SEQLENS: return "cu_seqlens is not a valid prefix sum of total_tokens";
+    case GQA_ERR_TIMEOUT: return "a bounded wait inside the kernel ran out";
+    case GQA_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int gqa_rope_attn_abi_version(void) { return GQA_ROPE_ATTN_ABI_VERSION; }
+
+extern "C" int gqa_rope_attn_last_launch_count(void) { return t_last_launches; }
+
+extern "C" void gqa_rope_attn_set_profile_events(void* ev_start, void* ev_mid, void* ev_end) {
+  t_prof_ev[0] = reinterpret_cast<cudaEvent_t>(ev_start);
+  t_prof_ev[1] = reinterpret_cast<cudaEvent_t>(ev_mid);
+  t_prof_ev[2] = reinterpret_cast<cudaEvent_t>(ev_end);
+}

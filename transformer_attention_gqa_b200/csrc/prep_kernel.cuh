@@ -1,0 +1,241 @@
+// Prologue kernel of the fused forward. Runs once per call, ahead of the
+// attention kernel (which it releases early through programmatic dependent
+// launch):
+//
+//  * block 0 checks cu_seqlens and builds the tile schedule: every
+//    (sequence, q-tile) pair, sorted by decreasing cost (number of KV tiles
+//    the causal q-tile visits), so that persistent CTAs take the longest
+//    tiles first;
+//  * the other blocks compute each token's RoPE (cos, sin) table row and
+//    write the RoPE'd K once, head-major, into the workspace. K is shared by
+//    every query tile that attends to it, so it is rotated once per
+//    (token, KV head) instead of once per visiting tile.
+//
+// RoPE ("Embeddings & the Residual Stream", section "Positional information:
+// RoPE, not a learned table"): inv_freq[i] = theta^(-2i/d); angle =
+// position * inv_freq[i]; feature i is rotated with feature i + d/2:
+//   out[i]       = x[i]       * cos - x[i + d/2] * sin
+//   out[i + d/2] = x[i + d/2] * cos + x[i]       * sin
+// The angle and cos/sin are evaluated in float64 and stored as fp32; the
+// rotation is one exact float64 fused multiply-add whose result is rounded
+// once, to nearest even, to bf16 (round-to-odd to fp32, then to bf16).
+#pragma once
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace gqa {
+
+
+__device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
+
+// Round a float64 value to the nearest bf16 (ties to even) in one rounding.
+__device__ __forceinline__ __nv_bfloat16 f64_to_bf16_rn(double x) {
+  float f = __double2float_rz(x);
+  if ((double)f != x) f = __uint_as_float(__float_as_uint(f) | 1u);  // round to odd
+  return __float2bfloat16_rn(f);
+}
+
+__device__ __forceinline__ void rope_pair(float xl, float xh, float c, float s, __nv_bfloat16& ol,
+                                          __nv_bfloat16& oh) {
+  const double dc = (double)c, ds = (double)s, dl = (double)xl, dh = (double)xh;
+  ol = f64_to_bf16_rn(fma(dl, dc, -(dh * ds)));
+  oh = f64_to_bf16_rn(fma(dh, dc, dl * ds));
+}
+
+// largest s in [0, n) with a[s] <= x (a nondecreasing, a[0] <= x)
+__device__ __forceinline__ int upper_index(const int* a, int n, int x) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(a + mid) <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int tile_cost(int L, int l, int tq, int causal) {
+  const int t_end = causal ? min((l + 1) * tq, L) : L;
+  return (t_end + BN - 1) / BN;
+}
+
+// Block-wide exclusive scan of one int per thread (PREP_THREADS threads).
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_buf, int& total) {
+  const int tid = threadIdx.x;
+  s_buf[tid] = v;
+  __syncthreads();
+  for (int off = 1; off < PREP_THREADS; off <<= 1) {
+    const int add = tid >= off ? s_buf[tid - off] : 0;
+    __syncthreads();
+    s_buf[tid] += add;
+    __syncthreads();
+  }
+  total = s_buf[PREP_THREADS - 1];
+  const int excl = s_buf[tid] - v;
+  __syncthreads();
+  return excl;
+}
+
+__device__ void build_schedule(const PrepParams& p) {
+  __shared__ int s_scan[PREP_THREADS];
+  __shared__ int s_bins[SCHED_BINS];
+  const int tid = threadIdx.x;
+  const int ns = p.num_seqs;
+
+  int bad = 0;
+  for (int s = tid; s < ns; s += PREP_THREADS)
+    if (__ldg(p.cu + s + 1) < __ldg(p.cu + s)) bad = 1;
+  if (tid == 0 && (__ldg(p.cu) != 0 || __ldg(p.cu + ns) != p.N)) bad = 1;
+  if (__syncthreads_or(bad)) {
+    if (tid == 0) {
+      set_status(kStatusBadSeqlens);
+      p.header[0] = 0;
+    }
+    return;
+  }
+
+  // First pair index of every sequence.
+  int running = 0;
+  for (int base = 0; base < ns; base += PREP_THREADS) {
+    const int s = base + tid;
+    int nt = 0;
+    if (s < ns) nt = (__ldg(p.cu + s + 1) - __ldg(p.cu + s) + p.tq - 1) / p.tq;
+    int tot;
+    const int ex = block_exclusive_scan(nt, s_scan, tot);
+    if (s < ns) p.seq_pfx[s] = running + ex;
+    running += tot;
+  }
+  if (tid == 0) p.seq_pfx[ns] = running;
+  const int P = running;
+
+  for (int i = tid; i < SCHED_BINS; i += PREP_THREADS) s_bins[i] = 0;
+  __syncthreads();  // seq_pfx (global) and s_bins visible to the whole block
+
+  for (int q = tid; q < P; q += PREP_THREADS) {
+    const int s = upper_index(p.seq_pfx, ns, q);
+    const int l = q - p.seq_pfx[s];
+    const int L = __ldg(p.cu + s + 1) - __ldg(p.cu + s);
+    const int c = min(tile_cost(L, l, p.tq, p.causal), SCHED_BINS - 1);
+    atomicAdd(&s_bins[c], 1);
+  }
+  __syncthreads();
+
+  // Offsets in decreasing-cost order: thread t owns reversed bins [8t, 8t+8).
+  constexpr int PER = SCHED_BINS / PREP_THREADS;
+  int local[PER];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    local[i] = s_bins[SCHED_BINS - 1 - (tid * PER + i)];
+    sum += local[i];
+  }
+  int tot;
+  int off = block_exclusive_scan(sum, s_scan, tot);
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    s_bins[SCHED_BINS - 1 - (tid * PER + i)] = off;  // each bin written by its owner only
+    off += local[i];
+  }
+  __syncthreads();
+
+  for (int q = tid; q < P; q += PREP_THREADS) {
+    const int s = upper_index(p.seq_pfx, ns, q);
+    const int l = q - p.seq_pfx[s];
+    const int L = __ldg(p.cu + s + 1) - __ldg(p.cu + s);
+    const int c = min(tile_cost(L, l, p.tq, p.causal), SCHED_BINS - 1);
+    const int slot = atomicAdd(&s_bins[c], 1);
+    p.pairs[slot] = make_int2(s, l);
+  }
+  if (tid == 0) p.header[0] = P;
+}
+
+template <int D, bool FP32_IN>
+__device__ void rope_k_and_table(const PrepParams& p, int block, int nblocks) {
+  constexpr int HALF = D / 2;
+  constexpr int PAIRS = HALF / 2;  // each thread handles frequencies i, i+1
+  __shared__ double s_invf[HALF];
+  for (int i = threadIdx.x; i < HALF; i += PREP_THREADS) s_invf[i] = pow(p.theta, -(2.0 * i) / D);
+  __syncthreads();
+
+  const long long total = (long long)p.N * PAIRS;
+  for (long long idx = (long long)block * PREP_THREADS + threadIdx.x; idx < total;
+       idx += (long long)nblocks * PREP_THREADS) {
+    const int t = (int)(idx / PAIRS);
+    const int i = (int)(idx % PAIRS) * 2;
+    int pos;
+    if (p.positions) {
+      pos = __ldg(p.positions + t);
+    } else {
+      const int s = upper_index(p.cu, p.num_seqs, t);
+      pos = t - __ldg(p.cu + s);
+    }
+    float c[2], sn[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      double sd, cd;
+      sincos((double)pos * s_invf[i + e], &sd, &cd);
+      c[e] = (float)cd;
+      sn[e] = (float)sd;
+    }
+    *reinterpret_cast<float4*>(p.table + (size_t)t * HALF + i) = make_float4(c[0], sn[0], c[1], sn[1]);
+
+    for (int h = 0; h < p.nkv; ++h) {
+      const size_t src = ((size_t)t * p.nkv + h) * D;
+      float xl[2], xh[2];
+      if constexpr (FP32_IN) {
+        const float2 a = *reinterpret_cast<const float2*>((const float*)p.k + src + i);
+        const float2 b = *reinterpret_cast<const float2*>((const float*)p.k + src + i + HALF);
+        // inputs are rounded to bf16 before anything else
+        xl[0] = __bfloat162float(__float2bfloat16_rn(a.x));
+        xl[1] = __bfloat162float(__float2bfloat16_rn(a.y));
+        xh[0] = __bfloat162float(__float2bfloat16_rn(b.x));
+        xh[1] = __bfloat162float(__float2bfloat16_rn(b.y));
+      } else {
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>((const __nv_bfloat16*)p.k + src + i);
+        const __nv_bfloat162 b =
+            *reinterpret_cast<const __nv_bfloat162*>((const __nv_bfloat16*)p.k + src + i + HALF);
+        xl[0] = __low2float(a);
+        xl[1] = __high2float(a);
+        xh[0] = __low2float(b);
+        xh[1] = __high2float(b);
+      }
+      __nv_bfloat16 ol[2], oh[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) rope_pair(xl[e], xh[e], c[e], sn[e], ol[e], oh[e]);
+      const size_t dst = ((size_t)h * p.N + t) * D;
+      *reinterpret_cast<__nv_bfloat162*>(p.kws + dst + i) = __halves2bfloat162(ol[0], ol[1]);
+      *reinterpret_cast<__nv_bfloat162*>(p.kws + dst + i + HALF) = __halves2bfloat162(oh[0], oh[1]);
+    }
+
+    if constexpr (FP32_IN) {
+      // bf16 copies of q (rotated later, in the attention kernel) and v.
+      for (int h = 0; h < p.nq; ++h) {
+        const size_t o = ((size_t)t * p.nq + h) * D;
+        const float2 a = *reinterpret_cast<const float2*>((const float*)p.q + o + i);
+        const float2 b = *reinterpret_cast<const float2*>((const float*)p.q + o + i + HALF);
+        *reinterpret_cast<__nv_bfloat162*>(p.qws + o + i) = __floats2bfloat162_rn(a.x, a.y);
+        *reinterpret_cast<__nv_bfloat162*>(p.qws + o + i + HALF) = __floats2bfloat162_rn(b.x, b.y);
+      }
+      for (int h = 0; h < p.nkv; ++h) {
+        const size_t o = ((size_t)t * p.nkv + h) * D;
+        const float2 a = *reinterpret_cast<const float2*>((const float*)p.v + o + i);
+        const float2 b = *reinterpret_cast<const float2*>((const float*)p.v + o + i + HALF);
+        *reinterpret_cast<__nv_bfloat162*>(p.vws + o + i) = __floats2bfloat162_rn(a.x, a.y);
+        *reinterpret_cast<__nv_bfloat162*>(p.vws + o + i + HALF) = __floats2bfloat162_rn(b.x, b.y);
+      }
+    }
+  }
+}
+
+template <int D, bool FP32_IN>
+__global__ void __launch_bounds__(PREP_THREADS) gqa_prep_kernel(const PrepParams p) {
+  // Let the attention grid start its prologue; it reads nothing written
+  // here before its griddepcontrol.wait.
+  ptx::griddep_launch_dependents();
+  if (blockIdx.x == 0) {
+    build_schedule(p);
+  } else {
+    rope_k_and_table<D, FP32_IN>(p, blockIdx.x - 1, gridDim.x - 1);
+  }
+}
+
+}  // namespace gqa
