@@ -195,16 +195,32 @@ def run_ours(args, rank, world, local_rank):
     total_ms = sum(step_ms)
 
     # per-kernel durations (second pass, same stream, events recorded by the library)
+    from cuda.bindings import runtime as rt
+
+    def _ev():
+        err, e = rt.cudaEventCreate()
+        assert int(err) == 0
+        return e
+
     kern = []
     for i in range(max(3, min(args.steps, 10))):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e = [_ev() for _ in range(3)]
         flush.zero_()
-        _abi.set_profile_events(e[0].cuda_event, e[1].cuda_event, e[2].cuda_event)
+        _abi.set_profile_events(int(e[0]), int(e[1]), int(e[2]))
         step()
         kern.append(e)
     torch.cuda.synchronize()
-    prep_ms = statistics.median(a.elapsed_time(b) for a, b, _ in kern)
-    attn_ms = statistics.median(b.elapsed_time(c) for _, b, c in kern)
+
+    def _ms(a, b):
+        err, ms = rt.cudaEventElapsedTime(a, b)
+        assert int(err) == 0
+        return float(ms)
+
+    prep_ms = statistics.median(_ms(a, b) for a, b, _ in kern)
+    attn_ms = statistics.median(_ms(b, c) for _, b, c in kern)
+    for e in kern:
+        for x in e:
+            rt.cudaEventDestroy(x)
     clk = clocks.stop()
 
     # end to end through the public API with host buffers

@@ -117,3 +117,27 @@ def test_bad_cu_seqlens_sets_status_and_writes_nothing():
         assert g.get_device_status() == 4
         assert g.get_device_status() == 0  # cleared by the read
         assert torch.all(out == 0)
+
+
+def test_workspace_reuse_with_garbage_contents():
+    """The kernels must read nothing from the workspace that the prologue of
+    the same call has not written: reuse one workspace across shapes, filled
+    with garbage bytes before every call."""
+    import torch
+    import transformer_attention_gqa_b200 as g
+
+    ws = g.Workspace(torch.device("cuda"))
+    shapes = [([400, 96], 8, 2, 128), ([33, 700, 5], 4, 1, 64), ([1], 16, 2, 128), ([2048], 14, 2, 64),
+              ([129, 127, 256], 6, 2, 128)]
+    for rep in range(3):
+        for idx, (lens, nq, nkv, d) in enumerate(shapes):
+            inp = wl.make_custom(lens, nq, nkv, d, 1e4, seed=100 * rep + idx)
+            q, k, v, cu, _ = H.to_device(inp)
+            buf = ws.get(g.workspace_size(len(lens), sum(lens), nq, nkv, d))
+            buf.fill_(0x7F if rep % 2 == 0 else 0xFF)
+            out, lse = g.gqa_rope_attn_fwd(q, k, v, cu, 1e4, workspace=ws)
+            torch.cuda.synchronize()
+            assert g.get_device_status() == 0
+            ref_out, ref_lse = H.oracle(inp)
+            H.compare(out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64),
+                      ref_out, ref_lse, what=f"reuse {rep} {lens}")

@@ -33,6 +33,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "exp2_poly.cuh"
 #include "ptx.cuh"
 
 namespace gqa {
@@ -78,6 +79,12 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (layout << 61);
 }
 
+constexpr int REG_PRODUCER = 56;
+constexpr int REG_SOFTMAX = 232;
+constexpr int REG_ROPE = 128;
+static_assert((REG_PRODUCER + REG_SOFTMAX + REG_ROPE) * 128 <= 65536 / ATTN_THREADS * ATTN_THREADS,
+              "register split exceeds the launch's register file share");
+
 struct Barriers {
   uint64_t q_loaded[2], q_ready[2], q_empty[2];
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
@@ -95,7 +102,7 @@ __device__ __forceinline__ WorkItem decode_item(const AttnParams& p, int w) {
   WorkItem it;
   const int pair = w / p.nkv;
   it.kvh = w - pair * p.nkv;
-  const int2 sl = p.pairs[pair];
+  const int2 sl = ptx::ld_cg_v2s32(p.pairs + pair);  // written by the prologue grid
   it.seq_start = __ldg(p.cu + sl.x);
   it.L = __ldg(p.cu + sl.x + 1) - it.seq_start;
   it.t0 = sl.y * p.tq;
@@ -131,6 +138,41 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
     }
   }
 }
+
+// 2^x on the FMA pipe, for x <= 8: x = n + f with n = rint(x) (the 1.5*2^23
+// addition leaves n in the low mantissa bits), 2^f from the degree-4
+// minimax polynomial of exp2_poly.cuh, n added to the exponent as an
+// integer. x is clamped to -125 so the result stays a normal number
+// (2^-125 is negligible next to the row maximum's 1).
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  float p = fmaf(kExp2C4, f, kExp2C3);
+  p = fmaf(p, f, kExp2C2);
+  p = fmaf(p, f, kExp2C1);
+  p = fmaf(p, f, kExp2C0);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// Two fp32 -> one bf16x2 word (lo in the low half), rounded to nearest (ties
+// away from zero), with integer ops instead of the conversion unit.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Of every EMU_PERIOD exponent pairs of a row, one is evaluated on the FMA
+// pipe, the rest on the special-function unit.
+#ifndef GQA_EMU_PERIOD
+#define GQA_EMU_PERIOD 4
+#endif
+constexpr int EMU_PERIOD = GQA_EMU_PERIOD;
 
 __device__ __forceinline__ uint32_t swz(uint32_t lin, int mask) { return lin ^ (((lin >> 7) & mask) << 4); }
 
@@ -189,9 +231,13 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
 
   // Everything below reads what the prologue kernel wrote.
   ptx::griddep_wait();
-  const int n_items = __ldg(p.header) * p.nkv;
+  const int n_items = ptx::ld_cg_s32(p.header) * p.nkv;
 
-  if (warp == 0) {
+  // Register split (launch: 384 threads x 168): producers/MMA 56, softmax
+  // 232, Q rotation 128 -> (56 + 232 + 128) x 128 = 53248 <= 64512.
+  if (warp < 4) {
+   ptx::setmaxnreg_dec<REG_PRODUCER>();
+   if (warp == 0) {
     // ------------------------------------------------------------ Q/K producer
     if (lane == 0) {
       int q_uses[2] = {0, 0};
@@ -226,7 +272,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           if (k_uses[i]) drain_wait(B(bars->k_full[i]), (k_uses[i] - 1) & 1);
       }
     }
-  } else if (warp == 2) {
+   } else if (warp == 2) {
     // ------------------------------------------------------------ V producer
     if (lane == 0) {
       int v_uses[C::VST];
@@ -250,7 +296,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           if (v_uses[i]) drain_wait(B(bars->v_full[i]), (v_uses[i] - 1) & 1);
       }
     }
-  } else if (warp == 1) {
+   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t g = 0;
@@ -310,7 +356,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       ptx::mma_commit(B(bars->drain));
       drain_wait(B(bars->drain), 0);
     }
-  } else if (warp >= 4 && warp < 8) {
+   }
+  } else if (warp < 8) {
+    ptx::setmaxnreg_inc<REG_SOFTMAX>();
     // ------------------------------------------------------------ softmax
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // row of the tile == TMEM lane
@@ -347,9 +395,15 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           for (int c = 0; c < BN; ++c)
             if (c > lim) sr[c] = __float_as_uint(-INFINITY);
         }
-        float mx = __uint_as_float(sr[0]);
+        // row max: 8 independent chains of 3-input max, then a tree
+        float mx8[8];
 #pragma unroll
-        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(__uint_as_float(sr[e]), __uint_as_float(sr[e + 8]));
+#pragma unroll
+        for (int c = 16; c < BN; c += 16)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], __uint_as_float(sr[c + e]), __uint_as_float(sr[c + 8 + e]));
+        const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
         float alpha = 1.f;
         bool need = false;
         if (j == 0) {
@@ -360,18 +414,32 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           need = true;
         }
         const float neg = -m * sl2;
-        float lsum = 0.f;
+        // p = 2^(s*log2e/sqrt(d) - m*log2e/sqrt(d)); 8 partial sums; P packed to
+        // bf16 pairs in place and stored to TMEM one half at a time
+        float ls8[8];
 #pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[c]), sl2, neg));
-          const float p1 = ptx::ex2(fmaf(__uint_as_float(sr[c + 1]), sl2, neg));
-          lsum += p0 + p1;
-          const __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
-          sr[c >> 1] = *reinterpret_cast<const uint32_t*>(&pk);
+        for (int e = 0; e < 8; ++e) ls8[e] = 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+          for (int c = half * 64; c < half * 64 + 64; c += 2) {
+            const float x0 = fmaf(__uint_as_float(sr[c]), sl2, neg);
+            const float x1 = fmaf(__uint_as_float(sr[c + 1]), sl2, neg);
+            float p0, p1;
+            if (((c >> 1) % EMU_PERIOD) == EMU_PERIOD - 1) {
+              p0 = exp2_fma(x0);
+              p1 = exp2_fma(x1);
+            } else {
+              p0 = ptx::ex2(x0);
+              p1 = ptx::ex2(x1);
+            }
+            ls8[(c >> 1) & 7] += p0 + p1;
+            sr[c >> 1] = pack_bf16x2(p0, p1);
+          }
+          ptx::tmem_st32(trow + b * 128 + half * 32, sr + half * 32);
         }
+        const float lsum = ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
         l = l * alpha + lsum;
-        ptx::tmem_st32(trow + b * 128, sr);
-        ptx::tmem_st32(trow + b * 128 + 32, sr + 32);
         if (__any_sync(0xffffffffu, need)) {
           // O holds the sum up to the previous tile: wait for PV(gg-1), then scale.
           const uint32_t gp = gg - 1;
@@ -435,7 +503,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       }
       g += wi.nkv;
     }
-  } else if (warp >= 8) {
+  } else {
+    ptx::setmaxnreg_dec<REG_ROPE>();
     // ------------------------------------------------------------ Q rotation
     const int tid = threadIdx.x - 256;
     const int G = p.G;
@@ -473,7 +542,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         float cs[8], sn[8];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float4 t4 = __ldg(tab + e);
+          const float4 t4 = ptx::ld_cg_v4f32(tab + e);
           cs[2 * e] = t4.x;
           sn[2 * e] = t4.y;
           cs[2 * e + 1] = t4.z;
