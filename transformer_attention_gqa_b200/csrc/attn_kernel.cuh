@@ -15,9 +15,9 @@
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer: Q tile and K tiles (K is RoPE'd already)
-//   warp 1      TMEM allocator and the single MMA-issuing thread
+//   warp 1      TMEM allocator; one thread issues the S = Q K^T MMAs
 //   warp 2      TMA producer: V tiles
-//   warp 3      idle
+//   warp 3      one thread issues the O += P V MMAs
 //   warps 4-7   softmax: one thread per row (TMEM lane), S -> P, running
 //               max/sum, O rescale, epilogue (O / l, LSE)
 //   warps 8-11  Q rotation: RoPE applied in shared memory to each Q tile
@@ -113,11 +113,35 @@ __device__ __forceinline__ WorkItem decode_item(const AttnParams& p, int w) {
 
 // Bounded wait on an mbarrier phase. Returns false if the CTA is aborting or
 // the wait exceeded WAIT_TIMEOUT_NS (then the abort flag and the device
-// status word are set).
+// status word are set). The abort flag and the clock are checked only every
+// 8 polls.
 __device__ __forceinline__ bool bwait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
   while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i)
+      if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (ptx::globaltimer() - t0 > WAIT_TIMEOUT_NS) {
+      *abort_flag = 1;
+      atomicCAS(&g_status, 0, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+// Bounded wait for waiters off the critical path (TMA producers, the Q
+// rotation warps): between polls the warp sleeps with exponential backoff
+// (32 ns .. 1 us), so that it takes no issue slots from the softmax warps
+// that share its scheduler.
+__device__ __forceinline__ bool bwait_lazy(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  uint32_t ns = 32;
+  while (true) {
+    __nanosleep(ns);
+    if (ns < 1024) ns <<= 1;
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (ptx::globaltimer() - t0 > WAIT_TIMEOUT_NS) {
@@ -168,13 +192,34 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 
 // Of every EMU_PERIOD exponent pairs of a row, one is evaluated on the FMA
-// pipe, the rest on the special-function unit.
+// pipe, the rest on the special-function unit (0: all on the SFU; measured
+// fastest while the softmax is latency-bound rather than SFU-bound).
 #ifndef GQA_EMU_PERIOD
-#define GQA_EMU_PERIOD 4
+#define GQA_EMU_PERIOD 0
 #endif
 constexpr int EMU_PERIOD = GQA_EMU_PERIOD;
 
 __device__ __forceinline__ uint32_t swz(uint32_t lin, int mask) { return lin ^ (((lin >> 7) & mask) << 4); }
+
+// S = Q K^T for one KV tile: D/16 K-steps, K-major A and B (SW128/SW64).
+template <class C>
+__device__ __forceinline__ void issue_s_mmas(uint32_t d_tmem, uint64_t dq, uint64_t dk) {
+#pragma unroll
+  for (int kk = 0; kk < C::KSTEPS_S; ++kk) {
+    const uint32_t off_q = (kk / C::STEPS_PER_BOX) * C::Q_BOX_BYTES + (kk % C::STEPS_PER_BOX) * 32;
+    const uint32_t off_k = (kk / C::STEPS_PER_BOX) * C::KV_BOX_BYTES + (kk % C::STEPS_PER_BOX) * 32;
+    ptx::mma_ss(d_tmem, dq + (uint64_t)(off_q >> 4), dk + (uint64_t)(off_k >> 4), C::IDESC_S, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O (+)= P V for one KV tile: 8 K-steps of 16 keys, P from TMEM, V MN-major.
+template <class C>
+__device__ __forceinline__ void issue_pv_mmas(uint32_t o_tmem, uint32_t p_tmem, uint64_t dv, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < C::KSTEPS_PV; ++kk)
+    ptx::mma_ts(o_tmem, p_tmem + kk * 8, dv + (uint64_t)((kk * 16 * C::ROWB) >> 4), C::IDESC_O,
+                (accumulate || kk > 0) ? 1u : 0u);
+}
 
 template <int D, bool OUT_FP32>
 __global__ void __launch_bounds__(ATTN_THREADS, 1)
@@ -211,7 +256,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       ptx::mbar_init(B(bars->pv_done[i]), 1);
     }
     ptx::mbar_init(B(bars->o_free), 128);
-    ptx::mbar_init(B(bars->drain), 1);
+    ptx::mbar_init(B(bars->drain), 2);  // one commit per MMA-issuing thread
     bars->abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -240,119 +285,120 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
    if (warp == 0) {
     // ------------------------------------------------------------ Q/K producer
     if (lane == 0) {
-      int q_uses[2] = {0, 0};
-      int k_uses[C::KST];
-      for (int i = 0; i < C::KST; ++i) k_uses[i] = 0;
       uint32_t g = 0;
-      int it = 0;
+      int it = 0, q_issued = 0;
       bool ok = true;
       for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
         const WorkItem wi = decode_item(p, w);
         const int qb = it & 1;
-        if (!(ok = bwait(B(bars->q_empty[qb]), ((it >> 1) & 1) ^ 1, abort_flag))) break;
+        if (!(ok = bwait_lazy(B(bars->q_empty[qb]), ((it >> 1) & 1) ^ 1, abort_flag))) break;
         ptx::mbar_arrive_expect_tx(B(bars->q_loaded[qb]), (uint32_t)(D * 2 * p.G * p.tq));
         for (int b = 0; b < C::NBOX; ++b)
           ptx::tma_load_3d(sbase + qb * C::Q_BYTES + b * C::Q_BOX_BYTES, &tmQ, B(bars->q_loaded[qb]),
                            b * C::BOXC, wi.kvh * p.G, wi.seq_start + wi.t0);
-        ++q_uses[qb];
+        ++q_issued;
         for (int j = 0; j < wi.nkv; ++j, ++g) {
           const int ks = g % C::KST;
-          if (!(ok = bwait(B(bars->k_empty[ks]), ((g / C::KST) & 1) ^ 1, abort_flag))) break;
+          if (!(ok = bwait_lazy(B(bars->k_empty[ks]), ((g / C::KST) & 1) ^ 1, abort_flag))) break;
           ptx::mbar_arrive_expect_tx(B(bars->k_full[ks]), (uint32_t)C::KV_BYTES);
           for (int b = 0; b < C::NBOX; ++b)
             ptx::tma_load_3d(sbase + C::OFF_K + ks * C::KV_BYTES + b * C::KV_BOX_BYTES, &tmK,
                              B(bars->k_full[ks]), b * C::BOXC, wi.seq_start + j * BN, wi.kvh);
-          ++k_uses[ks];
         }
       }
       if (!ok) {  // let every copy already issued land before the CTA exits
-        for (int i = 0; i < 2; ++i)
-          if (q_uses[i]) drain_wait(B(bars->q_loaded[i]), (q_uses[i] - 1) & 1);
-        for (int i = 0; i < C::KST; ++i)
-          if (k_uses[i]) drain_wait(B(bars->k_full[i]), (k_uses[i] - 1) & 1);
+        // loads issued: Q tiles 0..q_issued-1 (buffer t & 1), K tiles 0..g-1 (stage x % KST)
+        for (int i = 0; i < 2; ++i) {
+          const int uses = (q_issued - i + 1) / 2;
+          if (uses > 0) drain_wait(B(bars->q_loaded[i]), (uses - 1) & 1);
+        }
+        for (int i = 0; i < C::KST; ++i) {
+          const int uses = ((int)g - i + C::KST - 1) / C::KST;
+          if (uses > 0) drain_wait(B(bars->k_full[i]), (uses - 1) & 1);
+        }
       }
     }
    } else if (warp == 2) {
     // ------------------------------------------------------------ V producer
     if (lane == 0) {
-      int v_uses[C::VST];
-      for (int i = 0; i < C::VST; ++i) v_uses[i] = 0;
       uint32_t g = 0;
       bool ok = true;
       for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
         const WorkItem wi = decode_item(p, w);
         for (int j = 0; j < wi.nkv; ++j, ++g) {
           const int vs = g % C::VST;
-          if (!(ok = bwait(B(bars->v_empty[vs]), ((g / C::VST) & 1) ^ 1, abort_flag))) break;
+          if (!(ok = bwait_lazy(B(bars->v_empty[vs]), ((g / C::VST) & 1) ^ 1, abort_flag))) break;
           ptx::mbar_arrive_expect_tx(B(bars->v_full[vs]), (uint32_t)C::KV_BYTES);
           for (int b = 0; b < C::NBOX; ++b)
             ptx::tma_load_3d(sbase + C::OFF_V + vs * C::KV_BYTES + b * C::KV_BOX_BYTES, &tmV,
                              B(bars->v_full[vs]), b * C::BOXC, wi.kvh, wi.seq_start + j * BN);
-          ++v_uses[vs];
         }
       }
       if (!ok) {
-        for (int i = 0; i < C::VST; ++i)
-          if (v_uses[i]) drain_wait(B(bars->v_full[i]), (v_uses[i] - 1) & 1);
+        for (int i = 0; i < C::VST; ++i) {
+          const int uses = ((int)g - i + C::VST - 1) / C::VST;
+          if (uses > 0) drain_wait(B(bars->v_full[i]), (uses - 1) & 1);
+        }
       }
     }
    } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S issuer
+    // S(x) = Q K(x)^T into S buffer x % 3; it needs PV(x - 3) done (that PV
+    // read P from the same columns). Runs ahead of the softmax by up to three
+    // KV tiles; a tcgen05.mma blocks its issuing thread while the tensor core
+    // works, so S and PV have separate issuing threads.
     if (lane == 0) {
-      uint32_t g = 0;
+      const uint64_t dq_base = umma_desc(sbase, 16, C::SBO, C::UMMA_LAYOUT);
+      const uint64_t dk_base = umma_desc(sbase + C::OFF_K, 16, C::SBO, C::UMMA_LAYOUT);
+      const uint32_t bar_pv0 = B(bars->pv_done[0]), bar_s0 = B(bars->s_full[0]);
+      const uint32_t bar_kf0 = B(bars->k_full[0]), bar_ke0 = B(bars->k_empty[0]);
+      const uint32_t bar_qr0 = B(bars->q_ready[0]), bar_qe0 = B(bars->q_empty[0]);
+      uint32_t gs = 0;
       int it = 0;
       bool ok = true;
-      // S(gg) = Q K(gg)^T into S buffer gg % 3
-      auto issue_s = [&](uint32_t gg, int qb) -> bool {
-        const int b = gg % NUM_S_BUF;
-        if (gg >= NUM_S_BUF)  // PV(gg - 3) read P from this buffer
-          if (!bwait(B(bars->pv_done[b]), ((gg / NUM_S_BUF) - 1) & 1, abort_flag)) return false;
-        const int ks = gg % C::KST;
-        if (!bwait(B(bars->k_full[ks]), (gg / C::KST) & 1, abort_flag)) return false;
-        ptx::tc_fence_after();
-        const uint32_t qaddr = sbase + qb * C::Q_BYTES;
-        const uint32_t kaddr = sbase + C::OFF_K + ks * C::KV_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < C::KSTEPS_S; ++kk) {
-          const uint32_t off_q = (kk / C::STEPS_PER_BOX) * C::Q_BOX_BYTES + (kk % C::STEPS_PER_BOX) * 32;
-          const uint32_t off_k = (kk / C::STEPS_PER_BOX) * C::KV_BOX_BYTES + (kk % C::STEPS_PER_BOX) * 32;
-          ptx::mma_ss(tmem + b * 128, umma_desc(qaddr + off_q, 16, C::SBO, C::UMMA_LAYOUT),
-                      umma_desc(kaddr + off_k, 16, C::SBO, C::UMMA_LAYOUT), C::IDESC_S, kk > 0 ? 1u : 0u);
-        }
-        ptx::mma_commit(B(bars->s_full[b]));
-        ptx::mma_commit(B(bars->k_empty[ks]));
-        return true;
-      };
       for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
         const WorkItem wi = decode_item(p, w);
         const int qb = it & 1;
-        if (!(ok = bwait(B(bars->q_ready[qb]), (it >> 1) & 1, abort_flag))) break;
-        ptx::tc_fence_after();
-        const int npre = wi.nkv < 2 ? wi.nkv : 2;
-        for (int jj = 0; ok && jj < npre; ++jj) ok = issue_s(g + jj, qb);
-        for (int j = 0; ok && j < wi.nkv; ++j) {
-          const uint32_t gg = g + j;
-          const int b = gg % NUM_S_BUF;
-          const int vs = gg % C::VST;
-          if (!(ok = bwait(B(bars->p_full[b]), (gg / NUM_S_BUF) & 1, abort_flag))) break;
-          if (!(ok = bwait(B(bars->v_full[vs]), (gg / C::VST) & 1, abort_flag))) break;
-          if (j == 0 && !(ok = bwait(B(bars->o_free), (it & 1) ^ 1, abort_flag))) break;
+        if (!(ok = bwait(bar_qr0 + 8 * qb, (it >> 1) & 1, abort_flag))) break;
+        const uint64_t dq = dq_base + (uint64_t)((qb * C::Q_BYTES) >> 4);
+        for (int j = 0; j < wi.nkv; ++j, ++gs) {
+          const int bs = gs % NUM_S_BUF, ks = gs % C::KST;
+          if (gs >= NUM_S_BUF && !(ok = bwait(bar_pv0 + 8 * bs, ((gs / NUM_S_BUF) - 1) & 1, abort_flag))) break;
+          if (!(ok = bwait(bar_kf0 + 8 * ks, (gs / C::KST) & 1, abort_flag))) break;
           ptx::tc_fence_after();
-          const uint32_t vaddr = sbase + C::OFF_V + vs * C::KV_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < C::KSTEPS_PV; ++kk) {
-            ptx::mma_ts(tmem + C::O_COL, tmem + b * 128 + kk * 8,
-                        umma_desc(vaddr + kk * 16 * C::ROWB, C::KV_BOX_BYTES, C::SBO, C::UMMA_LAYOUT),
-                        C::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          ptx::mma_commit(B(bars->pv_done[b]));
-          ptx::mma_commit(B(bars->v_empty[vs]));
-          if (j == wi.nkv - 1) ptx::mma_commit(B(bars->q_empty[qb]));
-          if (j + 2 < wi.nkv) ok = issue_s(gg + 2, qb);
+          issue_s_mmas<C>(tmem + bs * 128, dq, dk_base + (uint64_t)((ks * C::KV_BYTES) >> 4));
+          ptx::mma_commit(bar_s0 + 8 * bs);
+          ptx::mma_commit(bar_ke0 + 8 * ks);
         }
-        g += wi.nkv;
+        if (ok) ptx::mma_commit(bar_qe0 + 8 * qb);  // every S of this tile read Q
       }
-      // all tensor-core work of this CTA has finished before TMEM is freed
+      // all tensor-core work issued here has finished before TMEM is freed
+      ptx::mma_commit(B(bars->drain));
+      drain_wait(B(bars->drain), 0);
+    }
+   } else if (warp == 3) {
+    // ------------------------------------------------------------ PV issuer
+    // O += P(x) V(x) once the softmax has written P(x) into S buffer x % 3.
+    if (lane == 0) {
+      const uint64_t dv_base = umma_desc(sbase + C::OFF_V, C::KV_BOX_BYTES, C::SBO, C::UMMA_LAYOUT);
+      const uint32_t bar_pv0 = B(bars->pv_done[0]), bar_p0 = B(bars->p_full[0]);
+      const uint32_t bar_vf0 = B(bars->v_full[0]), bar_ve0 = B(bars->v_empty[0]), bar_of = B(bars->o_free);
+      uint32_t g = 0;
+      int it = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
+        const WorkItem wi = decode_item(p, w);
+        for (int j = 0; j < wi.nkv; ++j, ++g) {
+          const int b = g % NUM_S_BUF, vs = g % C::VST;
+          if (!(ok = bwait(bar_vf0 + 8 * vs, (g / C::VST) & 1, abort_flag))) break;
+          if (j == 0 && !(ok = bwait(bar_of, (it & 1) ^ 1, abort_flag))) break;
+          if (!(ok = bwait(bar_p0 + 8 * b, (g / NUM_S_BUF) & 1, abort_flag))) break;
+          ptx::tc_fence_after();
+          issue_pv_mmas<C>(tmem + C::O_COL, tmem + b * 128, dv_base + (uint64_t)((vs * C::KV_BYTES) >> 4), j > 0);
+          ptx::mma_commit(bar_pv0 + 8 * b);
+          ptx::mma_commit(bar_ve0 + 8 * vs);
+        }
+      }
       ptx::mma_commit(B(bars->drain));
       drain_wait(B(bars->drain), 0);
     }
@@ -426,7 +472,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             const float x0 = fmaf(__uint_as_float(sr[c]), sl2, neg);
             const float x1 = fmaf(__uint_as_float(sr[c + 1]), sl2, neg);
             float p0, p1;
-            if (((c >> 1) % EMU_PERIOD) == EMU_PERIOD - 1) {
+            if (EMU_PERIOD > 0 && ((c >> 1) % (EMU_PERIOD > 0 ? EMU_PERIOD : 1)) == EMU_PERIOD - 1) {
               p0 = exp2_fma(x0);
               p1 = exp2_fma(x1);
             } else {
@@ -443,8 +489,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         if (__any_sync(0xffffffffu, need)) {
           // O holds the sum up to the previous tile: wait for PV(gg-1), then scale.
           const uint32_t gp = gg - 1;
-          ok = __all_sync(0xffffffffu,
-                          bwait(B(bars->pv_done[gp % NUM_S_BUF]), (gp / NUM_S_BUF) & 1, abort_flag));
+          ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[gp % NUM_S_BUF]), (gp / NUM_S_BUF) & 1, abort_flag));
           if (!ok) break;
           ptx::tc_fence_after();
 #pragma unroll
@@ -529,7 +574,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
       const WorkItem wi = decode_item(p, w);
       const int qb = it & 1;
-      ok = __all_sync(0xffffffffu, bwait(B(bars->q_loaded[qb]), (it >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, bwait_lazy(B(bars->q_loaded[qb]), (it >> 1) & 1, abort_flag));
       if (!ok) break;
       uint8_t* qbuf = smem + qb * C::Q_BYTES;
       const int items = p.tq * NCH;
