@@ -141,3 +141,26 @@ def test_workspace_reuse_with_garbage_contents():
             ref_out, ref_lse = H.oracle(inp)
             H.compare(out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64),
                       ref_out, ref_lse, what=f"reuse {rep} {lens}")
+
+
+def test_running_max_rescale_paths():
+    """Keys whose norm grows along the sequence make later tiles raise the
+    row max far past the running one, which exercises the O rescale path
+    (and the redo of a tile's exponentials) in every row; a single huge
+    score late in the row does the same for one key."""
+    import dataclasses
+
+    inp = wl.make_custom([700, 300], 8, 2, 128, 1e4, seed=21)
+    t = np.arange(inp.workload.total_tokens, dtype=np.float32)
+    inp.k = wl.to_bf16_values(inp.k * (1.0 + t / 48.0)[:, None, None])
+    inp.q = wl.to_bf16_values(inp.q * np.float32(1.5))
+    out, lse = H.run_gpu(inp)
+    ref_out, ref_lse = H.oracle(inp)
+    H.compare(out, lse, ref_out, ref_lse, what="growing keys")
+    # one very large key in the middle of a long row, positions all zero
+    inp2 = wl.make_custom([520], 4, 1, 64, 1e4, seed=22)
+    inp2.k[400, 0, :] = wl.to_bf16_values(inp2.q[450, 0, :] * np.float32(6.0))
+    pos = np.zeros(520, np.int32)
+    out, lse = H.run_gpu(inp2, positions=pos)
+    ref_out, ref_lse = H.oracle(inp2, positions=pos)
+    H.compare(out, lse, ref_out, ref_lse, what="spike key")

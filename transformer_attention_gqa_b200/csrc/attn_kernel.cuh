@@ -201,6 +201,92 @@ constexpr int EMU_PERIOD = GQA_EMU_PERIOD;
 
 __device__ __forceinline__ uint32_t swz(uint32_t lin, int mask) { return lin ^ (((lin >> 7) & mask) << 4); }
 
+// The packed P row (BN/2 words) into its TMEM columns.
+__device__ __forceinline__ void store_p_row(uint32_t taddr, const uint32_t* r) {
+#pragma unroll
+  for (int c = 0; c < BN / 64; ++c) ptx::tmem_st32(taddr + c * 32, r + c * 32);
+}
+
+// D = A * B + C and A + B on pairs of fp32 (packed .f32x2 instructions).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// ---- softmax row helpers (one thread = one row of the S tile) ----
+
+// All BN columns of the row from TMEM into r[] (fp32 bit patterns).
+__device__ __forceinline__ void load_s_row(uint32_t taddr, uint32_t* r) {
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) ptx::tmem_ld32(taddr + c * 32, r + c * 32);
+  ptx::tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) ptx::reg_fence32(r + c * 32);
+}
+
+// Columns > lim get -inf (causal diagonal tile, or keys past the sequence).
+__device__ __forceinline__ void mask_row(uint32_t* r, int lim) {
+#pragma unroll
+  for (int c = 0; c < BN; ++c)
+    if (c > lim) r[c] = __float_as_uint(-INFINITY);
+}
+
+// Row max: 8 independent chains of 3-input max, then a tree.
+__device__ __forceinline__ float row_max(const uint32_t* r) {
+  float mx8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(__uint_as_float(r[e]), __uint_as_float(r[e + 8]));
+#pragma unroll
+  for (int c = 16; c < BN; c += 16)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], __uint_as_float(r[c + e]), __uint_as_float(r[c + 8 + e]));
+  return fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
+}
+
+// p = 2^(s * scale + bias) for the row, packed in place to bf16 pairs
+// (r[c/2], c = 0..BN-1). Returns the fp32 sum of p; if mx_out is given, also
+// the row max of s.
+__device__ __forceinline__ float exp_pack(uint32_t* r, float bias, float scale, float* mx_out) {
+  float2 ls[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) ls[e] = make_float2(0.f, 0.f);
+  float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  const float2 sc2 = make_float2(scale, scale), bi2 = make_float2(bias, bias);
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+#pragma unroll
+    for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 4) {
+      const float2 s01 = make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+      const float2 s23 = make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+      if (mx_out) mx4[(c >> 2) & 3] = fmax3(mx4[(c >> 2) & 3], fmaxf(s01.x, s01.y), fmaxf(s23.x, s23.y));
+      const float2 x01 = ffma2(s01, sc2, bi2);
+      const float2 x23 = ffma2(s23, sc2, bi2);
+      const float2 p01 = make_float2(ptx::ex2(x01.x), ptx::ex2(x01.y));
+      const float2 p23 = make_float2(ptx::ex2(x23.x), ptx::ex2(x23.y));
+      ls[(c >> 2) & 3] = fadd2(ls[(c >> 2) & 3], fadd2(p01, p23));
+      r[c >> 1] = pack_bf16x2(p01.x, p01.y);
+      r[(c >> 1) + 1] = pack_bf16x2(p23.x, p23.y);
+    }
+  }
+  if (mx_out) *mx_out = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+  const float2 t = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
+  return t.x + t.y;
+}
+
 // S = Q K^T for one KV tile: D/16 K-steps, K-major A and B (SW128/SW64).
 template <class C>
 __device__ __forceinline__ void issue_s_mmas(uint32_t d_tmem, uint64_t dq, uint64_t dk) {
@@ -427,82 +513,53 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       for (int j = 0; j < wi.nkv; ++j) {
         const uint32_t gg = g + j;
         const int b = gg % NUM_S_BUF;
+        const uint32_t tS = trow + b * 128;
         ok = __all_sync(0xffffffffu, bwait(B(bars->s_full[b]), (gg / NUM_S_BUF) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(trow + b * 128 + c * 32, sr + c * 32);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ptx::reg_fence32(sr + c * 32);
+        load_s_row(tS, sr);
         const int lim = last_key - j * BN;  // columns > lim are masked
-        if (lim < BN - 1) {
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c > lim) sr[c] = __float_as_uint(-INFINITY);
-        }
-        // row max: 8 independent chains of 3-input max, then a tree
-        float mx8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(__uint_as_float(sr[e]), __uint_as_float(sr[e + 8]));
-#pragma unroll
-        for (int c = 16; c < BN; c += 16)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], __uint_as_float(sr[c + e]), __uint_as_float(sr[c + 8 + e]));
-        const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
+        if (lim < BN - 1) mask_row(sr, lim);
         float alpha = 1.f;
         bool need = false;
+        float lsum;
         if (j == 0) {
-          m = mx;
-        } else if (mx > m + p.rescale_thr) {
-          alpha = ptx::ex2((m - mx) * sl2);
-          m = mx;
-          need = true;
-        }
-        const float neg = -m * sl2;
-        // p = 2^(s*log2e/sqrt(d) - m*log2e/sqrt(d)); 8 partial sums; P packed to
-        // bf16 pairs in place and stored to TMEM one half at a time
-        float ls8[8];
+          m = row_max(sr);
+          lsum = exp_pack(sr, -m * sl2, sl2, nullptr);
+        } else {
+          // Exponentials with the running max m, the tile's row max alongside;
+          // if it exceeds m by more than the threshold (2^8 in p) the tile is
+          // redone below with the new max.
+          float mx;
+          lsum = exp_pack(sr, -m * sl2, sl2, &mx);
+          if (mx > m + p.rescale_thr) {
+            alpha = ptx::ex2((m - mx) * sl2);
+            m = mx;
+            need = true;
+          }
+          if (__any_sync(0xffffffffu, need)) {
+            load_s_row(tS, sr);  // S is intact: P has not been stored yet
+            if (lim < BN - 1) mask_row(sr, lim);
+            lsum = exp_pack(sr, -m * sl2, sl2, nullptr);
+            // O holds the sum up to the previous tile: wait for PV(gg-1), then scale.
+            const uint32_t gp = gg - 1;
+            ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[gp % NUM_S_BUF]), (gp / NUM_S_BUF) & 1, abort_flag));
+            if (!ok) break;
+            ptx::tc_fence_after();
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ls8[e] = 0.f;
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t* o = sr + 64;
+              ptx::tmem_ld32(trow + C::O_COL + c * 32, o);
+              ptx::tmem_wait_ld();
+              ptx::reg_fence32(o);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-#pragma unroll
-          for (int c = half * 64; c < half * 64 + 64; c += 2) {
-            const float x0 = fmaf(__uint_as_float(sr[c]), sl2, neg);
-            const float x1 = fmaf(__uint_as_float(sr[c + 1]), sl2, neg);
-            float p0, p1;
-            if (EMU_PERIOD > 0 && ((c >> 1) % (EMU_PERIOD > 0 ? EMU_PERIOD : 1)) == EMU_PERIOD - 1) {
-              p0 = exp2_fma(x0);
-              p1 = exp2_fma(x1);
-            } else {
-              p0 = ptx::ex2(x0);
-              p1 = ptx::ex2(x1);
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              ptx::tmem_st32(trow + C::O_COL + c * 32, o);
             }
-            ls8[(c >> 1) & 7] += p0 + p1;
-            sr[c >> 1] = pack_bf16x2(p0, p1);
           }
-          ptx::tmem_st32(trow + b * 128 + half * 32, sr + half * 32);
         }
-        const float lsum = ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
         l = l * alpha + lsum;
-        if (__any_sync(0xffffffffu, need)) {
-          // O holds the sum up to the previous tile: wait for PV(gg-1), then scale.
-          const uint32_t gp = gg - 1;
-          ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[gp % NUM_S_BUF]), (gp / NUM_S_BUF) & 1, abort_flag));
-          if (!ok) break;
-          ptx::tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t* o = sr + 64;
-            ptx::tmem_ld32(trow + C::O_COL + c * 32, o);
-            ptx::tmem_wait_ld();
-            ptx::reg_fence32(o);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            ptx::tmem_st32(trow + C::O_COL + c * 32, o);
-          }
-        }
+        store_p_row(tS, sr);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(B(bars->p_full[b]));
