@@ -164,3 +164,24 @@ def test_running_max_rescale_paths():
     out, lse = H.run_gpu(inp2, positions=pos)
     ref_out, ref_lse = H.oracle(inp2, positions=pos)
     H.compare(out, lse, ref_out, ref_lse, what="spike key")
+
+
+def test_single_key_rows_pin_operand_rounding():
+    """Rows with one visible key: softmax is exactly 1, so out must equal v
+    bit for bit, and lse is one score q~.k~/sqrt(d) of the bf16-rounded
+    rotated operands. A single operand element rounded differently from the
+    oracle moves that score by ~1e-3, far above the fp32 accumulation error;
+    near-cancelling feature pairs and large positions stress the rounding."""
+    rng = np.random.default_rng(31)
+    n = 3000
+    inp = wl.make_custom([1] * n, 8, 2, 128, 5e5, seed=31)
+    # features i and i + d/2 equal in a quarter of the tokens (x*cos - y*sin cancels near 45 degrees)
+    sel = rng.random(n) < 0.25
+    inp.q[sel, :, 64:] = inp.q[sel, :, :64]
+    inp.k[sel, :, 64:] = inp.k[sel, :, :64]
+    pos = rng.integers(0, 500000, n).astype(np.int32)
+    out, lse = H.run_gpu(inp, positions=pos)
+    v_rep = np.repeat(inp.v.astype(np.float64), 4, axis=1)
+    assert np.array_equal(out, v_rep)
+    _, ref_lse = H.oracle(inp, positions=pos)
+    assert np.max(np.abs(lse - ref_lse)) < 2e-5

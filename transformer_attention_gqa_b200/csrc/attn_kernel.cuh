@@ -35,6 +35,7 @@
 #include "common.cuh"
 #include "exp2_poly.cuh"
 #include "ptx.cuh"
+#include "rope_round.cuh"
 
 namespace gqa {
 
@@ -663,17 +664,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(&vhi);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const double dl = (double)__bfloat162float(xl[e]);
-            const double dh = (double)__bfloat162float(xh[e]);
-            const double dc = (double)cs[e], ds = (double)sn[e];
-            const double rl = fma(dl, dc, -(dh * ds));
-            const double rh = fma(dh, dc, dl * ds);
-            float fl = __double2float_rz(rl);
-            if ((double)fl != rl) fl = __uint_as_float(__float_as_uint(fl) | 1u);
-            float fh = __double2float_rz(rh);
-            if ((double)fh != rh) fh = __uint_as_float(__float_as_uint(fh) | 1u);
-            xl[e] = __float2bfloat16_rn(fl);
-            xh[e] = __float2bfloat16_rn(fh);
+            const float fl = __bfloat162float(xl[e]), fh = __bfloat162float(xh[e]);
+            xl[e] = __ushort_as_bfloat16(rope_round_bf16(fl, cs[e], fh, -sn[e]));
+            xh[e] = __ushort_as_bfloat16(rope_round_bf16(fh, cs[e], fl, sn[e]));
           }
           *plo = vlo;
           *phi = vhi;

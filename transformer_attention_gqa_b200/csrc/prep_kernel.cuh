@@ -17,30 +17,23 @@
 //   out[i]       = x[i]       * cos - x[i + d/2] * sin
 //   out[i + d/2] = x[i + d/2] * cos + x[i]       * sin
 // The angle and cos/sin are evaluated in float64 and stored as fp32; the
-// rotation is one exact float64 fused multiply-add whose result is rounded
-// once, to nearest even, to bf16 (round-to-odd to fp32, then to bf16).
+// rotated value is rounded once, to nearest even, to bf16 from its exact
+// value (rope_round.cuh).
 #pragma once
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "rope_round.cuh"
 
 namespace gqa {
 
 
 __device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
 
-// Round a float64 value to the nearest bf16 (ties to even) in one rounding.
-__device__ __forceinline__ __nv_bfloat16 f64_to_bf16_rn(double x) {
-  float f = __double2float_rz(x);
-  if ((double)f != x) f = __uint_as_float(__float_as_uint(f) | 1u);  // round to odd
-  return __float2bfloat16_rn(f);
-}
-
 __device__ __forceinline__ void rope_pair(float xl, float xh, float c, float s, __nv_bfloat16& ol,
                                           __nv_bfloat16& oh) {
-  const double dc = (double)c, ds = (double)s, dl = (double)xl, dh = (double)xh;
-  ol = f64_to_bf16_rn(fma(dl, dc, -(dh * ds)));
-  oh = f64_to_bf16_rn(fma(dh, dc, dl * ds));
+  ol = __ushort_as_bfloat16(rope_round_bf16(xl, c, xh, -s));
+  oh = __ushort_as_bfloat16(rope_round_bf16(xh, c, xl, s));
 }
 
 // largest s in [0, n) with a[s] <= x (a nondecreasing, a[0] <= x)
