@@ -100,34 +100,47 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle timing
-def cpu_baseline(workload, budget_s: float = 15.0, seed_rows: int = 0):
-    """Times the float64 oracle, as it stands, on a bounded sample of query
-    rows of the workload; returns (TFLOP/s by the metric's convention, info)."""
-    import oracle.gqa_oracle as orc
+_INPUTS = {}
+
+
+def _cached_inputs(workload):
     from transformer_attention_gqa_b200 import workloads as wl
 
-    inp = wl.make_inputs(workload)
-    w = workload
+    if workload.name not in _INPUTS:
+        _INPUTS[workload.name] = wl.make_inputs(workload)
+    return _INPUTS[workload.name]
+
+
+def _oracle_rows(inp, w, rows):
+    import oracle.gqa_oracle as orc
+
+    t0 = time.perf_counter()
+    orc.gqa_rope_attention(inp.q, inp.k, inp.v, inp.cu_seqlens, w.n_q_heads, w.n_kv_heads, w.rope_theta,
+                           causal=w.causal, query_rows=rows)
+    dt = time.perf_counter() - t0
     cu = inp.cu_seqlens
+    seq = np.searchsorted(cu, rows, side="right") - 1
+    tok = rows - cu[seq]
+    L = cu[seq + 1] - cu[seq]
+    keys = (tok + 1) if w.causal else L
+    # metric convention: 4*Tq*Tk*d per head, halved for causal == 4*d per (row, visible key, head)
+    return dt, float(np.sum(4.0 * keys * w.head_dim * w.n_q_heads))
+
+
+def cpu_baseline(workload, budget_s: float = 15.0, seed_rows: int = 0):
+    """Times the float64 oracle, as it stands, on a bounded sample of random
+    query rows of the workload (two small probes size the sample to about
+    budget_s seconds); returns its TFLOP/s by the metric's convention."""
+    w = workload
+    inp = _cached_inputs(w)
     rng = np.random.default_rng(seed_rows)
-    # grow the sample until the budget is used
-    n_rows = 8
-    spent, flops, rows_done = 0.0, 0.0, 0
-    while spent < budget_s:
-        rows = np.sort(rng.integers(0, w.total_tokens, n_rows))
-        t0 = time.perf_counter()
-        orc.gqa_rope_attention(inp.q, inp.k, inp.v, cu, w.n_q_heads, w.n_kv_heads, w.rope_theta,
-                               causal=w.causal, query_rows=rows)
-        dt = time.perf_counter() - t0
-        seq = np.searchsorted(cu, rows, side="right") - 1
-        tok = rows - cu[seq]
-        L = cu[seq + 1] - cu[seq]
-        keys = (tok + 1) if w.causal else L
-        # metric convention: 4*Tq*Tk*d per head halved for causal == 4*d per (row, visible key)
-        flops += float(np.sum(4.0 * keys * w.head_dim * w.n_q_heads))
-        spent += dt
-        rows_done += n_rows
-        n_rows = min(n_rows * 2, 4096)
+    pick = lambda n: np.sort(rng.choice(w.total_tokens, size=min(n, w.total_tokens), replace=False))
+    t8, _ = _oracle_rows(inp, w, pick(8))
+    t64, _ = _oracle_rows(inp, w, pick(64))
+    per_row = max((t64 - t8) / 56.0, 1e-6)
+    fixed = max(t8 - 8 * per_row, 0.0)
+    n = int(max(8, min(w.total_tokens, (budget_s - fixed) / per_row)))
+    dt, flops = _oracle_rows(inp, w, pick(n))
     cores = len(os.sched_getaffinity(0))
     threads = None
     try:
@@ -135,22 +148,22 @@ def cpu_baseline(workload, budget_s: float = 15.0, seed_rows: int = 0):
         threads = max((x.get("num_threads", 0) for x in threadpool_info()), default=None)
     except Exception:
         pass
-    info = {"value": flops / spent / 1e12, "unit": UNIT, "cores": threads or cores, "kind": "oracle",
-            "sample": f"{rows_done} random query rows x {w.n_q_heads} heads of {w.name}, float64 NumPy, "
-                      f"{spent:.1f} s", "host_cores": cores}
-    return info
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": threads or cores, "kind": "oracle",
+            "sample": f"{n} random query rows x {w.n_q_heads} heads of {w.name} (all their visible keys), "
+                      f"float64 NumPy, {dt:.1f} s", "host_cores": cores}
 
 
 # ------------------------------------------------------------------ GPU arm
 def run_ours(args, rank, world, local_rank):
     import torch
     import transformer_attention_gqa_b200 as g
-    from transformer_attention_gqa_b200 import _abi, workloads as wl
+    from transformer_attention_gqa_b200 import _abi, replicas, workloads as wl
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = wl.WORKLOADS[args.workload]
-    inp = wl.make_inputs(w)
+    # every rank runs its own batch of the same shape (weak scaling)
+    inp = wl.make_inputs(w, seed=w.seed if rank == 0 else replicas.replica_seed(w.seed, rank))
     dt = torch.float32 if w.io_dtype == "fp32" else torch.bfloat16
     q = torch.from_numpy(inp.q).to(dt).to(dev)
     k = torch.from_numpy(inp.k).to(dt).to(dev)
@@ -172,10 +185,7 @@ def run_ours(args, rank, world, local_rank):
     assert g.get_device_status() == 0
     launches_per_step = _abi.last_launch_count()
 
-    def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
+    barrier = replicas.barrier
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -256,11 +266,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1) / e_steps
     assert g.get_device_status() == 0
 
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms, e2e_ms, attn_ms, prep_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms, attn_ms, prep_ms = t.tolist()
+    total_ms, e2e_ms, attn_ms, prep_ms = replicas.max_over_ranks([total_ms, e2e_ms, attn_ms, prep_ms], device=dev)
 
     flops = w.flops()
     ms_per_step = total_ms / args.steps
@@ -316,11 +322,11 @@ def main():
         if rank != 0:
             return 0
         per_step = []
-        for _ in range(args.warmup):
-            cpu_baseline(w, budget_s=0.5)
+        for i in range(args.warmup):
+            cpu_baseline(w, budget_s=0.5, seed_rows=1000 + i)
         info = None
-        for _ in range(args.steps):
-            info = cpu_baseline(w, budget_s=max(1.0, 60.0 / max(args.steps, 1)))
+        for i in range(args.steps):
+            info = cpu_baseline(w, budget_s=max(1.0, min(5.0, 60.0 / max(args.steps, 1))), seed_rows=i)
             per_step.append(info["value"])
         val = statistics.median(per_step)
         res = {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": UNIT, "n_gpus": world,
@@ -333,17 +339,12 @@ def main():
         print(json.dumps(res))
         return 0
 
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from transformer_attention_gqa_b200 import replicas
+    replicas.init("nccl", timeout_s=120)
     res = run_ours(args, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
+    replicas.shutdown()
     if rank == 0:
         print(json.dumps(res))
     return 0

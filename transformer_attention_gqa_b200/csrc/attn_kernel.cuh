@@ -14,14 +14,15 @@
 // tile loaded by TMA is used by all G heads at once.
 //
 // Warp roles (384 threads):
-//   warp 0      TMA producer: Q tile and K tiles (K is RoPE'd already)
+//   warp 0      TMA producer: K tiles (K is RoPE'd already)
 //   warp 1      TMEM allocator; one thread issues the S = Q K^T MMAs
 //   warp 2      TMA producer: V tiles
 //   warp 3      one thread issues the O += P V MMAs
 //   warps 4-7   softmax: one thread per row (TMEM lane), S -> P, running
 //               max/sum, O rescale, epilogue (O / l, LSE)
-//   warps 8-11  Q rotation: RoPE applied in shared memory to each Q tile
-//               after its TMA load, before the first S MMA reads it
+//   warps 8-11  Q tiles: TMA load, RoPE applied in shared memory before the
+//               first S MMA reads it; epilogue: O / l from TMEM, TMA store,
+//               LSE
 //
 // Tensor memory (512 columns x 128 lanes of 32 bit):
 //   [0,128) [128,256) [256,384): three S buffers; the bf16 P of a tile
@@ -40,8 +41,25 @@
 namespace gqa {
 
 
-template <int D>
+constexpr int REG_PRODUCER = 56;
+constexpr int REG_SOFTMAX = 232;
+constexpr int REG_ROPE = 128;
+static_assert((REG_PRODUCER + REG_SOFTMAX + REG_ROPE) * 128 <= 65536 / ATTN_THREADS * ATTN_THREADS,
+              "register split exceeds the launch's register file share");
+
+struct Barriers {
+  uint64_t q_loaded[2], q_ready[2], q_empty[2];
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t s_full[NUM_S_BUF], p_full[NUM_S_BUF], pv_done[NUM_S_BUF];
+  uint64_t o_free, drain;
+  uint64_t stats_full, stats_empty;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D_>
 struct AttnCfg {
+  static constexpr int D = D_;
   static constexpr int BOXC = D >= 64 ? 64 : 32;   // columns per TMA box
   static constexpr int NBOX = D / BOXC;            // boxes per row of a tile
   static constexpr int ROWB = BOXC * 2;            // bytes per box row (swizzle span)
@@ -56,7 +74,8 @@ struct AttnCfg {
   static constexpr int VST = KST;
   static constexpr int OFF_K = 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
+  static constexpr int OFF_STATS = OFF_V + VST * KV_BYTES;  // float2 (m, l) per row, softmax -> epilogue
+  static constexpr int OFF_BAR = OFF_STATS + BM * 8;
   static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
@@ -70,6 +89,7 @@ struct AttnCfg {
   static constexpr uint32_t IDESC_O = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                                       ((uint32_t)(D >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(sizeof(Barriers) <= BAR_BYTES, "barrier area");
   static_assert(O_COL + D <= TMEM_COLS, "tensor memory budget");
 };
 
@@ -79,21 +99,6 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (layout << 61);
 }
-
-constexpr int REG_PRODUCER = 56;
-constexpr int REG_SOFTMAX = 232;
-constexpr int REG_ROPE = 128;
-static_assert((REG_PRODUCER + REG_SOFTMAX + REG_ROPE) * 128 <= 65536 / ATTN_THREADS * ATTN_THREADS,
-              "register split exceeds the launch's register file share");
-
-struct Barriers {
-  uint64_t q_loaded[2], q_ready[2], q_empty[2];
-  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[NUM_S_BUF], p_full[NUM_S_BUF], pv_done[NUM_S_BUF];
-  uint64_t o_free, drain;
-  uint32_t tmem_base;
-  int abort_flag;
-};
 
 struct WorkItem {
   int seq_start, L, t0, nkv, kvh;
@@ -288,6 +293,145 @@ __device__ __forceinline__ float exp_pack(uint32_t* r, float bias, float scale, 
   return t.x + t.y;
 }
 
+// Rotates the Q tile of work item `wi` in shared memory (buffer it & 1) once
+// its TMA load has landed, then releases it to the S issuer. Run by the 128
+// threads of the Q-rotation/epilogue warpgroup.
+template <class C>
+__device__ __forceinline__ bool rope_q_tile(const AttnParams& p, const WorkItem& wi, uint8_t* smem, Barriers* bars,
+                                            const CUtensorMap* tmQ, int it, int tid, volatile int* abort_flag) {
+  constexpr int D = C::D;
+  constexpr int NCH = D / 16;  // 16-byte chunks in the first half of a row
+  constexpr int HALF = D / 2;
+  const int qb = it & 1;
+  const int G = p.G;
+  bool issued = false;
+  if (tid == 0) {  // the buffer's previous tile has finished its S MMAs: load this tile's Q
+    if (bwait(ptx::smem_u32(&bars->q_empty[qb]), ((it >> 1) & 1) ^ 1, abort_flag)) {
+      issued = true;
+      const uint32_t bar = ptx::smem_u32(&bars->q_loaded[qb]);
+      ptx::mbar_arrive_expect_tx(bar, (uint32_t)(D * 2 * G * p.tq));
+#pragma unroll
+      for (int b = 0; b < C::NBOX; ++b)
+        ptx::tma_load_3d(ptx::smem_u32(smem + qb * C::Q_BYTES + b * C::Q_BOX_BYTES), tmQ, bar, b * C::BOXC,
+                         wi.kvh * G, wi.seq_start + wi.t0);
+    }
+  }
+  const bool ok = __all_sync(0xffffffffu, bwait_lazy(ptx::smem_u32(&bars->q_loaded[qb]), (it >> 1) & 1, abort_flag));
+  if (!ok) {  // a load issued above lands before the CTA may exit
+    if (issued) drain_wait(ptx::smem_u32(&bars->q_loaded[qb]), (it >> 1) & 1);
+    return false;
+  }
+  uint8_t* qbuf = smem + qb * C::Q_BYTES;
+  const int items = p.tq * NCH;
+  for (int item = tid; item < items; item += 128) {
+    const int tt = item / NCH;
+    const int ch = item - tt * NCH;
+    const int tok = wi.t0 + tt;
+    if (tok >= wi.L) continue;
+    const float4* tab = reinterpret_cast<const float4*>(p.table + (size_t)(wi.seq_start + tok) * HALF + ch * 8);
+    float cs[8], sn[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float4 t4 = ptx::ld_cg_v4f32(tab + e);
+      cs[2 * e] = t4.x;
+      sn[2 * e] = t4.y;
+      cs[2 * e + 1] = t4.z;
+      sn[2 * e + 1] = t4.w;
+    }
+    const int col_lo = ch * 8, col_hi = ch * 8 + HALF;
+    const int bx_lo = col_lo / C::BOXC, bx_hi = col_hi / C::BOXC;
+    for (int hh = 0; hh < G; ++hh) {
+      const int row = tt * G + hh;
+      uint4* plo = reinterpret_cast<uint4*>(qbuf + bx_lo * C::Q_BOX_BYTES +
+                                            swz(row * C::ROWB + (col_lo % C::BOXC) * 2, C::SWZ_MASK));
+      uint4* phi = reinterpret_cast<uint4*>(qbuf + bx_hi * C::Q_BOX_BYTES +
+                                            swz(row * C::ROWB + (col_hi % C::BOXC) * 2, C::SWZ_MASK));
+      uint4 vlo = *plo, vhi = *phi;
+      __nv_bfloat16* xl = reinterpret_cast<__nv_bfloat16*>(&vlo);
+      __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(&vhi);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float fl = __bfloat162float(xl[e]), fh = __bfloat162float(xh[e]);
+        xl[e] = __ushort_as_bfloat16(rope_round_bf16(fl, cs[e], fh, -sn[e]));
+        xh[e] = __ushort_as_bfloat16(rope_round_bf16(fh, cs[e], fl, sn[e]));
+      }
+      *plo = vlo;
+      *phi = vhi;
+    }
+  }
+  ptx::fence_proxy_async_smem();
+  ptx::mbar_arrive(ptx::smem_u32(&bars->q_ready[qb]));
+  return true;
+}
+
+// Epilogue of work item `wi` (the CTA's it-th): out = O / l (bf16 or fp32),
+// lse = (m log2e/sqrt(d) + log2 l) ln 2. One thread per row (TMEM lane),
+// 16-byte stores of the row. (Staging the tile in shared memory for a TMA
+// store was measured slower: this runs off the softmax's critical path.)
+template <class C, bool OUT_FP32>
+__device__ __forceinline__ bool epilogue_tile(const AttnParams& p, const WorkItem& wi, uint8_t* smem, Barriers* bars,
+                                              uint32_t tmem, int it, uint32_t g, int tid,
+                                              volatile int* abort_flag) {
+  constexpr int D = C::D;
+  const int warp = tid >> 5;  // 0..3 inside the warpgroup == TMEM lane quadrant
+  const int r = tid;
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  const int G = p.G;
+  const int tok_off = r / G;
+  const int hin = r - tok_off * G;
+  const int tok = wi.t0 + tok_off;
+  const bool row_valid = r < p.tq * G && tok < wi.L;
+  bool ok = __all_sync(0xffffffffu, bwait(ptx::smem_u32(&bars->stats_full), it & 1, abort_flag));
+  if (!ok) return false;
+  const float2 ml = reinterpret_cast<const float2*>(smem + C::OFF_STATS)[r];
+  ptx::mbar_arrive(ptx::smem_u32(&bars->stats_empty));
+  const uint32_t gl = g + wi.nkv - 1;
+  ok = __all_sync(0xffffffffu,
+                  bwait(ptx::smem_u32(&bars->pv_done[gl % NUM_S_BUF]), (gl / NUM_S_BUF) & 1, abort_flag));
+  if (!ok) return false;
+  ptx::tc_fence_after();
+
+  const float inv_l = 1.f / ml.y;
+  const int h = wi.kvh * G + hin;
+  const size_t orow = (size_t)(wi.seq_start + tok) * p.nq + h;
+  uint32_t o[32];
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    ptx::tmem_ld32(trow + C::O_COL + c * 32, o);
+    ptx::tmem_wait_ld();
+    ptx::reg_fence32(o);
+    if (c == D / 32 - 1) {  // O fully read: the next tile's first P.V may overwrite it
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(ptx::smem_u32(&bars->o_free));
+    }
+    if constexpr (OUT_FP32) {
+      if (row_valid) {
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + orow * D + c * 32);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
+                               __uint_as_float(o[4 * e + 2]) * inv_l, __uint_as_float(o[4 * e + 3]) * inv_l);
+      }
+    } else {
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv_l,
+                                                        __uint_as_float(o[2 * e + 1]) * inv_l);
+        pk[e] = *reinterpret_cast<const uint32_t*>(&v2);
+      }
+      if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + orow * D + c * 32);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+      }
+    }
+  }
+  if (row_valid && p.lse)
+    p.lse[(size_t)h * p.N + wi.seq_start + tok] = (ml.x * p.scale_log2 + __log2f(ml.y)) * 0.69314718055994531f;
+  return true;
+}
+
 // S = Q K^T for one KV tile: D/16 K-steps, K-major A and B (SW128/SW64).
 template <class C>
 __device__ __forceinline__ void issue_s_mmas(uint32_t d_tmem, uint64_t dq, uint64_t dk) {
@@ -343,6 +487,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       ptx::mbar_init(B(bars->pv_done[i]), 1);
     }
     ptx::mbar_init(B(bars->o_free), 128);
+    ptx::mbar_init(B(bars->stats_full), 128);
+    ptx::mbar_init(B(bars->stats_empty), 128);
     ptx::mbar_init(B(bars->drain), 2);  // one commit per MMA-issuing thread
     bars->abort_flag = 0;
     ptx::fence_mbar_init();
@@ -361,7 +507,10 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  // Everything below reads what the prologue kernel wrote.
+  // Everything below reads what the prologue kernel wrote. The attention
+  // kernel is launched in plain stream order (a programmatic dependent
+  // launch measured slower), so this wait returns at once; it would order
+  // the reads if the launch were made programmatic.
   ptx::griddep_wait();
   const int n_items = ptx::ld_cg_s32(p.header) * p.nkv;
 
@@ -370,20 +519,12 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   if (warp < 4) {
    ptx::setmaxnreg_dec<REG_PRODUCER>();
    if (warp == 0) {
-    // ------------------------------------------------------------ Q/K producer
+    // ------------------------------------------------------------ K producer
     if (lane == 0) {
       uint32_t g = 0;
-      int it = 0, q_issued = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
+      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
         const WorkItem wi = decode_item(p, w);
-        const int qb = it & 1;
-        if (!(ok = bwait_lazy(B(bars->q_empty[qb]), ((it >> 1) & 1) ^ 1, abort_flag))) break;
-        ptx::mbar_arrive_expect_tx(B(bars->q_loaded[qb]), (uint32_t)(D * 2 * p.G * p.tq));
-        for (int b = 0; b < C::NBOX; ++b)
-          ptx::tma_load_3d(sbase + qb * C::Q_BYTES + b * C::Q_BOX_BYTES, &tmQ, B(bars->q_loaded[qb]),
-                           b * C::BOXC, wi.kvh * p.G, wi.seq_start + wi.t0);
-        ++q_issued;
         for (int j = 0; j < wi.nkv; ++j, ++g) {
           const int ks = g % C::KST;
           if (!(ok = bwait_lazy(B(bars->k_empty[ks]), ((g / C::KST) & 1) ^ 1, abort_flag))) break;
@@ -394,11 +535,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         }
       }
       if (!ok) {  // let every copy already issued land before the CTA exits
-        // loads issued: Q tiles 0..q_issued-1 (buffer t & 1), K tiles 0..g-1 (stage x % KST)
-        for (int i = 0; i < 2; ++i) {
-          const int uses = (q_issued - i + 1) / 2;
-          if (uses > 0) drain_wait(B(bars->q_loaded[i]), (uses - 1) & 1);
-        }
+        // loads issued: K tiles 0..g-1 (stage x % KST)
         for (int i = 0; i < C::KST; ++i) {
           const int uses = ((int)g - i + C::KST - 1) / C::KST;
           if (uses > 0) drain_wait(B(bars->k_full[i]), (uses - 1) & 1);
@@ -498,9 +635,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
     const int G = p.G;
     const int tok_off = r / G;
-    const int hin = r - tok_off * G;
-    const bool row_in_tile = r < p.tq * G;
     const float sl2 = p.scale_log2;
+    float2* stats = reinterpret_cast<float2*>(smem + C::OFF_STATS);
     uint32_t g = 0;
     int it = 0;
     bool ok = true;
@@ -566,54 +702,18 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         ptx::mbar_arrive(B(bars->p_full[b]));
       }
       if (!ok) break;
-      // ---- epilogue: O / l and LSE
-      const uint32_t gl = g + wi.nkv - 1;
-      ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[gl % NUM_S_BUF]), (gl / NUM_S_BUF) & 1, abort_flag));
+      // ---- hand (m, l) of every row to the epilogue warps
+      ok = __all_sync(0xffffffffu, bwait(B(bars->stats_empty), (it & 1) ^ 1, abort_flag));
       if (!ok) break;
-      ptx::tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(trow + C::O_COL + c * 32, sr + c * 32);
-      ptx::tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) ptx::reg_fence32(sr + c * 32);
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(B(bars->o_free));
-      if (row_in_tile && tok < wi.L) {
-        const float inv_l = 1.f / l;
-        const int h = wi.kvh * G + hin;
-        const size_t row = (size_t)(wi.seq_start + tok) * p.nq + h;
-        if constexpr (OUT_FP32) {
-          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + row * D);
-#pragma unroll
-          for (int c = 0; c < D; c += 4)
-            dst[c / 4] = make_float4(__uint_as_float(sr[c]) * inv_l, __uint_as_float(sr[c + 1]) * inv_l,
-                                     __uint_as_float(sr[c + 2]) * inv_l, __uint_as_float(sr[c + 3]) * inv_l);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + row * D);
-#pragma unroll
-          for (int c = 0; c < D; c += 8) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(sr[c + 2 * e]) * inv_l,
-                                                             __uint_as_float(sr[c + 2 * e + 1]) * inv_l);
-              pk[e] = *reinterpret_cast<const uint32_t*>(&v);
-            }
-            dst[c / 8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
-        }
-        if (p.lse) p.lse[(size_t)h * p.N + wi.seq_start + tok] = (m * sl2 + __log2f(l)) * 0.69314718055994531f;
-      }
+      stats[r] = make_float2(m, l);
+      ptx::mbar_arrive(B(bars->stats_full));
       g += wi.nkv;
     }
   } else {
     ptx::setmaxnreg_dec<REG_ROPE>();
-    // ------------------------------------------------------------ Q rotation
+    // ------------------------------------------------------------ Q rotation + epilogue
     const int tid = threadIdx.x - 256;
-    const int G = p.G;
-    const int rows = p.tq * G;
-    constexpr int NCH = D / 16;  // 16-byte chunks in the first half of a row
-    constexpr int HALF = D / 2;
+    const int rows = p.tq * p.G;
     // padding rows (never written by TMA) are zero in both Q buffers
     for (int i = tid; i < 2 * C::NBOX * (BM - rows) * (C::ROWB / 16); i += 128) {
       const int per_buf = C::NBOX * (BM - rows) * (C::ROWB / 16);
@@ -627,53 +727,20 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
                                             swz(row * C::ROWB + ch * 16, C::SWZ_MASK));
       *dst = make_uint4(0, 0, 0, 0);
     }
-    int it = 0;
+    // Order: rope(0); then for every tile t: rope(t + 1), epilogue(t). The
+    // next tile's Q is rotated while tile t still runs; the epilogue of t
+    // runs once its last P.V is done.
     bool ok = true;
+    if (blockIdx.x < n_items) ok = rope_q_tile<C>(p, decode_item(p, blockIdx.x), smem, bars, &tmQ, 0, tid, abort_flag);
+    int it = 0;
+    uint32_t g = 0;
     for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
       const WorkItem wi = decode_item(p, w);
-      const int qb = it & 1;
-      ok = __all_sync(0xffffffffu, bwait_lazy(B(bars->q_loaded[qb]), (it >> 1) & 1, abort_flag));
+      if (w + (int)gridDim.x < n_items)
+        ok = rope_q_tile<C>(p, decode_item(p, w + gridDim.x), smem, bars, &tmQ, it + 1, tid, abort_flag);
       if (!ok) break;
-      uint8_t* qbuf = smem + qb * C::Q_BYTES;
-      const int items = p.tq * NCH;
-      for (int item = tid; item < items; item += 128) {
-        const int tt = item / NCH;
-        const int ch = item - tt * NCH;
-        const int tok = wi.t0 + tt;
-        if (tok >= wi.L) continue;
-        const float4* tab = reinterpret_cast<const float4*>(p.table + (size_t)(wi.seq_start + tok) * HALF + ch * 8);
-        float cs[8], sn[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float4 t4 = ptx::ld_cg_v4f32(tab + e);
-          cs[2 * e] = t4.x;
-          sn[2 * e] = t4.y;
-          cs[2 * e + 1] = t4.z;
-          sn[2 * e + 1] = t4.w;
-        }
-        const int col_lo = ch * 8, col_hi = ch * 8 + HALF;
-        const int bx_lo = col_lo / C::BOXC, bx_hi = col_hi / C::BOXC;
-        for (int hh = 0; hh < G; ++hh) {
-          const int row = tt * G + hh;
-          uint4* plo = reinterpret_cast<uint4*>(
-              qbuf + bx_lo * C::Q_BOX_BYTES + swz(row * C::ROWB + (col_lo % C::BOXC) * 2, C::SWZ_MASK));
-          uint4* phi = reinterpret_cast<uint4*>(
-              qbuf + bx_hi * C::Q_BOX_BYTES + swz(row * C::ROWB + (col_hi % C::BOXC) * 2, C::SWZ_MASK));
-          uint4 vlo = *plo, vhi = *phi;
-          __nv_bfloat16* xl = reinterpret_cast<__nv_bfloat16*>(&vlo);
-          __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(&vhi);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float fl = __bfloat162float(xl[e]), fh = __bfloat162float(xh[e]);
-            xl[e] = __ushort_as_bfloat16(rope_round_bf16(fl, cs[e], fh, -sn[e]));
-            xh[e] = __ushort_as_bfloat16(rope_round_bf16(fh, cs[e], fl, sn[e]));
-          }
-          *plo = vlo;
-          *phi = vhi;
-        }
-      }
-      ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(B(bars->q_ready[qb]));
+      ok = epilogue_tile<C, OUT_FP32>(p, wi, smem, bars, tmem, it, g, tid, abort_flag);
+      g += wi.nkv;
     }
   }
 

@@ -1,6 +1,6 @@
 // Host side of the C ABI (include/gqa_rope_attn.h): argument checks, TMA
 // descriptor cache, and the two launches of the fused forward (prologue,
-// then the attention kernel chained by programmatic dependent launch).
+// then the attention kernel, in stream order).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -180,6 +180,7 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
     if (!make_tmap(device, vsrc, dims, str, box, C::ROWB, &tmV)) return GQA_ERR_CUDA;
   }
 
+
   const long long work = (long long)N * (D / 4);
   long long nb = (work + PREP_THREADS - 1) / PREP_THREADS;
   const long long cap = (long long)sm_count * 8;
@@ -216,11 +217,8 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
   cfg.blockDim = dim3(ATTN_THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;  // plain stream order after the prologue kernel
   if (cudaLaunchKernelEx(&cfg, gqa_attn_fwd_kernel<D, FP32>, tmQ, tmK, tmV, ap) != cudaSuccess)
     return GQA_ERR_CUDA;
   if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;

@@ -1,6 +1,5 @@
 // Prologue kernel of the fused forward. Runs once per call, ahead of the
-// attention kernel (which it releases early through programmatic dependent
-// launch):
+// attention kernel:
 //
 //  * block 0 checks cu_seqlens and builds the tile schedule: every
 //    (sequence, q-tile) pair, sorted by decreasing cost (number of KV tiles
