@@ -74,7 +74,9 @@ enum {
   GQA_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed          */
   GQA_ERR_BAD_SEQLENS = 4, /* device: cu_seqlens not a valid prefix sum     */
   GQA_ERR_TIMEOUT = 5,     /* device: a bounded wait in the kernel ran out  */
-  GQA_ERR_WORKSPACE = 6    /* workspace missing, too small or misaligned    */
+  GQA_ERR_WORKSPACE = 6,   /* workspace missing, too small or misaligned    */
+  GQA_ERR_NOALLOC_LIMIT = 7 /* shape needs more scratch than the built-in
+                               buffer of gqa_rope_attn_fwd_noalloc holds    */
 };
 
 /* Bytes of scratch the caller must pass to gqa_rope_attn_fwd for this shape
@@ -133,6 +135,38 @@ int gqa_rope_attn_abi_version(void);
 /* Number of kernel launches the last successful gqa_rope_attn_fwd queued on
  * the calling thread (0 for a no-op). */
 int gqa_rope_attn_last_launch_count(void);
+
+/* Size of the scratch buffer built into the library for
+ * gqa_rope_attn_fwd_noalloc: 32 MiB of device memory per GPU that loads the
+ * library, held until the process exits. */
+#define GQA_ROPE_ATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* The fused forward for callers that cannot allocate device memory: for
+ * instance code running inside a host application that owns every device
+ * allocation and forbids its plug-ins from making their own, or callers that
+ * cannot afford the device-wide synchronisation cudaMalloc/cudaFree imply.
+ * (The pages have no counterpart; this is a deployment convenience.)
+ *
+ * Same arguments and results as gqa_rope_attn_fwd, minus the workspace: the
+ * scratch lives in a static device array of GQA_ROPE_ATTN_NOALLOC_SCRATCH_BYTES
+ * inside the library. The caller still provides q, k, v, positions,
+ * cu_seqlens, out and lse. Nothing is allocated, by this call or any library
+ * it uses.
+ *   - Shapes whose gqa_rope_attn_workspace_size() exceeds the buffer are
+ *     rejected with GQA_ERR_NOALLOC_LIMIT before any CUDA call.
+ *   - The first call on a device (per process) looks the buffer's device
+ *     address up with cudaGetSymbolAddress, with that device current; make
+ *     that first call before any stream capture on the device.
+ *   - All calls on a device share the one buffer: calls that may overlap on
+ *     the GPU (different streams without ordering, several host threads)
+ *     race on it and must be serialised by the caller. The buffer keeps the
+ *     last call's contents; nothing in it needs to start at zero, since each
+ *     call writes every byte it later reads.
+ */
+int gqa_rope_attn_fwd_noalloc(const void* q, const void* k, const void* v, const int32_t* positions,
+                              double rope_theta, const int32_t* cu_seqlens, int num_seqs,
+                              int total_tokens, int n_q_heads, int n_kv_heads, int head_dim,
+                              int causal, int dtype, void* out, float* lse, void* stream);
 
 /* Measurement aid. Arms the calling thread's next gqa_rope_attn_fwd call to
  * record three CUDA events (cudaEvent_t passed as void*, any may be NULL) on

@@ -20,6 +20,8 @@ GQA_ERR_CUDA = 3
 GQA_ERR_BAD_SEQLENS = 4
 GQA_ERR_TIMEOUT = 5
 GQA_ERR_WORKSPACE = 6
+GQA_ERR_NOALLOC_LIMIT = 7
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 EXPORTED = (
     "gqa_rope_attn_workspace_size",
@@ -29,6 +31,7 @@ EXPORTED = (
     "gqa_rope_attn_abi_version",
     "gqa_rope_attn_last_launch_count",
     "gqa_rope_attn_set_profile_events",
+    "gqa_rope_attn_fwd_noalloc",
 )
 
 _lib = None
@@ -64,6 +67,9 @@ def load() -> ctypes.CDLL:
     lib.gqa_rope_attn_abi_version.argtypes = []
     lib.gqa_rope_attn_last_launch_count.restype = c_int
     lib.gqa_rope_attn_last_launch_count.argtypes = []
+    lib.gqa_rope_attn_fwd_noalloc.restype = c_int
+    lib.gqa_rope_attn_fwd_noalloc.argtypes = [c_void, c_void, c_void, c_void, c_double, c_void, c_int, c_int, c_int,
+                                              c_int, c_int, c_int, c_int, c_void, c_void, c_void]
     lib.gqa_rope_attn_set_profile_events.restype = None
     lib.gqa_rope_attn_set_profile_events.argtypes = [c_void, c_void, c_void]
     _lib = lib
@@ -85,6 +91,15 @@ def gqa_rope_attn_fwd(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, tota
     return int(load().gqa_rope_attn_fwd(q, k, v, positions, float(rope_theta), cu_seqlens, int(num_seqs),
                                         int(total_tokens), int(n_q_heads), int(n_kv_heads), int(head_dim),
                                         int(causal), int(dtype), out, lse, workspace, int(workspace_bytes), stream))
+
+
+def gqa_rope_attn_fwd_noalloc(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads,
+                              n_kv_heads, head_dim, causal, dtype, out, lse, stream) -> int:
+    """Raw call of the no-allocation entry point (scratch built into the
+    library); integer device addresses, 0 for NULL; returns the status."""
+    return int(load().gqa_rope_attn_fwd_noalloc(q, k, v, positions, float(rope_theta), cu_seqlens, int(num_seqs),
+                                                int(total_tokens), int(n_q_heads), int(n_kv_heads), int(head_dim),
+                                                int(causal), int(dtype), out, lse, stream))
 
 
 def get_device_status(stream=None) -> int:

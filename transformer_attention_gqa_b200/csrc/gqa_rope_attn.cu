@@ -301,6 +301,43 @@ extern "C" int gqa_rope_attn_fwd(const void* q, const void* k, const void* v, co
   return rc;
 }
 
+// ---------------------------------------------------------------------------
+// No-allocation variant: the workspace is a static device array of the
+// library (one per device that loads it).
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[GQA_ROPE_ATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+}  // namespace
+
+extern "C" int gqa_rope_attn_fwd_noalloc(const void* q, const void* k, const void* v, const int32_t* positions,
+                                         double rope_theta, const int32_t* cu_seqlens, int num_seqs,
+                                         int total_tokens, int n_q_heads, int n_kv_heads, int head_dim,
+                                         int causal, int dtype, void* out, float* lse, void* stream) {
+  const size_t need =
+      gqa_rope_attn_workspace_size(num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim, dtype);
+  if (need > (size_t)GQA_ROPE_ATTN_NOALLOC_SCRATCH_BYTES) return GQA_ERR_NOALLOC_LIMIT;
+  void* scratch = nullptr;
+  if (total_tokens > 0 && need > 0) {
+    int device = 0;
+    if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices) return GQA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[device]) {
+      // The array's name is only a host-side handle; its device address is
+      // looked up once per device, with that device current.
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return GQA_ERR_CUDA;
+      g_noalloc_ptr[device] = ptr;
+    }
+    scratch = g_noalloc_ptr[device];
+  }
+  return gqa_rope_attn_fwd(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads,
+                           n_kv_heads, head_dim, causal, dtype, out, lse, scratch,
+                           scratch ? (size_t)GQA_ROPE_ATTN_NOALLOC_SCRATCH_BYTES : 0, stream);
+}
+
 extern "C" int gqa_rope_attn_get_device_status(void* stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GQA_ERR_CUDA;
   int v = 0;
@@ -321,6 +358,9 @@ extern "C" const char* gqa_rope_attn_strerror(int status) {
     case GQA_ERR_BAD_SEQLENS: return "cu_seqlens is not a valid prefix sum of total_tokens";
     case GQA_ERR_TIMEOUT: return "a bounded wait inside the kernel ran out";
     case GQA_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
+    case GQA_ERR_NOALLOC_LIMIT:
+      return "shape needs more scratch than the no-allocation entry point's built-in buffer "
+             "(GQA_ROPE_ATTN_NOALLOC_SCRATCH_BYTES)";
     default: return "unknown status";
   }
 }
