@@ -43,6 +43,30 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+KERNEL_SOURCES = ("attn_kernel.cuh", "prep_kernel.cuh", "common.cuh", "ptx.cuh", "rope_round.cuh",
+                  "exp2_poly.cuh", "gqa_rope_attn.cu")
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes (read + write) per launch of the attention kernel from the
+    committed ncu capture for this workload, or None when there is none or
+    when the kernel sources have changed since it was taken (the capture
+    records a SHA-256 over the sources)."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", f"gqa_attn_fwd_kernel.{workload}.traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "transformer_attention_gqa_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    if rec.get("sources_sha256") != h.hexdigest():
+        return None
+    return int(rec["dram_bytes_per_launch"])
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -285,7 +309,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "256 MiB written before every timed step, outside the step's events"},
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name),
                      "peak_source": f"{src} bf16_tflops (burst)", "kernel": "gqa_attn_fwd_kernel",
                      "kernel_ms": round(attn_ms, 4), "prologue_ms": round(prep_ms, 4)},
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
