@@ -8,8 +8,10 @@
 // are produced in tensor memory, turned into probabilities by an online
 // (running max / running sum) softmax and consumed by the P.V product.
 //
-// One persistent CTA per SM walks a static, longest-first list of work
-// items (sequence, q-tile, KV head). A q-tile packs tq = 128 / G tokens
+// One persistent CTA per SM takes work items (sequence, q-tile, KV head)
+// from a longest-first list: its first item statically, every further one
+// from a global counter (greedy list scheduling, so that faster CTAs take
+// more items), or, for short lists, from a static alternating deal. A q-tile packs tq = 128 / G tokens
 // times the G query heads of one KV head into 128 MMA rows, so every K/V
 // tile loaded by TMA is used by all G heads at once.
 //
@@ -41,6 +43,13 @@
 namespace gqa {
 
 
+// Work-item hand-off ring: the K producer takes item indices and publishes
+// them; every other role (V producer, S issuer, PV issuer: one thread each;
+// softmax warps: one arrival per warp; Q warps: their first thread, which
+// passes the index on with the tile's Q load) reads each slot once.
+constexpr int ITEM_SLOTS = 8;
+constexpr int ITEM_READERS = 3 + 4 + 1;
+
 constexpr int REG_PRODUCER = 56;
 constexpr int REG_SOFTMAX = 232;
 constexpr int REG_ROPE = 128;
@@ -53,6 +62,9 @@ struct Barriers {
   uint64_t s_full[NUM_S_BUF], p_full[NUM_S_BUF], pv_done[NUM_S_BUF];
   uint64_t o_free, drain;
   uint64_t stats_full, stats_empty;
+  uint64_t item_full[ITEM_SLOTS], item_empty[ITEM_SLOTS];
+  int item[ITEM_SLOTS];  // work-item index, -1 = no more items
+  int q_item[2];         // work item whose Q is in Q buffer 0 / 1 (-1: none left)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -167,6 +179,48 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
       return;
     }
   }
+}
+
+// Work item k of this CTA from the hand-off ring (-1: none left), read by one
+// thread (take_item) or by a whole warp (take_item_warp, one arrival).
+__device__ __forceinline__ bool take_item(Barriers* bars, int k, int& w, volatile int* abort_flag) {
+  const int slot = k & (ITEM_SLOTS - 1);
+  if (!bwait(ptx::smem_u32(&bars->item_full[slot]), (k / ITEM_SLOTS) & 1, abort_flag)) return false;
+  w = *reinterpret_cast<volatile int*>(&bars->item[slot]);
+  ptx::mbar_arrive(ptx::smem_u32(&bars->item_empty[slot]));
+  return true;
+}
+// Index of the CTA's k-th work item (k >= 1) in the longest-first list.
+// Dynamic: the next unclaimed item (greedy list scheduling; it adapts to
+// the actual duration of every item). Static, for lists of only a few items
+// per CTA, where a claim made two items ahead is too coarse: rounds of
+// gridDim.x items dealt in alternating direction (CTA b takes item b of even
+// rounds and gridDim.x - 1 - b of odd ones).
+__device__ __forceinline__ int next_item_index(const AttnParams& p, int k) {
+  const int G = (int)gridDim.x, b = (int)blockIdx.x;
+  if (p.sched_dynamic) return atomicAdd(p.item_counter, 1) + G;
+  return k * G + ((k & 1) ? G - 1 - b : b);
+}
+
+// Publishes work item k (index w, -1 = none left) once every reader has
+// taken item k - ITEM_SLOTS from the same slot.
+__device__ __forceinline__ bool publish_item(Barriers* bars, int k, int w, volatile int* abort_flag) {
+  const int slot = k & (ITEM_SLOTS - 1);
+  if (k >= ITEM_SLOTS &&
+      !bwait_lazy(ptx::smem_u32(&bars->item_empty[slot]), ((k / ITEM_SLOTS) - 1) & 1, abort_flag))
+    return false;
+  *reinterpret_cast<volatile int*>(&bars->item[slot]) = w;
+  ptx::mbar_arrive(ptx::smem_u32(&bars->item_full[slot]));
+  return true;
+}
+__device__ __forceinline__ bool take_item_warp(Barriers* bars, int k, int& w, volatile int* abort_flag) {
+  const int slot = k & (ITEM_SLOTS - 1);
+  if (!__all_sync(0xffffffffu, bwait(ptx::smem_u32(&bars->item_full[slot]), (k / ITEM_SLOTS) & 1, abort_flag)))
+    return false;
+  w = *reinterpret_cast<volatile int*>(&bars->item[slot]);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(ptx::smem_u32(&bars->item_empty[slot]));
+  return true;
 }
 
 // 2^x on the FMA pipe, for x <= 8: x = n + f with n = rint(x) (the 1.5*2^23
@@ -293,27 +347,40 @@ __device__ __forceinline__ float exp_pack(uint32_t* r, float bias, float scale, 
   return t.x + t.y;
 }
 
-// Rotates the Q tile of work item `wi` in shared memory (buffer it & 1) once
-// its TMA load has landed, then releases it to the S issuer. Run by the 128
-// threads of the Q-rotation/epilogue warpgroup.
+// Takes the CTA's it-th work item from the hand-off ring and rotates its Q
+// tile in shared memory (buffer it & 1) once the TMA load has landed, then
+// releases it to the S issuer. Run by the 128 threads of the
+// Q-rotation/epilogue warpgroup; thread 0 takes the item and loads Q, and
+// the item index reaches the others with the load's barrier. Returns false
+// on abort; w_out = the item's index, or -1 when no items are left.
 template <class C>
-__device__ __forceinline__ bool rope_q_tile(const AttnParams& p, const WorkItem& wi, uint8_t* smem, Barriers* bars,
-                                            const CUtensorMap* tmQ, int it, int tid, volatile int* abort_flag) {
+__device__ __forceinline__ bool rope_q_tile(const AttnParams& p, uint8_t* smem, Barriers* bars,
+                                            const CUtensorMap* tmQ, int it, int tid, volatile int* abort_flag,
+                                            int& w_out) {
   constexpr int D = C::D;
   constexpr int NCH = D / 16;  // 16-byte chunks in the first half of a row
   constexpr int HALF = D / 2;
   const int qb = it & 1;
   const int G = p.G;
   bool issued = false;
-  if (tid == 0) {  // the buffer's previous tile has finished its S MMAs: load this tile's Q
-    if (bwait(ptx::smem_u32(&bars->q_empty[qb]), ((it >> 1) & 1) ^ 1, abort_flag)) {
-      issued = true;
+  if (tid == 0) {
+    int w;
+    if (take_item(bars, it, w, abort_flag) &&
+        // the buffer's previous tile has finished its S MMAs: load this tile's Q
+        bwait(ptx::smem_u32(&bars->q_empty[qb]), ((it >> 1) & 1) ^ 1, abort_flag)) {
       const uint32_t bar = ptx::smem_u32(&bars->q_loaded[qb]);
-      ptx::mbar_arrive_expect_tx(bar, (uint32_t)(D * 2 * G * p.tq));
+      *reinterpret_cast<volatile int*>(&bars->q_item[qb]) = w;
+      if (w >= 0) {
+        issued = true;
+        const WorkItem wi = decode_item(p, w);
+        ptx::mbar_arrive_expect_tx(bar, (uint32_t)(D * 2 * G * p.tq));
 #pragma unroll
-      for (int b = 0; b < C::NBOX; ++b)
-        ptx::tma_load_3d(ptx::smem_u32(smem + qb * C::Q_BYTES + b * C::Q_BOX_BYTES), tmQ, bar, b * C::BOXC,
-                         wi.kvh * G, wi.seq_start + wi.t0);
+        for (int b = 0; b < C::NBOX; ++b)
+          ptx::tma_load_3d(ptx::smem_u32(smem + qb * C::Q_BYTES + b * C::Q_BOX_BYTES), tmQ, bar, b * C::BOXC,
+                           wi.kvh * G, wi.seq_start + wi.t0);
+      } else {
+        ptx::mbar_arrive(bar);
+      }
     }
   }
   const bool ok = __all_sync(0xffffffffu, bwait_lazy(ptx::smem_u32(&bars->q_loaded[qb]), (it >> 1) & 1, abort_flag));
@@ -321,6 +388,10 @@ __device__ __forceinline__ bool rope_q_tile(const AttnParams& p, const WorkItem&
     if (issued) drain_wait(ptx::smem_u32(&bars->q_loaded[qb]), (it >> 1) & 1);
     return false;
   }
+  const int w = *reinterpret_cast<volatile int*>(&bars->q_item[qb]);
+  w_out = w;
+  if (w < 0) return true;
+  const WorkItem wi = decode_item(p, w);
   uint8_t* qbuf = smem + qb * C::Q_BYTES;
   const int items = p.tq * NCH;
   for (int item = tid; item < items; item += 128) {
@@ -490,6 +561,10 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     ptx::mbar_init(B(bars->stats_full), 128);
     ptx::mbar_init(B(bars->stats_empty), 128);
     ptx::mbar_init(B(bars->drain), 2);  // one commit per MMA-issuing thread
+    for (int i = 0; i < ITEM_SLOTS; ++i) {
+      ptx::mbar_init(B(bars->item_full[i]), 1);
+      ptx::mbar_init(B(bars->item_empty[i]), ITEM_READERS);
+    }
     bars->abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -520,10 +595,20 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
    ptx::setmaxnreg_dec<REG_PRODUCER>();
    if (warp == 0) {
     // ------------------------------------------------------------ K producer
+    // Also the scheduler: when it starts the K loads of item k it publishes
+    // item k + 1 in ring slot (k + 1) % ITEM_SLOTS (so the Q warps can rotate
+    // that tile early) and asks the global counter for item k + 2, whose
+    // index is needed only one item later.
     if (lane == 0) {
       uint32_t g = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+      int w = (int)blockIdx.x < n_items ? (int)blockIdx.x : -1;  // first item of CTA b: item b
+      int nxt = w >= 0 ? next_item_index(p, 1) : n_items;
+      ok = publish_item(bars, 0, w, abort_flag);
+      for (int k = 0; ok && w >= 0; ++k) {
+        const int wn = nxt < n_items ? nxt : -1;
+        if (!(ok = publish_item(bars, k + 1, wn, abort_flag))) break;
+        if (wn >= 0) nxt = next_item_index(p, k + 2);
         const WorkItem wi = decode_item(p, w);
         for (int j = 0; j < wi.nkv; ++j, ++g) {
           const int ks = g % C::KST;
@@ -533,6 +618,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             ptx::tma_load_3d(sbase + C::OFF_K + ks * C::KV_BYTES + b * C::KV_BOX_BYTES, &tmK,
                              B(bars->k_full[ks]), b * C::BOXC, wi.seq_start + j * BN, wi.kvh);
         }
+        w = wn;
       }
       if (!ok) {  // let every copy already issued land before the CTA exits
         // loads issued: K tiles 0..g-1 (stage x % KST)
@@ -547,7 +633,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     if (lane == 0) {
       uint32_t g = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+      for (int k = 0; ok; ++k) {
+        int w;
+        if (!(ok = take_item(bars, k, w, abort_flag)) || w < 0) break;
         const WorkItem wi = decode_item(p, w);
         for (int j = 0; j < wi.nkv; ++j, ++g) {
           const int vs = g % C::VST;
@@ -580,7 +668,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       uint32_t gs = 0;
       int it = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
+      for (; ok; ++it) {
+        int w;
+        if (!(ok = take_item(bars, it, w, abort_flag)) || w < 0) break;
         const WorkItem wi = decode_item(p, w);
         const int qb = it & 1;
         if (!(ok = bwait(bar_qr0 + 8 * qb, (it >> 1) & 1, abort_flag))) break;
@@ -610,7 +700,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       uint32_t g = 0;
       int it = 0;
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
+      for (; ok; ++it) {
+        int w;
+        if (!(ok = take_item(bars, it, w, abort_flag)) || w < 0) break;
         const WorkItem wi = decode_item(p, w);
         for (int j = 0; j < wi.nkv; ++j, ++g) {
           const int b = g % NUM_S_BUF, vs = g % C::VST;
@@ -641,7 +733,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     int it = 0;
     bool ok = true;
     uint32_t sr[128];
-    for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
+    for (; ok; ++it) {
+      int w;
+      if (!(ok = take_item_warp(bars, it, w, abort_flag)) || w < 0) break;
       const WorkItem wi = decode_item(p, w);
       const int tok = wi.t0 + tok_off;  // index inside the sequence
       const int last_key = p.causal ? tok : wi.L - 1;
@@ -730,17 +824,18 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     // Order: rope(0); then for every tile t: rope(t + 1), epilogue(t). The
     // next tile's Q is rotated while tile t still runs; the epilogue of t
     // runs once its last P.V is done.
-    bool ok = true;
-    if (blockIdx.x < n_items) ok = rope_q_tile<C>(p, decode_item(p, blockIdx.x), smem, bars, &tmQ, 0, tid, abort_flag);
+    int w;
+    bool ok = rope_q_tile<C>(p, smem, bars, &tmQ, 0, tid, abort_flag, w);
     int it = 0;
     uint32_t g = 0;
-    for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++it) {
+    while (ok && w >= 0) {
+      int wn;
+      if (!(ok = rope_q_tile<C>(p, smem, bars, &tmQ, it + 1, tid, abort_flag, wn))) break;
       const WorkItem wi = decode_item(p, w);
-      if (w + (int)gridDim.x < n_items)
-        ok = rope_q_tile<C>(p, decode_item(p, w + gridDim.x), smem, bars, &tmQ, it + 1, tid, abort_flag);
-      if (!ok) break;
       ok = epilogue_tile<C, OUT_FP32>(p, wi, smem, bars, tmem, it, g, tid, abort_flag);
       g += wi.nkv;
+      w = wn;
+      ++it;
     }
   }
 

@@ -35,7 +35,7 @@ __host__ __device__ constexpr int tokens_per_tile(int G) { return BM / G; }
 
 // Workspace regions (byte offsets from the 256-byte aligned base).
 struct WsLayout {
-  size_t header;   // int[4]: number of (sequence, q-tile) pairs, ...
+  size_t header;   // int[16]: [0] number of (sequence, q-tile) pairs, [8] work-item counter
   size_t seq_pfx;  // int[num_seqs + 1]: first pair index of each sequence
   size_t pairs;    // int2[max_pairs]: (sequence, q-tile) in decreasing cost order
   size_t table;    // float2[N * d/2]: (cos, sin) of each token's angles
@@ -94,11 +94,13 @@ struct PrepParams {
 struct AttnParams {
   const int* cu;
   const int* header;
+  int* item_counter;    // work items taken so far beyond the first of each CTA (zeroed by the prologue)
   const int2* pairs;
   const float2* table;
   void* out;
   float* lse;
   int N, nq, nkv, G, tq, causal;
+  int sched_dynamic;    // 1: items beyond the first from item_counter; 0: static alternating deal
   float scale_log2;     // log2(e) / sqrt(d)
   float rescale_thr;    // raw-score growth that triggers an O rescale
 };

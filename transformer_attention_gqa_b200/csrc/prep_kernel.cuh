@@ -73,6 +73,7 @@ __device__ void build_schedule(const PrepParams& p) {
   const int tid = threadIdx.x;
   const int ns = p.num_seqs;
 
+  if (tid == 0) p.header[8] = 0;  // work-item counter of the attention kernel
   int bad = 0;
   for (int s = tid; s < ns; s += PREP_THREADS)
     if (__ldg(p.cu + s + 1) < __ldg(p.cu + s)) bad = 1;
