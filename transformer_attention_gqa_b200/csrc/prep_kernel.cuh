@@ -154,6 +154,30 @@ __device__ void rope_k_and_table(const PrepParams& p, int block, int nblocks) {
        idx += (long long)nblocks * PREP_THREADS) {
     const int t = (int)(idx / PAIRS);
     const int i = (int)(idx % PAIRS) * 2;
+    // K words of up to HB heads are loaded before the sincos, so that one
+    // memory latency covers them all.
+    constexpr int HB = 8;
+    uint32_t wl[HB], wh[HB];  // bf16 pairs (i, i + 1) and (i + d/2, i + d/2 + 1)
+    auto load_heads = [&](int h0) {
+#pragma unroll
+      for (int u = 0; u < HB; ++u) {
+        if (h0 + u >= p.nkv) break;
+        const size_t src = ((size_t)t * p.nkv + h0 + u) * D;
+        if constexpr (FP32_IN) {
+          // inputs are rounded to bf16 before anything else
+          const float2 a = *reinterpret_cast<const float2*>((const float*)p.k + src + i);
+          const float2 b = *reinterpret_cast<const float2*>((const float*)p.k + src + i + HALF);
+          const __nv_bfloat162 ra = __floats2bfloat162_rn(a.x, a.y), rb = __floats2bfloat162_rn(b.x, b.y);
+          wl[u] = *reinterpret_cast<const uint32_t*>(&ra);
+          wh[u] = *reinterpret_cast<const uint32_t*>(&rb);
+        } else {
+          wl[u] = *reinterpret_cast<const uint32_t*>((const __nv_bfloat16*)p.k + src + i);
+          wh[u] = *reinterpret_cast<const uint32_t*>((const __nv_bfloat16*)p.k + src + i + HALF);
+        }
+      }
+    };
+    load_heads(0);
+
     int pos;
     if (p.positions) {
       pos = __ldg(p.positions + t);
@@ -171,32 +195,24 @@ __device__ void rope_k_and_table(const PrepParams& p, int block, int nblocks) {
     }
     *reinterpret_cast<float4*>(p.table + (size_t)t * HALF + i) = make_float4(c[0], sn[0], c[1], sn[1]);
 
-    for (int h = 0; h < p.nkv; ++h) {
-      const size_t src = ((size_t)t * p.nkv + h) * D;
-      float xl[2], xh[2];
-      if constexpr (FP32_IN) {
-        const float2 a = *reinterpret_cast<const float2*>((const float*)p.k + src + i);
-        const float2 b = *reinterpret_cast<const float2*>((const float*)p.k + src + i + HALF);
-        // inputs are rounded to bf16 before anything else
-        xl[0] = __bfloat162float(__float2bfloat16_rn(a.x));
-        xl[1] = __bfloat162float(__float2bfloat16_rn(a.y));
-        xh[0] = __bfloat162float(__float2bfloat16_rn(b.x));
-        xh[1] = __bfloat162float(__float2bfloat16_rn(b.y));
-      } else {
-        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>((const __nv_bfloat16*)p.k + src + i);
-        const __nv_bfloat162 b =
-            *reinterpret_cast<const __nv_bfloat162*>((const __nv_bfloat16*)p.k + src + i + HALF);
-        xl[0] = __low2float(a);
-        xl[1] = __high2float(a);
-        xh[0] = __low2float(b);
-        xh[1] = __high2float(b);
-      }
-      __nv_bfloat16 ol[2], oh[2];
+    for (int h0 = 0; h0 < p.nkv; h0 += HB) {
+      if (h0 > 0) load_heads(h0);
 #pragma unroll
-      for (int e = 0; e < 2; ++e) rope_pair(xl[e], xh[e], c[e], sn[e], ol[e], oh[e]);
-      const size_t dst = ((size_t)h * p.N + t) * D;
-      *reinterpret_cast<__nv_bfloat162*>(p.kws + dst + i) = __halves2bfloat162(ol[0], ol[1]);
-      *reinterpret_cast<__nv_bfloat162*>(p.kws + dst + i + HALF) = __halves2bfloat162(oh[0], oh[1]);
+      for (int u = 0; u < HB; ++u) {
+        if (h0 + u >= p.nkv) break;
+        uint32_t ol[2], oh[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          __nv_bfloat16 lo, hi;
+          rope_pair(__uint_as_float(((wl[u] >> (16 * e)) & 0xFFFFu) << 16),
+                    __uint_as_float(((wh[u] >> (16 * e)) & 0xFFFFu) << 16), c[e], sn[e], lo, hi);
+          ol[e] = __bfloat16_as_ushort(lo);
+          oh[e] = __bfloat16_as_ushort(hi);
+        }
+        const size_t dst = ((size_t)(h0 + u) * p.N + t) * D;
+        *reinterpret_cast<uint32_t*>(p.kws + dst + i) = ol[0] | (ol[1] << 16);
+        *reinterpret_cast<uint32_t*>(p.kws + dst + i + HALF) = oh[0] | (oh[1] << 16);
+      }
     }
 
     if constexpr (FP32_IN) {
