@@ -67,17 +67,43 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_buf, int& tota
   return excl;
 }
 
+// largest s in [0, n) with a[s] <= x (a nondecreasing, a[0] <= x); plain
+// loads, for arrays this block has written (shared or global memory).
+__device__ __forceinline__ int upper_index_plain(const int* a, int n, int x) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Up to this many sequences, cu_seqlens and the per-sequence pair offsets are
+// kept in shared memory while the schedule is built (beyond: global memory).
+constexpr int SCHED_SMEM_SEQS = 2048;
+
 __device__ void build_schedule(const PrepParams& p) {
   __shared__ int s_scan[PREP_THREADS];
   __shared__ int s_bins[SCHED_BINS];
+  __shared__ int s_cu[SCHED_SMEM_SEQS + 1];
+  __shared__ int s_pfx[SCHED_SMEM_SEQS + 1];
   const int tid = threadIdx.x;
   const int ns = p.num_seqs;
 
+  const int* cu = p.cu;
+  int* pfx = p.seq_pfx;
+  if (ns <= SCHED_SMEM_SEQS) {
+    for (int i = tid; i <= ns; i += PREP_THREADS) s_cu[i] = __ldg(p.cu + i);
+    cu = s_cu;
+    pfx = s_pfx;
+  }
   if (tid == 0) p.header[8] = 0;  // work-item counter of the attention kernel
+  __syncthreads();
+
   int bad = 0;
   for (int s = tid; s < ns; s += PREP_THREADS)
-    if (__ldg(p.cu + s + 1) < __ldg(p.cu + s)) bad = 1;
-  if (tid == 0 && (__ldg(p.cu) != 0 || __ldg(p.cu + ns) != p.N)) bad = 1;
+    if (cu[s + 1] < cu[s]) bad = 1;
+  if (tid == 0 && (cu[0] != 0 || cu[ns] != p.N)) bad = 1;
   if (__syncthreads_or(bad)) {
     if (tid == 0) {
       set_status(kStatusBadSeqlens);
@@ -91,22 +117,22 @@ __device__ void build_schedule(const PrepParams& p) {
   for (int base = 0; base < ns; base += PREP_THREADS) {
     const int s = base + tid;
     int nt = 0;
-    if (s < ns) nt = (__ldg(p.cu + s + 1) - __ldg(p.cu + s) + p.tq - 1) / p.tq;
+    if (s < ns) nt = (cu[s + 1] - cu[s] + p.tq - 1) / p.tq;
     int tot;
     const int ex = block_exclusive_scan(nt, s_scan, tot);
-    if (s < ns) p.seq_pfx[s] = running + ex;
+    if (s < ns) pfx[s] = running + ex;
     running += tot;
   }
-  if (tid == 0) p.seq_pfx[ns] = running;
+  if (tid == 0) pfx[ns] = running;
   const int P = running;
 
   for (int i = tid; i < SCHED_BINS; i += PREP_THREADS) s_bins[i] = 0;
-  __syncthreads();  // seq_pfx (global) and s_bins visible to the whole block
+  __syncthreads();  // pfx and s_bins visible to the whole block
 
   for (int q = tid; q < P; q += PREP_THREADS) {
-    const int s = upper_index(p.seq_pfx, ns, q);
-    const int l = q - p.seq_pfx[s];
-    const int L = __ldg(p.cu + s + 1) - __ldg(p.cu + s);
+    const int s = upper_index_plain(pfx, ns, q);
+    const int l = q - pfx[s];
+    const int L = cu[s + 1] - cu[s];
     const int c = min(tile_cost(L, l, p.tq, p.causal), SCHED_BINS - 1);
     atomicAdd(&s_bins[c], 1);
   }
@@ -131,9 +157,9 @@ __device__ void build_schedule(const PrepParams& p) {
   __syncthreads();
 
   for (int q = tid; q < P; q += PREP_THREADS) {
-    const int s = upper_index(p.seq_pfx, ns, q);
-    const int l = q - p.seq_pfx[s];
-    const int L = __ldg(p.cu + s + 1) - __ldg(p.cu + s);
+    const int s = upper_index_plain(pfx, ns, q);
+    const int l = q - pfx[s];
+    const int L = cu[s + 1] - cu[s];
     const int c = min(tile_cost(L, l, p.tq, p.causal), SCHED_BINS - 1);
     const int slot = atomicAdd(&s_bins[c], 1);
     p.pairs[slot] = make_int2(s, l);
