@@ -15,20 +15,24 @@
 // times the G query heads of one KV head into 128 MMA rows, so every K/V
 // tile loaded by TMA is used by all G heads at once.
 //
-// Warp roles (384 threads):
-//   warp 0      TMA producer: K tiles (K is RoPE'd already)
+// Warp roles (512 threads):
+//   warp 0      TMA producer: K tiles (K is RoPE'd already); work items
 //   warp 1      TMEM allocator; one thread issues the S = Q K^T MMAs
 //   warp 2      TMA producer: V tiles
 //   warp 3      one thread issues the O += P V MMAs
-//   warps 4-7   softmax: one thread per row (TMEM lane), S -> P, running
-//               max/sum, O rescale, epilogue (O / l, LSE)
-//   warps 8-11  Q tiles: TMA load, RoPE applied in shared memory before the
-//               first S MMA reads it; epilogue: O / l from TMEM, TMA store,
-//               LSE
+//   warps 4-11  softmax: a row (TMEM lane) is shared by two threads, warps
+//               4-7 take its columns [0, 64) and warps 8-11 columns
+//               [64, 128); S -> P, running max (exchanged once per tile)
+//               and partial sums, O rescale of their half of O's columns
+//   warps 12-15 Q tiles: TMA load, RoPE applied in shared memory before the
+//               first S MMA reads it; epilogue: O / l from TMEM, LSE
+// Two softmax warps per SM sub-partition keep the special-function unit
+// busy while either one waits on its in-order instruction stream.
 //
 // Tensor memory (512 columns x 128 lanes of 32 bit):
-//   [0,128) [128,256) [256,384): three S buffers; the bf16 P of a tile
-//   overwrites the first 64 columns of its own S buffer; [384, 384+d): O.
+//   [0,128) [128,256) [256,384): three S buffers; the bf16 P of each column
+//   half overwrites the first 32 columns of that half's S columns (keys
+//   [0, 64) at +0, keys [64, 128) at +64); [384, 384+d): O.
 // MMAs: S = Q K^T   kind::f16, A = Q (smem, K-major), B = K (smem, K-major),
 //                   M = 128, N = 128, fp32 accumulate, d/16 steps;
 //       O += P V    A = P (tmem), B = V (smem, MN-major), M = 128, N = d,
@@ -48,12 +52,14 @@ namespace gqa {
 // softmax warps: one arrival per warp; Q warps: their first thread, which
 // passes the index on with the tile's Q load) reads each slot once.
 constexpr int ITEM_SLOTS = 8;
-constexpr int ITEM_READERS = 3 + 4 + 1;
+constexpr int ITEM_READERS = 3 + 8 + 1;
 
+// Register split (launch: 512 threads x 128): producers/MMA 56, softmax 160
+// (8 warps), Q rotation/epilogue 128 (the launch value).
 constexpr int REG_PRODUCER = 56;
-constexpr int REG_SOFTMAX = 232;
+constexpr int REG_SOFTMAX = 160;
 constexpr int REG_ROPE = 128;
-static_assert((REG_PRODUCER + REG_SOFTMAX + REG_ROPE) * 128 <= 65536 / ATTN_THREADS * ATTN_THREADS,
+static_assert(REG_PRODUCER * 128 + REG_SOFTMAX * 256 + REG_ROPE * 128 <= 65536 / ATTN_THREADS * ATTN_THREADS,
               "register split exceeds the launch's register file share");
 
 struct Barriers {
@@ -62,6 +68,7 @@ struct Barriers {
   uint64_t s_full[NUM_S_BUF], p_full[NUM_S_BUF], pv_done[NUM_S_BUF];
   uint64_t o_free, drain;
   uint64_t stats_full, stats_empty;
+  uint64_t xchg[2][4];  // row-max exchange of the two softmax halves: [tile parity][lane quadrant]
   uint64_t item_full[ITEM_SLOTS], item_empty[ITEM_SLOTS];
   int item[ITEM_SLOTS];  // work-item index, -1 = no more items
   int q_item[2];         // work item whose Q is in Q buffer 0 / 1 (-1: none left)
@@ -86,9 +93,10 @@ struct AttnCfg {
   static constexpr int VST = KST;
   static constexpr int OFF_K = 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr int OFF_STATS = OFF_V + VST * KV_BYTES;  // float2 (m, l) per row, softmax -> epilogue
-  static constexpr int OFF_BAR = OFF_STATS + BM * 8;
-  static constexpr int BAR_BYTES = 512;
+  static constexpr int OFF_STATS = OFF_V + VST * KV_BYTES;  // float2 (m, l_half) [2][BM], softmax -> epilogue
+  static constexpr int OFF_XMAX = OFF_STATS + 2 * BM * 8;   // float [2 parities][2 halves][BM]: row max exchange
+  static constexpr int OFF_BAR = OFF_XMAX + 4 * BM * 4;
+  static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t O_COL = 384;
@@ -239,10 +247,11 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
-// Two fp32 -> one bf16x2 word (lo in the low half), rounded to nearest (ties
-// away from zero), with integer ops instead of the conversion unit.
+// Two fp32 -> one bf16x2 word (lo in the low half), rounded to nearest even:
+// one cvt.rn.bf16x2.f32 (measured faster than packing with integer ops).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&b);
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -251,11 +260,12 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// Of every EMU_PERIOD exponent pairs of a row, one is evaluated on the FMA
-// pipe, the rest on the special-function unit (0: all on the SFU; measured
-// fastest while the softmax is latency-bound rather than SFU-bound).
+// Of every EMU_PERIOD groups of 4 exponentials of a row, one is evaluated on
+// the FMA pipe, the rest on the special-function unit (0: all on the SFU).
+// With two softmax warps per sub-partition the SFU is the limit; 1 in 8
+// measured fastest (1 in 4 and more run out of issue slots).
 #ifndef GQA_EMU_PERIOD
-#define GQA_EMU_PERIOD 0
+#define GQA_EMU_PERIOD 8
 #endif
 constexpr int EMU_PERIOD = GQA_EMU_PERIOD;
 
@@ -287,39 +297,43 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
-// ---- softmax row helpers (one thread = one row of the S tile) ----
+// ---- softmax helpers (one thread = NC columns of one row of the S tile) ----
 
-// All BN columns of the row from TMEM into r[] (fp32 bit patterns).
-__device__ __forceinline__ void load_s_row(uint32_t taddr, uint32_t* r) {
+// NC columns of the row from TMEM into r[] (fp32 bit patterns).
+template <int NC>
+__device__ __forceinline__ void load_s_cols(uint32_t taddr, uint32_t* r) {
 #pragma unroll
-  for (int c = 0; c < BN / 32; ++c) ptx::tmem_ld32(taddr + c * 32, r + c * 32);
+  for (int c = 0; c < NC / 32; ++c) ptx::tmem_ld32(taddr + c * 32, r + c * 32);
   ptx::tmem_wait_ld();
 #pragma unroll
-  for (int c = 0; c < BN / 32; ++c) ptx::reg_fence32(r + c * 32);
+  for (int c = 0; c < NC / 32; ++c) ptx::reg_fence32(r + c * 32);
 }
 
 // Columns > lim get -inf (causal diagonal tile, or keys past the sequence).
-__device__ __forceinline__ void mask_row(uint32_t* r, int lim) {
+template <int NC>
+__device__ __forceinline__ void mask_cols(uint32_t* r, int lim) {
 #pragma unroll
-  for (int c = 0; c < BN; ++c)
+  for (int c = 0; c < NC; ++c)
     if (c > lim) r[c] = __float_as_uint(-INFINITY);
 }
 
-// Row max: 8 independent chains of 3-input max, then a tree.
-__device__ __forceinline__ float row_max(const uint32_t* r) {
+// Max of the NC values: 8 independent chains of 3-input max, then a tree.
+template <int NC>
+__device__ __forceinline__ float cols_max(const uint32_t* r) {
   float mx8[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(__uint_as_float(r[e]), __uint_as_float(r[e + 8]));
 #pragma unroll
-  for (int c = 16; c < BN; c += 16)
+  for (int c = 16; c < NC; c += 16)
 #pragma unroll
     for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], __uint_as_float(r[c + e]), __uint_as_float(r[c + 8 + e]));
   return fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
 }
 
-// p = 2^(s * scale + bias) for the row, packed in place to bf16 pairs
-// (r[c/2], c = 0..BN-1). Returns the fp32 sum of p; if mx_out is given, also
-// the row max of s.
+// p = 2^(s * scale + bias) for the NC values, packed in place to bf16 pairs
+// (r[c/2], c = 0..NC-1). Returns the fp32 sum of p; if mx_out is given, also
+// the max of s.
+template <int NC>
 __device__ __forceinline__ float exp_pack(uint32_t* r, float bias, float scale, float* mx_out) {
   float2 ls[4];
 #pragma unroll
@@ -327,24 +341,58 @@ __device__ __forceinline__ float exp_pack(uint32_t* r, float bias, float scale, 
   float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   const float2 sc2 = make_float2(scale, scale), bi2 = make_float2(bias, bias);
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-#pragma unroll
-    for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 4) {
-      const float2 s01 = make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1]));
-      const float2 s23 = make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
-      if (mx_out) mx4[(c >> 2) & 3] = fmax3(mx4[(c >> 2) & 3], fmaxf(s01.x, s01.y), fmaxf(s23.x, s23.y));
-      const float2 x01 = ffma2(s01, sc2, bi2);
-      const float2 x23 = ffma2(s23, sc2, bi2);
-      const float2 p01 = make_float2(ptx::ex2(x01.x), ptx::ex2(x01.y));
-      const float2 p23 = make_float2(ptx::ex2(x23.x), ptx::ex2(x23.y));
-      ls[(c >> 2) & 3] = fadd2(ls[(c >> 2) & 3], fadd2(p01, p23));
-      r[c >> 1] = pack_bf16x2(p01.x, p01.y);
-      r[(c >> 1) + 1] = pack_bf16x2(p23.x, p23.y);
+  for (int c = 0; c < NC; c += 4) {
+    const float2 s01 = make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+    const float2 s23 = make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+    if (mx_out) mx4[(c >> 2) & 3] = fmax3(mx4[(c >> 2) & 3], fmaxf(s01.x, s01.y), fmaxf(s23.x, s23.y));
+    const float2 x01 = ffma2(s01, sc2, bi2);
+    const float2 x23 = ffma2(s23, sc2, bi2);
+    float2 p01, p23;
+    if (EMU_PERIOD > 0 && ((c >> 2) % (EMU_PERIOD > 0 ? EMU_PERIOD : 1)) == EMU_PERIOD - 1) {
+      p01 = make_float2(exp2_fma(x01.x), exp2_fma(x01.y));
+      p23 = make_float2(exp2_fma(x23.x), exp2_fma(x23.y));
+    } else {
+      p01 = make_float2(ptx::ex2(x01.x), ptx::ex2(x01.y));
+      p23 = make_float2(ptx::ex2(x23.x), ptx::ex2(x23.y));
     }
+    ls[(c >> 2) & 3] = fadd2(ls[(c >> 2) & 3], fadd2(p01, p23));
+    r[c >> 1] = pack_bf16x2(p01.x, p01.y);
+    r[(c >> 1) + 1] = pack_bf16x2(p23.x, p23.y);
   }
   if (mx_out) *mx_out = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
   const float2 t = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
   return t.x + t.y;
+}
+
+// The NC/2 packed P words into TMEM.
+template <int NC>
+__device__ __forceinline__ void store_p(uint32_t taddr, const uint32_t* r) {
+  static_assert(NC == 64, "one 32-column store per half row");
+  ptx::tmem_st32(taddr, r);
+}
+
+// Multiplies NCOL columns of O (this thread's row) by alpha.
+template <int NCOL>
+__device__ __forceinline__ void scale_o_cols(uint32_t taddr, float alpha, uint32_t* o) {
+  if constexpr (NCOL >= 32) {
+#pragma unroll
+    for (int c = 0; c < NCOL / 32; ++c) {
+      ptx::tmem_ld32(taddr + c * 32, o);
+      ptx::tmem_wait_ld();
+      ptx::reg_fence32(o);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+      ptx::tmem_st32(taddr + c * 32, o);
+    }
+  } else {
+    static_assert(NCOL == 16, "O half widths are 64, 32 or 16 columns");
+    ptx::tmem_ld16(taddr, o);
+    ptx::tmem_wait_ld();
+    ptx::reg_fence16(o);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+    ptx::tmem_st16(taddr, o);
+  }
 }
 
 // Takes the CTA's it-th work item from the hand-off ring and rotates its Q
@@ -454,7 +502,9 @@ __device__ __forceinline__ bool epilogue_tile(const AttnParams& p, const WorkIte
   const bool row_valid = r < p.tq * G && tok < wi.L;
   bool ok = __all_sync(0xffffffffu, bwait(ptx::smem_u32(&bars->stats_full), it & 1, abort_flag));
   if (!ok) return false;
-  const float2 ml = reinterpret_cast<const float2*>(smem + C::OFF_STATS)[r];
+  const float2 ml0 = reinterpret_cast<const float2*>(smem + C::OFF_STATS)[r];
+  const float2 ml1 = reinterpret_cast<const float2*>(smem + C::OFF_STATS)[BM + r];
+  const float2 ml = make_float2(ml0.x, ml0.y + ml1.y);  // both halves hold the same running max
   ptx::mbar_arrive(ptx::smem_u32(&bars->stats_empty));
   const uint32_t gl = g + wi.nkv - 1;
   ok = __all_sync(0xffffffffu,
@@ -514,13 +564,14 @@ __device__ __forceinline__ void issue_s_mmas(uint32_t d_tmem, uint64_t dq, uint6
   }
 }
 
-// O (+)= P V for one KV tile: 8 K-steps of 16 keys, P from TMEM, V MN-major.
+// O (+)= P V for one KV tile: 8 K-steps of 16 keys, P from TMEM (keys
+// [0, 64) at S buffer column 0, keys [64, 128) at column 64), V MN-major.
 template <class C>
 __device__ __forceinline__ void issue_pv_mmas(uint32_t o_tmem, uint32_t p_tmem, uint64_t dv, bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < C::KSTEPS_PV; ++kk)
-    ptx::mma_ts(o_tmem, p_tmem + kk * 8, dv + (uint64_t)((kk * 16 * C::ROWB) >> 4), C::IDESC_O,
-                (accumulate || kk > 0) ? 1u : 0u);
+    ptx::mma_ts(o_tmem, p_tmem + (kk >> 2) * 64 + (kk & 3) * 8, dv + (uint64_t)((kk * 16 * C::ROWB) >> 4),
+                C::IDESC_O, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D, bool OUT_FP32>
@@ -554,13 +605,15 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     }
     for (int i = 0; i < NUM_S_BUF; ++i) {
       ptx::mbar_init(B(bars->s_full[i]), 1);
-      ptx::mbar_init(B(bars->p_full[i]), 128);
+      ptx::mbar_init(B(bars->p_full[i]), 256);
       ptx::mbar_init(B(bars->pv_done[i]), 1);
     }
     ptx::mbar_init(B(bars->o_free), 128);
-    ptx::mbar_init(B(bars->stats_full), 128);
+    ptx::mbar_init(B(bars->stats_full), 256);
     ptx::mbar_init(B(bars->stats_empty), 128);
     ptx::mbar_init(B(bars->drain), 2);  // one commit per MMA-issuing thread
+    for (int i = 0; i < 2; ++i)
+      for (int qd = 0; qd < 4; ++qd) ptx::mbar_init(B(bars->xchg[i][qd]), 64);
     for (int i = 0; i < ITEM_SLOTS; ++i) {
       ptx::mbar_init(B(bars->item_full[i]), 1);
       ptx::mbar_init(B(bars->item_empty[i]), ITEM_READERS);
@@ -589,8 +642,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   ptx::griddep_wait();
   const int n_items = ptx::ld_cg_s32(p.header) * p.nkv;
 
-  // Register split (launch: 384 threads x 168): producers/MMA 56, softmax
-  // 232, Q rotation 128 -> (56 + 232 + 128) x 128 = 53248 <= 64512.
+  // Register split (launch: 512 threads x 128): producers/MMA 56, softmax
+  // 160, Q rotation 128 -> 56 x 128 + 160 x 256 + 128 x 128 = 64512 <= 65536.
   if (warp < 4) {
    ptx::setmaxnreg_dec<REG_PRODUCER>();
    if (warp == 0) {
@@ -719,20 +772,23 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       drain_wait(B(bars->drain), 0);
     }
    }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     ptx::setmaxnreg_inc<REG_SOFTMAX>();
     // ------------------------------------------------------------ softmax
+    constexpr int NC = BN / 2;           // columns per thread
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;  // row of the tile == TMEM lane
-    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const int half = (warp - 4) >> 2;    // 0: columns [0, 64), 1: [64, 128)
+    const int r = quad * 32 + lane;      // row of the tile == TMEM lane
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16) + half * NC;
     const int G = p.G;
     const int tok_off = r / G;
     const float sl2 = p.scale_log2;
-    float2* stats = reinterpret_cast<float2*>(smem + C::OFF_STATS);
+    float2* stats = reinterpret_cast<float2*>(smem + C::OFF_STATS) + half * BM;
+    float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);  // [parity][half][BM]
     uint32_t g = 0;
     int it = 0;
     bool ok = true;
-    uint32_t sr[128];
+    uint32_t sr[NC];
     for (; ok; ++it) {
       int w;
       if (!(ok = take_item_warp(bars, it, w, abort_flag)) || w < 0) break;
@@ -748,55 +804,67 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         ok = __all_sync(0xffffffffu, bwait(B(bars->s_full[b]), (gg / NUM_S_BUF) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
-        load_s_row(tS, sr);
-        const int lim = last_key - j * BN;  // columns > lim are masked
-        if (lim < BN - 1) mask_row(sr, lim);
+        load_s_cols<NC>(tS, sr);
+        const int lim = last_key - j * BN - half * NC;  // this half's columns > lim are masked
+        if (lim < NC - 1) mask_cols<NC>(sr, lim);
+        // Both halves publish their max, then read the other's (mbarrier of
+        // 64 arrivals per lane quadrant, alternating by tile parity).
+        const int xp = gg & 1;
+        float* xm_mine = xmax + (xp * 2 + half) * BM + r;
+        const float* xm_other = xmax + (xp * 2 + (half ^ 1)) * BM + r;
+        const uint32_t xbar = B(bars->xchg[xp][quad]);
+        const uint32_t xpar = (gg >> 1) & 1;
         float alpha = 1.f;
-        bool need = false;
         float lsum;
         if (j == 0) {
-          m = row_max(sr);
-          lsum = exp_pack(sr, -m * sl2, sl2, nullptr);
+          const float mh = cols_max<NC>(sr);
+          *xm_mine = mh;
+          ptx::mbar_arrive(xbar);
+          ok = __all_sync(0xffffffffu, bwait(xbar, xpar, abort_flag));
+          if (!ok) break;
+          m = fmaxf(mh, *xm_other);
+          lsum = exp_pack<NC>(sr, -m * sl2, sl2, nullptr);
         } else {
-          // Exponentials with the running max m, the tile's row max alongside;
-          // if it exceeds m by more than the threshold (2^8 in p) the tile is
-          // redone below with the new max.
-          float mx;
-          lsum = exp_pack(sr, -m * sl2, sl2, &mx);
+          // Exponentials with the running max m, the tile's max alongside;
+          // if the row's max exceeds m by more than the threshold (2^8 in p)
+          // the tile is redone below with the new max.
+          float mh;
+          lsum = exp_pack<NC>(sr, -m * sl2, sl2, &mh);
+          *xm_mine = mh;
+          ptx::mbar_arrive(xbar);
+          ok = __all_sync(0xffffffffu, bwait(xbar, xpar, abort_flag));
+          if (!ok) break;
+          const float mx = fmaxf(mh, *xm_other);
+          bool need = false;
           if (mx > m + p.rescale_thr) {
             alpha = ptx::ex2((m - mx) * sl2);
             m = mx;
             need = true;
           }
+          // Both halves see the same maxima, so they take this branch together.
           if (__any_sync(0xffffffffu, need)) {
-            load_s_row(tS, sr);  // S is intact: P has not been stored yet
-            if (lim < BN - 1) mask_row(sr, lim);
-            lsum = exp_pack(sr, -m * sl2, sl2, nullptr);
-            // O holds the sum up to the previous tile: wait for PV(gg-1), then scale.
+            load_s_cols<NC>(tS, sr);  // S is intact: P has not been stored yet
+            if (lim < NC - 1) mask_cols<NC>(sr, lim);
+            lsum = exp_pack<NC>(sr, -m * sl2, sl2, nullptr);
+            // O holds the sum up to the previous tile: wait for PV(gg-1), then
+            // scale this half's share of O's columns.
             const uint32_t gp = gg - 1;
             ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[gp % NUM_S_BUF]), (gp / NUM_S_BUF) & 1, abort_flag));
             if (!ok) break;
             ptx::tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t* o = sr + 64;
-              ptx::tmem_ld32(trow + C::O_COL + c * 32, o);
-              ptx::tmem_wait_ld();
-              ptx::reg_fence32(o);
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              ptx::tmem_st32(trow + C::O_COL + c * 32, o);
-            }
+            // (sr[0, NC/2) holds the packed P; the upper half is free scratch)
+            scale_o_cols<D / 2>(tmem + ((uint32_t)(quad * 32) << 16) + C::O_COL + half * (D / 2), alpha,
+                                sr + NC / 2);
           }
         }
         l = l * alpha + lsum;
-        store_p_row(tS, sr);
+        store_p<NC>(tS, sr);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(B(bars->p_full[b]));
       }
       if (!ok) break;
-      // ---- hand (m, l) of every row to the epilogue warps
+      // ---- hand (m, this half's l) of every row to the epilogue warps
       ok = __all_sync(0xffffffffu, bwait(B(bars->stats_empty), (it & 1) ^ 1, abort_flag));
       if (!ok) break;
       stats[r] = make_float2(m, l);
@@ -804,9 +872,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       g += wi.nkv;
     }
   } else {
-    ptx::setmaxnreg_dec<REG_ROPE>();
+    // (runs with the launch's REG_ROPE registers)
     // ------------------------------------------------------------ Q rotation + epilogue
-    const int tid = threadIdx.x - 256;
+    const int tid = threadIdx.x - 384;
     const int rows = p.tq * p.G;
     // padding rows (never written by TMA) are zero in both Q buffers
     for (int i = tid; i < 2 * C::NBOX * (BM - rows) * (C::ROWB / 16); i += 128) {

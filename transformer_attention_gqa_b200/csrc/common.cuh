@@ -15,7 +15,7 @@ namespace gqa {
 constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int NUM_S_BUF = 3;        // S/P buffers in tensor memory
-constexpr int ATTN_THREADS = 384;   // 12 warps, roles below
+constexpr int ATTN_THREADS = 512;   // 16 warps (roles: attention kernel)
 constexpr int PREP_THREADS = 256;
 constexpr int SCHED_BINS = 2048;    // cost histogram bins of the tile scheduler
 constexpr unsigned long long WAIT_TIMEOUT_NS = 2000000000ull;  // bounded waits: 2 s
