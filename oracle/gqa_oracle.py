@@ -43,6 +43,14 @@ page builds (here: the float64 cos/sin of the float64 angle, rounded once to
 fp32), evaluates x*cos - y*sin in float64 and rounds that once to bf16 (round
 to nearest, ties to even). With ``operand_rounding=False`` the rotation is
 exact float64 and nothing is rounded; the RoPE pins use that form.
+
+Decoding (``gqa_rope_decode``): one new token per sequence against a cache of
+the keys and values of every earlier token ("Attention from Scratch", section
+"Attention, the math: Grouped-Query Attention with RoPE'd Q/K", the paragraph
+on why GQA shrinks the KV cache: one K and one V vector per token and KV head
+is kept for every token generated so far). The new token is the last row of
+the causal mask, so the step is the forward's last row; the cache holds the
+keys after rotation, each at its own position.
 """
 from __future__ import annotations
 
@@ -64,6 +72,7 @@ __all__ = [
     "gather",
     "gqa_rope_attention",
     "brute_force_attention",
+    "gqa_rope_decode",
 ]
 
 
@@ -312,3 +321,56 @@ def brute_force_attention(q, k, v, cu_seqlens, n_q_heads: int, n_kv_heads: int, 
                     out[i][h][t] = sum(ex[n] * v[js[n], g, t] for n in range(len(js))) / z
                 lse[h][i] = mx + math.log(z)
     return np.array(out, dtype=np.float64).reshape(N, hq, d), np.array(lse, dtype=np.float64).reshape(hq, N)
+
+
+def gqa_rope_decode(q, k_new, v_new, k_cache, v_cache, cache_seqlens, n_q_heads: int, n_kv_heads: int,
+                    rope_theta: float, operand_rounding: bool = True):
+    """One decoding step for a batch of sequences.
+
+    q: [B, n_q, d] queries of each sequence's new token; k_new, v_new:
+    [B, n_kv, d] its key (not rotated yet) and value; k_cache, v_cache:
+    [B, max_len, n_kv, d] with rows 0..p-1 holding the rotated keys and the
+    values of the earlier tokens of sequence b, p = cache_seqlens[b] (rows
+    from p on are not read). The new token sits at position p: its key is
+    rotated at p and becomes cache row p, its value too, and its rotated
+    query attends to keys 0..p (step 5's causal row of the last token).
+
+    Returns (out [B, n_q, d], lse [n_q, B], k_row [B, n_kv, d],
+    v_row [B, n_kv, d]); k_row / v_row are the rows the step appends.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k_new = np.asarray(k_new, dtype=np.float64)
+    v_new = np.asarray(v_new, dtype=np.float64)
+    k_cache = np.asarray(k_cache, dtype=np.float64)
+    v_cache = np.asarray(v_cache, dtype=np.float64)
+    B, hq, d = q.shape
+    if hq != n_q_heads or n_q_heads % n_kv_heads:
+        raise ValueError("bad head counts")
+    if k_new.shape != (B, n_kv_heads, d) or v_new.shape != (B, n_kv_heads, d):
+        raise ValueError("shape mismatch")
+    if k_cache.shape[0] != B or k_cache.shape[2:] != (n_kv_heads, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape mismatch")
+    lens = np.asarray(cache_seqlens, dtype=np.int64).reshape(-1)
+    if lens.shape != (B,) or np.any(lens < 0) or np.any(lens >= k_cache.shape[1]):
+        raise ValueError("bad cache_seqlens")
+    G = n_q_heads // n_kv_heads
+    out = np.empty((B, n_q_heads, d))
+    lse = np.empty((n_q_heads, B))
+    k_row = np.empty((B, n_kv_heads, d))
+    for b in range(B):
+        p = int(lens[b])
+        # 2. Rotate the new token's query and key at its position p.
+        qr = apply_rope(q[b][None], [p], rope_theta, operand_rounding)[0]      # [n_q, d]
+        kr = apply_rope(k_new[b][None], [p], rope_theta, operand_rounding)[0]  # [n_kv, d]
+        k_row[b] = kr
+        keys = np.concatenate([k_cache[b, :p], kr[None]], axis=0)              # [p+1, n_kv, d]
+        vals = np.concatenate([v_cache[b, :p], v_new[b][None]], axis=0)
+        # 3. Share each KV head across its group; head-major views.
+        kh = np.transpose(share_kv_heads(keys, G, axis=1), (1, 0, 2))          # [n_q, p+1, d]
+        vh = np.transpose(share_kv_heads(vals, G, axis=1), (1, 0, 2))
+        qh = qr[:, None, :]                                                     # [n_q, 1, d]
+        # 4.-6. Score, softmax over the p + 1 visible keys, gather.
+        w, row_lse = softmax_with_lse(score(qh, kh))
+        out[b] = gather(w, vh)[:, 0, :]
+        lse[:, b] = row_lse[:, 0]
+    return out, lse, k_row, v_new.copy()
