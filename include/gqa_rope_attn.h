@@ -23,6 +23,8 @@
  *     batches (cu_seqlens prefix sums).
  *   The log-sum-exp output is not on the pages; it is the natural-log
  *   normaliser of each row's scaled, masked scores.
+ * A decoding step against a KV cache (gqa_rope_attn_decode) is declared
+ * further down.
  *
  * Precision: q, k, v, out are bf16 (or fp32 with dtype GQA_DTYPE_FP32; then
  * q, k, v are rounded to bf16 on load and out is written as fp32). cos/sin
@@ -168,10 +170,53 @@ int gqa_rope_attn_fwd_noalloc(const void* q, const void* k, const void* v, const
                               int total_tokens, int n_q_heads, int n_kv_heads, int head_dim,
                               int causal, int dtype, void* out, float* lse, void* stream);
 
-/* Measurement aid. Arms the calling thread's next gqa_rope_attn_fwd call to
- * record three CUDA events (cudaEvent_t passed as void*, any may be NULL) on
- * its stream: before the prologue kernel, between the prologue and the
- * attention kernel, and after the attention kernel, so that each kernel's
+/* ---- Decoding step (one new token per sequence against a KV cache) ------
+ *
+ * "Attention from Scratch", section "Attention, the math: Grouped-Query
+ * Attention with RoPE'd Q/K", the paragraph on the KV cache GQA shrinks: one
+ * K and one V vector per token and KV head is kept for every token so far.
+ * For sequence b the new token sits at position p = cache_seqlens[b]:
+ *
+ *   k_cache[b, p, kv, :] = rope(k_new[b, kv], p)   (rounded once to bf16)
+ *   v_cache[b, p, kv, :] = v_new[b, kv]
+ *   out[b, h, :] = softmax_j( rope(q[b, h], p) . k_cache[b, j, kv] / sqrt(d) ) v_cache[b, j, kv],
+ *                  j = 0 .. p, kv = h / G
+ *   lse[h, b]    = ln sum_j exp( rope(q[b, h], p) . k_cache[b, j, kv] / sqrt(d) )
+ *
+ * i.e. the causal mask's last row of the prefill above, with the earlier
+ * keys read from the cache (which holds keys after rotation). RoPE and the
+ * rounding of the rotated operands are those of gqa_rope_attn_fwd.
+ *
+ * All tensors bf16 (lse fp32), contiguous, device memory, 16-byte aligned:
+ *   q          [batch, n_q_heads, head_dim]
+ *   k_new      [batch, n_kv_heads, head_dim]   (not rotated)
+ *   v_new      [batch, n_kv_heads, head_dim]
+ *   k_cache    [batch, max_cache_len, n_kv_heads, head_dim]  rotated keys;
+ *              rows 0 .. p-1 are read, row p is written
+ *   v_cache    same layout; rows 0 .. p-1 read, row p written
+ *   cache_seqlens  int32 [batch]: tokens already cached, 0 <= p < max_cache_len.
+ *              Checked on the device: a sequence outside the range gets no
+ *              output and sets GQA_ERR_BAD_SEQLENS in the status word.
+ *   out        [batch, n_q_heads, head_dim]
+ *   lse        [n_q_heads, batch] fp32, or NULL
+ * head_dim 32, 64 or 128; n_q_heads / n_kv_heads <= 16; batch <= 65535.
+ * workspace: at least gqa_rope_attn_decode_workspace_size() bytes, 256-byte
+ * aligned, contents need not be initialised, not shared by calls that may
+ * overlap. Two kernels are queued on `stream`; the call does not wait.
+ * Returns GQA_OK or an error code; on an error nothing has been queued.
+ */
+size_t gqa_rope_attn_decode_workspace_size(int batch, int max_cache_len, int n_q_heads, int n_kv_heads,
+                                           int head_dim);
+
+int gqa_rope_attn_decode(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                         const int32_t* cache_seqlens, double rope_theta, int batch, int max_cache_len,
+                         int n_q_heads, int n_kv_heads, int head_dim, void* out, float* lse, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Measurement aid. Arms the calling thread's next gqa_rope_attn_fwd or
+ * gqa_rope_attn_decode call to record three CUDA events (cudaEvent_t passed
+ * as void*, any may be NULL) on its stream: before its first kernel, between
+ * its two kernels, and after the second, so that each kernel's
  * duration can be read with cudaEventElapsedTime. The arming is consumed by
  * that one call (also when it fails). The caller owns the events. */
 void gqa_rope_attn_set_profile_events(void* ev_start, void* ev_mid, void* ev_end);

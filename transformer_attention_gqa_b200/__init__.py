@@ -4,9 +4,10 @@ PyTorch-facing binding. PyTorch provides device memory and streams only."""
 from __future__ import annotations
 
 from . import _abi
-from ._abi import GqaError, workspace_size, get_device_status  # noqa: F401
+from ._abi import GqaError, workspace_size, decode_workspace_size, get_device_status  # noqa: F401
 
-__all__ = ["gqa_rope_attn_fwd", "workspace_size", "get_device_status", "GqaError", "Workspace"]
+__all__ = ["gqa_rope_attn_fwd", "gqa_rope_attn_decode", "workspace_size", "decode_workspace_size",
+           "get_device_status", "GqaError", "Workspace"]
 
 
 def _ptr(t):
@@ -65,4 +66,44 @@ def gqa_rope_attn_fwd(q, k, v, cu_seqlens, rope_theta: float, positions=None, ca
                                 ws.numel() * ws.element_size(), stream)
     if rc != _abi.GQA_OK:
         raise GqaError(rc)
+    return out, lse
+
+
+def gqa_rope_attn_decode(q, k_new, v_new, k_cache, v_cache, cache_seqlens, rope_theta: float, out=None, lse=None,
+                         workspace=None, stream=None, need_lse: bool = True):
+    """One decoding step: the new token of each sequence b sits at position
+    p = cache_seqlens[b]; its key is rotated at p and written, with its
+    value, to cache row p; out = softmax(rope(q) . K[0..p]^T / sqrt(d)) V[0..p].
+
+    q: [B, n_q, d]; k_new, v_new: [B, n_kv, d]; k_cache, v_cache:
+    [B, max_len, n_kv, d] (rotated keys) -- bf16 CUDA tensors;
+    cache_seqlens: int32 [B] on the device. The caches are updated in place.
+    Returns (out [B, n_q, d] bf16, lse [n_q, B] fp32 or None). Raises
+    GqaError on a non-OK status.
+    """
+    import torch
+
+    B, nq, d = q.shape
+    nkv = k_new.shape[1]
+    Lmax = k_cache.shape[1]
+    for t in (q, k_new, v_new, k_cache, v_cache, cache_seqlens):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    if any(t.dtype != torch.bfloat16 for t in (q, k_new, v_new, k_cache, v_cache)):
+        raise TypeError("decode tensors must be bfloat16")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and need_lse:
+        lse = torch.empty((nq, B), dtype=torch.float32, device=q.device)
+    nbytes = decode_workspace_size(B, Lmax, nq, nkv, d)
+    if workspace is None:
+        workspace = Workspace(q.device)
+    ws = workspace.get(nbytes) if isinstance(workspace, Workspace) else workspace
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    rc = _abi.gqa_rope_attn_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                   _ptr(cache_seqlens), rope_theta, B, Lmax, nq, nkv, d, _ptr(out), _ptr(lse),
+                                   _ptr(ws), ws.numel() * ws.element_size(), stream)
+    if rc != _abi.GQA_OK:
+        raise GqaError(rc, "gqa_rope_attn_decode")
     return out, lse

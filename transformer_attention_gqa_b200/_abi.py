@@ -32,6 +32,8 @@ EXPORTED = (
     "gqa_rope_attn_last_launch_count",
     "gqa_rope_attn_set_profile_events",
     "gqa_rope_attn_fwd_noalloc",
+    "gqa_rope_attn_decode_workspace_size",
+    "gqa_rope_attn_decode",
 )
 
 _lib = None
@@ -70,6 +72,11 @@ def load() -> ctypes.CDLL:
     lib.gqa_rope_attn_fwd_noalloc.restype = c_int
     lib.gqa_rope_attn_fwd_noalloc.argtypes = [c_void, c_void, c_void, c_void, c_double, c_void, c_int, c_int, c_int,
                                               c_int, c_int, c_int, c_int, c_void, c_void, c_void]
+    lib.gqa_rope_attn_decode_workspace_size.restype = c_size
+    lib.gqa_rope_attn_decode_workspace_size.argtypes = [c_int] * 5
+    lib.gqa_rope_attn_decode.restype = c_int
+    lib.gqa_rope_attn_decode.argtypes = [c_void, c_void, c_void, c_void, c_void, c_void, c_double, c_int, c_int,
+                                         c_int, c_int, c_int, c_void, c_void, c_void, c_size, c_void]
     lib.gqa_rope_attn_set_profile_events.restype = None
     lib.gqa_rope_attn_set_profile_events.argtypes = [c_void, c_void, c_void]
     _lib = lib
@@ -100,6 +107,19 @@ def gqa_rope_attn_fwd_noalloc(q, k, v, positions, rope_theta, cu_seqlens, num_se
     return int(load().gqa_rope_attn_fwd_noalloc(q, k, v, positions, float(rope_theta), cu_seqlens, int(num_seqs),
                                                 int(total_tokens), int(n_q_heads), int(n_kv_heads), int(head_dim),
                                                 int(causal), int(dtype), out, lse, stream))
+
+
+def decode_workspace_size(batch: int, max_cache_len: int, n_q_heads: int, n_kv_heads: int, head_dim: int) -> int:
+    return int(load().gqa_rope_attn_decode_workspace_size(batch, max_cache_len, n_q_heads, n_kv_heads, head_dim))
+
+
+def gqa_rope_attn_decode(q, k_new, v_new, k_cache, v_cache, cache_seqlens, rope_theta, batch, max_cache_len,
+                         n_q_heads, n_kv_heads, head_dim, out, lse, workspace, workspace_bytes, stream) -> int:
+    """Raw call of the decoding step; integer device addresses (0 for NULL);
+    returns the status."""
+    return int(load().gqa_rope_attn_decode(q, k_new, v_new, k_cache, v_cache, cache_seqlens, float(rope_theta),
+                                           int(batch), int(max_cache_len), int(n_q_heads), int(n_kv_heads),
+                                           int(head_dim), out, lse, workspace, int(workspace_bytes), stream))
 
 
 def get_device_status(stream=None) -> int:

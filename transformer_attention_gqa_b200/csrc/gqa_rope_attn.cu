@@ -1,6 +1,7 @@
 // Host side of the C ABI (include/gqa_rope_attn.h): argument checks, TMA
-// descriptor cache, and the two launches of the fused forward (prologue,
-// then the attention kernel, in stream order).
+// descriptor cache, the two launches of the fused forward (prologue, then
+// the attention kernel, in stream order) and the two of the decoding step
+// (key-range kernel, then the merge).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -12,6 +13,7 @@
 #include "../../include/gqa_rope_attn.h"
 #include "attn_kernel.cuh"
 #include "common.cuh"
+#include "decode_kernel.cuh"
 #include "prep_kernel.cuh"
 
 namespace gqa {
@@ -24,6 +26,7 @@ struct DeviceState {
   bool init = false;
   int sm_count = 0;
   bool attr_set[3][2] = {};
+  bool dec_attr_set[3][3] = {};
 };
 
 std::mutex g_mu;
@@ -231,10 +234,157 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
   return GQA_OK;
 }
 
+// ---------------------------------------------------------------- decoding
+
+struct DecLayout {
+  size_t part_o, part_ml, total;
+  int splits, kps;
+};
+
+// Key ranges: whole 64-key tiles, about DEC_TARGET_CTAS CTAs over the batch
+// (a rule of the shape alone, so the workspace size needs no device query).
+DecLayout dec_layout(int B, int Lmax, int nq, int nkv, int d) {
+  DecLayout L{};
+  const int G = nq / nkv;
+  const long long tiles = (Lmax + DEC_KT - 1) / DEC_KT;
+  long long want = (DEC_TARGET_CTAS + (long long)B * nkv - 1) / ((long long)B * nkv);
+  if (want < 1) want = 1;
+  if (want > tiles) want = tiles;
+  const long long tps = (tiles + want - 1) / want;
+  L.kps = (int)(tps * DEC_KT);
+  L.splits = (int)((tiles + tps - 1) / tps);
+  size_t off = 0;
+  L.part_o = off;
+  off = align_up(off + (size_t)B * nkv * L.splits * G * d * sizeof(float), 256);
+  L.part_ml = off;
+  off = align_up(off + (size_t)B * nkv * L.splits * G * sizeof(float2), 256);
+  L.total = off;
+  return L;
+}
+
+template <int D, int GM>
+int launch_decode(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                  const int32_t* lens, double theta, int B, int Lmax, int nq, int nkv, void* out, float* lse,
+                  uint8_t* ws, const DecLayout& lay, cudaStream_t stream, int device) {
+  using C = DecCfg<D, GM>;
+  constexpr int gi = GM == 4 ? 0 : (GM == 8 ? 1 : 2);
+  {  // caller holds g_mu
+    DeviceState& ds = g_dev[device];
+    if (!ds.dec_attr_set[dim_index(D)][gi]) {
+      if (cudaFuncSetAttribute(gqa_decode_split_kernel<D, GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_BYTES) != cudaSuccess)
+        return GQA_ERR_CUDA;
+      ds.dec_attr_set[dim_index(D)][gi] = true;
+    }
+  }
+  // Cache maps: [B*Lmax rows][nkv][d], box (BOXC columns, 1 head, 64 rows).
+  CUtensorMap tmK, tmV;
+  const uint64_t dims[3] = {(uint64_t)D, (uint64_t)nkv, (uint64_t)B * (uint64_t)Lmax};
+  const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)nkv * D * 2};
+  const uint32_t box[3] = {(uint32_t)C::BOXC, 1u, (uint32_t)DEC_KT};
+  if (!make_tmap(device, k_cache, dims, str, box, C::ROWB, &tmK)) return GQA_ERR_CUDA;
+  if (!make_tmap(device, v_cache, dims, str, box, C::ROWB, &tmV)) return GQA_ERR_CUDA;
+
+  DecodeParams dp{};
+  dp.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  dp.k_new = reinterpret_cast<const __nv_bfloat16*>(k_new);
+  dp.v_new = reinterpret_cast<const __nv_bfloat16*>(v_new);
+  dp.k_cache = reinterpret_cast<__nv_bfloat16*>(k_cache);
+  dp.v_cache = reinterpret_cast<__nv_bfloat16*>(v_cache);
+  dp.cache_seqlens = lens;
+  dp.part_o = reinterpret_cast<float*>(ws + lay.part_o);
+  dp.part_ml = reinterpret_cast<float2*>(ws + lay.part_ml);
+  dp.out = reinterpret_cast<__nv_bfloat16*>(out);
+  dp.lse = lse;
+  dp.theta = theta;
+  dp.B = B;
+  dp.Lmax = Lmax;
+  dp.nq = nq;
+  dp.nkv = nkv;
+  dp.G = nq / nkv;
+  dp.splits = lay.splits;
+  dp.kps = lay.kps;
+  dp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+
+  if (t_prof_ev[0] && cudaEventRecord(t_prof_ev[0], stream) != cudaSuccess) return GQA_ERR_CUDA;
+  gqa_decode_split_kernel<D, GM><<<dim3(lay.splits, nkv, B), DEC_THREADS, C::SMEM_BYTES, stream>>>(tmK, tmV, dp);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+  if (t_prof_ev[1] && cudaEventRecord(t_prof_ev[1], stream) != cudaSuccess) return GQA_ERR_CUDA;
+  gqa_decode_combine_kernel<<<dim3(nkv, B), DEC_THREADS, 0, stream>>>(dp, D);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+  if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;
+  t_last_launches = 2;
+  return GQA_OK;
+}
+
 }  // namespace
 }  // namespace gqa
 
 using namespace gqa;
+
+extern "C" size_t gqa_rope_attn_decode_workspace_size(int batch, int max_cache_len, int n_q_heads,
+                                                      int n_kv_heads, int head_dim) {
+  if (batch < 0 || max_cache_len < 1 || n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return 0;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return 0;
+  if (n_q_heads / n_kv_heads > DEC_GMAX) return 0;
+  if (batch == 0) return 256;
+  return dec_layout(batch, max_cache_len, n_q_heads, n_kv_heads, head_dim).total;
+}
+
+extern "C" int gqa_rope_attn_decode(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                                    void* v_cache, const int32_t* cache_seqlens, double rope_theta, int batch,
+                                    int max_cache_len, int n_q_heads, int n_kv_heads, int head_dim, void* out,
+                                    float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  t_last_launches = 0;
+  struct Disarm {
+    ~Disarm() { t_prof_ev[0] = t_prof_ev[1] = t_prof_ev[2] = nullptr; }
+  } disarm;
+  if (batch < 0 || max_cache_len < 1) return GQA_ERR_INVALID_ARG;
+  if (n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return GQA_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.0) || !std::isfinite(rope_theta)) return GQA_ERR_INVALID_ARG;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED;
+  if (n_q_heads / n_kv_heads > DEC_GMAX) return GQA_ERR_UNSUPPORTED;
+  if (batch > 65535 || n_kv_heads > 65535) return GQA_ERR_UNSUPPORTED;
+  if ((long long)batch * max_cache_len >= (1ll << 31)) return GQA_ERR_UNSUPPORTED;
+  if (batch == 0) return GQA_OK;
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !cache_seqlens || !out) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(out))
+    return GQA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return GQA_ERR_INVALID_ARG;
+  const DecLayout lay = dec_layout(batch, max_cache_len, n_q_heads, n_kv_heads, head_dim);
+  if (!workspace || workspace_bytes < lay.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return GQA_ERR_WORKSPACE;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices) return GQA_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState& ds = g_dev[device];
+    if (!ds.init) {
+      int major = 0;
+      if (cudaDeviceGetAttribute(&ds.sm_count, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+          cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess)
+        return GQA_ERR_CUDA;
+      if (major != 10) return GQA_ERR_UNSUPPORTED;
+      ds.init = true;
+    }
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  std::lock_guard<std::mutex> lk(g_mu);  // descriptor cache
+  const int G = n_q_heads / n_kv_heads;
+  const int gb = G <= 4 ? 4 : (G <= 8 ? 8 : 16);
+#define GQA_DEC_CASE(DD, GG)                                                                                  \
+  if (head_dim == DD && gb == GG)                                                                             \
+    return launch_decode<DD, GG>(q, k_new, v_new, k_cache, v_cache, cache_seqlens, rope_theta, batch,         \
+                                 max_cache_len, n_q_heads, n_kv_heads, out, lse, ws, lay, st, device);
+  GQA_DEC_CASE(32, 4) GQA_DEC_CASE(32, 8) GQA_DEC_CASE(32, 16)
+  GQA_DEC_CASE(64, 4) GQA_DEC_CASE(64, 8) GQA_DEC_CASE(64, 16)
+  GQA_DEC_CASE(128, 4) GQA_DEC_CASE(128, 8) GQA_DEC_CASE(128, 16)
+#undef GQA_DEC_CASE
+  return GQA_ERR_UNSUPPORTED;
+}
 
 extern "C" size_t gqa_rope_attn_workspace_size(int num_seqs, int total_tokens, int n_q_heads, int n_kv_heads,
                                                int head_dim, int dtype) {
@@ -360,7 +510,9 @@ extern "C" const char* gqa_rope_attn_strerror(int status) {
     case GQA_ERR_INVALID_ARG: return "invalid argument";
     case GQA_ERR_UNSUPPORTED: return "unsupported shape or device";
     case GQA_ERR_CUDA: return "CUDA error";
-    case GQA_ERR_BAD_SEQLENS: return "cu_seqlens is not a valid prefix sum of total_tokens";
+    case GQA_ERR_BAD_SEQLENS:
+      return "cu_seqlens is not a valid prefix sum of total_tokens, or a decode cache_seqlens entry is "
+             "outside [0, max_cache_len)";
     case GQA_ERR_TIMEOUT: return "a bounded wait inside the kernel ran out";
     case GQA_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
     case GQA_ERR_NOALLOC_LIMIT:

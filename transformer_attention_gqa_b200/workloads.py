@@ -18,6 +18,21 @@ Qwen2.5-0.5B head layouts:
   varlen    16384 packed tokens, lengths ~ U{64..4096} (seed 0, last one
             truncated), n_q=32, n_kv=8, d=128, theta=5e5
 
+Decoding workloads (one new token per sequence against a KV cache of
+rotated keys; the "Kohaku-TT" page times a Qwen2.5-3B greedy decode):
+
+  decode_llama8b  B=32, 4096 cached tokens each, n_q=32, n_kv=8, d=128,
+                  theta=5e5 (537 MB of K and V read per step)
+  decode_qwen3b   B=64, 8192 cached tokens each, n_q=16, n_kv=2, d=128,
+                  theta=1e6 (Qwen2.5-3B head layout; 537 MB per step)
+  decode_ragged   B=64, cached lengths ~ U{1..8191} (seed 5), n_q=32,
+                  n_kv=8, d=128, theta=5e5
+  decode_small    B=5, lengths 0, 1, 63, 64, 190 in a 200-row cache,
+                  n_q=12, n_kv=4, d=64, theta=1e4
+The cache holds standard-normal bf16 values in the rows before each
+sequence's length (a rotation keeps that distribution, so no RoPE is applied
+here) and NaN in the rows after it, which the step must never read.
+
 Recipe: ``numpy.random.default_rng(seed)`` draws ``standard_normal`` float32
 arrays in the order q, k, v; values are then rounded to bfloat16 (round to
 nearest even, done by ``torch.Tensor.to(torch.bfloat16)``) because the kernel's
@@ -38,6 +53,10 @@ __all__ = [
     "make_inputs",
     "make_custom",
     "to_bf16_values",
+    "DecodeWorkload",
+    "DECODE_WORKLOADS",
+    "DecodeInputs",
+    "make_decode_inputs",
 ]
 
 
@@ -168,3 +187,80 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Inputs:
     q, k, v = to_bf16_values(q), to_bf16_values(k), to_bf16_values(v)
     cu, pos = _cu_and_positions(w.seq_lens)
     return Inputs(w, q, k, v, cu, pos)
+
+
+# ---------------------------------------------------------------- decoding
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    cache_lens: tuple  # tokens already cached per sequence (the new token's position)
+    max_cache_len: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    rope_theta: float
+    seed: int = 0
+    description: str = ""
+
+    @property
+    def batch(self) -> int:
+        return len(self.cache_lens)
+
+    def kv_bytes(self) -> int:
+        """K and V bytes one step must read: p + 1 rows (p cached, one new)
+        of n_kv heads x d bf16 each, per sequence."""
+        return int(sum(p + 1 for p in self.cache_lens)) * self.n_kv_heads * self.head_dim * 2 * 2
+
+    def step_bytes(self) -> int:
+        """Algorithmic HBM bytes of one step: the K/V rows read, q / k_new /
+        v_new read, the appended K/V rows and out written, lse written."""
+        B, nq, nkv, d = self.batch, self.n_q_heads, self.n_kv_heads, self.head_dim
+        return self.kv_bytes() + B * (nq + 2 * nkv) * d * 2 + B * (2 * nkv + nq) * d * 2 + B * nq * 4
+
+    def flops(self) -> float:
+        """Scores and weighted sum: 4 * (p + 1) * d per query head."""
+        return float(sum(4.0 * (p + 1) * self.head_dim * self.n_q_heads for p in self.cache_lens))
+
+
+def _ragged_lens(n: int, lo: int, hi: int, seed: int) -> tuple:
+    rng = np.random.default_rng(seed)
+    return tuple(int(x) for x in rng.integers(lo, hi, size=n, endpoint=True))
+
+
+DECODE_WORKLOADS: Dict[str, DecodeWorkload] = {
+    "decode_llama8b": DecodeWorkload("decode_llama8b", (4096,) * 32, 4097, 32, 8, 128, 5e5, seed=6,
+                                     description="B=32 cache 4096 n_q=32 n_kv=8 d=128 theta=5e5 bf16"),
+    "decode_qwen3b": DecodeWorkload("decode_qwen3b", (8192,) * 64, 8193, 16, 2, 128, 1e6, seed=7,
+                                    description="B=64 cache 8192 n_q=16 n_kv=2 d=128 theta=1e6 bf16"),
+    "decode_ragged": DecodeWorkload("decode_ragged", _ragged_lens(64, 1, 8191, 5), 8192, 32, 8, 128, 5e5,
+                                    seed=8, description="B=64 cache ~U{1..8191} n_q=32 n_kv=8 d=128 theta=5e5 bf16"),
+    "decode_small": DecodeWorkload("decode_small", (0, 1, 63, 64, 190), 200, 12, 4, 64, 1e4, seed=9,
+                                   description="B=5 cache 0,1,63,64,190 of 200 n_q=12 n_kv=4 d=64 theta=1e4 bf16"),
+}
+
+
+@dataclass
+class DecodeInputs:
+    workload: DecodeWorkload
+    q: np.ndarray        # [B, n_q, d] float32 holding bf16 values
+    k_new: np.ndarray    # [B, n_kv, d]
+    v_new: np.ndarray    # [B, n_kv, d]
+    k_cache: np.ndarray  # [B, max_len, n_kv, d]; NaN from each sequence's length on
+    v_cache: np.ndarray
+    cache_seqlens: np.ndarray  # [B] int32
+
+
+def make_decode_inputs(w: DecodeWorkload, seed: Optional[int] = None, nan_tail: bool = True) -> DecodeInputs:
+    rng = np.random.default_rng(w.seed if seed is None else seed)
+    B, L, nq, nkv, d = w.batch, w.max_cache_len, w.n_q_heads, w.n_kv_heads, w.head_dim
+    q = to_bf16_values(rng.standard_normal((B, nq, d), dtype=np.float32))
+    kn = to_bf16_values(rng.standard_normal((B, nkv, d), dtype=np.float32))
+    vn = to_bf16_values(rng.standard_normal((B, nkv, d), dtype=np.float32))
+    kc = np.full((B, L, nkv, d), np.nan if nan_tail else 0.0, dtype=np.float32)
+    vc = np.full((B, L, nkv, d), np.nan if nan_tail else 0.0, dtype=np.float32)
+    for b, p in enumerate(w.cache_lens):
+        kc[b, :p] = to_bf16_values(rng.standard_normal((p, nkv, d), dtype=np.float32))
+        vc[b, :p] = to_bf16_values(rng.standard_normal((p, nkv, d), dtype=np.float32))
+    lens = np.asarray(w.cache_lens, dtype=np.int32)
+    return DecodeInputs(w, q, kn, vn, kc, vc, lens)
