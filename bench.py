@@ -177,6 +177,176 @@ def cpu_baseline(workload, budget_s: float = 15.0, seed_rows: int = 0):
                       f"float64 NumPy, {dt:.1f} s", "host_cores": cores}
 
 
+# ------------------------------------------------------------------ decoding
+DECODE_METRIC = "GQA+RoPE decode step (KV cache read, new row appended) algorithmic HBM GB/s on 1 B200"
+DECODE_UNIT = "GB/s"
+
+
+def _decode_sample_bytes(w, sel):
+    lens = np.asarray(w.cache_lens)[sel]
+    return float(np.sum(lens + 1)) * w.n_kv_heads * w.head_dim * 2 * 2
+
+
+def cpu_baseline_decode(w, inp, budget_s: float = 15.0, seed: int = 0):
+    """Times the float64 oracle's decoding step on a bounded random sample of
+    the batch's sequences; returns the algorithmic K/V bytes of the sample
+    per second (GB/s), the decode metric's convention."""
+    import oracle.gqa_oracle as orc
+
+    rng = np.random.default_rng(seed)
+
+    def run(n):
+        sel = np.sort(rng.choice(w.batch, size=min(n, w.batch), replace=False))
+        t0 = time.perf_counter()
+        orc.gqa_rope_decode(inp.q[sel], inp.k_new[sel], inp.v_new[sel], inp.k_cache[sel], inp.v_cache[sel],
+                            inp.cache_seqlens[sel], w.n_q_heads, w.n_kv_heads, w.rope_theta)
+        return time.perf_counter() - t0, sel
+
+    t1, _ = run(1)
+    n = int(max(1, min(w.batch, budget_s / max(t1, 1e-3))))
+    dt, sel = run(n)
+    cores = len(os.sched_getaffinity(0))
+    return {"value": _decode_sample_bytes(w, sel) / dt / 1e9, "unit": DECODE_UNIT, "cores": cores,
+            "kind": "oracle", "sample": f"{len(sel)} of {w.batch} sequences of {w.name}, float64 NumPy, {dt:.1f} s"}
+
+
+def run_decode(args, rank, world, local_rank):
+    import torch
+    import transformer_attention_gqa_b200 as g
+    from transformer_attention_gqa_b200 import _abi, replicas, workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = wl.DECODE_WORKLOADS[args.workload]
+    inp = wl.make_decode_inputs(w, seed=w.seed if rank == 0 else replicas.replica_seed(w.seed, rank), nan_tail=False)
+    bf = torch.bfloat16
+    q = torch.from_numpy(inp.q).to(bf).to(dev)
+    kn = torch.from_numpy(inp.k_new).to(bf).to(dev)
+    vn = torch.from_numpy(inp.v_new).to(bf).to(dev)
+    kc = torch.from_numpy(inp.k_cache).to(bf).to(dev)
+    vc = torch.from_numpy(inp.v_cache).to(bf).to(dev)
+    lens = torch.from_numpy(inp.cache_seqlens).to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.n_q_heads, w.batch), dtype=torch.float32, device=dev)
+    ws = g.Workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+    big = w.kv_bytes() > 2 * (126 << 20)
+    flush = None if big else torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():  # the same token each step: row p is rewritten with the same values
+        g.gqa_rope_attn_decode(q, kn, vn, kc, vc, lens, w.rope_theta, out=out, lse=lse, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert g.get_device_status() == 0
+    launches_per_step = _abi.last_launch_count()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    replicas.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    replicas.barrier()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+
+    from cuda.bindings import runtime as rt
+
+    def _ev():
+        err, e = rt.cudaEventCreate()
+        assert int(err) == 0
+        return e
+
+    def _ms(a, b):
+        err, ms = rt.cudaEventElapsedTime(a, b)
+        assert int(err) == 0
+        return float(ms)
+
+    kern = []
+    for _ in range(max(3, min(args.steps, 10))):
+        e = [_ev() for _ in range(3)]
+        if flush is not None:
+            flush.zero_()
+        _abi.set_profile_events(int(e[0]), int(e[1]), int(e[2]))
+        step()
+        kern.append(e)
+    torch.cuda.synchronize()
+    split_ms = statistics.median(_ms(a, b) for a, b, _ in kern)
+    merge_ms = statistics.median(_ms(b, c) for _, b, c in kern)
+    for e in kern:
+        for x in e:
+            rt.cudaEventDestroy(x)
+    clk = clocks.stop()
+
+    # end to end: the token's q, k_new, v_new and the lengths from pinned host
+    # memory, out and lse back; the cache stays resident on the device
+    qh, knh, vnh = (torch.from_numpy(a).to(bf).pin_memory() for a in (inp.q, inp.k_new, inp.v_new))
+    lh = torch.from_numpy(inp.cache_seqlens).pin_memory()
+    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (qh, knh, vnh, lh))
+    d2h = outh.numel() * outh.element_size() + lseh.numel() * lseh.element_size()
+
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        kn.copy_(knh, non_blocking=True)
+        vn.copy_(vnh, non_blocking=True)
+        lens.copy_(lh, non_blocking=True)
+        step()
+        outh.copy_(out, non_blocking=True)
+        lseh.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    replicas.barrier()
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    assert g.get_device_status() == 0
+
+    total_ms, e2e_ms, split_ms, merge_ms = replicas.max_over_ranks([total_ms, e2e_ms, split_ms, merge_ms], device=dev)
+    ms_per_step = total_ms / args.steps
+    nbytes = w.step_bytes()
+    peaks, src = load_peaks()
+    peak = float(peaks["hbm_gbs"])
+    achieved = nbytes / ((split_ms + merge_ms) * 1e-3) / 1e9
+    res = {
+        "metric": DECODE_METRIC, "value": round(nbytes * world / (ms_per_step * 1e-3) / 1e9, 1),
+        "unit": DECODE_UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "shape": w.description, "batch": w.batch, "max_cache_len": w.max_cache_len,
+                   "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+                   "algorithmic_bytes_per_step": nbytes, "tokens_per_step": w.batch,
+                   "tokens_per_s": round(w.batch * world / (ms_per_step * 1e-3), 1),
+                   "parallelism": f"replicas x{world}",
+                   "l2": "K/V read per step larger than L2" if big else "256 MiB written before every timed step"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{src} hbm_gbs (copy)", "kernel": "gqa_decode_split_kernel + gqa_decode_combine_kernel",
+                     "split_ms": round(split_ms, 5), "merge_ms": round(merge_ms, 5)},
+        "e2e": {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": DECODE_UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if clk:
+        res["clocks"] = clk
+    res["_inputs"] = inp
+    return res
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -340,6 +510,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
     from transformer_attention_gqa_b200 import workloads as wl
+    if args.workload in wl.DECODE_WORKLOADS:
+        return main_decode(args, world, rank, local_rank)
     w = wl.WORKLOADS[args.workload]
 
     if args.impl == "reference":
@@ -368,6 +540,41 @@ def main():
     res = run_ours(args, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    replicas.shutdown()
+    if rank == 0:
+        print(json.dumps(res))
+    return 0
+
+
+def main_decode(args, world, rank, local_rank):
+    from transformer_attention_gqa_b200 import workloads as wl
+    w = wl.DECODE_WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        inp = wl.make_decode_inputs(w, nan_tail=False)
+        for i in range(args.warmup):
+            cpu_baseline_decode(w, inp, budget_s=0.5, seed=1000 + i)
+        vals, info = [], None
+        for i in range(args.steps):
+            info = cpu_baseline_decode(w, inp, budget_s=max(1.0, min(5.0, 60.0 / max(args.steps, 1))), seed=i)
+            vals.append(info["value"])
+        val = statistics.median(vals)
+        print(json.dumps({"impl": "reference", "metric": DECODE_METRIC, "value": round(val, 4), "unit": DECODE_UNIT,
+                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": {"workload": w.name, "shape": w.description},
+                          "cpu_baseline": {"value": round(val, 4), "unit": DECODE_UNIT, "cores": info["cores"],
+                                           "kind": "oracle", "sample": info["sample"]},
+                          "e2e": {"value": round(val, 4), "unit": DECODE_UNIT, "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return 0
+    from transformer_attention_gqa_b200 import replicas
+    replicas.init("nccl", timeout_s=120)
+    res = run_decode(args, rank, world, local_rank)
+    inp = res.pop("_inputs")
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_decode(w, inp, budget_s=args.cpu_budget)
     replicas.shutdown()
     if rank == 0:
         print(json.dumps(res))

@@ -29,7 +29,7 @@
 
 namespace gqa {
 
-constexpr int DEC_THREADS = 128;
+constexpr int DEC_THREADS = 256;
 constexpr int DEC_KT = 64;      // keys per tile
 constexpr int DEC_STAGES = 3;
 constexpr int DEC_GMAX = 16;    // query heads per KV head
@@ -61,19 +61,28 @@ struct DecCfg {
   static constexpr int SWZ_MASK = ROWB == 128 ? 7 : 3;
   static constexpr int BOX_BYTES = DEC_KT * ROWB;
   static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one K or V tile
-  // PV outputs (4 columns of one head each) per thread
-  static constexpr int UNITS = GM * (D / 4) > DEC_THREADS ? GM * (D / 4) / DEC_THREADS : 1;
+  // Score phase: 4 lanes per key (a quarter of d each: CPQ 16-byte chunks),
+  // 8 keys per warp. Weighted-sum phase: thread = (4 output columns, key
+  // group of KPG keys), all heads.
+  static constexpr int CPQ = D / 32;
+  // Query chunk c (8 features) is stored at slot (c % CPQ) * 4 + c / CPQ, so
+  // the four lanes of a key, reading chunk i of their quarters at once, hit
+  // four different bank groups.
+  static __device__ __forceinline__ int qslot(int c) { return (c % CPQ) * 4 + c / CPQ; }
+  static constexpr int KGROUPS = DEC_THREADS / (D / 4);
+  static constexpr int KPG = DEC_KT / KGROUPS;
   static constexpr int OFF_KV = 0;                                 // [stage][K tile, V tile]
   static constexpr int OFF_Q = OFF_KV + DEC_STAGES * 2 * TILE_BYTES;  // float [GM][D]
-  static constexpr int OFF_S = OFF_Q + GM * D * 4;                    // float [GM][KT]
+  static constexpr int OFF_S = OFF_Q + GM * D * 4;                    // float [KT][GM]
   static constexpr int OFF_CS = OFF_S + GM * DEC_KT * 4;              // float2 [D/2] (cos, sin)
   static constexpr int OFF_ML = OFF_CS + (D / 2) * 8;                 // float2 [GM] running (max, sum)
   static constexpr int OFF_A = OFF_ML + GM * 8;                       // float [GM] rescale of the tile
   static constexpr int OFF_NEW = OFF_A + GM * 4;                      // bf16 [2][D]: rotated new key, value
   static constexpr int OFF_BAR = OFF_NEW + 2 * D * 2;                 // mbarriers [STAGES]
   static constexpr int SMEM_BYTES = ((OFF_BAR + DEC_STAGES * 8 + 15) / 16) * 16 + 1024;  // + alignment slack
-  static_assert(GM * (D / 4) <= DEC_THREADS || GM * (D / 4) % DEC_THREADS == 0, "PV work split");
-  static_assert(DEC_THREADS == 2 * DEC_KT, "score phase: two threads per key");
+  static_assert(DEC_THREADS == 4 * DEC_KT, "score phase: four lanes per key");
+  static_assert(KPG * KGROUPS == DEC_KT, "weighted-sum key groups");
+  static_assert(GM * D * 4 <= DEC_STAGES * 2 * TILE_BYTES, "final reduction buffer in the stage area");
   static_assert(SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
 };
 
@@ -96,6 +105,17 @@ __device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity) {
   return true;
 }
 
+// d = a * b + c on pairs of fp32 (one packed .f32x2 instruction).
+__device__ __forceinline__ float2 dec_ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -113,7 +133,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 2)
                             const DecodeParams p) {
   using C = DecCfg<D, GM>;
   extern __shared__ uint8_t dec_smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dec_smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, derived from the shared array by pointer
+  // arithmetic so that accesses through it stay shared-memory accesses
+  uint8_t* sm = dec_smem_raw + ((1024u - (ptx::smem_u32(dec_smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int G = p.G;
@@ -178,8 +200,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 2)
     const float xl = __bfloat162float(src[i]), xh = __bfloat162float(src[i + D / 2]);
     const uint16_t lo = rope_round_bf16(xl, c.x, xh, -c.y), hi = rope_round_bf16(xh, c.x, xl, c.y);
     if (row < G) {
-      qs[row * D + i] = __uint_as_float((uint32_t)lo << 16);
-      qs[row * D + i + D / 2] = __uint_as_float((uint32_t)hi << 16);
+      qs[row * D + C::qslot(i / 8) * 8 + i % 8] = __uint_as_float((uint32_t)lo << 16);
+      qs[row * D + C::qslot((i + D / 2) / 8) * 8 + i % 8] = __uint_as_float((uint32_t)hi << 16);
     } else {
       knew[i] = __ushort_as_bfloat16(lo);
       knew[i + D / 2] = __ushort_as_bfloat16(hi);
@@ -193,15 +215,15 @@ __global__ void __launch_bounds__(DEC_THREADS, 2)
   if (tid < GM) mls[tid] = make_float2(-INFINITY, 0.f);
   __syncthreads();
 
-  // PV outputs of this thread: units u = tid + i*THREADS, head u / (D/4),
-  // columns 4 * (u % (D/4)) .. +3. All units of a thread share the columns.
+  // weighted-sum phase: this thread's columns and key group
   const int cq = tid % (D / 4);
+  const int kg = tid / (D / 4);
   const int col = cq * 4;
   const uint32_t vcol_off = (col / C::BOXC) * C::BOX_BYTES;
   const uint32_t vcol_in = (col % C::BOXC) * 2;
-  float o[C::UNITS][4];
+  float2 o[GM][2];  // columns (col, col + 1), (col + 2, col + 3) per head
 #pragma unroll
-  for (int i = 0; i < C::UNITS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  for (int g = 0; g < GM; ++g) o[g][0] = o[g][1] = make_float2(0.f, 0.f);
 
   int t_fail = -1;
   for (int t = 0; t < ntiles; ++t) {
@@ -228,51 +250,57 @@ __global__ void __launch_bounds__(DEC_THREADS, 2)
       __syncthreads();
     }
 
-    // ---- scores, log2 units: thread = (key, every other head)
+    // ---- scores, log2 units: lanes (key, d quarter), all heads
     {
-      const int key = tid & (DEC_KT - 1);
-      const int gh = tid >> 6;
-      float acc[GM / 2];
+      const int key = warp * 8 + (lane & 7);
+      const int dq = lane >> 3;
+      float2 acc2[GM];  // two partial sums per head (even / odd features)
 #pragma unroll
-      for (int j = 0; j < GM / 2; ++j) acc[j] = 0.f;
-#pragma unroll 2
-      for (int c = 0; c < D / 8; ++c) {
+      for (int g = 0; g < GM; ++g) acc2[g] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < C::CPQ; ++i) {
+        const int c = dq * C::CPQ + i;
         const int bx = c / (C::BOXC / 8), ch = c % (C::BOXC / 8);
         const uint4 kw = *reinterpret_cast<const uint4*>(kt + bx * C::BOX_BYTES +
                                                          dswz(key * C::ROWB + ch * 16, C::SWZ_MASK));
-        const float kf[8] = {bf_lo(kw.x), bf_hi(kw.x), bf_lo(kw.y), bf_hi(kw.y),
-                             bf_lo(kw.z), bf_hi(kw.z), bf_lo(kw.w), bf_hi(kw.w)};
+        const float2 k01 = make_float2(bf_lo(kw.x), bf_hi(kw.x)), k23 = make_float2(bf_lo(kw.y), bf_hi(kw.y));
+        const float2 k45 = make_float2(bf_lo(kw.z), bf_hi(kw.z)), k67 = make_float2(bf_lo(kw.w), bf_hi(kw.w));
 #pragma unroll
-        for (int j = 0; j < GM / 2; ++j) {
-          const int g = gh + 2 * j;
+        for (int g = 0; g < GM; ++g) {
           if (g < G) {
-            const float4 qa = *reinterpret_cast<const float4*>(qs + g * D + c * 8);
-            const float4 qb = *reinterpret_cast<const float4*>(qs + g * D + c * 8 + 4);
-            float a = acc[j];
-            a = fmaf(qa.x, kf[0], a); a = fmaf(qa.y, kf[1], a); a = fmaf(qa.z, kf[2], a); a = fmaf(qa.w, kf[3], a);
-            a = fmaf(qb.x, kf[4], a); a = fmaf(qb.y, kf[5], a); a = fmaf(qb.z, kf[6], a); a = fmaf(qb.w, kf[7], a);
-            acc[j] = a;
+            const float4 qa = *reinterpret_cast<const float4*>(qs + g * D + (i * 4 + dq) * 8);
+            const float4 qb = *reinterpret_cast<const float4*>(qs + g * D + (i * 4 + dq) * 8 + 4);
+            float2 a = acc2[g];
+            a = dec_ffma2(make_float2(qa.x, qa.y), k01, a);
+            a = dec_ffma2(make_float2(qa.z, qa.w), k23, a);
+            a = dec_ffma2(make_float2(qb.x, qb.y), k45, a);
+            a = dec_ffma2(make_float2(qb.z, qb.w), k67, a);
+            acc2[g] = a;
           }
         }
       }
+      float acc[GM];
 #pragma unroll
-      for (int j = 0; j < GM / 2; ++j) {
-        const int g = gh + 2 * j;
-        if (g < G) sp[g * DEC_KT + key] = key < nvalid ? acc[j] * p.scale_log2 : -INFINITY;
+      for (int g = 0; g < GM; ++g) acc[g] = acc2[g].x + acc2[g].y;
+#pragma unroll
+      for (int g = 0; g < GM; ++g) {
+        acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 8);
+        acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 16);
+        if (g < G && (g & 3) == dq) sp[key * GM + g] = key < nvalid ? acc[g] * p.scale_log2 : -INFINITY;
       }
     }
     __syncthreads();
 
-    // ---- online softmax: warp w takes heads w, w + 4, ...
+    // ---- online softmax: warp w takes heads w, w + 8
     for (int g = warp; g < G; g += DEC_THREADS / 32) {
-      const float s0 = sp[g * DEC_KT + lane], s1 = sp[g * DEC_KT + lane + 32];
+      const float s0 = sp[lane * GM + g], s1 = sp[(lane + 32) * GM + g];
       const float2 ml = mls[g];
       const float mnew = fmaxf(ml.x, warp_max(fmaxf(s0, s1)));  // finite: key tstart is visible
       const float p0 = ptx::ex2(s0 - mnew), p1 = ptx::ex2(s1 - mnew);
       const float sum = warp_sum(p0 + p1);
       const float a = ptx::ex2(ml.x - mnew);
-      sp[g * DEC_KT + lane] = p0;
-      sp[g * DEC_KT + lane + 32] = p1;
+      sp[lane * GM + g] = p0;
+      sp[(lane + 32) * GM + g] = p1;
       __syncwarp();
       if (lane == 0) {
         mls[g] = make_float2(mnew, ml.y * a + sum);
@@ -281,29 +309,36 @@ __global__ void __launch_bounds__(DEC_THREADS, 2)
     }
     __syncthreads();
 
-    // ---- O = O * a + P V over the tile's visible keys
+    // ---- O = O * a + P V: this thread's 4 columns, its key group, all heads
     {
-      float av[C::UNITS];
 #pragma unroll
-      for (int i = 0; i < C::UNITS; ++i) {
-        const int g = (tid + i * DEC_THREADS) / (D / 4);
-        av[i] = g < G ? alpha_s[g] : 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[i][e] *= av[i];
+      for (int g = 0; g < GM; ++g) {
+        if (g < G) {
+          const float a = alpha_s[g];
+          o[g][0].x *= a; o[g][0].y *= a; o[g][1].x *= a; o[g][1].y *= a;
+        }
       }
 #pragma unroll 2
-      for (int k = 0; k < nvalid; ++k) {
-        const uint2 vw = *reinterpret_cast<const uint2*>(vt + vcol_off + dswz(k * C::ROWB + vcol_in, C::SWZ_MASK));
-        const float v0 = bf_lo(vw.x), v1 = bf_hi(vw.x), v2 = bf_lo(vw.y), v3 = bf_hi(vw.y);
+      for (int j = 0; j < C::KPG; ++j) {
+        const int k = kg * C::KPG + j;
+        if (k < nvalid) {  // uniform across the warp
+          const uint2 vw = *reinterpret_cast<const uint2*>(vt + vcol_off + dswz(k * C::ROWB + vcol_in, C::SWZ_MASK));
+          const float2 v01 = make_float2(bf_lo(vw.x), bf_hi(vw.x)), v23 = make_float2(bf_lo(vw.y), bf_hi(vw.y));
 #pragma unroll
-        for (int i = 0; i < C::UNITS; ++i) {
-          const int g = (tid + i * DEC_THREADS) / (D / 4);
-          if (g < G) {
-            const float pk = sp[g * DEC_KT + k];
-            o[i][0] = fmaf(pk, v0, o[i][0]);
-            o[i][1] = fmaf(pk, v1, o[i][1]);
-            o[i][2] = fmaf(pk, v2, o[i][2]);
-            o[i][3] = fmaf(pk, v3, o[i][3]);
+          for (int g4 = 0; g4 < GM / 4; ++g4) {
+            if (4 * g4 < G) {
+              const float4 pk = *reinterpret_cast<const float4*>(sp + k * GM + 4 * g4);
+              const float pv[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int g = 4 * g4 + e;
+                if (g < G) {
+                  const float2 pp = make_float2(pv[e], pv[e]);
+                  o[g][0] = dec_ffma2(pp, v01, o[g][0]);
+                  o[g][1] = dec_ffma2(pp, v23, o[g][1]);
+                }
+              }
+            }
           }
         }
       }
@@ -322,12 +357,26 @@ __global__ void __launch_bounds__(DEC_THREADS, 2)
     return;
   }
 
-  // ---- this range's partial results
+  // ---- this range's partial results: the key groups' sums, added in a
+  // fixed order (group 0 first) in shared memory (the stage area is free)
+  float* red = reinterpret_cast<float*>(sm + C::OFF_KV);  // [G][D]
+  for (int i = tid; i < G * D; i += DEC_THREADS) red[i] = 0.f;
+  __syncthreads();
+  for (int r = 0; r < C::KGROUPS; ++r) {
+    if (kg == r) {
 #pragma unroll
-  for (int i = 0; i < C::UNITS; ++i) {
-    const int g = (tid + i * DEC_THREADS) / (D / 4);
-    if (g < G) *reinterpret_cast<float4*>(po + g * D + col) = make_float4(o[i][0], o[i][1], o[i][2], o[i][3]);
+      for (int g = 0; g < GM; ++g) {
+        if (g < G) {
+          float4* dst = reinterpret_cast<float4*>(red + g * D + col);
+          const float4 cur = *dst;
+          *dst = make_float4(cur.x + o[g][0].x, cur.y + o[g][0].y, cur.z + o[g][1].x, cur.w + o[g][1].y);
+        }
+      }
+    }
+    __syncthreads();
   }
+  for (int i = tid; i < G * D / 4; i += DEC_THREADS)
+    reinterpret_cast<float4*>(po)[i] = reinterpret_cast<const float4*>(red)[i];
   for (int i = tid; i < G; i += DEC_THREADS) pml[i] = mls[i];
   // the appended cache row (after every load of this CTA has landed)
   if (has_new) {
@@ -339,7 +388,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2)
   }
 }
 
-// Merge of the key ranges of one (sequence, KV head); 128 threads over
+// Merge of the key ranges of one (sequence, KV head); threads over
 // (head, column).
 __global__ void __launch_bounds__(DEC_THREADS) gqa_decode_combine_kernel(const DecodeParams p, int D) {
   const int h = blockIdx.x, b = blockIdx.y;
