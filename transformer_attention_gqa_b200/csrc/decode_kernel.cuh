@@ -15,7 +15,7 @@
 //
 // Kernel 1 (split): one CTA per (key range, KV head, sequence). It rotates
 // the G queries of the KV head at p (and the new key, in the CTA whose range
-// holds p), then walks its key range in tiles of 64 keys (3-stage TMA ring
+// holds p), then walks its key range in tiles of 64 keys (2-stage TMA ring
 // for K and V): scores of the tile for the G heads, an online softmax, and
 // the weighted sum of V. It leaves (running max, sum, un-normalised output)
 // per head in the workspace.
@@ -31,9 +31,9 @@ namespace gqa {
 
 constexpr int DEC_THREADS = 256;
 constexpr int DEC_KT = 64;      // keys per tile
-constexpr int DEC_STAGES = 3;
+constexpr int DEC_STAGES = 2;
 constexpr int DEC_GMAX = 16;    // query heads per KV head
-constexpr int DEC_TARGET_CTAS = 1024;  // split count aims at about this many CTAs
+constexpr int DEC_TARGET_CTAS = 256;   // split count aims at about this many CTAs (measured: fewer, longer CTAs amortise the per-CTA RoPE setup)
 
 struct DecodeParams {
   const __nv_bfloat16* q;        // [B, nq, d]
