@@ -51,6 +51,15 @@ on why GQA shrinks the KV cache: one K and one V vector per token and KV head
 is kept for every token generated so far). The new token is the last row of
 the causal mask, so the step is the forward's last row; the cache holds the
 keys after rotation, each at its own position.
+
+Backward (``gqa_rope_attention_backward``): the gradients of the forward's
+output with respect to q, k, v for an upstream gradient dout, i.e. of the
+scalar sum(dout * out). It is the training-time counterpart of the forward
+(the "Train and Run" page's training loop over SDPA-based attention); the
+formulas are the chain rule through the six steps: gather (dV = P^T dO,
+dP = dO V^T), softmax (dS = P * (dP - rowsum(dO * O))), score (dQ' = dS K' /
+sqrt(d), dK' = dS^T Q' / sqrt(d)), share (the G query heads of a group add
+their dK', dV), rotate (the transpose of the rotation: by -angle).
 """
 from __future__ import annotations
 
@@ -73,6 +82,8 @@ __all__ = [
     "gqa_rope_attention",
     "brute_force_attention",
     "gqa_rope_decode",
+    "rope_backward",
+    "gqa_rope_attention_backward",
 ]
 
 
@@ -374,3 +385,75 @@ def gqa_rope_decode(q, k_new, v_new, k_cache, v_cache, cache_seqlens, n_q_heads:
         out[b] = gather(w, vh)[:, 0, :]
         lse[:, b] = row_lse[:, 0]
     return out, lse, k_row, v_new.copy()
+
+
+def rope_backward(dx_rot: np.ndarray, positions, theta: float) -> np.ndarray:
+    """Gradient through x -> x*cos + rotate_half(x)*sin: the transpose of the
+    per-pair rotation, i.e. the rotation by the negative angle:
+    dx_i = g_i*cos + g_{i+d/2}*sin, dx_{i+d/2} = g_{i+d/2}*cos - g_i*sin."""
+    g = np.asarray(dx_rot, dtype=np.float64)
+    d = g.shape[-1]
+    c, s = rope_cos_sin(positions, d, theta, table_fp32=False)
+    c = c[:, None, :]
+    s = s[:, None, :]
+    return g * c - rotate_half(g) * s
+
+
+def gqa_rope_attention_backward(q, k, v, dout, cu_seqlens, n_q_heads: int, n_kv_heads: int, rope_theta: float,
+                                positions=None, causal: bool = True, operand_rounding: bool = False):
+    """Gradients (dq [N, n_q, d], dk [N, n_kv, d], dv [N, n_kv, d]) of
+    sum(dout * out) for the forward above, in float64.
+
+    With ``operand_rounding`` the scores and products use the bf16-rounded
+    rotated operands the forward uses, and the rounding is passed through as
+    the identity (its derivative is zero almost everywhere; the gradient of the
+    unrounded rotation is used instead)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    N, d, cu = _check_args(q, k, v, cu_seqlens, n_q_heads, n_kv_heads)
+    if dout.shape != q.shape:
+        raise ValueError("dout shape mismatch")
+    G = n_q_heads // n_kv_heads
+    if positions is None:
+        pos = np.concatenate([np.arange(cu[i + 1] - cu[i]) for i in range(len(cu) - 1)] + [np.zeros(0)])
+    else:
+        pos = np.asarray(positions, dtype=np.int64).reshape(-1)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    scale = 1.0 / math.sqrt(d)
+    for si in range(len(cu) - 1):
+        a, b = int(cu[si]), int(cu[si + 1])
+        L = b - a
+        if L == 0:
+            continue
+        p = pos[a:b]
+        qr = apply_rope(q[a:b], p, rope_theta, operand_rounding)
+        kr = apply_rope(k[a:b], p, rope_theta, operand_rounding)
+        qh = np.transpose(qr, (1, 0, 2))                                           # [n_q, L, d]
+        kh = np.transpose(share_kv_heads(kr, G, axis=1), (1, 0, 2))
+        vh = np.transpose(share_kv_heads(v[a:b], G, axis=1), (1, 0, 2))
+        doh = np.transpose(dout[a:b], (1, 0, 2))
+        scores = score(qh, kh)
+        if causal:
+            scores = causal_mask(scores, np.arange(L), np.arange(L))
+        w, _ = softmax_with_lse(scores)                                            # P [n_q, L, L]
+        o = gather(w, vh)
+        # gather: out = P V
+        dvh = np.matmul(np.swapaxes(w, -1, -2), doh)                               # [n_q, L, d]
+        dw = np.matmul(doh, np.swapaxes(vh, -1, -2))                               # dP
+        # softmax: dS = P * (dP - sum_j P_ij dP_ij); sum_j P_ij dP_ij = dO_i . O_i
+        delta = np.sum(doh * o, axis=-1, keepdims=True)
+        ds = w * (dw - delta)
+        # score: S = Q' K'^T / sqrt(d)
+        dqh = np.matmul(ds, kh) * scale
+        dkh = np.matmul(np.swapaxes(ds, -1, -2), qh) * scale
+        # share: the G query heads of a group add into their KV head
+        dkr = np.transpose(dkh, (1, 0, 2)).reshape(L, n_kv_heads, G, d).sum(axis=2)
+        dv[a:b] = np.transpose(dvh, (1, 0, 2)).reshape(L, n_kv_heads, G, d).sum(axis=2)
+        # rotate: transpose of the rotation
+        dq[a:b] = rope_backward(np.transpose(dqh, (1, 0, 2)), p, rope_theta)
+        dk[a:b] = rope_backward(dkr, p, rope_theta)
+    return dq, dk, dv
