@@ -104,3 +104,45 @@ def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_abi, "_lib", None)
     with pytest.raises(ImportError):
         _abi.load()
+
+
+def test_decode_workspace_size():
+    ws = _abi.decode_workspace_size(32, 4097, 32, 8, 128)
+    assert ws > 0 and ws % 256 == 0
+    # partial outputs of at least one key range per (sequence, KV head)
+    assert ws >= 32 * 8 * 4 * 128 * 4
+    assert _abi.decode_workspace_size(32, 4097, 32, 8, 96) == 0      # head_dim
+    assert _abi.decode_workspace_size(32, 4097, 32, 1, 128) == 0     # group of 32 > 16
+    assert _abi.decode_workspace_size(32, 4097, 30, 8, 128) == 0     # not a multiple
+    assert _abi.decode_workspace_size(32, 0, 32, 8, 128) == 0        # empty cache
+    assert _abi.decode_workspace_size(-1, 4097, 32, 8, 128) == 0
+    assert _abi.decode_workspace_size(0, 4097, 32, 8, 128) > 0       # empty batch: a no-op still accepted
+
+
+def dcall(**kw):
+    args = dict(q=A, k_new=A, v_new=A, k_cache=A, v_cache=A, cache_seqlens=A, rope_theta=1e4, batch=4,
+                max_cache_len=100, n_q_heads=8, n_kv_heads=2, head_dim=64, out=A, lse=0, workspace=A,
+                workspace_bytes=1 << 30, stream=None)
+    args.update(kw)
+    return _abi.gqa_rope_attn_decode(**args)
+
+
+def test_decode_host_rejections_before_any_cuda_call():
+    E = _abi
+    assert dcall(batch=0) == E.GQA_OK  # no-op
+    assert dcall(batch=-1) == E.GQA_ERR_INVALID_ARG
+    assert dcall(max_cache_len=0) == E.GQA_ERR_INVALID_ARG
+    assert dcall(n_q_heads=6, n_kv_heads=4) == E.GQA_ERR_INVALID_ARG
+    assert dcall(rope_theta=0.0) == E.GQA_ERR_INVALID_ARG
+    assert dcall(rope_theta=float("nan")) == E.GQA_ERR_INVALID_ARG
+    assert dcall(head_dim=96) == E.GQA_ERR_UNSUPPORTED
+    assert dcall(n_q_heads=64, n_kv_heads=2) == E.GQA_ERR_UNSUPPORTED  # group of 32
+    assert dcall(batch=70000) == E.GQA_ERR_UNSUPPORTED
+    assert dcall(q=0) == E.GQA_ERR_INVALID_ARG
+    assert dcall(k_cache=0) == E.GQA_ERR_INVALID_ARG
+    assert dcall(cache_seqlens=0) == E.GQA_ERR_INVALID_ARG
+    assert dcall(out=A + 8) == E.GQA_ERR_INVALID_ARG      # 16-byte alignment
+    assert dcall(lse=A + 2) == E.GQA_ERR_INVALID_ARG      # 4-byte alignment
+    assert dcall(workspace=0) == E.GQA_ERR_WORKSPACE
+    assert dcall(workspace=A + 16) == E.GQA_ERR_WORKSPACE  # 256-byte alignment
+    assert dcall(workspace_bytes=16) == E.GQA_ERR_WORKSPACE
