@@ -11,9 +11,9 @@
 // One persistent CTA per SM takes work items (sequence, q-tile, KV head)
 // from a longest-first list: its first item statically, every further one
 // from a global counter (greedy list scheduling, so that faster CTAs take
-// more items), or, for short lists, from a static alternating deal. A q-tile packs tq = 128 / G tokens
-// times the G query heads of one KV head into 128 MMA rows, so every K/V
-// tile loaded by TMA is used by all G heads at once.
+// more items), or, for short lists, from a static alternating deal. A q-tile
+// packs tq = 128 / G tokens times the G query heads of one KV head into 128
+// MMA rows, so every K/V tile loaded by TMA is used by all G heads at once.
 //
 // Warp roles (512 threads):
 //   warp 0      TMA producer: K tiles (K is RoPE'd already); work items
