@@ -33,7 +33,9 @@ constexpr int DEC_THREADS = 256;
 constexpr int DEC_KT = 64;      // keys per tile
 constexpr int DEC_STAGES = 2;
 constexpr int DEC_GMAX = 16;    // query heads per KV head
-constexpr int DEC_TARGET_CTAS = 256;   // split count aims at about this many CTAs (measured: fewer, longer CTAs amortise the per-CTA RoPE setup)
+// The split count aims at about this many CTAs over the batch (measured:
+// fewer, longer CTAs amortise the per-CTA RoPE setup).
+constexpr int DEC_TARGET_CTAS = 256;
 
 struct DecodeParams {
   const __nv_bfloat16* q;        // [B, nq, d]

@@ -445,14 +445,21 @@ extern "C" int gqa_rope_attn_fwd(const void* q, const void* k, const void* v, co
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   int rc;
   std::lock_guard<std::mutex> lk(g_mu);  // descriptor cache
+#define GQA_FWD_CASE(KEY, DD, FP)                                                                           \
+  case KEY:                                                                                                 \
+    rc = launch<DD, FP>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads,     \
+                        n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count);                       \
+    break;
   switch (head_dim * 2 + (fp32 ? 1 : 0)) {
-    case 64: rc = launch<32, false>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count); break;
-    case 65: rc = launch<32, true>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count); break;
-    case 128: rc = launch<64, false>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count); break;
-    case 129: rc = launch<64, true>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count); break;
-    case 256: rc = launch<128, false>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count); break;
-    default: rc = launch<128, true>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count); break;
+    GQA_FWD_CASE(64, 32, false)
+    GQA_FWD_CASE(65, 32, true)
+    GQA_FWD_CASE(128, 64, false)
+    GQA_FWD_CASE(129, 64, true)
+    GQA_FWD_CASE(256, 128, false)
+    GQA_FWD_CASE(257, 128, true)
+    default: rc = GQA_ERR_UNSUPPORTED; break;
   }
+#undef GQA_FWD_CASE
   return rc;
 }
 
