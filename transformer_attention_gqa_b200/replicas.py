@@ -27,10 +27,14 @@ def init(backend: str = "nccl", timeout_s: float = 120.0) -> None:
 
 
 def barrier() -> None:
+    import torch
     import torch.distributed as dist
 
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
-        dist.barrier()
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[torch.cuda.current_device()])  # the rank's own GPU, set by the caller
+        else:
+            dist.barrier()
 
 
 def max_over_ranks(values: Sequence[float], device=None) -> list:
@@ -55,5 +59,5 @@ def shutdown() -> None:
     import torch.distributed as dist
 
     if dist.is_available() and dist.is_initialized():
-        dist.barrier()
+        barrier()
         dist.destroy_process_group()
