@@ -82,6 +82,7 @@ struct PrepParams {
   const int* cu;
   int N, num_seqs, nq, nkv, tq, causal;
   double theta;
+  double inv_freq[64];  // theta^(-2i/d), i < d/2, evaluated once on the host
   int* header;
   int* seq_pfx;
   int2* pairs;

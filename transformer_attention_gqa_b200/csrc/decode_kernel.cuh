@@ -49,6 +49,7 @@ struct DecodeParams {
   __nv_bfloat16* out;            // [B, nq, d]
   float* lse;                    // [nq, B] or null
   double theta;
+  double inv_freq[64];           // theta^(-2i/d), i < d/2, evaluated once on the host
   int B, Lmax, nq, nkv, G, splits, kps;  // kps: keys per split, a multiple of DEC_KT
   float scale_log2;              // log2(e) / sqrt(d)
 };
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2)
   __nv_bfloat16* vnew = knew + D;
   for (int i = tid; i < D / 2; i += DEC_THREADS) {
     double sd, cd;
-    sincos((double)pos * pow(p.theta, -(2.0 * i) / D), &sd, &cd);
+    sincos((double)pos * p.inv_freq[i], &sd, &cd);
     cs[i] = make_float2((float)cd, (float)sd);
   }
   __syncthreads();

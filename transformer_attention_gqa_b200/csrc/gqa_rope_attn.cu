@@ -150,6 +150,7 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
   pp.tq = tq;
   pp.causal = causal;
   pp.theta = theta;
+  for (int i = 0; i < D / 2; ++i) pp.inv_freq[i] = std::pow(theta, -(2.0 * i) / D);
   pp.header = reinterpret_cast<int*>(ws + lay.header);
   pp.seq_pfx = reinterpret_cast<int*>(ws + lay.seq_pfx);
   pp.pairs = reinterpret_cast<int2*>(ws + lay.pairs);
@@ -297,6 +298,7 @@ int launch_decode(const void* q, const void* k_new, const void* v_new, void* k_c
   dp.out = reinterpret_cast<__nv_bfloat16*>(out);
   dp.lse = lse;
   dp.theta = theta;
+  for (int i = 0; i < D / 2; ++i) dp.inv_freq[i] = std::pow(theta, -(2.0 * i) / D);
   dp.B = B;
   dp.Lmax = Lmax;
   dp.nq = nq;

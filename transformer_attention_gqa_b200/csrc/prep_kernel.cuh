@@ -171,9 +171,6 @@ template <int D, bool FP32_IN>
 __device__ void rope_k_and_table(const PrepParams& p, int block, int nblocks) {
   constexpr int HALF = D / 2;
   constexpr int PAIRS = HALF / 2;  // each thread handles frequencies i, i+1
-  __shared__ double s_invf[HALF];
-  for (int i = threadIdx.x; i < HALF; i += PREP_THREADS) s_invf[i] = pow(p.theta, -(2.0 * i) / D);
-  __syncthreads();
 
   const long long total = (long long)p.N * PAIRS;
   for (long long idx = (long long)block * PREP_THREADS + threadIdx.x; idx < total;
@@ -215,7 +212,7 @@ __device__ void rope_k_and_table(const PrepParams& p, int block, int nblocks) {
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       double sd, cd;
-      sincos((double)pos * s_invf[i + e], &sd, &cd);
+      sincos((double)pos * p.inv_freq[i + e], &sd, &cd);
       c[e] = (float)cd;
       sn[e] = (float)sd;
     }
