@@ -14,8 +14,26 @@ def _ptr(t):
     return 0 if t is None else int(t.data_ptr())
 
 
+def _check(cond: bool, msg: str) -> None:
+    if not cond:
+        raise ValueError(msg)
+
+
+def _check_tensors(named: dict, device) -> None:
+    """Every given tensor is a contiguous CUDA tensor on `device`: the library
+    receives raw device addresses and cannot tell a host pointer or a
+    strided view from a valid operand."""
+    for name, t in named.items():
+        if t is None:
+            continue
+        _check(t.is_cuda, f"{name} must be a CUDA tensor")
+        _check(t.device == device, f"{name} is on {t.device}, expected {device}")
+        _check(t.is_contiguous(), f"{name} must be contiguous")
+
+
 class Workspace:
-    """Reusable device scratch for gqa_rope_attn_fwd (grown on demand)."""
+    """Reusable device scratch for gqa_rope_attn_fwd / gqa_rope_attn_decode
+    (grown on demand) on `device`, by default the current CUDA device."""
 
     def __init__(self, device=None):
         self.device = device
@@ -23,6 +41,8 @@ class Workspace:
 
     def get(self, nbytes: int):
         import torch
+        if self.device is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
         if self.buf is None or self.buf.numel() < nbytes:
             self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
         return self.buf
@@ -39,6 +59,7 @@ def gqa_rope_attn_fwd(q, k, v, cu_seqlens, rope_theta: float, positions=None, ca
     """
     import torch
 
+    _check(q.dim() == 3 and k.dim() == 3, "q must be [N, n_q, d] and k, v [N, n_kv, d]")
     N, nq, d = q.shape
     nkv = k.shape[1]
     if q.dtype == torch.bfloat16:
@@ -47,18 +68,26 @@ def gqa_rope_attn_fwd(q, k, v, cu_seqlens, rope_theta: float, positions=None, ca
         dt = _abi.GQA_DTYPE_FP32
     else:
         raise TypeError("q must be bfloat16 or float32")
-    for t in (q, k, v, cu_seqlens) + ((positions,) if positions is not None else ()):
-        if not t.is_contiguous():
-            raise ValueError("inputs must be contiguous")
+    _check(k.shape == (N, nkv, d) and v.shape == (N, nkv, d), "k and v must be [N, n_kv, d] matching q")
+    _check(k.dtype == q.dtype and v.dtype == q.dtype, "q, k and v must share one dtype")
+    _check(cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1 and cu_seqlens.numel() >= 1,
+           "cu_seqlens must be a 1-D int32 tensor")
+    if positions is not None:
+        _check(positions.dtype == torch.int32 and positions.shape == (N,), "positions must be int32 [N]")
     num_seqs = cu_seqlens.numel() - 1
     if out is None:
         out = torch.empty_like(q)
     if lse is None and need_lse:
         lse = torch.empty((nq, N), dtype=torch.float32, device=q.device)
+    _check(out.shape == q.shape and out.dtype == q.dtype, "out must match q's shape and dtype")
+    if lse is not None:
+        _check(lse.shape == (nq, N) and lse.dtype == torch.float32, "lse must be float32 [n_q, N]")
+    _check_tensors(dict(q=q, k=k, v=v, cu_seqlens=cu_seqlens, positions=positions, out=out, lse=lse), q.device)
     nbytes = workspace_size(num_seqs, N, nq, nkv, d, dt)
     if workspace is None:
         workspace = Workspace(q.device)
     ws = workspace.get(nbytes) if isinstance(workspace, Workspace) else workspace
+    _check_tensors(dict(workspace=ws), q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     rc = _abi.gqa_rope_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(positions), rope_theta, _ptr(cu_seqlens), num_seqs,
@@ -83,22 +112,31 @@ def gqa_rope_attn_decode(q, k_new, v_new, k_cache, v_cache, cache_seqlens, rope_
     """
     import torch
 
+    _check(q.dim() == 3 and k_new.dim() == 3 and k_cache.dim() == 4,
+           "q must be [B, n_q, d], k_new/v_new [B, n_kv, d], caches [B, max_len, n_kv, d]")
     B, nq, d = q.shape
     nkv = k_new.shape[1]
     Lmax = k_cache.shape[1]
-    for t in (q, k_new, v_new, k_cache, v_cache, cache_seqlens):
-        if not t.is_contiguous():
-            raise ValueError("inputs must be contiguous")
     if any(t.dtype != torch.bfloat16 for t in (q, k_new, v_new, k_cache, v_cache)):
         raise TypeError("decode tensors must be bfloat16")
+    _check(k_new.shape == (B, nkv, d) and v_new.shape == (B, nkv, d), "k_new and v_new must be [B, n_kv, d]")
+    _check(k_cache.shape == (B, Lmax, nkv, d) and v_cache.shape == k_cache.shape,
+           "k_cache and v_cache must be [B, max_len, n_kv, d]")
+    _check(cache_seqlens.dtype == torch.int32 and cache_seqlens.shape == (B,), "cache_seqlens must be int32 [B]")
     if out is None:
         out = torch.empty_like(q)
     if lse is None and need_lse:
         lse = torch.empty((nq, B), dtype=torch.float32, device=q.device)
+    _check(out.shape == q.shape and out.dtype == q.dtype, "out must match q's shape and dtype")
+    if lse is not None:
+        _check(lse.shape == (nq, B) and lse.dtype == torch.float32, "lse must be float32 [n_q, B]")
+    _check_tensors(dict(q=q, k_new=k_new, v_new=v_new, k_cache=k_cache, v_cache=v_cache,
+                        cache_seqlens=cache_seqlens, out=out, lse=lse), q.device)
     nbytes = decode_workspace_size(B, Lmax, nq, nkv, d)
     if workspace is None:
         workspace = Workspace(q.device)
     ws = workspace.get(nbytes) if isinstance(workspace, Workspace) else workspace
+    _check_tensors(dict(workspace=ws), q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     rc = _abi.gqa_rope_attn_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
