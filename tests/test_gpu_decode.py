@@ -135,3 +135,23 @@ def test_decode_workspace_reuse_with_garbage():
         buf.fill_(0xFF)  # NaN patterns everywhere
         t, out, lse = _run(inp, workspace=ws)
         _check(inp, t, out, lse, what=f"reuse {rep}")
+
+
+def test_decode_timeout_is_reported_and_the_context_stays_usable(monkeypatch):
+    """Failure detection without a fault: with the test hook set, the first
+    K/V tile of every key range is never loaded; each CTA's bounded wait (2 s)
+    runs out, the CTA drains what it issued and exits, and the status word
+    reads GQA_ERR_TIMEOUT. The next call must then be correct."""
+    import torch
+    import transformer_attention_gqa_b200 as g
+
+    w = wl.DecodeWorkload("timeout", (100, 5), 128, 8, 2, 64, 1e4, seed=12)
+    inp = wl.make_decode_inputs(w)
+    t = _dev(inp)
+    monkeypatch.setenv("GQA_ROPE_ATTN_TEST_DROP_FIRST_LOAD", "1")
+    g.gqa_rope_attn_decode(t["q"], t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], t["lens"], w.rope_theta)
+    torch.cuda.synchronize()
+    assert g.get_device_status() == 5
+    monkeypatch.delenv("GQA_ROPE_ATTN_TEST_DROP_FIRST_LOAD")
+    t2, out, lse = _run(inp)
+    _check(inp, t2, out, lse, what="after a timeout")

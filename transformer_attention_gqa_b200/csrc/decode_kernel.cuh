@@ -51,6 +51,7 @@ struct DecodeParams {
   double theta;
   double inv_freq[64];           // theta^(-2i/d), i < d/2, evaluated once on the host
   int B, Lmax, nq, nkv, G, splits, kps;  // kps: keys per split, a multiple of DEC_KT
+  int test_drop_first_load;      // failure-detection test: never issue the first tile's load (0 normally)
   float scale_log2;              // log2(e) / sqrt(d)
 };
 
@@ -179,7 +180,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 2)
     }
   };
   if (tid == 0)
-    for (int t = 0; t < min(DEC_STAGES, ntiles); ++t) issue(t);
+    for (int t = 0; t < min(DEC_STAGES, ntiles); ++t)
+      if (!(p.test_drop_first_load && t == 0)) issue(t);
 
   // ---- RoPE at position pos: cos/sin (float64 angle, fp32 values, as in the
   // prefill), the G queries of KV head h, and the new key if this range

@@ -7,6 +7,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -307,6 +308,11 @@ int launch_decode(const void* q, const void* k_new, const void* v_new, void* k_c
   dp.splits = lay.splits;
   dp.kps = lay.kps;
   dp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  // Failure-detection test hook (off unless the variable is set to 1): the
+  // first K/V tile of every key range is never loaded, so each CTA's bounded
+  // wait runs out and the status word reads GQA_ERR_TIMEOUT.
+  const char* drop = std::getenv("GQA_ROPE_ATTN_TEST_DROP_FIRST_LOAD");
+  dp.test_drop_first_load = (drop && drop[0] == '1' && drop[1] == '\0') ? 1 : 0;
 
   if (t_prof_ev[0] && cudaEventRecord(t_prof_ev[0], stream) != cudaSuccess) return GQA_ERR_CUDA;
   gqa_decode_split_kernel<D, GM><<<dim3(lay.splits, nkv, B), DEC_THREADS, C::SMEM_BYTES, stream>>>(tmK, tmV, dp);
