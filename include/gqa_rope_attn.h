@@ -23,8 +23,8 @@
  *     batches (cu_seqlens prefix sums).
  *   The log-sum-exp output is not on the pages; it is the natural-log
  *   normaliser of each row's scaled, masked scores.
- * A decoding step against a KV cache (gqa_rope_attn_decode) is declared
- * further down.
+ * A decoding step against a KV cache (gqa_rope_attn_decode) and the
+ * backward (gqa_rope_attn_bwd) are declared further down.
  *
  * Precision: q, k, v, out are bf16 (or fp32 with dtype GQA_DTYPE_FP32; then
  * q, k, v are rounded to bf16 on load and out is written as fp32). cos/sin
@@ -213,12 +213,54 @@ int gqa_rope_attn_decode(const void* q, const void* k_new, const void* v_new, vo
                          int n_q_heads, int n_kv_heads, int head_dim, void* out, float* lse, void* workspace,
                          size_t workspace_bytes, void* stream);
 
-/* Measurement aid. Arms the calling thread's next gqa_rope_attn_fwd or
- * gqa_rope_attn_decode call to record three CUDA events (cudaEvent_t passed
- * as void*, any may be NULL) on its stream: before its first kernel, between
- * its two kernels, and after the second, so that each kernel's
- * duration can be read with cudaEventElapsedTime. The arming is consumed by
- * that one call (also when it fails). The caller owns the events. */
+/* ---- Backward (gradients of the prefill) --------------------------------
+ *
+ * The chain rule through the forward's steps ("Attention from Scratch",
+ * section "Attention, the math"), for a loss with gradient dout = dL/dout:
+ *
+ *   P  = exp(S - lse),  S = rope(q) rope(k)^T / sqrt(d) + mask (per head)
+ *   dv = sum over the G heads of a group of P^T dout
+ *   dS = P * (dout v^T - Delta),  Delta[t, h] = sum_c dout[t, h, c] out[t, h, c]
+ *   dq = rope^T(dS rope(k) / sqrt(d)),  dk = rope^T(sum over the group of dS^T rope(q) / sqrt(d))
+ *
+ * where rope^T rotates each pair (i, i + d/2) by the negative angle (the
+ * transpose of the rotation). lse and out are the forward's outputs for the
+ * same q, k, v (lse is required: P is recomputed from it, not stored). The
+ * rotated q and k are rounded to bf16 exactly as the forward rounds them; the
+ * gradient passes that rounding unchanged. P and dS enter their products as
+ * bf16; every product accumulates in fp32; dq accumulates over key tiles in
+ * fp32 in the workspace.
+ *
+ * All of q, k, v, out, dout, dq, dk, dv are bf16 in the forward's layout
+ * (q, out, dout, dq: [total_tokens, n_q_heads, head_dim]; k, v, dk, dv:
+ * [total_tokens, n_kv_heads, head_dim]), contiguous device memory, 16-byte
+ * aligned; lse is fp32 [n_q_heads, total_tokens]. positions, rope_theta,
+ * cu_seqlens, num_seqs, total_tokens, the head counts, head_dim and causal
+ * are those of the forward call and obey its rules (a bad cu_seqlens sets
+ * GQA_ERR_BAD_SEQLENS in the status word; dk and dv are then not written).
+ * dq, dk and dv are overwritten (not accumulated into). workspace: at least
+ * gqa_rope_attn_bwd_workspace_size() bytes, 256-byte aligned, contents need
+ * not be initialised, not shared by calls that may overlap. Three kernels
+ * are queued on `stream`; the call does not wait. Returns GQA_OK or an
+ * error code; on an error nothing has been queued.
+ */
+size_t gqa_rope_attn_bwd_workspace_size(int num_seqs, int total_tokens, int n_q_heads, int n_kv_heads,
+                                        int head_dim);
+
+int gqa_rope_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                      const void* dout, const int32_t* positions, double rope_theta,
+                      const int32_t* cu_seqlens, int num_seqs, int total_tokens, int n_q_heads,
+                      int n_kv_heads, int head_dim, int causal, void* dq, void* dk, void* dv,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Measurement aid. Arms the calling thread's next gqa_rope_attn_fwd,
+ * gqa_rope_attn_decode or gqa_rope_attn_bwd call to record three CUDA events
+ * (cudaEvent_t passed as void*, any may be NULL) on its stream: before its
+ * first kernel, between its first two kernels, and after the second, so
+ * that each kernel's duration can be read with cudaEventElapsedTime (the
+ * backward's third kernel, the dq rotation, runs after the last event). The
+ * arming is consumed by that one call (also when it fails). The caller owns
+ * the events. */
 void gqa_rope_attn_set_profile_events(void* ev_start, void* ev_mid, void* ev_end);
 
 #ifdef __cplusplus

@@ -146,3 +146,46 @@ def test_decode_host_rejections_before_any_cuda_call():
     assert dcall(workspace=0) == E.GQA_ERR_WORKSPACE
     assert dcall(workspace=A + 16) == E.GQA_ERR_WORKSPACE  # 256-byte alignment
     assert dcall(workspace_bytes=16) == E.GQA_ERR_WORKSPACE
+
+
+def test_bwd_workspace_size():
+    ws = _abi.bwd_workspace_size(1, 8192, 32, 8, 128)
+    assert ws % 256 == 0
+    # at least K' (n_kv * N * d * 2), Q' (N * n_q * d * 2) and the fp32 dq accumulator (N * n_q * d * 4)
+    assert ws >= 8 * 8192 * 128 * 2 + 8192 * 32 * 128 * 6
+    assert _abi.bwd_workspace_size(1, 8192, 32, 8, 96) == 0
+    assert _abi.bwd_workspace_size(1, 8192, 30, 8, 128) == 0
+    assert _abi.bwd_workspace_size(1, 8192, 256, 1, 128) == 0
+    assert _abi.bwd_workspace_size(-1, 8192, 32, 8, 128) == 0
+    assert _abi.bwd_workspace_size(2, 100, 4, 2, 64) < _abi.bwd_workspace_size(2, 200, 4, 2, 64)
+
+
+def bcall(**kw):
+    args = dict(q=A, k=A, v=A, out=A, lse=A, dout=A, positions=0, rope_theta=1e4, cu_seqlens=A, num_seqs=1,
+                total_tokens=128, n_q_heads=4, n_kv_heads=2, head_dim=64, causal=1, dq=A, dk=A, dv=A, workspace=0,
+                workspace_bytes=0, stream=None)
+    args.update(kw)
+    return _abi.gqa_rope_attn_bwd(**args)
+
+
+def test_bwd_host_rejections_before_any_cuda_call():
+    E = _abi
+    assert bcall(total_tokens=0) == E.GQA_OK  # no-op
+    assert bcall(total_tokens=-1) == E.GQA_ERR_INVALID_ARG
+    assert bcall(n_q_heads=6, n_kv_heads=4) == E.GQA_ERR_INVALID_ARG
+    assert bcall(causal=2) == E.GQA_ERR_INVALID_ARG
+    assert bcall(rope_theta=-1.0) == E.GQA_ERR_INVALID_ARG
+    assert bcall(head_dim=80) == E.GQA_ERR_UNSUPPORTED
+    assert bcall(n_q_heads=256, n_kv_heads=1) == E.GQA_ERR_UNSUPPORTED
+    assert bcall(num_seqs=0) == E.GQA_ERR_INVALID_ARG
+    for name in ("q", "k", "v", "out", "lse", "dout", "cu_seqlens", "dq", "dk", "dv"):
+        assert bcall(**{name: 0}) == E.GQA_ERR_INVALID_ARG, name
+    for name in ("q", "k", "v", "out", "dout", "dq", "dk", "dv"):
+        assert bcall(**{name: A + 8}) == E.GQA_ERR_INVALID_ARG, name  # 16-byte alignment
+    assert bcall(lse=A + 2) == E.GQA_ERR_INVALID_ARG
+    assert bcall(positions=A + 2) == E.GQA_ERR_INVALID_ARG
+    assert bcall() == E.GQA_ERR_WORKSPACE
+    need = _abi.bwd_workspace_size(1, 128, 4, 2, 64)
+    assert bcall(workspace=A, workspace_bytes=need - 1) == E.GQA_ERR_WORKSPACE
+    assert bcall(workspace=A + 16, workspace_bytes=need) == E.GQA_ERR_WORKSPACE
+    assert _abi.last_launch_count() == 0

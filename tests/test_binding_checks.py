@@ -81,3 +81,39 @@ def test_decode_rejects_other_dtypes():
     q, kn, vn, kc, vc, lens = _dec_args()
     with pytest.raises(TypeError):
         g.gqa_rope_attn_decode(q.float(), kn, vn, kc, vc, lens, 1e4)
+
+
+def _bwd_args(N=16, nq=4, nkv=2, d=32):
+    bf = torch.bfloat16
+    q, k, v, cu = _fwd_args(N, nq, nkv, d)
+    return q, k, v, torch.zeros(N, nq, d, dtype=bf), torch.zeros(nq, N), torch.zeros(N, nq, d, dtype=bf), cu
+
+
+def test_bwd_rejects_host_tensors():
+    q, k, v, out, lse, dout, cu = _bwd_args()
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        g.gqa_rope_attn_bwd(q, k, v, out, lse, dout, cu, 1e4)
+
+
+@pytest.mark.parametrize("bad", ["lse_shape", "lse_dtype", "dout_shape", "dk_shape", "positions"])
+def test_bwd_rejects_inconsistent_arguments(bad):
+    q, k, v, out, lse, dout, cu = _bwd_args()
+    kw = {}
+    if bad == "lse_shape":
+        lse = torch.zeros(16, 4)
+    elif bad == "lse_dtype":
+        lse = lse.double()
+    elif bad == "dout_shape":
+        dout = dout[:8]
+    elif bad == "dk_shape":
+        kw["dk"] = torch.zeros(16, 4, 32, dtype=torch.bfloat16)
+    elif bad == "positions":
+        kw["positions"] = torch.zeros(16, dtype=torch.int64)
+    with pytest.raises(ValueError):
+        g.gqa_rope_attn_bwd(q, k, v, out, lse, dout, cu, 1e4, **kw)
+
+
+def test_bwd_rejects_other_dtypes():
+    q, k, v, out, lse, dout, cu = _bwd_args()
+    with pytest.raises(TypeError):
+        g.gqa_rope_attn_bwd(q.float(), k.float(), v.float(), out.float(), lse, dout.float(), cu, 1e4)

@@ -4,10 +4,10 @@ PyTorch-facing binding. PyTorch provides device memory and streams only."""
 from __future__ import annotations
 
 from . import _abi
-from ._abi import GqaError, workspace_size, decode_workspace_size, get_device_status  # noqa: F401
+from ._abi import GqaError, workspace_size, decode_workspace_size, bwd_workspace_size, get_device_status  # noqa: F401
 
-__all__ = ["gqa_rope_attn_fwd", "gqa_rope_attn_decode", "workspace_size", "decode_workspace_size",
-           "get_device_status", "GqaError", "Workspace"]
+__all__ = ["gqa_rope_attn_fwd", "gqa_rope_attn_decode", "gqa_rope_attn_bwd", "workspace_size",
+           "decode_workspace_size", "bwd_workspace_size", "get_device_status", "GqaError", "Workspace"]
 
 
 def _ptr(t):
@@ -32,8 +32,9 @@ def _check_tensors(named: dict, device) -> None:
 
 
 class Workspace:
-    """Reusable device scratch for gqa_rope_attn_fwd / gqa_rope_attn_decode
-    (grown on demand) on `device`, by default the current CUDA device."""
+    """Reusable device scratch for gqa_rope_attn_fwd / gqa_rope_attn_decode /
+    gqa_rope_attn_bwd (grown on demand) on `device`, by default the current
+    CUDA device."""
 
     def __init__(self, device=None):
         self.device = device
@@ -145,3 +146,51 @@ def gqa_rope_attn_decode(q, k_new, v_new, k_cache, v_cache, cache_seqlens, rope_
     if rc != _abi.GQA_OK:
         raise GqaError(rc, "gqa_rope_attn_decode")
     return out, lse
+
+
+def gqa_rope_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, rope_theta: float, positions=None, causal: bool = True,
+                      dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of sum(dout * out) for out, lse =
+    gqa_rope_attn_fwd(q, k, v, cu_seqlens, rope_theta, positions, causal).
+
+    q, out, dout: [N, n_q, d]; k, v: [N, n_kv, d] -- bf16 CUDA tensors; lse:
+    fp32 [n_q, N], the forward's; cu_seqlens and positions as for the
+    forward. Returns bf16 dq [N, n_q, d], dk and dv [N, n_kv, d] (written
+    into dq/dk/dv when given). Raises GqaError on a non-OK status.
+    """
+    import torch
+
+    _check(q.dim() == 3 and k.dim() == 3, "q must be [N, n_q, d] and k, v [N, n_kv, d]")
+    N, nq, d = q.shape
+    nkv = k.shape[1]
+    if any(t.dtype != torch.bfloat16 for t in (q, k, v, out, dout)):
+        raise TypeError("q, k, v, out and dout must be bfloat16")
+    _check(k.shape == (N, nkv, d) and v.shape == (N, nkv, d), "k and v must be [N, n_kv, d] matching q")
+    _check(out.shape == q.shape and dout.shape == q.shape, "out and dout must match q's shape")
+    _check(lse.shape == (nq, N) and lse.dtype == torch.float32, "lse must be float32 [n_q, N]")
+    _check(cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1 and cu_seqlens.numel() >= 1,
+           "cu_seqlens must be a 1-D int32 tensor")
+    if positions is not None:
+        _check(positions.dtype == torch.int32 and positions.shape == (N,), "positions must be int32 [N]")
+    num_seqs = cu_seqlens.numel() - 1
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(dq.shape == q.shape and dq.dtype == q.dtype, "dq must match q's shape and dtype")
+    _check(dk.shape == k.shape and dk.dtype == k.dtype and dv.shape == v.shape and dv.dtype == v.dtype,
+           "dk and dv must match k's and v's shapes and dtype")
+    _check_tensors(dict(q=q, k=k, v=v, out=out, lse=lse, dout=dout, cu_seqlens=cu_seqlens, positions=positions,
+                        dq=dq, dk=dk, dv=dv), q.device)
+    nbytes = bwd_workspace_size(num_seqs, N, nq, nkv, d)
+    if workspace is None:
+        workspace = Workspace(q.device)
+    ws = workspace.get(nbytes) if isinstance(workspace, Workspace) else workspace
+    _check_tensors(dict(workspace=ws), q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    rc = _abi.gqa_rope_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(positions),
+                                rope_theta, _ptr(cu_seqlens), num_seqs, N, nq, nkv, d, 1 if causal else 0,
+                                _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel() * ws.element_size(), stream)
+    if rc != _abi.GQA_OK:
+        raise GqaError(rc, "gqa_rope_attn_bwd")
+    return dq, dk, dv

@@ -34,6 +34,8 @@ EXPORTED = (
     "gqa_rope_attn_fwd_noalloc",
     "gqa_rope_attn_decode_workspace_size",
     "gqa_rope_attn_decode",
+    "gqa_rope_attn_bwd_workspace_size",
+    "gqa_rope_attn_bwd",
 )
 
 _lib = None
@@ -77,6 +79,12 @@ def load() -> ctypes.CDLL:
     lib.gqa_rope_attn_decode.restype = c_int
     lib.gqa_rope_attn_decode.argtypes = [c_void, c_void, c_void, c_void, c_void, c_void, c_double, c_int, c_int,
                                          c_int, c_int, c_int, c_void, c_void, c_void, c_size, c_void]
+    lib.gqa_rope_attn_bwd_workspace_size.restype = c_size
+    lib.gqa_rope_attn_bwd_workspace_size.argtypes = [c_int] * 5
+    lib.gqa_rope_attn_bwd.restype = c_int
+    lib.gqa_rope_attn_bwd.argtypes = [c_void, c_void, c_void, c_void, c_void, c_void, c_void, c_double, c_void,
+                                      c_int, c_int, c_int, c_int, c_int, c_int, c_void, c_void, c_void, c_void,
+                                      c_size, c_void]
     lib.gqa_rope_attn_set_profile_events.restype = None
     lib.gqa_rope_attn_set_profile_events.argtypes = [c_void, c_void, c_void]
     _lib = lib
@@ -122,6 +130,20 @@ def gqa_rope_attn_decode(q, k_new, v_new, k_cache, v_cache, cache_seqlens, rope_
                                            int(head_dim), out, lse, workspace, int(workspace_bytes), stream))
 
 
+def bwd_workspace_size(num_seqs: int, total_tokens: int, n_q_heads: int, n_kv_heads: int, head_dim: int) -> int:
+    return int(load().gqa_rope_attn_bwd_workspace_size(num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim))
+
+
+def gqa_rope_attn_bwd(q, k, v, out, lse, dout, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads,
+                      n_kv_heads, head_dim, causal, dq, dk, dv, workspace, workspace_bytes, stream) -> int:
+    """Raw call of the backward; integer device addresses (0 for NULL);
+    returns the status."""
+    return int(load().gqa_rope_attn_bwd(q, k, v, out, lse, dout, positions, float(rope_theta), cu_seqlens,
+                                        int(num_seqs), int(total_tokens), int(n_q_heads), int(n_kv_heads),
+                                        int(head_dim), int(causal), dq, dk, dv, workspace, int(workspace_bytes),
+                                        stream))
+
+
 def get_device_status(stream=None) -> int:
     return int(load().gqa_rope_attn_get_device_status(stream))
 
@@ -136,5 +158,5 @@ def last_launch_count() -> int:
 
 def set_profile_events(ev_start=None, ev_mid=None, ev_end=None) -> None:
     """Arm the next call on this thread to record the given cudaEvent_t
-    handles (ints) around its two kernels."""
+    handles (ints) around its first two kernels."""
     load().gqa_rope_attn_set_profile_events(ev_start, ev_mid, ev_end)

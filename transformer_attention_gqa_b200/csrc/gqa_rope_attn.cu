@@ -1,7 +1,8 @@
 // Host side of the C ABI (include/gqa_rope_attn.h): argument checks, TMA
 // descriptor cache, the two launches of the fused forward (prologue, then
-// the attention kernel, in stream order) and the two of the decoding step
-// (key-range kernel, then the merge).
+// the attention kernel, in stream order), the two of the decoding step
+// (key-range kernel, then the merge) and the three of the backward
+// (prologue, attention backward, dq rotation).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -13,6 +14,7 @@
 
 #include "../../include/gqa_rope_attn.h"
 #include "attn_kernel.cuh"
+#include "bwd_kernel.cuh"
 #include "common.cuh"
 #include "decode_kernel.cuh"
 #include "prep_kernel.cuh"
@@ -28,6 +30,7 @@ struct DeviceState {
   int sm_count = 0;
   bool attr_set[3][2] = {};
   bool dec_attr_set[3][3] = {};
+  bool bwd_attr_set[3] = {};
 };
 
 std::mutex g_mu;
@@ -325,6 +328,120 @@ int launch_decode(const void* q, const void* k_new, const void* v_new, void* k_c
   return GQA_OK;
 }
 
+// ---------------------------------------------------------------- backward
+
+template <int D>
+int launch_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+               const int32_t* positions, double theta, const int32_t* cu, int num_seqs, int N, int nq, int nkv,
+               int causal, void* dq, void* dk, void* dv, uint8_t* ws, const BwdWsLayout& lay, cudaStream_t stream,
+               int device, int sm_count) {
+  using C = BwdCfg<D>;
+  const int G = nq / nkv;
+  const int tq = tokens_per_tile(G);
+  {  // caller holds g_mu
+    DeviceState& ds = g_dev[device];
+    if (!ds.bwd_attr_set[dim_index(D)]) {
+      if (cudaFuncSetAttribute(gqa_attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_BYTES) != cudaSuccess)
+        return GQA_ERR_CUDA;
+      ds.bwd_attr_set[dim_index(D)] = true;
+    }
+  }
+  BwdPrepParams pp{};
+  pp.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  pp.k = reinterpret_cast<const __nv_bfloat16*>(k);
+  pp.out = reinterpret_cast<const __nv_bfloat16*>(out);
+  pp.dout = reinterpret_cast<const __nv_bfloat16*>(dout);
+  pp.lse = lse;
+  pp.positions = positions;
+  pp.cu = cu;
+  pp.N = N;
+  pp.num_seqs = num_seqs;
+  pp.nq = nq;
+  pp.nkv = nkv;
+  pp.tq = tq;
+  pp.causal = causal;
+  for (int i = 0; i < D / 2; ++i) pp.inv_freq[i] = std::pow(theta, -(2.0 * i) / D);
+  pp.header = reinterpret_cast<int*>(ws + lay.header);
+  pp.seq_pfx = reinterpret_cast<int*>(ws + lay.seq_pfx);
+  pp.pairs = reinterpret_cast<int2*>(ws + lay.pairs);
+  pp.table = reinterpret_cast<float2*>(ws + lay.table);
+  pp.kws = reinterpret_cast<__nv_bfloat16*>(ws + lay.kws);
+  pp.qws = reinterpret_cast<__nv_bfloat16*>(ws + lay.qws);
+  pp.lse2 = reinterpret_cast<float*>(ws + lay.lse2);
+  pp.delta = reinterpret_cast<float*>(ws + lay.delta);
+  pp.dq_acc = reinterpret_cast<float*>(ws + lay.dq_acc);
+
+  // Q' and dO: [N][nq][d], box (BOXC, G heads, tq tokens); K': [nkv][N][d],
+  // box (BOXC, BN keys, 1); V: [N][nkv][d], box (BOXC, 1, BN keys).
+  CUtensorMap tmQ, tmDO, tmK, tmV;
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)nq, (uint64_t)N};
+    const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)nq * D * 2};
+    const uint32_t box[3] = {(uint32_t)C::BOXC, (uint32_t)G, (uint32_t)tq};
+    if (!make_tmap(device, ws + lay.qws, dims, str, box, C::ROWB, &tmQ)) return GQA_ERR_CUDA;
+    if (!make_tmap(device, dout, dims, str, box, C::ROWB, &tmDO)) return GQA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)N, (uint64_t)nkv};
+    const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)N * D * 2};
+    const uint32_t box[3] = {(uint32_t)C::BOXC, (uint32_t)BN, 1u};
+    if (!make_tmap(device, ws + lay.kws, dims, str, box, C::ROWB, &tmK)) return GQA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)nkv, (uint64_t)N};
+    const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)nkv * D * 2};
+    const uint32_t box[3] = {(uint32_t)C::BOXC, 1u, (uint32_t)BN};
+    if (!make_tmap(device, v, dims, str, box, C::ROWB, &tmV)) return GQA_ERR_CUDA;
+  }
+
+  const long long work = (long long)N * (D / 4);
+  long long nb = (work + PREP_THREADS - 1) / PREP_THREADS;
+  const long long cap = (long long)sm_count * 8;
+  if (nb > cap) nb = cap;
+  if (nb < 1) nb = 1;
+  if (t_prof_ev[0] && cudaEventRecord(t_prof_ev[0], stream) != cudaSuccess) return GQA_ERR_CUDA;
+  gqa_bwd_prep_kernel<D><<<(unsigned)(nb + 1), PREP_THREADS, 0, stream>>>(pp);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+  if (t_prof_ev[1] && cudaEventRecord(t_prof_ev[1], stream) != cudaSuccess) return GQA_ERR_CUDA;
+
+  BwdParams bp{};
+  bp.cu = cu;
+  bp.header = pp.header;
+  bp.pairs = pp.pairs;
+  bp.table = pp.table;
+  bp.lse2 = pp.lse2;
+  bp.delta = pp.delta;
+  bp.dq_acc = pp.dq_acc;
+  bp.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+  bp.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+  bp.N = N;
+  bp.nq = nq;
+  bp.nkv = nkv;
+  bp.G = G;
+  bp.tq = tq;
+  bp.causal = causal;
+  bp.scale = (float)(1.0 / std::sqrt((double)D));
+  bp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  // one CTA per (sequence, key tile, KV head); CTAs past the prologue's
+  // pair count exit at once
+  const unsigned grid = (unsigned)(lay.max_pairs * (long long)nkv);
+  gqa_attn_bwd_kernel<D><<<grid, BWD_THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmDO, bp);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+  if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;
+
+  const long long rows4 = (long long)N * nq * (D / 8);
+  long long nbq = (rows4 + PREP_THREADS - 1) / PREP_THREADS;
+  if (nbq > cap) nbq = cap;
+  if (nbq < 1) nbq = 1;
+  gqa_bwd_dq_kernel<D><<<(unsigned)nbq, PREP_THREADS, 0, stream>>>(pp.dq_acc, pp.table,
+                                                                 reinterpret_cast<__nv_bfloat16*>(dq), N, nq,
+                                                                 bp.scale);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+  t_last_launches = 3;
+  return GQA_OK;
+}
+
 }  // namespace
 }  // namespace gqa
 
@@ -545,4 +662,73 @@ extern "C" void gqa_rope_attn_set_profile_events(void* ev_start, void* ev_mid, v
   t_prof_ev[0] = reinterpret_cast<cudaEvent_t>(ev_start);
   t_prof_ev[1] = reinterpret_cast<cudaEvent_t>(ev_mid);
   t_prof_ev[2] = reinterpret_cast<cudaEvent_t>(ev_end);
+}
+
+// ---------------------------------------------------------------------------
+// Backward
+
+extern "C" size_t gqa_rope_attn_bwd_workspace_size(int num_seqs, int total_tokens, int n_q_heads, int n_kv_heads,
+                                                   int head_dim) {
+  if (num_seqs < 0 || total_tokens < 0 || n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return 0;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return 0;
+  if (n_q_heads / n_kv_heads > BM) return 0;
+  return bwd_ws_layout(num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim).total;
+}
+
+extern "C" int gqa_rope_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                                 const void* dout, const int32_t* positions, double rope_theta,
+                                 const int32_t* cu_seqlens, int num_seqs, int total_tokens, int n_q_heads,
+                                 int n_kv_heads, int head_dim, int causal, void* dq, void* dk, void* dv,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  t_last_launches = 0;
+  struct Disarm {
+    ~Disarm() { t_prof_ev[0] = t_prof_ev[1] = t_prof_ev[2] = nullptr; }
+  } disarm;
+  if (total_tokens < 0 || num_seqs < 0) return GQA_ERR_INVALID_ARG;
+  if (n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return GQA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return GQA_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.0) || !std::isfinite(rope_theta)) return GQA_ERR_INVALID_ARG;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED;
+  if (n_q_heads / n_kv_heads > BM) return GQA_ERR_UNSUPPORTED;
+  if ((long long)total_tokens * n_q_heads * head_dim > (1ll << 40)) return GQA_ERR_UNSUPPORTED;
+  if (total_tokens == 0) return GQA_OK;
+  if (num_seqs < 1) return GQA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !lse || !dout || !cu_seqlens || !dq || !dk || !dv) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv))
+    return GQA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(positions) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return GQA_ERR_INVALID_ARG;
+  const BwdWsLayout lay = bwd_ws_layout(num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim);
+  if (lay.max_pairs * (long long)n_kv_heads > 0x7fffffffll) return GQA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < lay.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return GQA_ERR_WORKSPACE;
+
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices) return GQA_ERR_CUDA;
+  int sm_count = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState& ds = g_dev[device];
+    if (!ds.init) {
+      int major = 0;
+      if (cudaDeviceGetAttribute(&ds.sm_count, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+          cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess)
+        return GQA_ERR_CUDA;
+      if (major != 10) return GQA_ERR_UNSUPPORTED;
+      ds.init = true;
+    }
+    sm_count = ds.sm_count;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  std::lock_guard<std::mutex> lk(g_mu);  // descriptor cache
+#define GQA_BWD_CASE(DD)                                                                                        \
+  if (head_dim == DD)                                                                                           \
+    return launch_bwd<DD>(q, k, v, out, lse, dout, positions, rope_theta, cu_seqlens, num_seqs, total_tokens,  \
+                          n_q_heads, n_kv_heads, causal, dq, dk, dv, ws, lay, st, device, sm_count);
+  GQA_BWD_CASE(32) GQA_BWD_CASE(64) GQA_BWD_CASE(128)
+#undef GQA_BWD_CASE
+  return GQA_ERR_UNSUPPORTED;
 }

@@ -189,6 +189,14 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Inputs:
     return Inputs(w, q, k, v, cu, pos)
 
 
+def make_grad_output(inp: Inputs, seed: int = 1) -> np.ndarray:
+    """Seeded upstream gradient dL/dout for the backward: standard normal
+    values rounded to bf16, shape [N, n_q, d] like out."""
+    w = inp.workload
+    rng = np.random.default_rng(w.seed * 7919 + seed)
+    return to_bf16_values(rng.standard_normal((w.total_tokens, w.n_q_heads, w.head_dim), dtype=np.float32))
+
+
 # ---------------------------------------------------------------- decoding
 
 @dataclass(frozen=True)
