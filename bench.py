@@ -9,6 +9,8 @@ in HBM. Default workload: Llama-3-8B-shaped causal prefill (B=1, T=8192,
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   (the float64 CPU oracle, timed)
+  --workload decode_llama8b | decode_qwen3b | ...   one decoding step
+  --workload bwd_llama8b | bwd_varlen | bwd_nano    the backward (dq, dk, dv)
 
 Under torchrun each rank runs its own replica of the workload (independent
 problems, weak scaling); the elapsed time is the max over ranks.
@@ -347,6 +349,208 @@ def run_decode(args, rank, world, local_rank):
     return res
 
 
+# ------------------------------------------------------------------ backward
+# Backward workloads: the gradients of a forward workload's shape. One step =
+# one gqa_rope_attn_bwd call (prologue, attention backward, dq rotation) on
+# the forward's out and lse, computed once before timing.
+BWD_WORKLOADS = {"bwd_llama8b": "llama8b", "bwd_varlen": "varlen", "bwd_nano": "nano"}
+BWD_METRIC = "causal GQA+RoPE attention bwd (dq, dk, dv) TFLOP/s on 1 B200; % of dense-BF16 tensor peak"
+BWD_FLOP_FACTOR = 2.5  # five products of the forward's two sizes (S recomputed, dP, dV, dK, dQ)
+
+
+def cpu_baseline_bwd(w, budget_s: float = 15.0, max_len: int = 1024):
+    """Times the float64 oracle's backward, as it stands, on a prefix of the
+    workload's first sequence (its length sized by two probes to about
+    budget_s, at most max_len tokens: the oracle holds [n_q, L, L] float64
+    matrices); returns TFLOP/s by the backward's convention."""
+    import oracle.gqa_oracle as orc
+    from transformer_attention_gqa_b200 import workloads as wl
+
+    inp = _cached_inputs(w)
+    dout = wl.make_grad_output(inp)
+    first = int(inp.cu_seqlens[1])
+
+    def run(L):
+        cu = np.array([0, L], dtype=np.int64)
+        t0 = time.perf_counter()
+        orc.gqa_rope_attention_backward(inp.q[:L], inp.k[:L], inp.v[:L], dout[:L], cu, w.n_q_heads, w.n_kv_heads,
+                                        w.rope_theta, causal=w.causal, operand_rounding=True)
+        return time.perf_counter() - t0
+
+    L0 = min(first, 128)
+    t0 = run(L0)
+    L = int(max(L0, min(first, max_len, L0 * np.sqrt(max(budget_s, 0.1) / max(t0, 1e-3)))))
+    dt = run(L)
+    flops = BWD_FLOP_FACTOR * 4.0 * L * L * w.head_dim * w.n_q_heads / (2.0 if w.causal else 1.0)
+    cores = len(os.sched_getaffinity(0))
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"first {L} tokens of {w.name}'s first sequence, all {w.n_q_heads} heads, float64 NumPy, "
+                      f"{dt:.1f} s"}
+
+
+def run_bwd(args, rank, world, local_rank):
+    import torch
+    import transformer_attention_gqa_b200 as g
+    from transformer_attention_gqa_b200 import _abi, replicas, workloads as wl
+    from cuda.bindings import runtime as rt
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = wl.WORKLOADS[BWD_WORKLOADS[args.workload]]
+    inp = wl.make_inputs(w, seed=w.seed if rank == 0 else replicas.replica_seed(w.seed, rank))
+    bf = torch.bfloat16
+    q = torch.from_numpy(inp.q).to(bf).to(dev)
+    k = torch.from_numpy(inp.k).to(bf).to(dev)
+    v = torch.from_numpy(inp.v).to(bf).to(dev)
+    do = torch.from_numpy(wl.make_grad_output(inp)).to(bf).to(dev)
+    cu = torch.from_numpy(inp.cu_seqlens).to(dev)
+    out, lse = g.gqa_rope_attn_fwd(q, k, v, cu, w.rope_theta, causal=w.causal)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = g.Workspace(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        g.gqa_rope_attn_bwd(q, k, v, out, lse, do, cu, w.rope_theta, causal=w.causal, dq=dq, dk=dk, dv=dv,
+                            workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert g.get_device_status() == 0
+    launches_per_step = _abi.last_launch_count()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    replicas.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    replicas.barrier()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+
+    def _ev():
+        err, e = rt.cudaEventCreate()
+        assert int(err) == 0
+        return e
+
+    def _ms(a, b):
+        err, ms = rt.cudaEventElapsedTime(a, b)
+        assert int(err) == 0
+        return float(ms)
+
+    kern = []
+    for _ in range(max(3, min(args.steps, 10))):
+        e = [_ev() for _ in range(3)]
+        flush.zero_()
+        _abi.set_profile_events(int(e[0]), int(e[1]), int(e[2]))
+        step()
+        kern.append(e)
+    torch.cuda.synchronize()
+    prep_ms = statistics.median(_ms(a, b) for a, b, _ in kern)
+    bwd_ms = statistics.median(_ms(b, c) for _, b, c in kern)
+    for e in kern:
+        for x in e:
+            rt.cudaEventDestroy(x)
+    clk = clocks.stop()
+
+    # end to end: q, k, v, out, lse, dout and cu_seqlens from pinned host
+    # memory every step, dq, dk, dv back
+    hosts = [t.cpu().pin_memory() for t in (q, k, v, out, lse, do, cu)]
+    devs = (q, k, v, out, lse, do, cu)
+    backs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+    h2d = sum(t.numel() * t.element_size() for t in hosts)
+    d2h = sum(t.numel() * t.element_size() for t in backs)
+
+    def e2e_step():
+        for d_, h_ in zip(devs, hosts):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        for h_, d_ in zip(backs, (dq, dk, dv)):
+            h_.copy_(d_, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    replicas.barrier()
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    assert g.get_device_status() == 0
+    assert torch.equal(backs[0], dq.cpu())
+
+    total_ms, e2e_ms, bwd_ms, prep_ms = replicas.max_over_ranks([total_ms, e2e_ms, bwd_ms, prep_ms], device=dev)
+    flops = BWD_FLOP_FACTOR * w.flops()
+    ms_per_step = total_ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (bwd_ms * 1e-3) / 1e12
+    res = {
+        "metric": BWD_METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "shape": w.description, "total_tokens": w.total_tokens,
+                   "num_seqs": w.num_seqs, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+                   "head_dim": w.head_dim, "rope_theta": w.rope_theta, "causal": w.causal,
+                   "flops_per_step": flops, "parallelism": f"replicas x{world}",
+                   "l2": "256 MiB written before every timed step, outside the step's events"},
+        "pct_of_peak": round(100.0 * value / world / peak, 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{src} bf16_tflops (burst)", "kernel": "gqa_attn_bwd_kernel",
+                     "kernel_ms": round(bwd_ms, 4), "prologue_ms": round(prep_ms, 4)},
+        "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if clk:
+        res["clocks"] = clk
+    return res
+
+
+def main_bwd(args, world, rank, local_rank):
+    from transformer_attention_gqa_b200 import workloads as wl
+    w = wl.WORKLOADS[BWD_WORKLOADS[args.workload]]
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cpu_baseline_bwd(w, budget_s=0.5)
+        vals, info = [], None
+        for _ in range(args.steps):
+            info = cpu_baseline_bwd(w, budget_s=max(1.0, min(5.0, 60.0 / max(args.steps, 1))))
+            vals.append(info["value"])
+        val = statistics.median(vals)
+        print(json.dumps({"impl": "reference", "metric": BWD_METRIC, "value": round(val, 6), "unit": UNIT,
+                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": {"workload": args.workload, "shape": w.description},
+                          "cpu_baseline": {"value": round(val, 6), "unit": UNIT, "cores": info["cores"],
+                                           "kind": "oracle", "sample": info["sample"]},
+                          "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return 0
+    from transformer_attention_gqa_b200 import replicas
+    replicas.init("nccl", timeout_s=120)
+    res = run_bwd(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_bwd(w, budget_s=args.cpu_budget)
+    replicas.shutdown()
+    if rank == 0:
+        print(json.dumps(res))
+    return 0
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -535,6 +739,8 @@ def main():
     from transformer_attention_gqa_b200 import workloads as wl
     if args.workload in wl.DECODE_WORKLOADS:
         return main_decode(args, world, rank, local_rank)
+    if args.workload in BWD_WORKLOADS:
+        return main_bwd(args, world, rank, local_rank)
     w = wl.WORKLOADS[args.workload]
 
     if args.impl == "reference":
