@@ -345,7 +345,8 @@ struct BwdCfg {
   static constexpr int OFF_Q = OFF_V + TILE_BYTES;   // two stages
   static constexpr int OFF_DO = OFF_Q + 2 * TILE_BYTES;  // two stages
   static constexpr int OFF_DS = DS_IN_DO ? OFF_DO : OFF_DO + 2 * TILE_BYTES;
-  static constexpr int OFF_ST = OFF_DS + (DS_IN_DO ? 0 : DS_BYTES);  // float [2 stages][lse2, Delta][128]
+  // float [2 stages][lse2, Delta][128], after the dO stages and the dS buffer
+  static constexpr int OFF_ST = DS_IN_DO ? OFF_DO + 2 * TILE_BYTES : OFF_DS + DS_BYTES;
   static constexpr int OFF_BAR = OFF_ST + 2 * 2 * BM * 4;
   static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM_USED = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
@@ -366,6 +367,13 @@ struct BwdCfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(DK_COL + D <= TMEM_COLS, "tensor memory budget");
   static_assert(OFF_DS % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_DO % 1024 == 0, "swizzle atoms 1024-aligned");
+  // regions in order, none overlapping the next
+  static_assert(OFF_V >= OFF_K + TILE_BYTES && OFF_Q >= OFF_V + TILE_BYTES && OFF_DO >= OFF_Q + 2 * TILE_BYTES,
+                "K', V, Q' regions overlap");
+  static_assert(DS_IN_DO ? (OFF_DS == OFF_DO && DS_BYTES <= TILE_BYTES) : OFF_DS >= OFF_DO + 2 * TILE_BYTES,
+                "dS region");
+  static_assert(OFF_ST >= OFF_DO + 2 * TILE_BYTES && OFF_ST >= OFF_DS + DS_BYTES, "statistics overlap dO or dS");
+  static_assert(OFF_BAR >= OFF_ST + 2 * 2 * BM * 4, "barriers overlap the statistics");
 };
 
 struct BwdBarriers {
