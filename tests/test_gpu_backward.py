@@ -8,12 +8,7 @@ writes bf16 gradients (relative 2^-9). The products sum O(100-1000) terms of
 either sign (dS sums to zero over the keys of a row), so the rounding errors
 average instead of adding up, and each gradient stays within a few 2^-9
 of its own scale: max |gpu - ref| <= 3e-2 * max |ref| and
-mean |gpu - ref| <= 1e-2 * mean |ref|, per gradient.
-
-Opt-in (GQA_BWD_GPU_TESTS=1) until the kernels have had their first
-supervised run on a B200."""
-import os
-
+mean |gpu - ref| <= 1e-2 * mean |ref|, per gradient."""
 import numpy as np
 import pytest
 
@@ -22,12 +17,7 @@ from tests.conftest import gpu_available
 from tests import gpu_helpers as H
 from transformer_attention_gqa_b200 import workloads as wl
 
-pytestmark = [
-    pytest.mark.gpu,
-    pytest.mark.skipif(not gpu_available(), reason="needs a CUDA device"),
-    pytest.mark.skipif(os.environ.get("GQA_BWD_GPU_TESTS") != "1",
-                       reason="backward kernels not yet run on a GPU: opt in with GQA_BWD_GPU_TESTS=1"),
-]
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not gpu_available(), reason="needs a CUDA device")]
 
 MAX_REL = 3e-2
 MEAN_REL = 1e-2
