@@ -52,6 +52,12 @@ is kept for every token generated so far). The new token is the last row of
 the causal mask, so the step is the forward's last row; the cache holds the
 keys after rotation, each at its own position.
 
+Projection (``qkv_rope_projection``): steps 1 and 2 of the same walk-through
+for the tokens x of the residual stream: q_proj, k_proj, v_proj are linears
+without bias (y = x W^T), q_proj n_q heads wide and k_proj, v_proj n_kv heads
+wide, each output split into heads as view(tokens, heads, head_dim); then Q
+and K are rotated and V is not.
+
 Backward (``gqa_rope_attention_backward``): the gradients of the forward's
 output with respect to q, k, v for an upstream gradient dout, i.e. of the
 scalar sum(dout * out). It is the training-time counterpart of the forward
@@ -84,6 +90,7 @@ __all__ = [
     "gqa_rope_decode",
     "rope_backward",
     "gqa_rope_attention_backward",
+    "qkv_rope_projection",
 ]
 
 
@@ -457,3 +464,48 @@ def gqa_rope_attention_backward(q, k, v, dout, cu_seqlens, n_q_heads: int, n_kv_
         dq[a:b] = rope_backward(np.transpose(dqh, (1, 0, 2)), p, rope_theta)
         dk[a:b] = rope_backward(dkr, p, rope_theta)
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------
+# Projection ("Attention from Scratch", section "Attention, the math", steps
+# 1 Project and 2 Rotate)
+# ---------------------------------------------------------------------------
+
+def qkv_rope_projection(x, w_q, w_k, w_v, n_q_heads: int, n_kv_heads: int, rope_theta: float, positions=None,
+                        cu_seqlens=None, operand_rounding: bool = False):
+    """q = rope(x W_q^T), k = rope(x W_k^T), v = x W_v^T for tokens x [N, C].
+
+    W_q: [n_q * d, C]; W_k, W_v: [n_kv * d, C] (the linear layers' weight
+    layout, out_features x in_features). Feature h*d + c of a projection is
+    column c of head h. Each token is rotated by positions[t] if given, else
+    by its index inside its sequence of ``cu_seqlens`` if given, else by t.
+    Returns q [N, n_q, d], k [N, n_kv, d], v [N, n_kv, d] in float64. With
+    ``operand_rounding`` the rotation takes the fp32 cos/sin table and every
+    output is rounded once, to bf16, from its float64 value (no rounding
+    between the projection and the rotation)."""
+    x = np.asarray(x, dtype=np.float64)
+    w_q = np.asarray(w_q, dtype=np.float64)
+    w_k = np.asarray(w_k, dtype=np.float64)
+    w_v = np.asarray(w_v, dtype=np.float64)
+    N, C = x.shape
+    d = w_q.shape[0] // n_q_heads
+    if w_q.shape != (n_q_heads * d, C) or w_k.shape != (n_kv_heads * d, C) or w_v.shape != (n_kv_heads * d, C):
+        raise ValueError("weight shapes must be [heads * head_dim, C]")
+    if positions is not None:
+        pos = np.asarray(positions, dtype=np.int64).reshape(-1)
+    elif cu_seqlens is not None:
+        cu = np.asarray(cu_seqlens, dtype=np.int64)
+        pos = np.concatenate([np.arange(cu[i + 1] - cu[i]) for i in range(len(cu) - 1)] + [np.zeros(0)])
+    else:
+        pos = np.arange(N)
+    if pos.shape != (N,):
+        raise ValueError("one position per token")
+    # 1. Project: y = x W^T, then split the features into heads.
+    yq = np.matmul(x, w_q.T).reshape(N, n_q_heads, d)
+    yk = np.matmul(x, w_k.T).reshape(N, n_kv_heads, d)
+    yv = np.matmul(x, w_v.T).reshape(N, n_kv_heads, d)
+    # 2. Rotate Q and K, never V.
+    q = apply_rope(yq, pos, rope_theta, operand_rounding)
+    k = apply_rope(yk, pos, rope_theta, operand_rounding)
+    v = round_to_bf16(yv) if operand_rounding else yv
+    return q, k, v
