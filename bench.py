@@ -11,6 +11,7 @@ in HBM. Default workload: Llama-3-8B-shaped causal prefill (B=1, T=8192,
   python bench.py --impl reference ...   (the float64 CPU oracle, timed)
   --workload decode_llama8b | decode_qwen3b | ...   one decoding step
   --workload bwd_llama8b | bwd_varlen | bwd_nano    the backward (dq, dk, dv)
+  --workload qkv_llama8b | qkv_nano                 the QKV projection with its RoPE epilogue
 
 Under torchrun each rank runs its own replica of the workload (independent
 problems, weak scaling); the elapsed time is the max over ranks.
@@ -551,6 +552,206 @@ def main_bwd(args, world, rank, local_rank):
     return 0
 
 
+# ------------------------------------------------------------------ QKV projection
+# The projection with its RoPE epilogue for a forward workload's tokens and
+# heads, hidden = n_q * d (the model width): one gqa_rope_attn_qkv_proj call
+# per step, 2 * N * hidden * (n_q + 2 n_kv) * d FLOPs.
+PROJ_WORKLOADS = {"qkv_llama8b": "llama8b", "qkv_nano": "nano"}
+PROJ_METRIC = "GQA QKV projection + RoPE epilogue TFLOP/s on 1 B200; % of dense-BF16 tensor peak"
+
+
+def _proj_shape(w):
+    return w.n_q_heads * w.head_dim, (w.n_q_heads + 2 * w.n_kv_heads) * w.head_dim
+
+
+def cpu_baseline_proj(w, inp, budget_s: float = 15.0):
+    """Times the float64 oracle's projection, as it stands, on the first n
+    tokens (n sized by a probe to about budget_s); returns TFLOP/s."""
+    import oracle.gqa_oracle as orc
+
+    C, F = _proj_shape(w)
+    f, fk = w.n_q_heads * w.head_dim, w.n_kv_heads * w.head_dim
+    W = inp.w_qkv
+
+    def run(n):
+        t0 = time.perf_counter()
+        orc.qkv_rope_projection(inp.x[:n], W[:f], W[f:f + fk], W[f + fk:], w.n_q_heads, w.n_kv_heads, w.rope_theta,
+                                positions=inp.positions[:n])
+        return time.perf_counter() - t0
+
+    n0 = min(w.total_tokens, 64)
+    t0 = run(n0)
+    n = int(max(n0, min(w.total_tokens, n0 * budget_s / max(t0, 1e-3))))
+    dt = run(n)
+    return {"value": 2.0 * n * C * F / dt / 1e12, "unit": UNIT, "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle", "sample": f"first {n} tokens of {w.name} (hidden {C}, {F} output features), "
+                                        f"float64 NumPy, {dt:.1f} s"}
+
+
+def run_proj(args, rank, world, local_rank, inp):
+    import torch
+    import transformer_attention_gqa_b200 as g
+    from transformer_attention_gqa_b200 import _abi, replicas, workloads as wl
+    from cuda.bindings import runtime as rt
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = wl.WORKLOADS[PROJ_WORKLOADS[args.workload]]
+    C, F = _proj_shape(w)
+    bf = torch.bfloat16
+    x = torch.from_numpy(inp.x).to(bf).to(dev)
+    wq = torch.from_numpy(inp.w_qkv).to(bf).to(dev)
+    cu = torch.from_numpy(inp.cu_seqlens).to(dev)
+    N = w.total_tokens
+    q = torch.empty((N, w.n_q_heads, w.head_dim), dtype=bf, device=dev)
+    k = torch.empty((N, w.n_kv_heads, w.head_dim), dtype=bf, device=dev)
+    v = torch.empty_like(k)
+    ws = g.Workspace(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        g.gqa_rope_attn_qkv_proj(x, wq, w.n_q_heads, w.n_kv_heads, w.rope_theta, cu_seqlens=cu, q=q, k=k, v=v,
+                                 workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert g.get_device_status() == 0
+    launches_per_step = _abi.last_launch_count()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    replicas.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    replicas.barrier()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+
+    def _ev():
+        err, e = rt.cudaEventCreate()
+        assert int(err) == 0
+        return e
+
+    def _ms(a, b):
+        err, ms = rt.cudaEventElapsedTime(a, b)
+        assert int(err) == 0
+        return float(ms)
+
+    kern = []
+    for _ in range(max(3, min(args.steps, 10))):
+        e = [_ev() for _ in range(3)]
+        flush.zero_()
+        _abi.set_profile_events(int(e[0]), int(e[1]), int(e[2]))
+        step()
+        kern.append(e)
+    torch.cuda.synchronize()
+    table_ms = statistics.median(_ms(a, b) for a, b, _ in kern)
+    proj_ms = statistics.median(_ms(b, c) for _, b, c in kern)
+    for e in kern:
+        for t in e:
+            rt.cudaEventDestroy(t)
+    clk = clocks.stop()
+
+    # end to end: x and cu_seqlens from pinned host memory every step (the
+    # weights stay resident), q, k, v back
+    xh, cuh = x.cpu().pin_memory(), cu.cpu().pin_memory()
+    backs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (q, k, v)]
+    h2d = xh.numel() * xh.element_size() + cuh.numel() * cuh.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in backs)
+
+    def e2e_step():
+        x.copy_(xh, non_blocking=True)
+        cu.copy_(cuh, non_blocking=True)
+        step()
+        for h_, d_ in zip(backs, (q, k, v)):
+            h_.copy_(d_, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    replicas.barrier()
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    assert g.get_device_status() == 0
+    assert torch.equal(backs[0], q.cpu())
+
+    total_ms, e2e_ms, proj_ms, table_ms = replicas.max_over_ranks([total_ms, e2e_ms, proj_ms, table_ms], device=dev)
+    flops = 2.0 * N * C * F
+    ms_per_step = total_ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (proj_ms * 1e-3) / 1e12
+    res = {
+        "metric": PROJ_METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "shape": w.description, "total_tokens": N, "hidden": C,
+                   "out_features": F, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+                   "head_dim": w.head_dim, "rope_theta": w.rope_theta, "flops_per_step": flops,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "256 MiB written before every timed step, outside the step's events"},
+        "pct_of_peak": round(100.0 * value / world / peak, 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{src} bf16_tflops (burst)", "kernel": "gqa_qkv_proj_kernel",
+                     "kernel_ms": round(proj_ms, 4), "table_ms": round(table_ms, 4)},
+        "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if clk:
+        res["clocks"] = clk
+    return res
+
+
+def main_proj(args, world, rank, local_rank):
+    from transformer_attention_gqa_b200 import replicas, workloads as wl
+    w = wl.WORKLOADS[PROJ_WORKLOADS[args.workload]]
+    C, _ = _proj_shape(w)
+    seed = w.seed if rank == 0 else replicas.replica_seed(w.seed, rank)
+    inp = wl.make_projection_inputs(w.seq_lens, C, w.n_q_heads, w.n_kv_heads, w.head_dim, w.rope_theta, seed=seed)
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cpu_baseline_proj(w, inp, budget_s=0.5)
+        vals, info = [], None
+        for _ in range(args.steps):
+            info = cpu_baseline_proj(w, inp, budget_s=max(1.0, min(5.0, 60.0 / max(args.steps, 1))))
+            vals.append(info["value"])
+        val = statistics.median(vals)
+        print(json.dumps({"impl": "reference", "metric": PROJ_METRIC, "value": round(val, 6), "unit": UNIT,
+                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": {"workload": args.workload, "shape": w.description},
+                          "cpu_baseline": {"value": round(val, 6), "unit": UNIT, "cores": info["cores"],
+                                           "kind": "oracle", "sample": info["sample"]},
+                          "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return 0
+    replicas.init("nccl", timeout_s=120)
+    res = run_proj(args, rank, world, local_rank, inp)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_proj(w, inp, budget_s=args.cpu_budget)
+    replicas.shutdown()
+    if rank == 0:
+        print(json.dumps(res))
+    return 0
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -741,6 +942,8 @@ def main():
         return main_decode(args, world, rank, local_rank)
     if args.workload in BWD_WORKLOADS:
         return main_bwd(args, world, rank, local_rank)
+    if args.workload in PROJ_WORKLOADS:
+        return main_proj(args, world, rank, local_rank)
     w = wl.WORKLOADS[args.workload]
 
     if args.impl == "reference":

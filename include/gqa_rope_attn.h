@@ -23,8 +23,9 @@
  *     batches (cu_seqlens prefix sums).
  *   The log-sum-exp output is not on the pages; it is the natural-log
  *   normaliser of each row's scaled, masked scores.
- * A decoding step against a KV cache (gqa_rope_attn_decode) and the
- * backward (gqa_rope_attn_bwd) are declared further down.
+ * A decoding step against a KV cache (gqa_rope_attn_decode), the backward
+ * (gqa_rope_attn_bwd) and the QKV projection with its RoPE epilogue
+ * (gqa_rope_attn_qkv_proj) are declared further down.
  *
  * Precision: q, k, v, out are bf16 (or fp32 with dtype GQA_DTYPE_FP32; then
  * q, k, v are rounded to bf16 on load and out is written as fp32). cos/sin
@@ -253,8 +254,46 @@ int gqa_rope_attn_bwd(const void* q, const void* k, const void* v, const void* o
                       int n_kv_heads, int head_dim, int causal, void* dq, void* dk, void* dv,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- QKV projection with the RoPE epilogue -------------------------------
+ *
+ * Steps 1 and 2 of the attention module ("Attention from Scratch", section
+ * "Attention, the math": Project, then Rotate) for tokens x of the residual
+ * stream, with the three bias-free linear layers stacked into one weight:
+ *
+ *   [q | k | v] = x W_qkv^T,   W_qkv = [W_q; W_k; W_v]
+ *   q[t, h, :] = rope(row t of x W_q^T, head h),  k likewise,  v not rotated
+ *
+ * Feature h * head_dim + c of each projection is column c of head h. RoPE
+ * is that of gqa_rope_attn_fwd (feature i rotated with i + d/2 by
+ * position * theta^(-2i/d)); the rotation is applied to the fp32
+ * accumulator and rounded once to bf16 (no rounding in between).
+ *
+ *   x          [total_tokens, hidden] bf16
+ *   w_qkv      [(n_q_heads + 2 n_kv_heads) head_dim, hidden] bf16, the rows
+ *              of W_q, then W_k, then W_v (out_features x in_features)
+ *   positions  int32 [total_tokens] or NULL: then each token's index inside
+ *              its sequence of cu_seqlens ([num_seqs + 1], as for the
+ *              forward; required when positions is NULL)
+ *   q          [total_tokens, n_q_heads, head_dim] bf16, rotated
+ *   k, v       [total_tokens, n_kv_heads, head_dim] bf16, k rotated
+ * All device memory, contiguous, 16-byte aligned; hidden a multiple of 8;
+ * head_dim 32, 64 or 128; n_q_heads a multiple of n_kv_heads. workspace: at
+ * least gqa_rope_attn_qkv_proj_workspace_size() bytes (the cos/sin table),
+ * 256-byte aligned. Two kernels are queued on `stream`; the call does not
+ * wait. Returns GQA_OK or an error code; on an error nothing has been queued.
+ * The outputs feed gqa_rope_attn_fwd only through its unrotated inputs: q
+ * and k leave this call already rotated.
+ */
+size_t gqa_rope_attn_qkv_proj_workspace_size(int total_tokens, int head_dim);
+
+int gqa_rope_attn_qkv_proj(const void* x, const void* w_qkv, const int32_t* positions, double rope_theta,
+                           const int32_t* cu_seqlens, int num_seqs, int total_tokens, int hidden,
+                           int n_q_heads, int n_kv_heads, int head_dim, void* q, void* k, void* v,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* Measurement aid. Arms the calling thread's next gqa_rope_attn_fwd,
- * gqa_rope_attn_decode or gqa_rope_attn_bwd call to record three CUDA events
+ * gqa_rope_attn_decode, gqa_rope_attn_bwd or gqa_rope_attn_qkv_proj call to
+ * record three CUDA events
  * (cudaEvent_t passed as void*, any may be NULL) on its stream: before its
  * first kernel, between its first two kernels, and after the second, so
  * that each kernel's duration can be read with cudaEventElapsedTime (the

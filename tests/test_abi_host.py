@@ -189,3 +189,38 @@ def test_bwd_host_rejections_before_any_cuda_call():
     assert bcall(workspace=A, workspace_bytes=need - 1) == E.GQA_ERR_WORKSPACE
     assert bcall(workspace=A + 16, workspace_bytes=need) == E.GQA_ERR_WORKSPACE
     assert _abi.last_launch_count() == 0
+
+
+def test_qkv_proj_workspace_size():
+    ws = _abi.qkv_proj_workspace_size(8192, 128)
+    assert ws >= 8192 * 64 * 8 and ws % 256 == 0
+    assert _abi.qkv_proj_workspace_size(8192, 96) == 0
+    assert _abi.qkv_proj_workspace_size(-1, 128) == 0
+
+
+def pcall(**kw):
+    args = dict(x=A, w_qkv=A, positions=0, rope_theta=1e4, cu_seqlens=A, num_seqs=1, total_tokens=128, hidden=256,
+                n_q_heads=4, n_kv_heads=2, head_dim=64, q=A, k=A, v=A, workspace=0, workspace_bytes=0, stream=None)
+    args.update(kw)
+    return _abi.gqa_rope_attn_qkv_proj(**args)
+
+
+def test_qkv_proj_host_rejections_before_any_cuda_call():
+    E = _abi
+    assert pcall(total_tokens=0) == E.GQA_OK  # no-op
+    assert pcall(total_tokens=-1) == E.GQA_ERR_INVALID_ARG
+    assert pcall(hidden=0) == E.GQA_ERR_INVALID_ARG
+    assert pcall(n_q_heads=6, n_kv_heads=4) == E.GQA_ERR_INVALID_ARG
+    assert pcall(rope_theta=float("inf")) == E.GQA_ERR_INVALID_ARG
+    assert pcall(head_dim=96) == E.GQA_ERR_UNSUPPORTED
+    assert pcall(hidden=100) == E.GQA_ERR_UNSUPPORTED  # rows not 16-byte aligned
+    for name in ("x", "w_qkv", "q", "k", "v"):
+        assert pcall(**{name: 0}) == E.GQA_ERR_INVALID_ARG, name
+        assert pcall(**{name: A + 8}) == E.GQA_ERR_INVALID_ARG, name
+    assert pcall(cu_seqlens=0) == E.GQA_ERR_INVALID_ARG        # neither positions nor cu_seqlens
+    assert pcall(cu_seqlens=0, positions=A) == E.GQA_ERR_WORKSPACE  # positions alone are enough
+    assert pcall(positions=A + 2) == E.GQA_ERR_INVALID_ARG
+    assert pcall() == E.GQA_ERR_WORKSPACE
+    need = _abi.qkv_proj_workspace_size(128, 64)
+    assert pcall(workspace=A, workspace_bytes=need - 1) == E.GQA_ERR_WORKSPACE
+    assert _abi.last_launch_count() == 0

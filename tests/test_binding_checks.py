@@ -117,3 +117,20 @@ def test_bwd_rejects_other_dtypes():
     q, k, v, out, lse, dout, cu = _bwd_args()
     with pytest.raises(TypeError):
         g.gqa_rope_attn_bwd(q.float(), k.float(), v.float(), out.float(), lse, dout.float(), cu, 1e4)
+
+
+def test_qkv_proj_rejects_host_tensors_and_bad_shapes():
+    bf = torch.bfloat16
+    x = torch.zeros(16, 64, dtype=bf)
+    w = torch.zeros((4 + 2 * 2) * 32, 64, dtype=bf)
+    cu = torch.tensor([0, 16], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        g.gqa_rope_attn_qkv_proj(x, w, 4, 2, 1e4, cu_seqlens=cu)
+    with pytest.raises(ValueError):
+        g.gqa_rope_attn_qkv_proj(x, w[:, :32], 4, 2, 1e4, cu_seqlens=cu)  # C mismatch
+    with pytest.raises(ValueError):
+        g.gqa_rope_attn_qkv_proj(x, w[:250], 4, 2, 1e4, cu_seqlens=cu)    # rows not heads x d
+    with pytest.raises(ValueError):
+        g.gqa_rope_attn_qkv_proj(x, w, 4, 2, 1e4)                          # no positions, no cu_seqlens
+    with pytest.raises(TypeError):
+        g.gqa_rope_attn_qkv_proj(x.float(), w, 4, 2, 1e4, cu_seqlens=cu)

@@ -4,10 +4,12 @@ PyTorch-facing binding. PyTorch provides device memory and streams only."""
 from __future__ import annotations
 
 from . import _abi
-from ._abi import GqaError, workspace_size, decode_workspace_size, bwd_workspace_size, get_device_status  # noqa: F401
+from ._abi import (GqaError, workspace_size, decode_workspace_size, bwd_workspace_size,  # noqa: F401
+                   qkv_proj_workspace_size, get_device_status)
 
-__all__ = ["gqa_rope_attn_fwd", "gqa_rope_attn_decode", "gqa_rope_attn_bwd", "workspace_size",
-           "decode_workspace_size", "bwd_workspace_size", "get_device_status", "GqaError", "Workspace"]
+__all__ = ["gqa_rope_attn_fwd", "gqa_rope_attn_decode", "gqa_rope_attn_bwd", "gqa_rope_attn_qkv_proj",
+           "workspace_size", "decode_workspace_size", "bwd_workspace_size", "qkv_proj_workspace_size",
+           "get_device_status", "GqaError", "Workspace"]
 
 
 def _ptr(t):
@@ -32,9 +34,8 @@ def _check_tensors(named: dict, device) -> None:
 
 
 class Workspace:
-    """Reusable device scratch for gqa_rope_attn_fwd / gqa_rope_attn_decode /
-    gqa_rope_attn_bwd (grown on demand) on `device`, by default the current
-    CUDA device."""
+    """Reusable device scratch for the library's calls (grown on demand) on
+    `device`, by default the current CUDA device."""
 
     def __init__(self, device=None):
         self.device = device
@@ -194,3 +195,50 @@ def gqa_rope_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, rope_theta: float, po
     if rc != _abi.GQA_OK:
         raise GqaError(rc, "gqa_rope_attn_bwd")
     return dq, dk, dv
+
+
+def gqa_rope_attn_qkv_proj(x, w_qkv, n_q_heads: int, n_kv_heads: int, rope_theta: float, cu_seqlens=None,
+                           positions=None, q=None, k=None, v=None, workspace=None, stream=None):
+    """q, k, v = rope(x W_q^T), rope(x W_k^T), x W_v^T split into heads, with
+    W_qkv = [W_q; W_k; W_v] ([(n_q + 2 n_kv) d, C] bf16) and x [N, C] bf16
+    CUDA tensors. Each token is rotated by positions[t] (int32 [N]) or, when
+    positions is None, by its index inside its sequence of cu_seqlens.
+    Returns bf16 q [N, n_q, d], k and v [N, n_kv, d]. Raises GqaError on a
+    non-OK status.
+    """
+    import torch
+
+    _check(x.dim() == 2 and w_qkv.dim() == 2, "x must be [N, C] and w_qkv [(n_q + 2 n_kv) d, C]")
+    if x.dtype != torch.bfloat16 or w_qkv.dtype != torch.bfloat16:
+        raise TypeError("x and w_qkv must be bfloat16")
+    N, C = x.shape
+    heads = n_q_heads + 2 * n_kv_heads
+    _check(w_qkv.shape[1] == C and w_qkv.shape[0] % heads == 0, "w_qkv must be [(n_q + 2 n_kv) d, C]")
+    d = w_qkv.shape[0] // heads
+    _check(positions is not None or cu_seqlens is not None, "give positions or cu_seqlens")
+    if positions is not None:
+        _check(positions.dtype == torch.int32 and positions.shape == (N,), "positions must be int32 [N]")
+    if cu_seqlens is not None:
+        _check(cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1 and cu_seqlens.numel() >= 1,
+               "cu_seqlens must be a 1-D int32 tensor")
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    q = torch.empty((N, n_q_heads, d), dtype=torch.bfloat16, device=x.device) if q is None else q
+    k = torch.empty((N, n_kv_heads, d), dtype=torch.bfloat16, device=x.device) if k is None else k
+    v = torch.empty((N, n_kv_heads, d), dtype=torch.bfloat16, device=x.device) if v is None else v
+    _check(q.shape == (N, n_q_heads, d) and k.shape == (N, n_kv_heads, d) and v.shape == (N, n_kv_heads, d),
+           "q, k, v must be [N, n_q, d], [N, n_kv, d], [N, n_kv, d]")
+    _check(all(t.dtype == torch.bfloat16 for t in (q, k, v)), "q, k, v must be bfloat16")
+    _check_tensors(dict(x=x, w_qkv=w_qkv, positions=positions, cu_seqlens=cu_seqlens, q=q, k=k, v=v), x.device)
+    nbytes = qkv_proj_workspace_size(N, d)
+    if workspace is None:
+        workspace = Workspace(x.device)
+    ws = workspace.get(nbytes) if isinstance(workspace, Workspace) else workspace
+    _check_tensors(dict(workspace=ws), x.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(x.device).cuda_stream
+    rc = _abi.gqa_rope_attn_qkv_proj(_ptr(x), _ptr(w_qkv), _ptr(positions), rope_theta, _ptr(cu_seqlens), num_seqs,
+                                     N, C, n_q_heads, n_kv_heads, d, _ptr(q), _ptr(k), _ptr(v), _ptr(ws),
+                                     ws.numel() * ws.element_size(), stream)
+    if rc != _abi.GQA_OK:
+        raise GqaError(rc, "gqa_rope_attn_qkv_proj")
+    return q, k, v

@@ -36,6 +36,8 @@ EXPORTED = (
     "gqa_rope_attn_decode",
     "gqa_rope_attn_bwd_workspace_size",
     "gqa_rope_attn_bwd",
+    "gqa_rope_attn_qkv_proj_workspace_size",
+    "gqa_rope_attn_qkv_proj",
 )
 
 _lib = None
@@ -85,6 +87,11 @@ def load() -> ctypes.CDLL:
     lib.gqa_rope_attn_bwd.argtypes = [c_void, c_void, c_void, c_void, c_void, c_void, c_void, c_double, c_void,
                                       c_int, c_int, c_int, c_int, c_int, c_int, c_void, c_void, c_void, c_void,
                                       c_size, c_void]
+    lib.gqa_rope_attn_qkv_proj_workspace_size.restype = c_size
+    lib.gqa_rope_attn_qkv_proj_workspace_size.argtypes = [c_int, c_int]
+    lib.gqa_rope_attn_qkv_proj.restype = c_int
+    lib.gqa_rope_attn_qkv_proj.argtypes = [c_void, c_void, c_void, c_double, c_void, c_int, c_int, c_int, c_int,
+                                           c_int, c_int, c_void, c_void, c_void, c_void, c_size, c_void]
     lib.gqa_rope_attn_set_profile_events.restype = None
     lib.gqa_rope_attn_set_profile_events.argtypes = [c_void, c_void, c_void]
     _lib = lib
@@ -142,6 +149,19 @@ def gqa_rope_attn_bwd(q, k, v, out, lse, dout, positions, rope_theta, cu_seqlens
                                         int(num_seqs), int(total_tokens), int(n_q_heads), int(n_kv_heads),
                                         int(head_dim), int(causal), dq, dk, dv, workspace, int(workspace_bytes),
                                         stream))
+
+
+def qkv_proj_workspace_size(total_tokens: int, head_dim: int) -> int:
+    return int(load().gqa_rope_attn_qkv_proj_workspace_size(total_tokens, head_dim))
+
+
+def gqa_rope_attn_qkv_proj(x, w_qkv, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, hidden, n_q_heads,
+                           n_kv_heads, head_dim, q, k, v, workspace, workspace_bytes, stream) -> int:
+    """Raw call of the QKV projection with the RoPE epilogue; integer device
+    addresses (0 for NULL); returns the status."""
+    return int(load().gqa_rope_attn_qkv_proj(x, w_qkv, positions, float(rope_theta), cu_seqlens, int(num_seqs),
+                                             int(total_tokens), int(hidden), int(n_q_heads), int(n_kv_heads),
+                                             int(head_dim), q, k, v, workspace, int(workspace_bytes), stream))
 
 
 def get_device_status(stream=None) -> int:

@@ -1,8 +1,9 @@
 // Host side of the C ABI (include/gqa_rope_attn.h): argument checks, TMA
 // descriptor cache, the two launches of the fused forward (prologue, then
 // the attention kernel, in stream order), the two of the decoding step
-// (key-range kernel, then the merge) and the three of the backward
-// (prologue, attention backward, dq rotation).
+// (key-range kernel, then the merge), the three of the backward (prologue,
+// attention backward, dq rotation) and the two of the QKV projection with
+// its RoPE epilogue (cos/sin table, projection).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -18,6 +19,7 @@
 #include "common.cuh"
 #include "decode_kernel.cuh"
 #include "prep_kernel.cuh"
+#include "proj_kernel.cuh"
 
 namespace gqa {
 
@@ -31,6 +33,7 @@ struct DeviceState {
   bool attr_set[3][2] = {};
   bool dec_attr_set[3][3] = {};
   bool bwd_attr_set[3] = {};
+  bool proj_attr_set[3] = {};
 };
 
 std::mutex g_mu;
@@ -442,6 +445,68 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   return GQA_OK;
 }
 
+// ---------------------------------------------------------------- QKV projection
+
+template <int D>
+int launch_qkv_proj(const void* x, const void* w, const int32_t* positions, double theta, const int32_t* cu,
+                    int num_seqs, int N, int C, int nq, int nkv, void* q, void* k, void* v, uint8_t* ws,
+                    cudaStream_t stream, int device, int sm_count) {
+  {  // caller holds g_mu
+    DeviceState& ds = g_dev[device];
+    if (!ds.proj_attr_set[dim_index(D)]) {
+      if (cudaFuncSetAttribute(gqa_qkv_proj_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PJ_SMEM_BYTES) != cudaSuccess)
+        return GQA_ERR_CUDA;
+      ds.proj_attr_set[dim_index(D)] = true;
+    }
+  }
+  const int F = (nq + 2 * nkv) * D;
+  // x: [N][C], box (64 of C, 128 tokens); W: [F][C], box (64 of C, 256 features)
+  CUtensorMap tmX, tmW;
+  {
+    const uint64_t dims[3] = {(uint64_t)C, (uint64_t)N, 1u};
+    const uint64_t str[2] = {(uint64_t)C * 2, (uint64_t)C * N * 2};
+    const uint32_t box[3] = {(uint32_t)PJ_BK, (uint32_t)PJ_BM, 1u};
+    if (!make_tmap(device, x, dims, str, box, 128, &tmX)) return GQA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)C, (uint64_t)F, 1u};
+    const uint64_t str[2] = {(uint64_t)C * 2, (uint64_t)C * F * 2};
+    const uint32_t box[3] = {(uint32_t)PJ_BK, (uint32_t)PJ_BN, 1u};
+    if (!make_tmap(device, w, dims, str, box, 128, &tmW)) return GQA_ERR_CUDA;
+  }
+  ProjTableParams tp{};
+  tp.positions = positions;
+  tp.cu = cu;
+  tp.N = N;
+  tp.num_seqs = num_seqs;
+  tp.half = D / 2;
+  for (int i = 0; i < D / 2; ++i) tp.inv_freq[i] = std::pow(theta, -(2.0 * i) / D);
+  tp.table = reinterpret_cast<float2*>(ws);
+  long long nb = ((long long)N * (D / 4) + PREP_THREADS - 1) / PREP_THREADS;
+  if (nb > (long long)sm_count * 8) nb = (long long)sm_count * 8;
+  if (nb < 1) nb = 1;
+  if (t_prof_ev[0] && cudaEventRecord(t_prof_ev[0], stream) != cudaSuccess) return GQA_ERR_CUDA;
+  gqa_qkv_table_kernel<<<(unsigned)nb, PREP_THREADS, 0, stream>>>(tp);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+  if (t_prof_ev[1] && cudaEventRecord(t_prof_ev[1], stream) != cudaSuccess) return GQA_ERR_CUDA;
+  ProjParams pp{};
+  pp.table = tp.table;
+  pp.q = reinterpret_cast<__nv_bfloat16*>(q);
+  pp.k = reinterpret_cast<__nv_bfloat16*>(k);
+  pp.v = reinterpret_cast<__nv_bfloat16*>(v);
+  pp.N = N;
+  pp.C = C;
+  pp.nq = nq;
+  pp.nkv = nkv;
+  const dim3 grid((unsigned)((F + PJ_BN - 1) / PJ_BN), (unsigned)((N + PJ_BM - 1) / PJ_BM), 1);
+  gqa_qkv_proj_kernel<D><<<grid, PJ_THREADS, PJ_SMEM_BYTES, stream>>>(tmX, tmW, pp);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+  if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;
+  t_last_launches = 2;
+  return GQA_OK;
+}
+
 }  // namespace
 }  // namespace gqa
 
@@ -730,5 +795,65 @@ extern "C" int gqa_rope_attn_bwd(const void* q, const void* k, const void* v, co
                           n_q_heads, n_kv_heads, causal, dq, dk, dv, ws, lay, st, device, sm_count);
   GQA_BWD_CASE(32) GQA_BWD_CASE(64) GQA_BWD_CASE(128)
 #undef GQA_BWD_CASE
+  return GQA_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------------------
+// QKV projection with the RoPE epilogue
+
+extern "C" size_t gqa_rope_attn_qkv_proj_workspace_size(int total_tokens, int head_dim) {
+  if (total_tokens < 0 || (head_dim != 32 && head_dim != 64 && head_dim != 128)) return 0;
+  return align_up((size_t)total_tokens * (head_dim / 2) * sizeof(float2), 256) + 256;
+}
+
+extern "C" int gqa_rope_attn_qkv_proj(const void* x, const void* w_qkv, const int32_t* positions, double rope_theta,
+                                      const int32_t* cu_seqlens, int num_seqs, int total_tokens, int hidden,
+                                      int n_q_heads, int n_kv_heads, int head_dim, void* q, void* k, void* v,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+  t_last_launches = 0;
+  struct Disarm {
+    ~Disarm() { t_prof_ev[0] = t_prof_ev[1] = t_prof_ev[2] = nullptr; }
+  } disarm;
+  if (total_tokens < 0 || num_seqs < 0 || hidden < 1) return GQA_ERR_INVALID_ARG;
+  if (n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return GQA_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.0) || !std::isfinite(rope_theta)) return GQA_ERR_INVALID_ARG;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED;
+  if (hidden % 8) return GQA_ERR_UNSUPPORTED;  // rows of x and W start on 16-byte boundaries
+  if ((long long)(n_q_heads + 2 * n_kv_heads) * head_dim > (1ll << 24)) return GQA_ERR_UNSUPPORTED;
+  if ((long long)total_tokens > 65535ll * PJ_BM) return GQA_ERR_UNSUPPORTED;
+  if (total_tokens == 0) return GQA_OK;
+  if (!x || !w_qkv || !q || !k || !v) return GQA_ERR_INVALID_ARG;
+  if (!positions && (!cu_seqlens || num_seqs < 1)) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q) || !aligned16(k) || !aligned16(v)) return GQA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(positions) & 3u))
+    return GQA_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < gqa_rope_attn_qkv_proj_workspace_size(total_tokens, head_dim) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return GQA_ERR_WORKSPACE;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices) return GQA_ERR_CUDA;
+  int sm_count = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState& ds = g_dev[device];
+    if (!ds.init) {
+      int major = 0;
+      if (cudaDeviceGetAttribute(&ds.sm_count, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+          cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess)
+        return GQA_ERR_CUDA;
+      if (major != 10) return GQA_ERR_UNSUPPORTED;
+      ds.init = true;
+    }
+    sm_count = ds.sm_count;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  std::lock_guard<std::mutex> lk(g_mu);  // descriptor cache
+#define GQA_PROJ_CASE(DD)                                                                                   \
+  if (head_dim == DD)                                                                                       \
+    return launch_qkv_proj<DD>(x, w_qkv, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, hidden, \
+                               n_q_heads, n_kv_heads, q, k, v, ws, st, device, sm_count);
+  GQA_PROJ_CASE(32) GQA_PROJ_CASE(64) GQA_PROJ_CASE(128)
+#undef GQA_PROJ_CASE
   return GQA_ERR_UNSUPPORTED;
 }

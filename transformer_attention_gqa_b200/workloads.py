@@ -197,6 +197,32 @@ def make_grad_output(inp: Inputs, seed: int = 1) -> np.ndarray:
     return to_bf16_values(rng.standard_normal((w.total_tokens, w.n_q_heads, w.head_dim), dtype=np.float32))
 
 
+@dataclass
+class ProjectionInputs:
+    x: np.ndarray       # [N, C] float32 holding bf16 values
+    w_qkv: np.ndarray   # [(n_q + 2 n_kv) d, C] float32 holding bf16 values: rows of W_q, W_k, W_v
+    cu_seqlens: np.ndarray
+    positions: np.ndarray
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    rope_theta: float
+
+
+def make_projection_inputs(seq_lens, hidden: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
+                           rope_theta: float = 1e4, seed: int = 0) -> ProjectionInputs:
+    """Seeded tokens x ~ N(0, 1) and stacked q/k/v projection weights ~
+    N(0, 1/hidden) (the scale of randomly initialised linear layers, so the
+    projections are of unit scale), both rounded to bf16."""
+    rng = np.random.default_rng(seed)
+    n = int(sum(seq_lens))
+    f = (n_q_heads + 2 * n_kv_heads) * head_dim
+    x = to_bf16_values(rng.standard_normal((n, hidden), dtype=np.float32))
+    w = to_bf16_values(rng.standard_normal((f, hidden), dtype=np.float32) / np.float32(np.sqrt(hidden)))
+    cu, pos = _cu_and_positions(seq_lens)
+    return ProjectionInputs(x, w, cu, pos, n_q_heads, n_kv_heads, head_dim, float(rope_theta))
+
+
 # ---------------------------------------------------------------- decoding
 
 @dataclass(frozen=True)
