@@ -58,6 +58,13 @@ without bias (y = x W^T), q_proj n_q heads wide and k_proj, v_proj n_kv heads
 wide, each output split into heads as view(tokens, heads, head_dim); then Q
 and K are rotated and V is not.
 
+Masks (``gqa_rope_attention_masked``): the attention kernel of the same
+page adds a mask tile to the scaled scores (scores * scale + mask, the mask
+holding -inf where a key is hidden), and the "Kohaku-TT" page lists masks
+among its flash-attention features. Here: an additive float mask over
+in-sequence (query, key) indices, shared by all sequences and heads, added
+after the 1/sqrt(d) scaling and combined with the causal mask when asked.
+
 Backward (``gqa_rope_attention_backward``): the gradients of the forward's
 output with respect to q, k, v for an upstream gradient dout, i.e. of the
 scalar sum(dout * out). It is the training-time counterpart of the forward
@@ -91,6 +98,7 @@ __all__ = [
     "rope_backward",
     "gqa_rope_attention_backward",
     "qkv_rope_projection",
+    "gqa_rope_attention_masked",
 ]
 
 
@@ -509,3 +517,52 @@ def qkv_rope_projection(x, w_q, w_k, w_v, n_q_heads: int, n_kv_heads: int, rope_
     k = apply_rope(yk, pos, rope_theta, operand_rounding)
     v = round_to_bf16(yv) if operand_rounding else yv
     return q, k, v
+
+
+# ---------------------------------------------------------------------------
+# Additive masks ("Attention from Scratch", section "The compute thread":
+# scores * scale + mask)
+# ---------------------------------------------------------------------------
+
+def gqa_rope_attention_masked(q, k, v, cu_seqlens, n_q_heads: int, n_kv_heads: int, rope_theta: float, attn_mask,
+                              positions=None, causal: bool = False, operand_rounding: bool = True):
+    """The forward with an additive mask: score(i, j) = q_i . k_j / sqrt(d) +
+    attn_mask[i, j], i and j indices inside the sequence (attn_mask is
+    [Lm, Lm] with Lm >= every sequence length, the same for every sequence
+    and head; -inf hides a key), then the causal mask if ``causal``, softmax,
+    weights @ v. A row whose scores are all -inf has no distribution: its out
+    is 0 and its lse -inf. Returns (out [N, n_q, d], lse [n_q, N]) in float64."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    mask = np.asarray(attn_mask, dtype=np.float64)
+    N, d, cu = _check_args(q, k, v, cu_seqlens, n_q_heads, n_kv_heads)
+    G = n_q_heads // n_kv_heads
+    if positions is None:
+        pos = np.concatenate([np.arange(cu[i + 1] - cu[i]) for i in range(len(cu) - 1)] + [np.zeros(0)])
+    else:
+        pos = np.asarray(positions, dtype=np.int64).reshape(-1)
+    out = np.zeros((N, n_q_heads, d))
+    lse = np.full((n_q_heads, N), -np.inf)
+    for si in range(len(cu) - 1):
+        a, b = int(cu[si]), int(cu[si + 1])
+        L = b - a
+        if L == 0:
+            continue
+        if mask.shape[0] < L or mask.shape[1] < L:
+            raise ValueError("attn_mask smaller than a sequence")
+        qh = np.transpose(apply_rope(q[a:b], pos[a:b], rope_theta, operand_rounding), (1, 0, 2))
+        kh = np.transpose(share_kv_heads(apply_rope(k[a:b], pos[a:b], rope_theta, operand_rounding), G, axis=1),
+                          (1, 0, 2))
+        vh = np.transpose(share_kv_heads(v[a:b], G, axis=1), (1, 0, 2))
+        scores = score(qh, kh) + mask[None, :L, :L]
+        if causal:
+            scores = causal_mask(scores, np.arange(L), np.arange(L))
+        m = np.max(scores, axis=-1, keepdims=True)
+        live = np.isfinite(m)
+        e = np.where(live, np.exp(scores - np.where(live, m, 0.0)), 0.0)
+        z = np.sum(e, axis=-1, keepdims=True)
+        w = e / np.where(z > 0, z, 1.0)
+        out[a:b] = np.transpose(gather(w, vh), (1, 0, 2))
+        lse[:, a:b] = np.where(live, m + np.log(np.where(z > 0, z, 1.0)), -np.inf)[..., 0]
+    return out, lse
