@@ -180,6 +180,122 @@ def cpu_baseline(workload, budget_s: float = 15.0, seed_rows: int = 0):
                       f"float64 NumPy, {dt:.1f} s", "host_cores": cores}
 
 
+# ------------------------------------------------------------------ shared timing
+def _rt_events():
+    """cudaEvent_t create / elapsed-ms / destroy through cuda.bindings (for
+    events handed to the library, which records them on its own stream)."""
+    from cuda.bindings import runtime as rt
+
+    def create():
+        err, e = rt.cudaEventCreate()
+        assert int(err) == 0
+        return e
+
+    def elapsed(a, b):
+        err, ms = rt.cudaEventElapsedTime(a, b)
+        assert int(err) == 0
+        return float(ms)
+
+    return create, elapsed, rt.cudaEventDestroy
+
+
+def _timed_steps(step, steps, stream, flush=None):
+    """Total device ms of `steps` calls of step(), each between CUDA events on
+    `stream`, with the L2 flushed before each outside its events, bracketed
+    by barriers and synchronisation."""
+    import torch
+    from transformer_attention_gqa_b200 import replicas
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    replicas.barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        if flush is not None:
+            flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    replicas.barrier()
+    return sum(a.elapsed_time(b) for a, b in ev)
+
+
+def _library_kernel_ms(step, calls, flush=None):
+    """Median durations (ms) of the first and the second kernel of the library
+    call step() makes, from events the library records around them on its
+    stream (gqa_rope_attn_set_profile_events), over `calls` calls."""
+    import torch
+    from transformer_attention_gqa_b200 import _abi
+
+    create, elapsed, destroy = _rt_events()
+    kern = []
+    for _ in range(calls):
+        e = [create() for _ in range(3)]
+        if flush is not None:
+            flush.zero_()
+        _abi.set_profile_events(int(e[0]), int(e[1]), int(e[2]))
+        step()
+        kern.append(e)
+    torch.cuda.synchronize()
+    first = statistics.median(elapsed(a, b) for a, b, _ in kern)
+    second = statistics.median(elapsed(b, c) for _, b, c in kern)
+    for e in kern:
+        for x in e:
+            destroy(x)
+    return first, second
+
+
+def _e2e_serial_ms(step, ins, outs, stream, steps):
+    """Mean ms per end-to-end step on `stream`: every step copies each
+    (device, pinned host) pair of `ins` to the device, runs step(), and
+    copies each (pinned host, device) pair of `outs` back."""
+    import torch
+    from transformer_attention_gqa_b200 import replicas
+
+    def one():
+        for d_, h_ in ins:
+            d_.copy_(h_, non_blocking=True)
+        step()
+        for h_, d_ in outs:
+            h_.copy_(d_, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    replicas.barrier()
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def _nbytes(tensors):
+    return sum(t.numel() * t.element_size() for t in tensors)
+
+
+def _reference_line(args, world, metric, unit, workload, shape, sample, digits=6):
+    """The --impl reference JSON line: the oracle, as it stands, on bounded
+    samples of the workload (sample(budget_s, index) -> cpu_baseline dict;
+    index 1000 + i for the args.warmup short warm-up samples, i for the
+    args.steps timed ones), reporting the median."""
+    for i in range(args.warmup):
+        sample(0.5, 1000 + i)
+    vals, info = [], None
+    for i in range(args.steps):
+        info = sample(max(1.0, min(5.0, 60.0 / max(args.steps, 1))), i)
+        vals.append(info["value"])
+    val = round(statistics.median(vals), digits)
+    return {"impl": "reference", "metric": metric, "value": val, "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": {"workload": workload, "shape": shape},
+            "cpu_baseline": {"value": val, "unit": unit, "cores": info["cores"], "kind": "oracle",
+                             "sample": info["sample"]},
+            "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 # ------------------------------------------------------------------ decoding
 DECODE_METRIC = "GQA+RoPE decode step (KV cache read, new row appended) algorithmic HBM GB/s on 1 B200"
 DECODE_UNIT = "GB/s"
@@ -246,77 +362,16 @@ def run_decode(args, rank, world, local_rank):
     launches_per_step = _abi.last_launch_count()
     clocks = ClockSampler(local_rank)
     clocks.start()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    replicas.barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        if flush is not None:
-            flush.zero_()
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    replicas.barrier()
-    total_ms = sum(a.elapsed_time(b) for a, b in ev)
-
-    from cuda.bindings import runtime as rt
-
-    def _ev():
-        err, e = rt.cudaEventCreate()
-        assert int(err) == 0
-        return e
-
-    def _ms(a, b):
-        err, ms = rt.cudaEventElapsedTime(a, b)
-        assert int(err) == 0
-        return float(ms)
-
-    kern = []
-    for _ in range(max(3, min(args.steps, 10))):
-        e = [_ev() for _ in range(3)]
-        if flush is not None:
-            flush.zero_()
-        _abi.set_profile_events(int(e[0]), int(e[1]), int(e[2]))
-        step()
-        kern.append(e)
-    torch.cuda.synchronize()
-    split_ms = statistics.median(_ms(a, b) for a, b, _ in kern)
-    merge_ms = statistics.median(_ms(b, c) for _, b, c in kern)
-    for e in kern:
-        for x in e:
-            rt.cudaEventDestroy(x)
+    total_ms = _timed_steps(step, args.steps, stream, flush)
+    split_ms, merge_ms = _library_kernel_ms(step, max(3, min(args.steps, 10)), flush)
     clk = clocks.stop()
 
     # end to end: the token's q, k_new, v_new and the lengths from pinned host
     # memory, out and lse back; the cache stays resident on the device
-    qh, knh, vnh = (torch.from_numpy(a).to(bf).pin_memory() for a in (inp.q, inp.k_new, inp.v_new))
-    lh = torch.from_numpy(inp.cache_seqlens).pin_memory()
-    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (qh, knh, vnh, lh))
-    d2h = outh.numel() * outh.element_size() + lseh.numel() * lseh.element_size()
-
-    def e2e_step():
-        q.copy_(qh, non_blocking=True)
-        kn.copy_(knh, non_blocking=True)
-        vn.copy_(vnh, non_blocking=True)
-        lens.copy_(lh, non_blocking=True)
-        step()
-        outh.copy_(out, non_blocking=True)
-        lseh.copy_(lse, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    e_steps = max(3, min(args.steps, 10))
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    replicas.barrier()
-    e0.record(stream)
-    for _ in range(e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e_steps
+    ins = [(d_, d_.cpu().pin_memory()) for d_ in (q, kn, vn, lens)]
+    outs = [(torch.empty(d_.shape, dtype=d_.dtype).pin_memory(), d_) for d_ in (out, lse)]
+    h2d, d2h = _nbytes(h_ for _, h_ in ins), _nbytes(h_ for h_, _ in outs)
+    e2e_ms = _e2e_serial_ms(step, ins, outs, stream, max(3, min(args.steps, 10)))
     assert g.get_device_status() == 0
 
     total_ms, e2e_ms, split_ms, merge_ms = replicas.max_over_ranks([total_ms, e2e_ms, split_ms, merge_ms], device=dev)
@@ -393,7 +448,6 @@ def run_bwd(args, rank, world, local_rank):
     import torch
     import transformer_attention_gqa_b200 as g
     from transformer_attention_gqa_b200 import _abi, replicas, workloads as wl
-    from cuda.bindings import runtime as rt
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -423,72 +477,18 @@ def run_bwd(args, rank, world, local_rank):
     launches_per_step = _abi.last_launch_count()
     clocks = ClockSampler(local_rank)
     clocks.start()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    replicas.barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.zero_()
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    replicas.barrier()
-    total_ms = sum(a.elapsed_time(b) for a, b in ev)
-
-    def _ev():
-        err, e = rt.cudaEventCreate()
-        assert int(err) == 0
-        return e
-
-    def _ms(a, b):
-        err, ms = rt.cudaEventElapsedTime(a, b)
-        assert int(err) == 0
-        return float(ms)
-
-    kern = []
-    for _ in range(max(3, min(args.steps, 10))):
-        e = [_ev() for _ in range(3)]
-        flush.zero_()
-        _abi.set_profile_events(int(e[0]), int(e[1]), int(e[2]))
-        step()
-        kern.append(e)
-    torch.cuda.synchronize()
-    prep_ms = statistics.median(_ms(a, b) for a, b, _ in kern)
-    bwd_ms = statistics.median(_ms(b, c) for _, b, c in kern)
-    for e in kern:
-        for x in e:
-            rt.cudaEventDestroy(x)
+    total_ms = _timed_steps(step, args.steps, stream, flush)
+    prep_ms, bwd_ms = _library_kernel_ms(step, max(3, min(args.steps, 10)), flush)
     clk = clocks.stop()
 
     # end to end: q, k, v, out, lse, dout and cu_seqlens from pinned host
     # memory every step, dq, dk, dv back
-    hosts = [t.cpu().pin_memory() for t in (q, k, v, out, lse, do, cu)]
-    devs = (q, k, v, out, lse, do, cu)
-    backs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
-    h2d = sum(t.numel() * t.element_size() for t in hosts)
-    d2h = sum(t.numel() * t.element_size() for t in backs)
-
-    def e2e_step():
-        for d_, h_ in zip(devs, hosts):
-            d_.copy_(h_, non_blocking=True)
-        step()
-        for h_, d_ in zip(backs, (dq, dk, dv)):
-            h_.copy_(d_, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    e_steps = max(3, min(args.steps, 10))
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    replicas.barrier()
-    e0.record(stream)
-    for _ in range(e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e_steps
+    ins = [(d_, d_.cpu().pin_memory()) for d_ in (q, k, v, out, lse, do, cu)]
+    outs = [(torch.empty(d_.shape, dtype=d_.dtype).pin_memory(), d_) for d_ in (dq, dk, dv)]
+    h2d, d2h = _nbytes(h_ for _, h_ in ins), _nbytes(h_ for h_, _ in outs)
+    e2e_ms = _e2e_serial_ms(step, ins, outs, stream, max(3, min(args.steps, 10)))
     assert g.get_device_status() == 0
-    assert torch.equal(backs[0], dq.cpu())
+    assert torch.equal(outs[0][0], dq.cpu())
 
     total_ms, e2e_ms, bwd_ms, prep_ms = replicas.max_over_ranks([total_ms, e2e_ms, bwd_ms, prep_ms], device=dev)
     flops = BWD_FLOP_FACTOR * w.flops()
@@ -524,22 +524,9 @@ def main_bwd(args, world, rank, local_rank):
     from transformer_attention_gqa_b200 import workloads as wl
     w = wl.WORKLOADS[BWD_WORKLOADS[args.workload]]
     if args.impl == "reference":
-        if rank != 0:
-            return 0
-        cpu_baseline_bwd(w, budget_s=0.5)
-        vals, info = [], None
-        for _ in range(args.steps):
-            info = cpu_baseline_bwd(w, budget_s=max(1.0, min(5.0, 60.0 / max(args.steps, 1))))
-            vals.append(info["value"])
-        val = statistics.median(vals)
-        print(json.dumps({"impl": "reference", "metric": BWD_METRIC, "value": round(val, 6), "unit": UNIT,
-                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
-                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                          "config": {"workload": args.workload, "shape": w.description},
-                          "cpu_baseline": {"value": round(val, 6), "unit": UNIT, "cores": info["cores"],
-                                           "kind": "oracle", "sample": info["sample"]},
-                          "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
-                                  "d2h_bytes_per_step": 0}}))
+        if rank == 0:
+            print(json.dumps(_reference_line(args, world, BWD_METRIC, UNIT, args.workload, w.description,
+                                             lambda budget, _: cpu_baseline_bwd(w, budget_s=budget))))
         return 0
     from transformer_attention_gqa_b200 import replicas
     replicas.init("nccl", timeout_s=120)
@@ -592,7 +579,6 @@ def run_proj(args, rank, world, local_rank, inp):
     import torch
     import transformer_attention_gqa_b200 as g
     from transformer_attention_gqa_b200 import _abi, replicas, workloads as wl
-    from cuda.bindings import runtime as rt
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -622,71 +608,18 @@ def run_proj(args, rank, world, local_rank, inp):
     launches_per_step = _abi.last_launch_count()
     clocks = ClockSampler(local_rank)
     clocks.start()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    replicas.barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.zero_()
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    replicas.barrier()
-    total_ms = sum(a.elapsed_time(b) for a, b in ev)
-
-    def _ev():
-        err, e = rt.cudaEventCreate()
-        assert int(err) == 0
-        return e
-
-    def _ms(a, b):
-        err, ms = rt.cudaEventElapsedTime(a, b)
-        assert int(err) == 0
-        return float(ms)
-
-    kern = []
-    for _ in range(max(3, min(args.steps, 10))):
-        e = [_ev() for _ in range(3)]
-        flush.zero_()
-        _abi.set_profile_events(int(e[0]), int(e[1]), int(e[2]))
-        step()
-        kern.append(e)
-    torch.cuda.synchronize()
-    table_ms = statistics.median(_ms(a, b) for a, b, _ in kern)
-    proj_ms = statistics.median(_ms(b, c) for _, b, c in kern)
-    for e in kern:
-        for t in e:
-            rt.cudaEventDestroy(t)
+    total_ms = _timed_steps(step, args.steps, stream, flush)
+    table_ms, proj_ms = _library_kernel_ms(step, max(3, min(args.steps, 10)), flush)
     clk = clocks.stop()
 
     # end to end: x and cu_seqlens from pinned host memory every step (the
     # weights stay resident), q, k, v back
-    xh, cuh = x.cpu().pin_memory(), cu.cpu().pin_memory()
-    backs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (q, k, v)]
-    h2d = xh.numel() * xh.element_size() + cuh.numel() * cuh.element_size()
-    d2h = sum(t.numel() * t.element_size() for t in backs)
-
-    def e2e_step():
-        x.copy_(xh, non_blocking=True)
-        cu.copy_(cuh, non_blocking=True)
-        step()
-        for h_, d_ in zip(backs, (q, k, v)):
-            h_.copy_(d_, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    e_steps = max(3, min(args.steps, 10))
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    replicas.barrier()
-    e0.record(stream)
-    for _ in range(e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e_steps
+    ins = [(d_, d_.cpu().pin_memory()) for d_ in (x, cu)]
+    outs = [(torch.empty(d_.shape, dtype=d_.dtype).pin_memory(), d_) for d_ in (q, k, v)]
+    h2d, d2h = _nbytes(h_ for _, h_ in ins), _nbytes(h_ for h_, _ in outs)
+    e2e_ms = _e2e_serial_ms(step, ins, outs, stream, max(3, min(args.steps, 10)))
     assert g.get_device_status() == 0
-    assert torch.equal(backs[0], q.cpu())
+    assert torch.equal(outs[0][0], q.cpu())
 
     total_ms, e2e_ms, proj_ms, table_ms = replicas.max_over_ranks([total_ms, e2e_ms, proj_ms, table_ms], device=dev)
     flops = 2.0 * N * C * F
@@ -725,22 +658,9 @@ def main_proj(args, world, rank, local_rank):
     seed = w.seed if rank == 0 else replicas.replica_seed(w.seed, rank)
     inp = wl.make_projection_inputs(w.seq_lens, C, w.n_q_heads, w.n_kv_heads, w.head_dim, w.rope_theta, seed=seed)
     if args.impl == "reference":
-        if rank != 0:
-            return 0
-        cpu_baseline_proj(w, inp, budget_s=0.5)
-        vals, info = [], None
-        for _ in range(args.steps):
-            info = cpu_baseline_proj(w, inp, budget_s=max(1.0, min(5.0, 60.0 / max(args.steps, 1))))
-            vals.append(info["value"])
-        val = statistics.median(vals)
-        print(json.dumps({"impl": "reference", "metric": PROJ_METRIC, "value": round(val, 6), "unit": UNIT,
-                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
-                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                          "config": {"workload": args.workload, "shape": w.description},
-                          "cpu_baseline": {"value": round(val, 6), "unit": UNIT, "cores": info["cores"],
-                                           "kind": "oracle", "sample": info["sample"]},
-                          "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
-                                  "d2h_bytes_per_step": 0}}))
+        if rank == 0:
+            print(json.dumps(_reference_line(args, world, PROJ_METRIC, UNIT, args.workload, w.description,
+                                             lambda budget, _: cpu_baseline_proj(w, inp, budget_s=budget))))
         return 0
     replicas.init("nccl", timeout_s=120)
     res = run_proj(args, rank, world, local_rank, inp)
@@ -982,24 +902,11 @@ def main_decode(args, world, rank, local_rank):
     from transformer_attention_gqa_b200 import workloads as wl
     w = wl.DECODE_WORKLOADS[args.workload]
     if args.impl == "reference":
-        if rank != 0:
-            return 0
-        inp = wl.make_decode_inputs(w, nan_tail=False)
-        for i in range(args.warmup):
-            cpu_baseline_decode(w, inp, budget_s=0.5, seed=1000 + i)
-        vals, info = [], None
-        for i in range(args.steps):
-            info = cpu_baseline_decode(w, inp, budget_s=max(1.0, min(5.0, 60.0 / max(args.steps, 1))), seed=i)
-            vals.append(info["value"])
-        val = statistics.median(vals)
-        print(json.dumps({"impl": "reference", "metric": DECODE_METRIC, "value": round(val, 4), "unit": DECODE_UNIT,
-                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
-                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                          "config": {"workload": w.name, "shape": w.description},
-                          "cpu_baseline": {"value": round(val, 4), "unit": DECODE_UNIT, "cores": info["cores"],
-                                           "kind": "oracle", "sample": info["sample"]},
-                          "e2e": {"value": round(val, 4), "unit": DECODE_UNIT, "h2d_bytes_per_step": 0,
-                                  "d2h_bytes_per_step": 0}}))
+        if rank == 0:
+            inp = wl.make_decode_inputs(w, nan_tail=False)
+            print(json.dumps(_reference_line(args, world, DECODE_METRIC, DECODE_UNIT, w.name, w.description,
+                                             lambda budget, i: cpu_baseline_decode(w, inp, budget_s=budget, seed=i),
+                                             digits=4)))
         return 0
     from transformer_attention_gqa_b200 import replicas
     replicas.init("nccl", timeout_s=120)
