@@ -12,6 +12,7 @@ in HBM. Default workload: Llama-3-8B-shaped causal prefill (B=1, T=8192,
   --workload decode_llama8b | decode_qwen3b | ...   one decoding step
   --workload bwd_llama8b | bwd_varlen | bwd_nano    the backward (dq, dk, dv)
   --workload qkv_llama8b | qkv_nano                 the QKV projection with its RoPE epilogue
+  --workload masked_llama8b | masked_nano           the forward with an additive mask
 
 Under torchrun each rank runs its own replica of the workload (independent
 problems, weak scaling); the elapsed time is the max over ranks.
@@ -672,6 +673,144 @@ def main_proj(args, world, rank, local_rank):
     return 0
 
 
+# ------------------------------------------------------------------ masked forward
+# The forward with an additive mask: a forward workload's shape, causal, with
+# a seeded bf16 bias over every in-sequence (query, key) pair (N(0, 1) values,
+# no hidden keys beyond the causal ones); one gqa_rope_attn_fwd_masked call
+# per step, the forward's FLOP convention.
+MASKED_WORKLOADS = {"masked_llama8b": "llama8b", "masked_nano": "nano"}
+MASKED_METRIC = "causal GQA+RoPE attention fwd with an additive mask TFLOP/s on 1 B200; % of dense-BF16 tensor peak"
+
+
+def _bench_mask(w, seed):
+    from transformer_attention_gqa_b200 import workloads as wl
+
+    Lm = max(w.seq_lens)
+    Lp = (Lm + 7) // 8 * 8
+    rng = np.random.default_rng(seed)
+    return wl.to_bf16_values(rng.standard_normal((Lp, Lp), dtype=np.float32))
+
+
+def cpu_baseline_masked(w, inp, mask, budget_s: float = 15.0, max_len: int = 2048):
+    """Times the float64 oracle's masked forward, as it stands, on a prefix of
+    the workload's first sequence (length sized by a probe to about
+    budget_s); returns TFLOP/s by the forward's convention."""
+    import oracle.gqa_oracle as orc
+
+    first = int(inp.cu_seqlens[1])
+
+    def run(L):
+        t0 = time.perf_counter()
+        orc.gqa_rope_attention_masked(inp.q[:L], inp.k[:L], inp.v[:L], [0, L], w.n_q_heads, w.n_kv_heads,
+                                      w.rope_theta, mask, causal=True)
+        return time.perf_counter() - t0
+
+    L0 = min(first, 128)
+    t0 = run(L0)
+    L = int(max(L0, min(first, max_len, L0 * np.sqrt(max(budget_s, 0.1) / max(t0, 1e-3)))))
+    dt = run(L)
+    flops = 4.0 * L * L * w.head_dim * w.n_q_heads / 2.0
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"first {L} tokens of {w.name}'s first sequence, all {w.n_q_heads} heads, float64 NumPy, "
+                      f"{dt:.1f} s"}
+
+
+def run_masked(args, rank, world, local_rank, inp, mask_np):
+    import torch
+    import transformer_attention_gqa_b200 as g
+    from transformer_attention_gqa_b200 import _abi, replicas, workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = wl.WORKLOADS[MASKED_WORKLOADS[args.workload]]
+    bf = torch.bfloat16
+    q = torch.from_numpy(inp.q).to(bf).to(dev)
+    k = torch.from_numpy(inp.k).to(bf).to(dev)
+    v = torch.from_numpy(inp.v).to(bf).to(dev)
+    cu = torch.from_numpy(inp.cu_seqlens).to(dev)
+    mask = torch.from_numpy(mask_np).to(bf).to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.n_q_heads, w.total_tokens), dtype=torch.float32, device=dev)
+    ws = g.Workspace(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        g.gqa_rope_attn_fwd_masked(q, k, v, cu, w.rope_theta, mask, causal=True, out=out, lse=lse, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert g.get_device_status() == 0
+    launches_per_step = _abi.last_launch_count()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    total_ms = _timed_steps(step, args.steps, stream, flush)
+    prep_ms, attn_ms = _library_kernel_ms(step, max(3, min(args.steps, 10)), flush)
+    clk = clocks.stop()
+
+    # end to end: q, k, v and cu_seqlens from pinned host memory every step
+    # (the mask stays resident), out and lse back
+    ins = [(d_, d_.cpu().pin_memory()) for d_ in (q, k, v, cu)]
+    outs = [(torch.empty(d_.shape, dtype=d_.dtype).pin_memory(), d_) for d_ in (out, lse)]
+    h2d, d2h = _nbytes(h_ for _, h_ in ins), _nbytes(h_ for h_, _ in outs)
+    e2e_ms = _e2e_serial_ms(step, ins, outs, stream, max(3, min(args.steps, 10)))
+    assert g.get_device_status() == 0
+    assert torch.equal(outs[0][0], out.cpu())
+
+    total_ms, e2e_ms, attn_ms, prep_ms = replicas.max_over_ranks([total_ms, e2e_ms, attn_ms, prep_ms], device=dev)
+    flops = w.flops()
+    ms_per_step = total_ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    res = {
+        "metric": MASKED_METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "shape": w.description, "total_tokens": w.total_tokens,
+                   "num_seqs": w.num_seqs, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+                   "head_dim": w.head_dim, "rope_theta": w.rope_theta, "causal": True,
+                   "mask": f"bf16 [{mask_np.shape[0]}, {mask_np.shape[1]}] seeded N(0, 1) bias",
+                   "flops_per_step": flops, "parallelism": f"replicas x{world}",
+                   "l2": "256 MiB written before every timed step, outside the step's events"},
+        "pct_of_peak": round(100.0 * value / world / peak, 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{src} bf16_tflops (burst)", "kernel": "gqa_attn_fwd_masked_kernel",
+                     "kernel_ms": round(attn_ms, 4), "prologue_ms": round(prep_ms, 4)},
+        "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if clk:
+        res["clocks"] = clk
+    return res
+
+
+def main_masked(args, world, rank, local_rank):
+    from transformer_attention_gqa_b200 import replicas, workloads as wl
+    w = wl.WORKLOADS[MASKED_WORKLOADS[args.workload]]
+    seed = w.seed if rank == 0 else replicas.replica_seed(w.seed, rank)
+    inp = wl.make_inputs(w, seed=seed)
+    mask = _bench_mask(w, seed + 1)
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(_reference_line(args, world, MASKED_METRIC, UNIT, args.workload, w.description,
+                                             lambda budget, _: cpu_baseline_masked(w, inp, mask, budget_s=budget))))
+        return 0
+    replicas.init("nccl", timeout_s=120)
+    res = run_masked(args, rank, world, local_rank, inp, mask)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_masked(w, inp, mask, budget_s=args.cpu_budget)
+    replicas.shutdown()
+    if rank == 0:
+        print(json.dumps(res))
+    return 0
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -864,6 +1003,8 @@ def main():
         return main_bwd(args, world, rank, local_rank)
     if args.workload in PROJ_WORKLOADS:
         return main_proj(args, world, rank, local_rank)
+    if args.workload in MASKED_WORKLOADS:
+        return main_masked(args, world, rank, local_rank)
     w = wl.WORKLOADS[args.workload]
 
     if args.impl == "reference":

@@ -23,7 +23,8 @@
  *     batches (cu_seqlens prefix sums).
  *   The log-sum-exp output is not on the pages; it is the natural-log
  *   normaliser of each row's scaled, masked scores.
- * A decoding step against a KV cache (gqa_rope_attn_decode), the backward
+ * A forward with an additive mask (gqa_rope_attn_fwd_masked), a decoding
+ * step against a KV cache (gqa_rope_attn_decode), the backward
  * (gqa_rope_attn_bwd) and the QKV projection with its RoPE epilogue
  * (gqa_rope_attn_qkv_proj) are declared further down.
  *
@@ -171,6 +172,31 @@ int gqa_rope_attn_fwd_noalloc(const void* q, const void* k, const void* v, const
                               int total_tokens, int n_q_heads, int n_kv_heads, int head_dim,
                               int causal, int dtype, void* out, float* lse, void* stream);
 
+/* ---- Forward with an additive mask -----------------------------------------
+ *
+ * The attention kernel of "Attention from Scratch" (section "The compute
+ * thread") adds a mask tile to the scaled scores: here
+ *
+ *   score(t, j) = rope(q[t, h]) . rope(k[j, kv]) / sqrt(d) + mask[t', j']
+ *
+ * with t', j' the indices of query t and key j inside their sequence; -inf
+ * hides a key. The mask is shared by every sequence and head and is combined
+ * with the causal mask when causal = 1. A row that sees no key gets out = 0
+ * and lse = -inf. Arguments as for gqa_rope_attn_fwd (bf16 only), plus:
+ *   mask      bf16 [mask_len, mask_ld] device array, 16-byte aligned
+ *   mask_len  >= the longest sequence (checked on the device: a longer one
+ *             gets no output and sets GQA_ERR_BAD_SEQLENS)
+ *   mask_ld   elements between mask rows, >= mask_len, a multiple of 8
+ * workspace: gqa_rope_attn_workspace_size(..., GQA_DTYPE_BF16) bytes. Two
+ * kernels are queued (the forward's prologue, then the masked attention
+ * kernel); the call does not wait.
+ */
+int gqa_rope_attn_fwd_masked(const void* q, const void* k, const void* v, const int32_t* positions,
+                             double rope_theta, const int32_t* cu_seqlens, int num_seqs, int total_tokens,
+                             int n_q_heads, int n_kv_heads, int head_dim, int causal, const void* mask,
+                             int mask_len, int mask_ld, void* out, float* lse, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
 /* ---- Decoding step (one new token per sequence against a KV cache) ------
  *
  * "Attention from Scratch", section "Attention, the math: Grouped-Query
@@ -292,8 +318,8 @@ int gqa_rope_attn_qkv_proj(const void* x, const void* w_qkv, const int32_t* posi
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /* Measurement aid. Arms the calling thread's next gqa_rope_attn_fwd,
- * gqa_rope_attn_decode, gqa_rope_attn_bwd or gqa_rope_attn_qkv_proj call to
- * record three CUDA events
+ * gqa_rope_attn_fwd_masked, gqa_rope_attn_decode, gqa_rope_attn_bwd or
+ * gqa_rope_attn_qkv_proj call to record three CUDA events
  * (cudaEvent_t passed as void*, any may be NULL) on its stream: before its
  * first kernel, between its first two kernels, and after the second, so
  * that each kernel's duration can be read with cudaEventElapsedTime (the

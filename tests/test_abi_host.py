@@ -224,3 +224,25 @@ def test_qkv_proj_host_rejections_before_any_cuda_call():
     need = _abi.qkv_proj_workspace_size(128, 64)
     assert pcall(workspace=A, workspace_bytes=need - 1) == E.GQA_ERR_WORKSPACE
     assert _abi.last_launch_count() == 0
+
+
+def mcall(**kw):
+    args = dict(q=A, k=A, v=A, positions=0, rope_theta=1e4, cu_seqlens=A, num_seqs=1, total_tokens=128,
+                n_q_heads=4, n_kv_heads=2, head_dim=64, causal=0, mask=A, mask_len=128, mask_ld=128, out=A, lse=0,
+                workspace=0, workspace_bytes=0, stream=None)
+    args.update(kw)
+    return _abi.gqa_rope_attn_fwd_masked(**args)
+
+
+def test_masked_host_rejections_before_any_cuda_call():
+    E = _abi
+    assert mcall(total_tokens=0) == E.GQA_OK
+    assert mcall(mask_len=0) == E.GQA_ERR_INVALID_ARG
+    assert mcall(mask_ld=100) == E.GQA_ERR_INVALID_ARG       # < mask_len
+    assert mcall(mask_ld=132) == E.GQA_ERR_INVALID_ARG       # not a multiple of 8
+    assert mcall(mask=0) == E.GQA_ERR_INVALID_ARG
+    assert mcall(mask=A + 8) == E.GQA_ERR_INVALID_ARG
+    assert mcall(causal=3) == E.GQA_ERR_INVALID_ARG
+    assert mcall(head_dim=48) == E.GQA_ERR_UNSUPPORTED
+    assert mcall() == E.GQA_ERR_WORKSPACE
+    assert _abi.last_launch_count() == 0

@@ -1,6 +1,6 @@
 """The benchmark's reference arm (the float64 oracle on host cores) prints
 one JSON line with the contract's keys, for a prefill, a decoding, a
-backward and a projection workload. CPU only: the reference arm needs no GPU."""
+backward, a projection and a masked-attention workload. CPU only: the reference arm needs no GPU."""
 import json
 import os
 import subprocess
@@ -13,7 +13,7 @@ KEYS = {"impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "higher_
         "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"}
 
 
-@pytest.mark.parametrize("workload", ["tiny", "decode_small", "bwd_nano", "qkv_nano"])
+@pytest.mark.parametrize("workload", ["tiny", "decode_small", "bwd_nano", "qkv_nano", "masked_nano"])
 def test_reference_arm_json_line(workload):
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", workload,
                         "--steps", "2", "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=300)

@@ -134,3 +134,16 @@ def test_qkv_proj_rejects_host_tensors_and_bad_shapes():
         g.gqa_rope_attn_qkv_proj(x, w, 4, 2, 1e4)                          # no positions, no cu_seqlens
     with pytest.raises(TypeError):
         g.gqa_rope_attn_qkv_proj(x.float(), w, 4, 2, 1e4, cu_seqlens=cu)
+
+
+def test_masked_rejects_host_tensors_and_bad_masks():
+    q, k, v, cu = _fwd_args()
+    bf = torch.bfloat16
+    with pytest.raises(TypeError):
+        g.gqa_rope_attn_fwd_masked(q, k, v, cu, 1e4, torch.zeros(16, 16))          # fp32 mask
+    with pytest.raises(ValueError):
+        g.gqa_rope_attn_fwd_masked(q, k, v, cu, 1e4, torch.zeros(16, 12, dtype=bf))  # fewer columns than rows
+    with pytest.raises(ValueError):
+        g.gqa_rope_attn_fwd_masked(q, k, v, cu, 1e4, torch.zeros(12, 12, dtype=bf))  # row stride 12
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        g.gqa_rope_attn_fwd_masked(q, k, v, cu, 1e4, torch.zeros(16, 16, dtype=bf))

@@ -7,7 +7,7 @@ from . import _abi
 from ._abi import (GqaError, workspace_size, decode_workspace_size, bwd_workspace_size,  # noqa: F401
                    qkv_proj_workspace_size, get_device_status)
 
-__all__ = ["gqa_rope_attn_fwd", "gqa_rope_attn_decode", "gqa_rope_attn_bwd", "gqa_rope_attn_qkv_proj",
+__all__ = ["gqa_rope_attn_fwd", "gqa_rope_attn_fwd_masked", "gqa_rope_attn_decode", "gqa_rope_attn_bwd", "gqa_rope_attn_qkv_proj",
            "workspace_size", "decode_workspace_size", "bwd_workspace_size", "qkv_proj_workspace_size",
            "get_device_status", "GqaError", "Workspace"]
 
@@ -242,3 +242,51 @@ def gqa_rope_attn_qkv_proj(x, w_qkv, n_q_heads: int, n_kv_heads: int, rope_theta
     if rc != _abi.GQA_OK:
         raise GqaError(rc, "gqa_rope_attn_qkv_proj")
     return q, k, v
+
+
+def gqa_rope_attn_fwd_masked(q, k, v, cu_seqlens, rope_theta: float, mask, positions=None, causal: bool = False,
+                             out=None, lse=None, workspace=None, stream=None):
+    """out, lse of softmax(rope(q) rope(k)^T / sqrt(d) + mask [+ causal mask]) v.
+
+    mask: bf16 [Lm, ld] CUDA tensor (ld >= Lm, a multiple of 8; a contiguous
+    [Lm, Lm] tensor needs Lm a multiple of 8) over in-sequence (query, key)
+    indices, shared by every sequence and head, -inf hiding a key; Lm must
+    be at least the longest sequence. Other arguments as for
+    gqa_rope_attn_fwd (bf16 only). Rows that see no key get out 0 and lse
+    -inf. Raises GqaError on a non-OK status.
+    """
+    import torch
+
+    _check(q.dim() == 3 and k.dim() == 3, "q must be [N, n_q, d] and k, v [N, n_kv, d]")
+    N, nq, d = q.shape
+    nkv = k.shape[1]
+    if any(t.dtype != torch.bfloat16 for t in (q, k, v, mask)):
+        raise TypeError("q, k, v and mask must be bfloat16")
+    _check(k.shape == (N, nkv, d) and v.shape == (N, nkv, d), "k and v must be [N, n_kv, d] matching q")
+    _check(mask.dim() == 2 and mask.stride(1) == 1, "mask must be a 2-D tensor with unit column stride")
+    mask_len, ld = mask.shape[0], mask.stride(0)
+    _check(mask.shape[1] >= mask_len and ld % 8 == 0, "mask must be [Lm, >= Lm] with a row stride divisible by 8")
+    _check(cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1 and cu_seqlens.numel() >= 1,
+           "cu_seqlens must be a 1-D int32 tensor")
+    if positions is not None:
+        _check(positions.dtype == torch.int32 and positions.shape == (N,), "positions must be int32 [N]")
+    num_seqs = cu_seqlens.numel() - 1
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((nq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(out.shape == q.shape and out.dtype == q.dtype, "out must match q's shape and dtype")
+    _check(lse.shape == (nq, N) and lse.dtype == torch.float32, "lse must be float32 [n_q, N]")
+    _check_tensors(dict(q=q, k=k, v=v, cu_seqlens=cu_seqlens, positions=positions, out=out, lse=lse), q.device)
+    _check(mask.is_cuda and mask.device == q.device, "mask must be a CUDA tensor on q's device")
+    nbytes = workspace_size(num_seqs, N, nq, nkv, d, _abi.GQA_DTYPE_BF16)
+    if workspace is None:
+        workspace = Workspace(q.device)
+    ws = workspace.get(nbytes) if isinstance(workspace, Workspace) else workspace
+    _check_tensors(dict(workspace=ws), q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    rc = _abi.gqa_rope_attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(positions), rope_theta, _ptr(cu_seqlens),
+                                       num_seqs, N, nq, nkv, d, 1 if causal else 0, _ptr(mask), mask_len, ld,
+                                       _ptr(out), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), stream)
+    if rc != _abi.GQA_OK:
+        raise GqaError(rc, "gqa_rope_attn_fwd_masked")
+    return out, lse

@@ -38,6 +38,7 @@ EXPORTED = (
     "gqa_rope_attn_bwd",
     "gqa_rope_attn_qkv_proj_workspace_size",
     "gqa_rope_attn_qkv_proj",
+    "gqa_rope_attn_fwd_masked",
 )
 
 _lib = None
@@ -92,6 +93,10 @@ def load() -> ctypes.CDLL:
     lib.gqa_rope_attn_qkv_proj.restype = c_int
     lib.gqa_rope_attn_qkv_proj.argtypes = [c_void, c_void, c_void, c_double, c_void, c_int, c_int, c_int, c_int,
                                            c_int, c_int, c_void, c_void, c_void, c_void, c_size, c_void]
+    lib.gqa_rope_attn_fwd_masked.restype = c_int
+    lib.gqa_rope_attn_fwd_masked.argtypes = [c_void, c_void, c_void, c_void, c_double, c_void, c_int, c_int, c_int,
+                                             c_int, c_int, c_int, c_void, c_int, c_int, c_void, c_void, c_void,
+                                             c_size, c_void]
     lib.gqa_rope_attn_set_profile_events.restype = None
     lib.gqa_rope_attn_set_profile_events.argtypes = [c_void, c_void, c_void]
     _lib = lib
@@ -162,6 +167,17 @@ def gqa_rope_attn_qkv_proj(x, w_qkv, positions, rope_theta, cu_seqlens, num_seqs
     return int(load().gqa_rope_attn_qkv_proj(x, w_qkv, positions, float(rope_theta), cu_seqlens, int(num_seqs),
                                              int(total_tokens), int(hidden), int(n_q_heads), int(n_kv_heads),
                                              int(head_dim), q, k, v, workspace, int(workspace_bytes), stream))
+
+
+def gqa_rope_attn_fwd_masked(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads,
+                             n_kv_heads, head_dim, causal, mask, mask_len, mask_ld, out, lse, workspace,
+                             workspace_bytes, stream) -> int:
+    """Raw call of the forward with an additive mask; integer device
+    addresses (0 for NULL); returns the status."""
+    return int(load().gqa_rope_attn_fwd_masked(q, k, v, positions, float(rope_theta), cu_seqlens, int(num_seqs),
+                                               int(total_tokens), int(n_q_heads), int(n_kv_heads), int(head_dim),
+                                               int(causal), mask, int(mask_len), int(mask_ld), out, lse, workspace,
+                                               int(workspace_bytes), stream))
 
 
 def get_device_status(stream=None) -> int:

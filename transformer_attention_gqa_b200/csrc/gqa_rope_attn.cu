@@ -1,9 +1,10 @@
 // Host side of the C ABI (include/gqa_rope_attn.h): argument checks, TMA
 // descriptor cache, the two launches of the fused forward (prologue, then
-// the attention kernel, in stream order), the two of the decoding step
-// (key-range kernel, then the merge), the three of the backward (prologue,
-// attention backward, dq rotation) and the two of the QKV projection with
-// its RoPE epilogue (cos/sin table, projection).
+// the attention kernel, in stream order), the two of the masked forward (the
+// same prologue, then the masked attention kernel), the two of the decoding
+// step (key-range kernel, then the merge), the three of the backward
+// (prologue, attention backward, dq rotation) and the two of the QKV
+// projection with its RoPE epilogue (cos/sin table, projection).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -18,6 +19,7 @@
 #include "bwd_kernel.cuh"
 #include "common.cuh"
 #include "decode_kernel.cuh"
+#include "masked_kernel.cuh"
 #include "prep_kernel.cuh"
 #include "proj_kernel.cuh"
 
@@ -34,6 +36,7 @@ struct DeviceState {
   bool dec_attr_set[3][3] = {};
   bool bwd_attr_set[3] = {};
   bool proj_attr_set[3] = {};
+  bool masked_attr_set[3] = {};
 };
 
 std::mutex g_mu;
@@ -507,6 +510,108 @@ int launch_qkv_proj(const void* x, const void* w, const int32_t* positions, doub
   return GQA_OK;
 }
 
+// ---------------------------------------------------------------- masked forward
+
+template <int D>
+int launch_masked(const void* q, const void* k, const void* v, const int32_t* positions, double theta,
+                  const int32_t* cu, int num_seqs, int N, int nq, int nkv, int causal, const void* mask,
+                  int mask_len, int mask_ld, void* out, float* lse, uint8_t* ws, const WsLayout& lay,
+                  cudaStream_t stream, int device, int sm_count) {
+  using A = AttnCfg<D>;
+  using C = MaskedCfg<D>;
+  const int G = nq / nkv;
+  const int tq = tokens_per_tile(G);
+  {  // caller holds g_mu
+    DeviceState& ds = g_dev[device];
+    if (!ds.masked_attr_set[dim_index(D)]) {
+      if (cudaFuncSetAttribute(gqa_attn_fwd_masked_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_BYTES) != cudaSuccess)
+        return GQA_ERR_CUDA;
+      ds.masked_attr_set[dim_index(D)] = true;
+    }
+  }
+  // the forward's prologue: schedule, cos/sin table, K' head-major
+  PrepParams pp{};
+  pp.q = q;
+  pp.k = k;
+  pp.v = v;
+  pp.positions = positions;
+  pp.cu = cu;
+  pp.N = N;
+  pp.num_seqs = num_seqs;
+  pp.nq = nq;
+  pp.nkv = nkv;
+  pp.tq = tq;
+  pp.causal = causal;
+  pp.theta = theta;
+  for (int i = 0; i < D / 2; ++i) pp.inv_freq[i] = std::pow(theta, -(2.0 * i) / D);
+  pp.header = reinterpret_cast<int*>(ws + lay.header);
+  pp.seq_pfx = reinterpret_cast<int*>(ws + lay.seq_pfx);
+  pp.pairs = reinterpret_cast<int2*>(ws + lay.pairs);
+  pp.table = reinterpret_cast<float2*>(ws + lay.table);
+  pp.kws = reinterpret_cast<__nv_bfloat16*>(ws + lay.kws);
+  pp.qws = nullptr;
+  pp.vws = nullptr;
+
+  CUtensorMap tmQ, tmK, tmV;
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)nq, (uint64_t)N};
+    const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)nq * D * 2};
+    const uint32_t box[3] = {(uint32_t)A::BOXC, (uint32_t)G, (uint32_t)tq};
+    if (!make_tmap(device, q, dims, str, box, A::ROWB, &tmQ)) return GQA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)N, (uint64_t)nkv};
+    const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)N * D * 2};
+    const uint32_t box[3] = {(uint32_t)A::BOXC, (uint32_t)BN, 1u};
+    if (!make_tmap(device, ws + lay.kws, dims, str, box, A::ROWB, &tmK)) return GQA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)nkv, (uint64_t)N};
+    const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)nkv * D * 2};
+    const uint32_t box[3] = {(uint32_t)A::BOXC, 1u, (uint32_t)BN};
+    if (!make_tmap(device, v, dims, str, box, A::ROWB, &tmV)) return GQA_ERR_CUDA;
+  }
+  long long nb = ((long long)N * (D / 4) + PREP_THREADS - 1) / PREP_THREADS;
+  if (nb > (long long)sm_count * 8) nb = (long long)sm_count * 8;
+  if (nb < 1) nb = 1;
+  if (t_prof_ev[0] && cudaEventRecord(t_prof_ev[0], stream) != cudaSuccess) return GQA_ERR_CUDA;
+  gqa_prep_kernel<D, false><<<(unsigned)(nb + 1), PREP_THREADS, 0, stream>>>(pp);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+  if (t_prof_ev[1] && cudaEventRecord(t_prof_ev[1], stream) != cudaSuccess) return GQA_ERR_CUDA;
+
+  MaskedParams mp{};
+  AttnParams& ap = mp.base;
+  ap.cu = cu;
+  ap.header = pp.header;
+  ap.item_counter = pp.header + 8;
+  ap.pairs = pp.pairs;
+  ap.table = pp.table;
+  ap.out = out;
+  ap.lse = lse;
+  ap.N = N;
+  ap.nq = nq;
+  ap.nkv = nkv;
+  ap.G = G;
+  ap.tq = tq;
+  ap.causal = causal;
+  ap.sched_dynamic = 0;
+  ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  ap.rescale_thr = 0.f;
+  mp.mask = reinterpret_cast<const __nv_bfloat16*>(mask);
+  mp.mask_len = mask_len;
+  mp.mask_ld = mask_ld;
+  mp.sqrt_d = (float)std::sqrt((double)D);
+  // one CTA per (sequence, q-tile, KV head) work item; CTAs past the
+  // prologue's item count exit at once
+  const unsigned grid = (unsigned)(lay.max_pairs * (long long)nkv);
+  gqa_attn_fwd_masked_kernel<D><<<grid, MK_THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, mp);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+  if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;
+  t_last_launches = 2;
+  return GQA_OK;
+}
+
 }  // namespace
 }  // namespace gqa
 
@@ -855,5 +960,66 @@ extern "C" int gqa_rope_attn_qkv_proj(const void* x, const void* w_qkv, const in
                                n_q_heads, n_kv_heads, q, k, v, ws, st, device, sm_count);
   GQA_PROJ_CASE(32) GQA_PROJ_CASE(64) GQA_PROJ_CASE(128)
 #undef GQA_PROJ_CASE
+  return GQA_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------------------
+// Forward with an additive mask
+
+extern "C" int gqa_rope_attn_fwd_masked(const void* q, const void* k, const void* v, const int32_t* positions,
+                                        double rope_theta, const int32_t* cu_seqlens, int num_seqs,
+                                        int total_tokens, int n_q_heads, int n_kv_heads, int head_dim, int causal,
+                                        const void* mask, int mask_len, int mask_ld, void* out, float* lse,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+  t_last_launches = 0;
+  struct Disarm {
+    ~Disarm() { t_prof_ev[0] = t_prof_ev[1] = t_prof_ev[2] = nullptr; }
+  } disarm;
+  if (total_tokens < 0 || num_seqs < 0) return GQA_ERR_INVALID_ARG;
+  if (n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return GQA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return GQA_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.0) || !std::isfinite(rope_theta)) return GQA_ERR_INVALID_ARG;
+  if (mask_len < 1 || mask_ld < mask_len || mask_ld % 8) return GQA_ERR_INVALID_ARG;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED;
+  if (n_q_heads / n_kv_heads > BM) return GQA_ERR_UNSUPPORTED;
+  if ((long long)total_tokens * n_q_heads * head_dim > (1ll << 40)) return GQA_ERR_UNSUPPORTED;
+  if (total_tokens == 0) return GQA_OK;
+  if (num_seqs < 1) return GQA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !cu_seqlens || !mask) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(mask))
+    return GQA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(positions) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return GQA_ERR_INVALID_ARG;
+  const WsLayout lay = ws_layout(num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim, false);
+  if (lay.max_pairs * (long long)n_kv_heads > 0x7fffffffll) return GQA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < lay.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return GQA_ERR_WORKSPACE;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices) return GQA_ERR_CUDA;
+  int sm_count = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState& ds = g_dev[device];
+    if (!ds.init) {
+      int major = 0;
+      if (cudaDeviceGetAttribute(&ds.sm_count, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+          cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess)
+        return GQA_ERR_CUDA;
+      if (major != 10) return GQA_ERR_UNSUPPORTED;
+      ds.init = true;
+    }
+    sm_count = ds.sm_count;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  std::lock_guard<std::mutex> lk(g_mu);  // descriptor cache
+#define GQA_MASKED_CASE(DD)                                                                                   \
+  if (head_dim == DD)                                                                                         \
+    return launch_masked<DD>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads,  \
+                             n_kv_heads, causal, mask, mask_len, mask_ld, out, lse, ws, lay, st, device,      \
+                             sm_count);
+  GQA_MASKED_CASE(32) GQA_MASKED_CASE(64) GQA_MASKED_CASE(128)
+#undef GQA_MASKED_CASE
   return GQA_ERR_UNSUPPORTED;
 }
