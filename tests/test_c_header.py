@@ -47,6 +47,9 @@ int main(void) {
   /* projection: hidden not a multiple of 8 */
   CHECK(gqa_rope_attn_qkv_proj(a, a, NULL, 1e4, (const int32_t*)a, 1, 128, 100, 4, 2, 64, a, a, a, NULL, 0,
                                NULL) == GQA_ERR_UNSUPPORTED);
+  /* masked forward: mask row stride not a multiple of 8 */
+  CHECK(gqa_rope_attn_fwd_masked(a, a, a, NULL, 1e4, (const int32_t*)a, 1, 128, 4, 2, 64, 1, a, 128, 132, a, NULL,
+                                 NULL, 0, NULL) == GQA_ERR_INVALID_ARG);
   CHECK(gqa_rope_attn_last_launch_count() == 0);
   gqa_rope_attn_set_profile_events(NULL, NULL, NULL);
   printf("ok\n");
