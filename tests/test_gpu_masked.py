@@ -80,3 +80,27 @@ def test_zero_mask_equals_the_forward():
     torch.cuda.synchronize()
     assert (out_m.float() - out_f.float()).abs().max().item() <= 2e-2
     assert ((lse_m - lse_f).abs() / lse_f.abs().clamp(min=1.0)).max().item() <= 1e-5
+
+
+def test_mask_with_a_wider_row_stride():
+    """A mask whose rows are longer than mask_len (ld > Lm): only the first
+    Lm columns of each row are read."""
+    import torch
+    import transformer_attention_gqa_b200 as g
+
+    lens = (120, 9)
+    inp = wl.make_custom(lens, 8, 2, 64, causal=True, seed=14, name="wide_ld")
+    mask = _mask(15, 120, 0.2, ())                        # [120, 120]
+    wide = np.full((mask.shape[0], mask.shape[1] + 16), np.nan)
+    wide[:, : mask.shape[1]] = mask                       # never-read columns hold NaN
+    q, k, v, cu, _ = H.to_device(inp)
+    mt = torch.from_numpy(wide.astype(np.float32)).to(torch.bfloat16).cuda()
+    out, lse = g.gqa_rope_attn_fwd_masked(q, k, v, cu, inp.workload.rope_theta, mt, causal=True)
+    torch.cuda.synchronize()
+    assert g.get_device_status() == 0
+    ro, rl = orc.gqa_rope_attention_masked(inp.q, inp.k, inp.v, inp.cu_seqlens, 8, 2, inp.workload.rope_theta, mask,
+                                           causal=True)
+    o = out.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(o))
+    err = np.abs(o - ro)
+    assert err.max() <= H.OUT_MAX_ABS and err.mean() <= H.OUT_MEAN_ABS

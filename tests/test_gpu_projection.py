@@ -28,11 +28,13 @@ pytestmark = [
 
 # (sequence lengths, hidden, n_q, n_kv, d, theta): ragged token tails; the
 # Llama-3-8B layer's widths (4096 -> 32/8 heads of 128); feature counts that
-# end inside a 256-wide tile (6/2 heads of 64 = 640 features); d = 32.
+# end inside a 256-wide tile (6/2 heads of 64 = 640 features); d = 32; a
+# hidden size that is not a multiple of 64.
 CASES = {
     "llama_widths": ((200, 77), 4096, 32, 8, 128, 5e5),
     "nano_ragged_features": ((300,), 384, 6, 2, 64, 1e4),
     "d32": ((130, 1, 60), 256, 8, 4, 32, 1e4),
+    "hidden_tail": ((70,), 200, 4, 2, 32, 1e4),  # the last 64-wide block of C is partly past the rows
 }
 
 
