@@ -7,7 +7,7 @@ from . import _abi
 from ._abi import (GqaError, workspace_size, decode_workspace_size, bwd_workspace_size,  # noqa: F401
                    qkv_proj_workspace_size, get_device_status)
 
-__all__ = ["gqa_rope_attn_fwd", "gqa_rope_attn_fwd_masked", "gqa_rope_attn_decode", "gqa_rope_attn_bwd", "gqa_rope_attn_qkv_proj",
+__all__ = ["gqa_rope_attention", "gqa_rope_attn_fwd", "gqa_rope_attn_fwd_masked", "gqa_rope_attn_decode", "gqa_rope_attn_bwd", "gqa_rope_attn_qkv_proj",
            "workspace_size", "decode_workspace_size", "bwd_workspace_size", "qkv_proj_workspace_size",
            "get_device_status", "GqaError", "Workspace"]
 
@@ -290,3 +290,46 @@ def gqa_rope_attn_fwd_masked(q, k, v, cu_seqlens, rope_theta: float, mask, posit
     if rc != _abi.GQA_OK:
         raise GqaError(rc, "gqa_rope_attn_fwd_masked")
     return out, lse
+
+
+def _autograd_function():
+    """The torch.autograd.Function over the library's forward and backward
+    (built on first use, so that importing the package needs no torch)."""
+    global _GqaRopeAttention
+    if _GqaRopeAttention is not None:
+        return _GqaRopeAttention
+    import torch
+
+    class GqaRopeAttention(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, q, k, v, cu_seqlens, rope_theta, positions, causal):
+            out, lse = gqa_rope_attn_fwd(q, k, v, cu_seqlens, rope_theta, positions=positions, causal=causal)
+            ctx.save_for_backward(q, k, v, out, lse, cu_seqlens)
+            ctx.positions = positions
+            ctx.rope_theta = rope_theta
+            ctx.causal = causal
+            ctx.mark_non_differentiable(lse)
+            return out, lse
+
+        @staticmethod
+        def backward(ctx, dout, _dlse):
+            q, k, v, out, lse, cu = ctx.saved_tensors
+            dq, dk, dv = gqa_rope_attn_bwd(q, k, v, out, lse, dout.contiguous(), cu, ctx.rope_theta,
+                                           positions=ctx.positions, causal=ctx.causal)
+            return dq, dk, dv, None, None, None, None
+
+    _GqaRopeAttention = GqaRopeAttention
+    return GqaRopeAttention
+
+
+_GqaRopeAttention = None
+
+
+def gqa_rope_attention(q, k, v, cu_seqlens, rope_theta: float, positions=None, causal: bool = True):
+    """softmax(rope(q) rope(k)^T / sqrt(d) + causal mask) v with gradients:
+    out = gqa_rope_attn_fwd(...) in the forward pass, and dq, dk, dv from
+    gqa_rope_attn_bwd (which reuses the forward's out and lse) in the
+    backward pass. bf16 q, k, v [N, heads, d]; returns out (lse is kept for
+    the backward and not returned)."""
+    out, _ = _autograd_function().apply(q, k, v, cu_seqlens, rope_theta, positions, causal)
+    return out
