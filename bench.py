@@ -277,11 +277,12 @@ def _nbytes(tensors):
     return sum(t.numel() * t.element_size() for t in tensors)
 
 
-def _reference_line(args, world, metric, unit, workload, shape, sample, digits=6):
+def _reference_line(args, world, metric, unit, config, sample, digits=6):
     """The --impl reference JSON line: the oracle, as it stands, on bounded
     samples of the workload (sample(budget_s, index) -> cpu_baseline dict;
     index 1000 + i for the args.warmup short warm-up samples, i for the
-    args.steps timed ones), reporting the median."""
+    args.steps timed ones), reporting the median. ``config`` is the GPU
+    arm's config dict for the same workload."""
     for i in range(args.warmup):
         sample(0.5, 1000 + i)
     vals, info = [], None
@@ -291,7 +292,7 @@ def _reference_line(args, world, metric, unit, workload, shape, sample, digits=6
     val = round(statistics.median(vals), digits)
     return {"impl": "reference", "metric": metric, "value": val, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": {"workload": workload, "shape": shape},
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
             "cpu_baseline": {"value": val, "unit": unit, "cores": info["cores"], "kind": "oracle",
                              "sample": info["sample"]},
             "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -305,6 +306,15 @@ DECODE_UNIT = "GB/s"
 def _decode_sample_bytes(w, sel):
     lens = np.asarray(w.cache_lens)[sel]
     return float(np.sum(lens + 1)) * w.n_kv_heads * w.head_dim * 2 * 2
+
+
+def decode_config(w, world):
+    big = w.kv_bytes() > 2 * (126 << 20)
+    return {"workload": w.name, "shape": w.description, "batch": w.batch, "max_cache_len": w.max_cache_len,
+            "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+            "algorithmic_bytes_per_step": w.step_bytes(), "tokens_per_step": w.batch,
+            "parallelism": f"replicas x{world}",
+            "l2": "K/V read per step larger than L2" if big else "256 MiB written before every timed step"}
 
 
 def cpu_baseline_decode(w, inp, budget_s: float = 15.0, seed: int = 0):
@@ -386,12 +396,8 @@ def run_decode(args, rank, world, local_rank):
         "unit": DECODE_UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "shape": w.description, "batch": w.batch, "max_cache_len": w.max_cache_len,
-                   "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
-                   "algorithmic_bytes_per_step": nbytes, "tokens_per_step": w.batch,
-                   "tokens_per_s": round(w.batch * world / (ms_per_step * 1e-3), 1),
-                   "parallelism": f"replicas x{world}",
-                   "l2": "K/V read per step larger than L2" if big else "256 MiB written before every timed step"},
+        "config": decode_config(w, world),
+        "tokens_per_s": round(w.batch * world / (ms_per_step * 1e-3), 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": None,
                      "peak_source": f"{src} hbm_gbs (copy)", "kernel": "gqa_decode_split_kernel + gqa_decode_combine_kernel",
@@ -502,11 +508,7 @@ def run_bwd(args, rank, world, local_rank):
         "metric": BWD_METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "shape": w.description, "total_tokens": w.total_tokens,
-                   "num_seqs": w.num_seqs, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
-                   "head_dim": w.head_dim, "rope_theta": w.rope_theta, "causal": w.causal,
-                   "flops_per_step": flops, "parallelism": f"replicas x{world}",
-                   "l2": "256 MiB written before every timed step, outside the step's events"},
+        "config": bwd_config(args.workload, w, world, flops),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": None,
@@ -521,12 +523,21 @@ def run_bwd(args, rank, world, local_rank):
     return res
 
 
+def bwd_config(name, w, world, flops):
+    return {"workload": name, "shape": w.description, "total_tokens": w.total_tokens,
+            "num_seqs": w.num_seqs, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim, "rope_theta": w.rope_theta, "causal": w.causal,
+            "flops_per_step": flops, "parallelism": f"replicas x{world}",
+            "l2": "256 MiB written before every timed step, outside the step's events"}
+
+
 def main_bwd(args, world, rank, local_rank):
     from transformer_attention_gqa_b200 import workloads as wl
     w = wl.WORKLOADS[BWD_WORKLOADS[args.workload]]
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(_reference_line(args, world, BWD_METRIC, UNIT, args.workload, w.description,
+            print(json.dumps(_reference_line(args, world, BWD_METRIC, UNIT,
+                                             bwd_config(args.workload, w, world, BWD_FLOP_FACTOR * w.flops()),
                                              lambda budget, _: cpu_baseline_bwd(w, budget_s=budget))))
         return 0
     from transformer_attention_gqa_b200 import replicas
@@ -633,11 +644,7 @@ def run_proj(args, rank, world, local_rank, inp):
         "metric": PROJ_METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "shape": w.description, "total_tokens": N, "hidden": C,
-                   "out_features": F, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
-                   "head_dim": w.head_dim, "rope_theta": w.rope_theta, "flops_per_step": flops,
-                   "parallelism": f"replicas x{world}",
-                   "l2": "256 MiB written before every timed step, outside the step's events"},
+        "config": proj_config(args.workload, w, world),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": None,
@@ -652,6 +659,16 @@ def run_proj(args, rank, world, local_rank, inp):
     return res
 
 
+def proj_config(name, w, world):
+    C, F = _proj_shape(w)
+    N = w.total_tokens
+    return {"workload": name, "shape": w.description, "total_tokens": N, "hidden": C,
+            "out_features": F, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim, "rope_theta": w.rope_theta, "flops_per_step": 2.0 * N * C * F,
+            "parallelism": f"replicas x{world}",
+            "l2": "256 MiB written before every timed step, outside the step's events"}
+
+
 def main_proj(args, world, rank, local_rank):
     from transformer_attention_gqa_b200 import replicas, workloads as wl
     w = wl.WORKLOADS[PROJ_WORKLOADS[args.workload]]
@@ -660,7 +677,7 @@ def main_proj(args, world, rank, local_rank):
     inp = wl.make_projection_inputs(w.seq_lens, C, w.n_q_heads, w.n_kv_heads, w.head_dim, w.rope_theta, seed=seed)
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(_reference_line(args, world, PROJ_METRIC, UNIT, args.workload, w.description,
+            print(json.dumps(_reference_line(args, world, PROJ_METRIC, UNIT, proj_config(args.workload, w, world),
                                              lambda budget, _: cpu_baseline_proj(w, inp, budget_s=budget))))
         return 0
     replicas.init("nccl", timeout_s=120)
@@ -770,12 +787,7 @@ def run_masked(args, rank, world, local_rank, inp, mask_np):
         "metric": MASKED_METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "shape": w.description, "total_tokens": w.total_tokens,
-                   "num_seqs": w.num_seqs, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
-                   "head_dim": w.head_dim, "rope_theta": w.rope_theta, "causal": True,
-                   "mask": f"bf16 [{mask_np.shape[0]}, {mask_np.shape[1]}] seeded N(0, 1) bias",
-                   "flops_per_step": flops, "parallelism": f"replicas x{world}",
-                   "l2": "256 MiB written before every timed step, outside the step's events"},
+        "config": masked_config(args.workload, w, world, mask_np.shape),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": None,
@@ -790,6 +802,15 @@ def run_masked(args, rank, world, local_rank, inp, mask_np):
     return res
 
 
+def masked_config(name, w, world, mask_shape):
+    return {"workload": name, "shape": w.description, "total_tokens": w.total_tokens,
+            "num_seqs": w.num_seqs, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim, "rope_theta": w.rope_theta, "causal": True,
+            "mask": f"bf16 [{mask_shape[0]}, {mask_shape[1]}] seeded N(0, 1) bias",
+            "flops_per_step": w.flops(), "parallelism": f"replicas x{world}",
+            "l2": "256 MiB written before every timed step, outside the step's events"}
+
+
 def main_masked(args, world, rank, local_rank):
     from transformer_attention_gqa_b200 import replicas, workloads as wl
     w = wl.WORKLOADS[MASKED_WORKLOADS[args.workload]]
@@ -798,7 +819,8 @@ def main_masked(args, world, rank, local_rank):
     mask = _bench_mask(w, seed + 1)
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(_reference_line(args, world, MASKED_METRIC, UNIT, args.workload, w.description,
+            print(json.dumps(_reference_line(args, world, MASKED_METRIC, UNIT,
+                                             masked_config(args.workload, w, world, mask.shape),
                                              lambda budget, _: cpu_baseline_masked(w, inp, mask, budget_s=budget))))
         return 0
     replicas.init("nccl", timeout_s=120)
@@ -812,6 +834,14 @@ def main_masked(args, world, rank, local_rank):
 
 
 # ------------------------------------------------------------------ GPU arm
+def fwd_config(w, world):
+    return {"workload": w.name, "shape": w.description, "total_tokens": w.total_tokens,
+            "num_seqs": w.num_seqs, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim, "rope_theta": w.rope_theta, "causal": w.causal,
+            "flops_per_step": w.flops(), "parallelism": f"replicas x{world}",
+            "l2": "256 MiB written before every timed step, outside the step's events"}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import transformer_attention_gqa_b200 as g
@@ -957,11 +987,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "shape": w.description, "total_tokens": w.total_tokens,
-                   "num_seqs": w.num_seqs, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
-                   "head_dim": w.head_dim, "rope_theta": w.rope_theta, "causal": w.causal,
-                   "flops_per_step": flops, "parallelism": f"replicas x{world}",
-                   "l2": "256 MiB written before every timed step, outside the step's events"},
+        "config": fwd_config(w, world),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name),
@@ -1021,7 +1047,7 @@ def main():
         res = {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": UNIT, "n_gpus": world,
                "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-               "config": {"workload": w.name, "shape": w.description},
+               "config": fwd_config(w, world),
                "cpu_baseline": {"value": round(val, 6), "unit": UNIT, "cores": info["cores"], "kind": "oracle",
                                 "sample": info["sample"]},
                "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -1045,7 +1071,7 @@ def main_decode(args, world, rank, local_rank):
     if args.impl == "reference":
         if rank == 0:
             inp = wl.make_decode_inputs(w, nan_tail=False)
-            print(json.dumps(_reference_line(args, world, DECODE_METRIC, DECODE_UNIT, w.name, w.description,
+            print(json.dumps(_reference_line(args, world, DECODE_METRIC, DECODE_UNIT, decode_config(w, world),
                                              lambda budget, i: cpu_baseline_decode(w, inp, budget_s=budget, seed=i),
                                              digits=4)))
         return 0

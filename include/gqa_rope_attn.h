@@ -141,8 +141,8 @@ int gqa_rope_attn_abi_version(void);
 int gqa_rope_attn_last_launch_count(void);
 
 /* Size of the scratch buffer built into the library for
- * gqa_rope_attn_fwd_noalloc: 32 MiB of device memory per GPU that loads the
- * library, held until the process exits. */
+ * gqa_rope_attn_fwd_noalloc: 32 MiB of device memory on every GPU where the
+ * library's device code is loaded, held until the process exits. */
 #define GQA_ROPE_ATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
 
 /* The fused forward for callers that cannot allocate device memory: for
@@ -154,13 +154,21 @@ int gqa_rope_attn_last_launch_count(void);
  * Same arguments and results as gqa_rope_attn_fwd, minus the workspace: the
  * scratch lives in a static device array of GQA_ROPE_ATTN_NOALLOC_SCRATCH_BYTES
  * inside the library. The caller still provides q, k, v, positions,
- * cu_seqlens, out and lse. Nothing is allocated, by this call or any library
- * it uses.
- *   - Shapes whose gqa_rope_attn_workspace_size() exceeds the buffer are
- *     rejected with GQA_ERR_NOALLOC_LIMIT before any CUDA call.
+ * cu_seqlens, out and lse. The call makes no cudaMalloc or cudaFree, and
+ * neither does anything it calls.
+ *   - Invalid arguments get the same codes as from gqa_rope_attn_fwd, before
+ *     any CUDA call. Shapes whose gqa_rope_attn_workspace_size() exceeds the
+ *     buffer are then rejected with GQA_ERR_NOALLOC_LIMIT, also before any
+ *     CUDA call.
  *   - The first call on a device (per process) looks the buffer's device
  *     address up with cudaGetSymbolAddress, with that device current; make
- *     that first call before any stream capture on the device.
+ *     that first call before any stream capture on the device. CUDA loads a
+ *     library's device code lazily by default, so this first call may be
+ *     the one that loads it onto the device: that reserves the buffer there
+ *     and may synchronise the device.
+ *   - The buffer is reserved on every device where the library's device
+ *     code is loaded (by any of its entry points), whether or not this entry
+ *     point is ever called, and held until the process exits.
  *   - All calls on a device share the one buffer: calls that may overlap on
  *     the GPU (different streams without ordering, several host threads)
  *     race on it and must be serialised by the caller. The buffer keeps the

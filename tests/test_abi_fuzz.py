@@ -35,6 +35,11 @@ def fwd(q, k, v, pos, th, cu, ns, n, hq, hk, d, causal, dt, out, lse, ws, wb):
     assert _abi.gqa_rope_attn_fwd(q, k, v, pos, th, cu, ns, n, hq, hk, d, causal, dt, out, lse, ws, wb, None) in CODES
 
 @cfg
+@given(ptr, ptr, ptr, ptr, theta, ptr, small, small, heads, heads, dims, flags, flags, ptr, ptr)
+def fwd_noalloc(q, k, v, pos, th, cu, ns, n, hq, hk, d, causal, dt, out, lse):
+    assert _abi.gqa_rope_attn_fwd_noalloc(q, k, v, pos, th, cu, ns, n, hq, hk, d, causal, dt, out, lse, None) in CODES
+
+@cfg
 @given(ptr, ptr, ptr, ptr, ptr, ptr, theta, small, small, heads, heads, dims, ptr, ptr, ptr, size)
 def dec(q, kn, vn, kc, vc, lens, th, b, lm, hq, hk, d, out, lse, ws, wb):
     assert _abi.gqa_rope_attn_decode(q, kn, vn, kc, vc, lens, th, b, lm, hq, hk, d, out, lse, ws, wb, None) in CODES
@@ -56,7 +61,7 @@ def masked(q, k, v, pos, th, cu, ns, n, hq, hk, d, causal, m, ml, ld, out, lse, 
     assert _abi.gqa_rope_attn_fwd_masked(q, k, v, pos, th, cu, ns, n, hq, hk, d, causal, m, ml, ld, out, lse, ws, wb,
                                          None) in CODES
 
-for f in (fwd, dec, bwd, proj, masked):
+for f in (fwd, fwd_noalloc, dec, bwd, proj, masked):
     f()
 print("fuzz ok")
 """

@@ -2,7 +2,7 @@
 two calls are replaced by float64 oracle stand-ins, so that only the
 binding's plumbing is under test (what it saves, what reaches the backward
 call, what it returns to autograd). CPU only; the GPU path of the same
-function is in tests/test_gpu_autograd.py."""
+function is in tests/test_gpu_backward_autograd.py."""
 import numpy as np
 import pytest
 import torch
@@ -31,6 +31,7 @@ def oracle_library(monkeypatch):
 
     monkeypatch.setattr(g, "gqa_rope_attn_fwd", fwd)
     monkeypatch.setattr(g, "gqa_rope_attn_bwd", bwd)
+    monkeypatch.setattr(g, "_AUTOGRAD_DTYPES", ("float64",))  # the stand-ins work in float64
     return calls
 
 
@@ -64,3 +65,13 @@ def test_non_contiguous_upstream_gradient_is_made_contiguous(oracle_library):
     big = torch.tensor(rng.standard_normal((N, nq, 2 * d)), dtype=torch.float64)
     out.backward(big[..., ::2])  # a strided view
     assert oracle_library["bwd"][5]
+
+
+def test_dtypes_the_backward_cannot_take_are_refused_before_the_forward(monkeypatch):
+    called = []
+    monkeypatch.setattr(g, "gqa_rope_attn_fwd", lambda *a, **kw: called.append(1))
+    cu = torch.tensor([0, 4], dtype=torch.int32)
+    q, k, v = (torch.zeros((4, 2, 8), dtype=torch.float32, requires_grad=True) for _ in range(3))
+    with pytest.raises(TypeError, match="bfloat16"):
+        g.gqa_rope_attention(q, k, v, cu, 1e4)
+    assert not called

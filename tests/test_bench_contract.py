@@ -24,5 +24,24 @@ def test_reference_arm_json_line(workload):
     assert KEYS <= set(res)
     assert res["impl"] == "reference" and res["value"] > 0 and res["steps"] == 2 and res["warmup"] == 3
     assert res["config"]["workload"] == workload
+    assert res["config"] == json.loads(json.dumps(_gpu_arm_config(workload)))  # the GPU arm's config, key for key
     assert res["cpu_baseline"]["kind"] == "oracle" and res["cpu_baseline"]["cores"] >= 1
     assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def _gpu_arm_config(workload):
+    sys.path.insert(0, ROOT)
+    import bench
+    from transformer_attention_gqa_b200 import workloads as wl
+
+    if workload in wl.DECODE_WORKLOADS:
+        return bench.decode_config(wl.DECODE_WORKLOADS[workload], 1)
+    if workload in bench.BWD_WORKLOADS:
+        w = wl.WORKLOADS[bench.BWD_WORKLOADS[workload]]
+        return bench.bwd_config(workload, w, 1, bench.BWD_FLOP_FACTOR * w.flops())
+    if workload in bench.PROJ_WORKLOADS:
+        return bench.proj_config(workload, wl.WORKLOADS[bench.PROJ_WORKLOADS[workload]], 1)
+    if workload in bench.MASKED_WORKLOADS:
+        w = wl.WORKLOADS[bench.MASKED_WORKLOADS[workload]]
+        return bench.masked_config(workload, w, 1, bench._bench_mask(w, w.seed + 1).shape)
+    return bench.fwd_config(wl.WORKLOADS[workload], 1)

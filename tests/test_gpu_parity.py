@@ -1,8 +1,8 @@
 """GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
-the same seeded, bf16-rounded inputs. Small workloads are compared element
-by element in full; the Llama-3-8B-shaped and packed variable-length
-workloads run at full size in the benchmark's launch configuration and are
-compared on sampled rows the oracle computes one by one."""
+the same seeded, bf16-rounded inputs, element by element on every row and
+head: the small workloads, and the Llama-3-8B-shaped and packed
+variable-length workloads at full size in the benchmark's launch
+configuration."""
 import numpy as np
 import pytest
 
@@ -25,13 +25,26 @@ def test_named_workload_full(name):
 
 
 @pytest.mark.parametrize("name", ["llama8b", "varlen"])
-def test_named_workload_sampled_rows(name):
+def test_named_workload_full_size(name, record_property):
+    """The full-size workloads in the benchmark's launch configuration,
+    compared with the oracle on every row and head (the oracle works through
+    256-row blocks to bound its memory). The LSE against the exact-rotation
+    oracle (no bf16 rounding of the rotated operands) is reported, not
+    gated: that rounding moves each score by up to ~1e-3 relative."""
     inp = wl.make_inputs(wl.WORKLOADS[name])
     out, lse = H.run_gpu(inp)
-    assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
-    rows = H.sample_rows(inp.cu_seqlens, per_seq=16 if name == "varlen" else 48)
-    ref_out, ref_lse = H.oracle(inp, rows=rows)
-    H.compare(out, lse, ref_out, ref_lse, rows=rows, what=name)
+    ref_out, ref_lse = H.oracle(inp, row_block=256)
+    stats = H.compare(out, lse, ref_out, ref_lse, what=name)
+    ex_out, ex_lse = H.oracle(inp, operand_rounding=False, row_block=256)
+    ex = H.compare(out, None, ex_out, None, what=name + " vs exact RoPE")
+    d = np.abs(lse - ex_lse)
+    stats.update({"exact_out_max_abs": ex["out_max_abs"], "exact_out_mean_abs": ex["out_mean_abs"],
+                  "exact_lse_rel_plain": float(np.max(d / np.abs(ex_lse))),
+                  "exact_lse_rel_floored": float(np.max(d / np.maximum(np.abs(ex_lse), 1.0))),
+                  "exact_lse_abs": float(d.max()), "min_abs_lse": float(np.min(np.abs(ex_lse)))})
+    for key, val in stats.items():
+        record_property(key, val)
+    print(name, stats)
 
 
 CASES = [

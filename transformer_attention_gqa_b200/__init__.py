@@ -323,6 +323,8 @@ def _autograd_function():
 
 
 _GqaRopeAttention = None
+# dtypes both library calls under gqa_rope_attention accept
+_AUTOGRAD_DTYPES = ("bfloat16",)
 
 
 def gqa_rope_attention(q, k, v, cu_seqlens, rope_theta: float, positions=None, causal: bool = True):
@@ -330,6 +332,10 @@ def gqa_rope_attention(q, k, v, cu_seqlens, rope_theta: float, positions=None, c
     out = gqa_rope_attn_fwd(...) in the forward pass, and dq, dk, dv from
     gqa_rope_attn_bwd (which reuses the forward's out and lse) in the
     backward pass. bf16 q, k, v [N, heads, d]; returns out (lse is kept for
-    the backward and not returned)."""
+    the backward and not returned). The backward takes bf16 only, so other
+    dtypes are refused here, before the forward runs."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if str(t.dtype).replace("torch.", "") not in _AUTOGRAD_DTYPES:
+            raise TypeError(f"gqa_rope_attention: {name} must be bfloat16 (the backward is bf16 only), got {t.dtype}")
     out, _ = _autograd_function().apply(q, k, v, cu_seqlens, rope_theta, positions, causal)
     return out

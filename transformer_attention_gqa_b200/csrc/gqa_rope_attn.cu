@@ -690,6 +690,34 @@ extern "C" size_t gqa_rope_attn_workspace_size(int num_seqs, int total_tokens, i
   return ws_layout(num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim, dtype == GQA_DTYPE_FP32).total;
 }
 
+// The forward's argument checks that need no CUDA call (shared by the
+// forward and its no-allocation variant). GQA_OK with *empty set means there
+// is nothing to compute (no tokens).
+static int fwd_check_args(const void* q, const void* k, const void* v, const int32_t* positions, double rope_theta,
+                          const int32_t* cu_seqlens, int num_seqs, int total_tokens, int n_q_heads, int n_kv_heads,
+                          int head_dim, int causal, int dtype, const void* out, const float* lse, bool* empty) {
+  *empty = false;
+  if (total_tokens < 0 || num_seqs < 0) return GQA_ERR_INVALID_ARG;
+  if (n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return GQA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return GQA_ERR_INVALID_ARG;
+  if (dtype != GQA_DTYPE_BF16 && dtype != GQA_DTYPE_FP32) return GQA_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.0) || !std::isfinite(rope_theta)) return GQA_ERR_INVALID_ARG;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED;
+  if (n_q_heads / n_kv_heads > BM) return GQA_ERR_UNSUPPORTED;
+  if ((long long)total_tokens * n_q_heads * head_dim > (1ll << 40)) return GQA_ERR_UNSUPPORTED;
+  if (total_tokens == 0) {
+    *empty = true;
+    return GQA_OK;
+  }
+  if (num_seqs < 1) return GQA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !cu_seqlens) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GQA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(positions) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return GQA_ERR_INVALID_ARG;
+  return GQA_OK;
+}
+
 extern "C" int gqa_rope_attn_fwd(const void* q, const void* k, const void* v, const int32_t* positions,
                                  double rope_theta, const int32_t* cu_seqlens, int num_seqs, int total_tokens,
                                  int n_q_heads, int n_kv_heads, int head_dim, int causal, int dtype, void* out,
@@ -699,21 +727,10 @@ extern "C" int gqa_rope_attn_fwd(const void* q, const void* k, const void* v, co
     ~Disarm() { t_prof_ev[0] = t_prof_ev[1] = t_prof_ev[2] = nullptr; }
   } disarm;
   // ---- checks that need no CUDA call
-  if (total_tokens < 0 || num_seqs < 0) return GQA_ERR_INVALID_ARG;
-  if (n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads) return GQA_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return GQA_ERR_INVALID_ARG;
-  if (dtype != GQA_DTYPE_BF16 && dtype != GQA_DTYPE_FP32) return GQA_ERR_INVALID_ARG;
-  if (!(rope_theta > 0.0) || !std::isfinite(rope_theta)) return GQA_ERR_INVALID_ARG;
-  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED;
-  if (n_q_heads / n_kv_heads > BM) return GQA_ERR_UNSUPPORTED;
-  if ((long long)total_tokens * n_q_heads * head_dim > (1ll << 40)) return GQA_ERR_UNSUPPORTED;
-  if (total_tokens == 0) return GQA_OK;
-  if (num_seqs < 1) return GQA_ERR_INVALID_ARG;
-  if (!q || !k || !v || !out || !cu_seqlens) return GQA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GQA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(positions) & 3u) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u))
-    return GQA_ERR_INVALID_ARG;
+  bool empty = false;
+  const int arg_rc = fwd_check_args(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads,
+                                    n_kv_heads, head_dim, causal, dtype, out, lse, &empty);
+  if (arg_rc != GQA_OK || empty) return arg_rc;
   const bool fp32 = dtype == GQA_DTYPE_FP32;
   const WsLayout lay = ws_layout(num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim, fp32);
   if (!workspace || workspace_bytes < lay.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -773,13 +790,18 @@ extern "C" int gqa_rope_attn_fwd_noalloc(const void* q, const void* k, const voi
                                          double rope_theta, const int32_t* cu_seqlens, int num_seqs,
                                          int total_tokens, int n_q_heads, int n_kv_heads, int head_dim,
                                          int causal, int dtype, void* out, float* lse, void* stream) {
+  // the same argument checks as the forward, before any CUDA call
+  bool empty = false;
+  const int arg_rc = fwd_check_args(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads,
+                                    n_kv_heads, head_dim, causal, dtype, out, lse, &empty);
+  if (arg_rc != GQA_OK || empty) return arg_rc;
   const size_t need =
       gqa_rope_attn_workspace_size(num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim, dtype);
   if (need > (size_t)GQA_ROPE_ATTN_NOALLOC_SCRATCH_BYTES) return GQA_ERR_NOALLOC_LIMIT;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices) return GQA_ERR_CUDA;
   void* scratch = nullptr;
-  if (total_tokens > 0 && need > 0) {
-    int device = 0;
-    if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices) return GQA_ERR_CUDA;
+  {
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
     if (!g_noalloc_ptr[device]) {
       // The array's name is only a host-side handle; its device address is
@@ -792,7 +814,7 @@ extern "C" int gqa_rope_attn_fwd_noalloc(const void* q, const void* k, const voi
   }
   return gqa_rope_attn_fwd(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads,
                            n_kv_heads, head_dim, causal, dtype, out, lse, scratch,
-                           scratch ? (size_t)GQA_ROPE_ATTN_NOALLOC_SCRATCH_BYTES : 0, stream);
+                           (size_t)GQA_ROPE_ATTN_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 extern "C" int gqa_rope_attn_get_device_status(void* stream) {
