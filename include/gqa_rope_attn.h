@@ -23,7 +23,8 @@
  *     batches (cu_seqlens prefix sums).
  *   The log-sum-exp output is not on the pages; it is the natural-log
  *   normaliser of each row's scaled, masked scores.
- * A forward with an additive mask (gqa_rope_attn_fwd_masked), a decoding
+ * A forward on already rotated q and k (gqa_rope_attn_fwd_rotated), a
+ * forward with an additive mask (gqa_rope_attn_fwd_masked), a decoding
  * step against a KV cache (gqa_rope_attn_decode), the backward
  * (gqa_rope_attn_bwd) and the QKV projection with its RoPE epilogue
  * (gqa_rope_attn_qkv_proj) are declared further down.
@@ -123,6 +124,25 @@ int gqa_rope_attn_fwd(const void* q, const void* k, const void* v, const int32_t
                       int total_tokens, int n_q_heads, int n_kv_heads, int head_dim,
                       int causal, int dtype, void* out, float* lse, void* workspace,
                       size_t workspace_bytes, void* stream);
+
+/* The forward on q and k that are already rotated, e.g. the outputs of
+ * gqa_rope_attn_qkv_proj. "Attention from Scratch", section "Attention, the
+ * math": the module rotates Q and K once (step 2) and then scores, masks and
+ * normalises them (steps 4-6); this call is steps 4-6 alone:
+ *
+ *   out[t, h, :] = softmax_j( q[t, h] . k[j, kv] / sqrt(d) ) v[j, kv]
+ *
+ * with lse, masks, GQA sharing and packed sequences as in gqa_rope_attn_fwd.
+ * bf16 only; no positions or rope_theta (nothing is rotated); K is read in
+ * place from the caller's [total_tokens, n_kv_heads, head_dim] tensor, so
+ * the call skips the forward's K pass (its prologue only builds the tile
+ * schedule). Arguments, alignment, workspace (gqa_rope_attn_workspace_size()
+ * with GQA_DTYPE_BF16 is enough), status codes and stream behaviour as for
+ * gqa_rope_attn_fwd. */
+int gqa_rope_attn_fwd_rotated(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                              int num_seqs, int total_tokens, int n_q_heads, int n_kv_heads,
+                              int head_dim, int causal, void* out, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream);
 
 /* Waits for `stream` (a cudaStream_t as void*, NULL for the default stream),
  * then returns and clears the current device's status word: GQA_OK, or the

@@ -40,6 +40,11 @@ def fwd_noalloc(q, k, v, pos, th, cu, ns, n, hq, hk, d, causal, dt, out, lse):
     assert _abi.gqa_rope_attn_fwd_noalloc(q, k, v, pos, th, cu, ns, n, hq, hk, d, causal, dt, out, lse, None) in CODES
 
 @cfg
+@given(ptr, ptr, ptr, ptr, small, small, heads, heads, dims, flags, ptr, ptr, ptr, size)
+def fwd_rotated(q, k, v, cu, ns, n, hq, hk, d, causal, out, lse, ws, wb):
+    assert _abi.gqa_rope_attn_fwd_rotated(q, k, v, cu, ns, n, hq, hk, d, causal, out, lse, ws, wb, None) in CODES
+
+@cfg
 @given(ptr, ptr, ptr, ptr, ptr, ptr, theta, small, small, heads, heads, dims, ptr, ptr, ptr, size)
 def dec(q, kn, vn, kc, vc, lens, th, b, lm, hq, hk, d, out, lse, ws, wb):
     assert _abi.gqa_rope_attn_decode(q, kn, vn, kc, vc, lens, th, b, lm, hq, hk, d, out, lse, ws, wb, None) in CODES
@@ -61,7 +66,7 @@ def masked(q, k, v, pos, th, cu, ns, n, hq, hk, d, causal, m, ml, ld, out, lse, 
     assert _abi.gqa_rope_attn_fwd_masked(q, k, v, pos, th, cu, ns, n, hq, hk, d, causal, m, ml, ld, out, lse, ws, wb,
                                          None) in CODES
 
-for f in (fwd, fwd_noalloc, dec, bwd, proj, masked):
+for f in (fwd, fwd_noalloc, fwd_rotated, dec, bwd, proj, masked):
     f()
 print("fuzz ok")
 """

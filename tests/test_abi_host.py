@@ -99,6 +99,30 @@ def test_host_rejections_before_any_cuda_call():
     assert _abi.last_launch_count() == 0
 
 
+def test_rotated_forward_host_rejections_before_any_cuda_call():
+    E = _abi
+
+    def rot(**kw):
+        args = dict(q=A, k=A, v=A, cu_seqlens=A, num_seqs=1, total_tokens=128, n_q_heads=4, n_kv_heads=2,
+                    head_dim=64, causal=1, out=A, lse=0, workspace=0, workspace_bytes=0, stream=None)
+        args.update(kw)
+        return _abi.gqa_rope_attn_fwd_rotated(**args)
+
+    assert rot(total_tokens=0) == E.GQA_OK
+    assert rot(total_tokens=-1) == E.GQA_ERR_INVALID_ARG
+    assert rot(n_q_heads=6, n_kv_heads=4) == E.GQA_ERR_INVALID_ARG
+    assert rot(causal=3) == E.GQA_ERR_INVALID_ARG
+    assert rot(head_dim=48) == E.GQA_ERR_UNSUPPORTED
+    assert rot(n_q_heads=256, n_kv_heads=1) == E.GQA_ERR_UNSUPPORTED
+    assert rot(num_seqs=0) == E.GQA_ERR_INVALID_ARG
+    assert rot(k=0) == E.GQA_ERR_INVALID_ARG
+    assert rot(v=A + 4) == E.GQA_ERR_INVALID_ARG
+    assert rot() == E.GQA_ERR_WORKSPACE
+    need = _abi.workspace_size(1, 128, 4, 2, 64)
+    assert rot(workspace=A, workspace_bytes=need - 1) == E.GQA_ERR_WORKSPACE
+    assert _abi.last_launch_count() == 0
+
+
 def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(_abi, "_lib", None)

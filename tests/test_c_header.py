@@ -36,6 +36,11 @@ int main(void) {
   /* forward: head_dim unsupported */
   CHECK(gqa_rope_attn_fwd(a, a, a, NULL, 1e4, (const int32_t*)a, 1, 128, 4, 2, 80, 1, GQA_DTYPE_BF16, a, NULL,
                           NULL, 0, NULL) == GQA_ERR_UNSUPPORTED);
+  /* forward on rotated inputs: workspace missing; group of 256 heads unsupported */
+  CHECK(gqa_rope_attn_fwd_rotated(a, a, a, (const int32_t*)a, 1, 128, 4, 2, 64, 1, a, NULL, NULL, 0, NULL) ==
+        GQA_ERR_WORKSPACE);
+  CHECK(gqa_rope_attn_fwd_rotated(a, a, a, (const int32_t*)a, 1, 128, 256, 1, 64, 1, a, NULL, NULL, 0, NULL) ==
+        GQA_ERR_UNSUPPORTED);
   CHECK(gqa_rope_attn_fwd_noalloc(a, a, a, NULL, 1e4, (const int32_t*)a, 1, 1 << 22, 32, 8, 128, 1,
                                   GQA_DTYPE_BF16, a, NULL, NULL) == GQA_ERR_NOALLOC_LIMIT);
   /* decoding step: group of 32 query heads per KV head is unsupported */

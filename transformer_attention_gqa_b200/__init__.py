@@ -7,7 +7,7 @@ from . import _abi
 from ._abi import (GqaError, workspace_size, decode_workspace_size, bwd_workspace_size,  # noqa: F401
                    qkv_proj_workspace_size, get_device_status)
 
-__all__ = ["gqa_rope_attention", "gqa_rope_attn_fwd", "gqa_rope_attn_fwd_masked", "gqa_rope_attn_decode", "gqa_rope_attn_bwd", "gqa_rope_attn_qkv_proj",
+__all__ = ["gqa_rope_attention", "gqa_rope_attn_fwd", "gqa_rope_attn_fwd_rotated", "gqa_rope_attn_fwd_masked", "gqa_rope_attn_decode", "gqa_rope_attn_bwd", "gqa_rope_attn_qkv_proj",
            "workspace_size", "decode_workspace_size", "bwd_workspace_size", "qkv_proj_workspace_size",
            "get_device_status", "GqaError", "Workspace"]
 
@@ -97,6 +97,48 @@ def gqa_rope_attn_fwd(q, k, v, cu_seqlens, rope_theta: float, positions=None, ca
                                 ws.numel() * ws.element_size(), stream)
     if rc != _abi.GQA_OK:
         raise GqaError(rc)
+    return out, lse
+
+
+def gqa_rope_attn_fwd_rotated(q, k, v, cu_seqlens, causal: bool = True, out=None, lse=None, workspace=None,
+                              stream=None, need_lse: bool = True):
+    """out, lse = softmax(q k^T / sqrt(d) + causal mask) v on q and k that are
+    already rotated (e.g. gqa_rope_attn_qkv_proj's outputs): the attention
+    steps after the rotation. bf16 CUDA tensors q [N, n_q, d], k/v
+    [N, n_kv, d]; cu_seqlens int32 [num_seqs+1]. Returns (out, lse [n_q, N]
+    fp32 or None). Raises GqaError on a non-OK status."""
+    import torch
+
+    _check(q.dim() == 3 and k.dim() == 3, "q must be [N, n_q, d] and k, v [N, n_kv, d]")
+    N, nq, d = q.shape
+    nkv = k.shape[1]
+    if q.dtype != torch.bfloat16:
+        raise TypeError("q must be bfloat16")
+    _check(k.shape == (N, nkv, d) and v.shape == (N, nkv, d), "k and v must be [N, n_kv, d] matching q")
+    _check(k.dtype == q.dtype and v.dtype == q.dtype, "q, k and v must share one dtype")
+    _check(cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1 and cu_seqlens.numel() >= 1,
+           "cu_seqlens must be a 1-D int32 tensor")
+    num_seqs = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and need_lse:
+        lse = torch.empty((nq, N), dtype=torch.float32, device=q.device)
+    _check(out.shape == q.shape and out.dtype == q.dtype, "out must match q's shape and dtype")
+    if lse is not None:
+        _check(lse.shape == (nq, N) and lse.dtype == torch.float32, "lse must be float32 [n_q, N]")
+    _check_tensors(dict(q=q, k=k, v=v, cu_seqlens=cu_seqlens, out=out, lse=lse), q.device)
+    nbytes = workspace_size(num_seqs, N, nq, nkv, d, _abi.GQA_DTYPE_BF16)
+    if workspace is None:
+        workspace = Workspace(q.device)
+    ws = workspace.get(nbytes) if isinstance(workspace, Workspace) else workspace
+    _check_tensors(dict(workspace=ws), q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    rc = _abi.gqa_rope_attn_fwd_rotated(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), num_seqs, N, nq, nkv, d,
+                                        1 if causal else 0, _ptr(out), _ptr(lse), _ptr(ws),
+                                        ws.numel() * ws.element_size(), stream)
+    if rc != _abi.GQA_OK:
+        raise GqaError(rc, "gqa_rope_attn_fwd_rotated")
     return out, lse
 
 

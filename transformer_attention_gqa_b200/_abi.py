@@ -39,6 +39,7 @@ EXPORTED = (
     "gqa_rope_attn_qkv_proj_workspace_size",
     "gqa_rope_attn_qkv_proj",
     "gqa_rope_attn_fwd_masked",
+    "gqa_rope_attn_fwd_rotated",
 )
 
 _lib = None
@@ -97,6 +98,9 @@ def load() -> ctypes.CDLL:
     lib.gqa_rope_attn_fwd_masked.argtypes = [c_void, c_void, c_void, c_void, c_double, c_void, c_int, c_int, c_int,
                                              c_int, c_int, c_int, c_void, c_int, c_int, c_void, c_void, c_void,
                                              c_size, c_void]
+    lib.gqa_rope_attn_fwd_rotated.restype = c_int
+    lib.gqa_rope_attn_fwd_rotated.argtypes = [c_void, c_void, c_void, c_void, c_int, c_int, c_int, c_int, c_int,
+                                              c_int, c_void, c_void, c_void, c_size, c_void]
     lib.gqa_rope_attn_set_profile_events.restype = None
     lib.gqa_rope_attn_set_profile_events.argtypes = [c_void, c_void, c_void]
     _lib = lib
@@ -118,6 +122,15 @@ def gqa_rope_attn_fwd(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, tota
     return int(load().gqa_rope_attn_fwd(q, k, v, positions, float(rope_theta), cu_seqlens, int(num_seqs),
                                         int(total_tokens), int(n_q_heads), int(n_kv_heads), int(head_dim),
                                         int(causal), int(dtype), out, lse, workspace, int(workspace_bytes), stream))
+
+
+def gqa_rope_attn_fwd_rotated(q, k, v, cu_seqlens, num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim, causal,
+                              out, lse, workspace, workspace_bytes, stream) -> int:
+    """Raw call of the forward on already rotated q and k; integer device
+    addresses, 0 for NULL; returns the status."""
+    return int(load().gqa_rope_attn_fwd_rotated(q, k, v, cu_seqlens, int(num_seqs), int(total_tokens),
+                                                int(n_q_heads), int(n_kv_heads), int(head_dim), int(causal), out, lse,
+                                                workspace, int(workspace_bytes), stream))
 
 
 def gqa_rope_attn_fwd_noalloc(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads,

@@ -441,7 +441,7 @@ __device__ __forceinline__ bool rope_q_tile(const AttnParams& p, uint8_t* smem, 
   if (w < 0) return true;
   const WorkItem wi = decode_item(p, w);
   uint8_t* qbuf = smem + qb * C::Q_BYTES;
-  const int items = p.tq * NCH;
+  const int items = p.prerotated ? 0 : p.tq * NCH;  // rotated inputs: Q is used as loaded
   for (int item = tid; item < items; item += 128) {
     const int tt = item / NCH;
     const int ch = item - tt * NCH;
@@ -669,9 +669,13 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           const int ks = g % C::KST;
           if (!(ok = bwait_lazy(B(bars->k_empty[ks]), ((g / C::KST) & 1) ^ 1, abort_flag))) break;
           ptx::mbar_arrive_expect_tx(B(bars->k_full[ks]), (uint32_t)C::KV_BYTES);
+          // K' head-major (token, head) or, for rotated inputs, the caller's
+          // token-major K (head, token): the same 128-byte rows in shared memory
+          const int c1 = p.prerotated ? wi.kvh : wi.seq_start + j * BN;
+          const int c2 = p.prerotated ? wi.seq_start + j * BN : wi.kvh;
           for (int b = 0; b < C::NBOX; ++b)
             ptx::tma_load_3d(sbase + C::OFF_K + ks * C::KV_BYTES + b * C::KV_BOX_BYTES, &tmK,
-                             B(bars->k_full[ks]), b * C::BOXC, wi.seq_start + j * BN, wi.kvh);
+                             B(bars->k_full[ks]), b * C::BOXC, c1, c2);
         }
         w = wn;
       }

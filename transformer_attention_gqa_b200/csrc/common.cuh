@@ -104,6 +104,8 @@ struct AttnParams {
   int sched_dynamic;    // 1: items beyond the first from item_counter; 0: static alternating deal
   float scale_log2;     // log2(e) / sqrt(d)
   float rescale_thr;    // raw-score growth that triggers an O rescale
+  int prerotated;       // 1: q and k arrive rotated; K is read token-major [N][n_kv][d] from the
+                        // caller's tensor and Q is not rotated again; 0: K' head-major from the prologue
 };
 
 }  // namespace gqa

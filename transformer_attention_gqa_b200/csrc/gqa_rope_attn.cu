@@ -129,10 +129,14 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int dim_index(int d) { return d == 32 ? 0 : (d == 64 ? 1 : 2); }
 
+// prerotated: q and k are already rotated (bf16 only); the prologue builds
+// the schedule alone and K is read from the caller's token-major tensor.
 template <int D, bool FP32>
 int launch(const void* q, const void* k, const void* v, const int32_t* positions, double theta,
            const int32_t* cu, int num_seqs, int N, int nq, int nkv, int causal, void* out, float* lse,
-           uint8_t* ws, const WsLayout& lay, cudaStream_t stream, int device, int sm_count) {
+           uint8_t* ws, const WsLayout& lay, cudaStream_t stream, int device, int sm_count,
+           bool prerotated = false) {
+  if (FP32 && prerotated) return GQA_ERR_UNSUPPORTED;
   using C = AttnCfg<D>;
   const int G = nq / nkv;
   const int tq = tokens_per_tile(G);
@@ -181,7 +185,12 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
     const uint32_t box[3] = {(uint32_t)C::BOXC, (uint32_t)G, (uint32_t)tq};
     if (!make_tmap(device, qsrc, dims, str, box, C::ROWB, &tmQ)) return GQA_ERR_CUDA;
   }
-  {
+  if (prerotated) {  // the caller's K, token-major like V
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)nkv, (uint64_t)N};
+    const uint64_t str[2] = {(uint64_t)D * es, (uint64_t)nkv * D * es};
+    const uint32_t box[3] = {(uint32_t)C::BOXC, 1u, (uint32_t)BN};
+    if (!make_tmap(device, k, dims, str, box, C::ROWB, &tmK)) return GQA_ERR_CUDA;
+  } else {
     const uint64_t dims[3] = {(uint64_t)D, (uint64_t)N, (uint64_t)nkv};
     const uint64_t str[2] = {(uint64_t)D * es, (uint64_t)N * D * es};
     const uint32_t box[3] = {(uint32_t)C::BOXC, (uint32_t)BN, 1u};
@@ -200,6 +209,7 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
   const long long cap = (long long)sm_count * 8;
   if (nb > cap) nb = cap;
   if (nb < 1) nb = 1;
+  if (prerotated) nb = 0;  // block 0 alone: the schedule
   if (t_prof_ev[0] && cudaEventRecord(t_prof_ev[0], stream) != cudaSuccess) return GQA_ERR_CUDA;
   gqa_prep_kernel<D, FP32><<<(unsigned)(nb + 1), PREP_THREADS, 0, stream>>>(pp);
   if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
@@ -222,6 +232,7 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
   ap.causal = causal;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   ap.rescale_thr = (float)(8.0 / (1.4426950408889634 / std::sqrt((double)D)));
+  ap.prerotated = prerotated ? 1 : 0;
 
   const long long max_items = lay.max_pairs * (long long)nkv;
   const unsigned grid = (unsigned)(max_items < sm_count ? max_items : sm_count);
@@ -690,6 +701,26 @@ extern "C" size_t gqa_rope_attn_workspace_size(int num_seqs, int total_tokens, i
   return ws_layout(num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim, dtype == GQA_DTYPE_FP32).total;
 }
 
+// Current device and its SM count; the first call per device checks that it
+// is a compute capability 10.x part.
+static int device_init(int* device_out, int* sm_count_out) {
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess || device < 0 || device >= kMaxDevices) return GQA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& ds = g_dev[device];
+  if (!ds.init) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&ds.sm_count, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess)
+      return GQA_ERR_CUDA;
+    if (major != 10) return GQA_ERR_UNSUPPORTED;
+    ds.init = true;
+  }
+  *device_out = device;
+  *sm_count_out = ds.sm_count;
+  return GQA_OK;
+}
+
 // The forward's argument checks that need no CUDA call (shared by the
 // forward and its no-allocation variant). GQA_OK with *empty set means there
 // is nothing to compute (no tokens).
@@ -773,6 +804,36 @@ extern "C" int gqa_rope_attn_fwd(const void* q, const void* k, const void* v, co
   }
 #undef GQA_FWD_CASE
   return rc;
+}
+
+extern "C" int gqa_rope_attn_fwd_rotated(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                                         int num_seqs, int total_tokens, int n_q_heads, int n_kv_heads,
+                                         int head_dim, int causal, void* out, float* lse, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  t_last_launches = 0;
+  struct Disarm {
+    ~Disarm() { t_prof_ev[0] = t_prof_ev[1] = t_prof_ev[2] = nullptr; }
+  } disarm;
+  bool empty = false;
+  const int arg_rc = fwd_check_args(q, k, v, nullptr, 1.0, cu_seqlens, num_seqs, total_tokens, n_q_heads,
+                                    n_kv_heads, head_dim, causal, GQA_DTYPE_BF16, out, lse, &empty);
+  if (arg_rc != GQA_OK || empty) return arg_rc;
+  const WsLayout lay = ws_layout(num_seqs, total_tokens, n_q_heads, n_kv_heads, head_dim, false);
+  if (!workspace || workspace_bytes < lay.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return GQA_ERR_WORKSPACE;
+  int device = 0, sm_count = 0;
+  const int init_rc = device_init(&device, &sm_count);
+  if (init_rc != GQA_OK) return init_rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  std::lock_guard<std::mutex> lk(g_mu);  // descriptor cache
+#define GQA_ROT_CASE(DD)                                                                                    \
+  if (head_dim == DD)                                                                                       \
+    return launch<DD, false>(q, k, v, nullptr, 1.0, cu_seqlens, num_seqs, total_tokens, n_q_heads,          \
+                             n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count, true);
+  GQA_ROT_CASE(32) GQA_ROT_CASE(64) GQA_ROT_CASE(128)
+#undef GQA_ROT_CASE
+  return GQA_ERR_UNSUPPORTED;
 }
 
 // ---------------------------------------------------------------------------
