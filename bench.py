@@ -13,6 +13,7 @@ in HBM. Default workload: Llama-3-8B-shaped causal prefill (B=1, T=8192,
   --workload bwd_llama8b | bwd_varlen | bwd_nano    the backward (dq, dk, dv)
   --workload qkv_llama8b | qkv_nano                 the QKV projection with its RoPE epilogue
   --workload masked_llama8b | masked_nano           the forward with an additive mask
+  --workload rot_llama8b | rot_varlen | ...          the forward on already rotated q and k
 
 Under torchrun each rank runs its own replica of the workload (independent
 problems, weak scaling); the elapsed time is the max over ranks.
@@ -834,7 +835,22 @@ def main_masked(args, world, rank, local_rank):
 
 
 # ------------------------------------------------------------------ GPU arm
-def fwd_config(w, world):
+# The forward on already rotated q and k (gqa_rope_attn_fwd_rotated): a
+# forward workload's shape, its seeded N(0, 1) q and k taken as the rotated
+# operands (a rotation keeps that distribution), the forward's FLOP count.
+ROT_WORKLOADS = {"rot_llama8b": "llama8b", "rot_varlen": "varlen", "rot_qwen05b": "qwen05b", "rot_nano": "nano"}
+ROT_METRIC = "causal GQA attention fwd on pre-rotated q/k TFLOP/s on 1 B200; % of dense-BF16 tensor peak"
+
+
+def fwd_config(w, world, name=None):
+    cfg = _fwd_config(w, world)
+    if name is not None:
+        cfg["workload"] = name
+        cfg["inputs"] = "q and k taken as already rotated"
+    return cfg
+
+
+def _fwd_config(w, world):
     return {"workload": w.name, "shape": w.description, "total_tokens": w.total_tokens,
             "num_seqs": w.num_seqs, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
             "head_dim": w.head_dim, "rope_theta": w.rope_theta, "causal": w.causal,
@@ -842,7 +858,7 @@ def fwd_config(w, world):
             "l2": "256 MiB written before every timed step, outside the step's events"}
 
 
-def run_ours(args, rank, world, local_rank):
+def run_ours(args, rank, world, local_rank, rotated=False):
     import torch
     import transformer_attention_gqa_b200 as g
     from transformer_attention_gqa_b200 import _abi, replicas, workloads as wl
@@ -864,7 +880,10 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        g.gqa_rope_attn_fwd(q, k, v, cu, w.rope_theta, causal=w.causal, out=out, lse=lse, workspace=ws)
+        if rotated:
+            g.gqa_rope_attn_fwd_rotated(q, k, v, cu, causal=w.causal, out=out, lse=lse, workspace=ws)
+        else:
+            g.gqa_rope_attn_fwd(q, k, v, cu, w.rope_theta, causal=w.causal, out=out, lse=lse, workspace=ws)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -948,8 +967,13 @@ def run_ours(args, rank, world, local_rank):
             sl["k"].copy_(kh, non_blocking=True)
             sl["v"].copy_(vh, non_blocking=True)
             sl["cu"].copy_(cuh, non_blocking=True)
-            g.gqa_rope_attn_fwd(sl["q"], sl["k"], sl["v"], sl["cu"], w.rope_theta, causal=w.causal, out=sl["out"],
-                                lse=sl["lse"], workspace=sl["ws"], stream=sl["stream"].cuda_stream)
+            if rotated:
+                g.gqa_rope_attn_fwd_rotated(sl["q"], sl["k"], sl["v"], sl["cu"], causal=w.causal, out=sl["out"],
+                                            lse=sl["lse"], workspace=sl["ws"], stream=sl["stream"].cuda_stream)
+            else:
+                g.gqa_rope_attn_fwd(sl["q"], sl["k"], sl["v"], sl["cu"], w.rope_theta, causal=w.causal,
+                                    out=sl["out"], lse=sl["lse"], workspace=sl["ws"],
+                                    stream=sl["stream"].cuda_stream)
             sl["outh"].copy_(sl["out"], non_blocking=True)
             sl["lseh"].copy_(sl["lse"], non_blocking=True)
 
@@ -984,13 +1008,13 @@ def run_ours(args, rank, world, local_rank):
     peak = float(peaks["bf16_tflops"])
     achieved = flops / (attn_ms * 1e-3) / 1e12
     res = {
-        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "metric": ROT_METRIC if rotated else METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": fwd_config(w, world),
+        "config": fwd_config(w, world, args.workload if rotated else None),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name),
+                     "frac": round(achieved / peak, 4), "traffic": None if rotated else recorded_traffic(w.name),
                      "peak_source": f"{src} bf16_tflops (burst)", "kernel": "gqa_attn_fwd_kernel",
                      "kernel_ms": round(attn_ms, 4), "prologue_ms": round(prep_ms, 4)},
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
@@ -1031,7 +1055,10 @@ def main():
         return main_proj(args, world, rank, local_rank)
     if args.workload in MASKED_WORKLOADS:
         return main_masked(args, world, rank, local_rank)
-    w = wl.WORKLOADS[args.workload]
+    rotated = args.workload in ROT_WORKLOADS
+    w = wl.WORKLOADS[ROT_WORKLOADS[args.workload] if rotated else args.workload]
+    metric = ROT_METRIC if rotated else METRIC
+    cfg_name = args.workload if rotated else None
 
     if args.impl == "reference":
         if rank != 0:
@@ -1044,10 +1071,10 @@ def main():
             info = cpu_baseline(w, budget_s=max(1.0, min(5.0, 60.0 / max(args.steps, 1))), seed_rows=i)
             per_step.append(info["value"])
         val = statistics.median(per_step)
-        res = {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": UNIT, "n_gpus": world,
+        res = {"impl": "reference", "metric": metric, "value": round(val, 6), "unit": UNIT, "n_gpus": world,
                "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-               "config": fwd_config(w, world),
+               "config": fwd_config(w, world, cfg_name),
                "cpu_baseline": {"value": round(val, 6), "unit": UNIT, "cores": info["cores"], "kind": "oracle",
                                 "sample": info["sample"]},
                "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -1056,7 +1083,7 @@ def main():
 
     from transformer_attention_gqa_b200 import replicas
     replicas.init("nccl", timeout_s=120)
-    res = run_ours(args, rank, world, local_rank)
+    res = run_ours(args, rank, world, local_rank, rotated=rotated)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
     replicas.shutdown()

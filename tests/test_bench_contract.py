@@ -13,7 +13,7 @@ KEYS = {"impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "higher_
         "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"}
 
 
-@pytest.mark.parametrize("workload", ["tiny", "decode_small", "bwd_nano", "qkv_nano", "masked_nano"])
+@pytest.mark.parametrize("workload", ["tiny", "decode_small", "bwd_nano", "qkv_nano", "masked_nano", "rot_nano"])
 def test_reference_arm_json_line(workload):
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", workload,
                         "--steps", "2", "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=300)
@@ -44,4 +44,6 @@ def _gpu_arm_config(workload):
     if workload in bench.MASKED_WORKLOADS:
         w = wl.WORKLOADS[bench.MASKED_WORKLOADS[workload]]
         return bench.masked_config(workload, w, 1, bench._bench_mask(w, w.seed + 1).shape)
+    if workload in bench.ROT_WORKLOADS:
+        return bench.fwd_config(wl.WORKLOADS[bench.ROT_WORKLOADS[workload]], 1, workload)
     return bench.fwd_config(wl.WORKLOADS[workload], 1)

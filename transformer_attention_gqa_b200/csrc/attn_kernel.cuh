@@ -260,14 +260,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// Of every EMU_PERIOD groups of 4 exponentials of a row, one is evaluated on
-// the FMA pipe, the rest on the special-function unit (0: all on the SFU).
-// With two softmax warps per sub-partition the SFU is the limit; 1 in 8
-// measured fastest (1 in 4 and more run out of issue slots).
-#ifndef GQA_EMU_PERIOD
-#define GQA_EMU_PERIOD 8
-#endif
-constexpr int EMU_PERIOD = GQA_EMU_PERIOD;
+// Of every emu_period(d) groups of 4 exponentials of a row, one is evaluated
+// on the FMA pipe, the rest on the special-function unit (0: all on the
+// SFU). With two softmax warps per sub-partition the SFU is the limit; at
+// d = 128, 1 in 8 measured fastest (1 in 4 and more run out of issue slots).
+__host__ __device__ constexpr int emu_period(int d) { return d == 128 ? 8 : (d == 64 ? 8 : 8); }
 
 __device__ __forceinline__ uint32_t swz(uint32_t lin, int mask) { return lin ^ (((lin >> 7) & mask) << 4); }
 
@@ -333,7 +330,7 @@ __device__ __forceinline__ float cols_max(const uint32_t* r) {
 // p = 2^(s * scale + bias) for the NC values, packed in place to bf16 pairs
 // (r[c/2], c = 0..NC-1). Returns the fp32 sum of p; if mx_out is given, also
 // the max of s.
-template <int NC>
+template <int NC, int EMU_PERIOD>
 __device__ __forceinline__ float exp_pack(uint32_t* r, float bias, float scale, float* mx_out) {
   float2 ls[4];
 #pragma unroll
@@ -829,13 +826,13 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           ok = __all_sync(0xffffffffu, bwait(xbar, xpar, abort_flag));
           if (!ok) break;
           m = fmaxf(mh, *xm_other);
-          lsum = exp_pack<NC>(sr, -m * sl2, sl2, nullptr);
+          lsum = exp_pack<NC, emu_period(D)>(sr, -m * sl2, sl2, nullptr);
         } else {
           // Exponentials with the running max m, the tile's max alongside;
           // if the row's max exceeds m by more than the threshold (2^8 in p)
           // the tile is redone below with the new max.
           float mh;
-          lsum = exp_pack<NC>(sr, -m * sl2, sl2, &mh);
+          lsum = exp_pack<NC, emu_period(D)>(sr, -m * sl2, sl2, &mh);
           *xm_mine = mh;
           ptx::mbar_arrive(xbar);
           ok = __all_sync(0xffffffffu, bwait(xbar, xpar, abort_flag));
@@ -851,7 +848,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           if (__any_sync(0xffffffffu, need)) {
             load_s_cols<NC>(tS, sr);  // S is intact: P has not been stored yet
             if (lim < NC - 1) mask_cols<NC>(sr, lim);
-            lsum = exp_pack<NC>(sr, -m * sl2, sl2, nullptr);
+            lsum = exp_pack<NC, emu_period(D)>(sr, -m * sl2, sl2, nullptr);
             // O holds the sum up to the previous tile: wait for PV(gg-1), then
             // scale this half's share of O's columns.
             const uint32_t gp = gg - 1;

@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(MK_THREADS, 1)
       m = m_new;
       // a row that has seen no visible key yet keeps p = 0 (bias 0, scores -inf)
       const float bias = m == -INFINITY ? 0.f : -m * sl2;
-      l += exp_pack<BN>(sr, bias, sl2, nullptr);
+      l += exp_pack<BN, emu_period(D)>(sr, bias, sl2, nullptr);
       ptx::tmem_st32(trow + s * 128, sr);            // keys [0, 64): columns 0..31
       ptx::tmem_st32(trow + s * 128 + 64, sr + 32);  // keys [64, 128): columns 64..95
       ptx::tmem_wait_st();
