@@ -6,12 +6,7 @@ Tolerance, from the arithmetic: the kernel accumulates x W^T in fp32 (for C
 up to 4096 and unit-scale outputs, errors of order 1e-5) and rounds each
 rotated output once to bf16 (at most 2^-9 relative, 2^-8 allowing the fp32
 error to cross a rounding midpoint); per element
-|gpu - ref| <= 2^-8 |ref| + 1e-4 max|ref|.
-
-Opt-in (GQA_PROJ_GPU_TESTS=1) until the kernel has had its first supervised
-run on a B200."""
-import os
-
+|gpu - ref| <= 2^-8 |ref| + 1e-4 max|ref|."""
 import numpy as np
 import pytest
 
@@ -19,12 +14,7 @@ import oracle.gqa_oracle as orc
 from tests.conftest import gpu_available
 from transformer_attention_gqa_b200 import workloads as wl
 
-pytestmark = [
-    pytest.mark.gpu,
-    pytest.mark.skipif(not gpu_available(), reason="needs a CUDA device"),
-    pytest.mark.skipif(os.environ.get("GQA_PROJ_GPU_TESTS") != "1",
-                       reason="projection kernel not yet run on a GPU: opt in with GQA_PROJ_GPU_TESTS=1"),
-]
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not gpu_available(), reason="needs a CUDA device")]
 
 # (sequence lengths, hidden, n_q, n_kv, d, theta): ragged token tails; the
 # Llama-3-8B layer's widths (4096 -> 32/8 heads of 128); feature counts that

@@ -305,9 +305,13 @@ __global__ void __launch_bounds__(MK_THREADS, 1)
       if (lim < BN - 1) mask_cols<BN>(sr, lim);
       const float mx = cols_max<BN>(sr);
       const float m_new = fmaxf(m, mx);
-      if (j > 0 && m != -INFINITY && m_new > m) {
+      // The rescale is decided per row, but its wait and the tensor-memory
+      // accesses are warp-collective (.sync.aligned): the whole warp enters
+      // the branch when any of its rows needs it, the others scale by 1.
+      const bool need = j > 0 && m != -INFINITY && m_new > m;
+      if (__any_sync(0xffffffffu, need)) {
         // O holds the sum up to tile j - 1: wait for P V(j - 1), then rescale
-        const float alpha = ptx::ex2((m - m_new) * sl2);
+        const float alpha = need ? ptx::ex2((m - m_new) * sl2) : 1.f;
         const uint32_t jp = j - 1;
         ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[jp & 1]), (jp >> 1) & 1, abort_flag));
         if (!ok) break;
