@@ -1,11 +1,7 @@
 """The autograd binding (``gqa_rope_attention``) on the GPU: out.backward()
 runs the library's backward on the forward's saved out and lse; the
 gradients match the float64 oracle's backward at the backward's bar
-(tests/test_gpu_backward.py).
-
-Opt-in (GQA_AUTOGRAD_GPU_TESTS=1) until its first supervised run on a B200."""
-import os
-
+(tests/test_gpu_backward.py)."""
 import numpy as np
 import pytest
 
@@ -13,12 +9,7 @@ import oracle.gqa_oracle as orc
 from tests.conftest import gpu_available
 from transformer_attention_gqa_b200 import workloads as wl
 
-pytestmark = [
-    pytest.mark.gpu,
-    pytest.mark.skipif(not gpu_available(), reason="needs a CUDA device"),
-    pytest.mark.skipif(os.environ.get("GQA_AUTOGRAD_GPU_TESTS") != "1",
-                       reason="autograd binding not yet run on a GPU: opt in with GQA_AUTOGRAD_GPU_TESTS=1"),
-]
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not gpu_available(), reason="needs a CUDA device")]
 
 
 def test_autograd_gradients_match_the_oracle():

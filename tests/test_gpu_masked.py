@@ -2,12 +2,7 @@
 through the C ABI) against the float64 oracle (``gqa_rope_attention_masked``)
 on the same seeded bf16 inputs and bf16 mask values, at the forward's bar
 (out max-abs <= 2e-2 and mean-abs <= 2e-3; lse |d| / max(|lse|, 1) <= 1e-4),
-rows that see no key compared exactly (out 0, lse -inf).
-
-Opt-in (GQA_MASK_GPU_TESTS=1) until the kernel has had its first supervised
-run on a B200."""
-import os
-
+rows that see no key compared exactly (out 0, lse -inf)."""
 import numpy as np
 import pytest
 
@@ -16,12 +11,7 @@ from tests.conftest import gpu_available
 from tests import gpu_helpers as H
 from transformer_attention_gqa_b200 import workloads as wl
 
-pytestmark = [
-    pytest.mark.gpu,
-    pytest.mark.skipif(not gpu_available(), reason="needs a CUDA device"),
-    pytest.mark.skipif(os.environ.get("GQA_MASK_GPU_TESTS") != "1",
-                       reason="masked kernel not yet run on a GPU: opt in with GQA_MASK_GPU_TESTS=1"),
-]
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not gpu_available(), reason="needs a CUDA device")]
 
 # (sequence lengths, n_q, n_kv, d, causal, share of hidden entries, rows hidden entirely)
 CASES = {
