@@ -783,7 +783,7 @@ def run_masked(args, rank, world, local_rank, inp, mask_np):
     value = flops * world / (ms_per_step * 1e-3) / 1e12
     peaks, src = load_peaks()
     peak = float(peaks["bf16_tflops"])
-    achieved = flops / (attn_ms * 1e-3) / 1e12
+    roof = fwd_roofline(w, attn_ms, peaks, src, clk, torch.cuda.get_device_properties(dev).multi_processor_count)
     res = {
         "metric": MASKED_METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
@@ -835,6 +835,31 @@ def main_masked(args, world, rank, local_rank):
 
 
 # ------------------------------------------------------------------ GPU arm
+SFU_EXP_PER_CLK_PER_SM = 16  # ex2 lanes per clock per SM (special-function unit)
+
+
+def fwd_roofline(w, kernel_ms, peaks, src, clk, sm_count):
+    """The attention kernel's binding roofline among three: dense bf16 tensor
+    throughput (the metric's FLOPs), the special-function unit's exponentials
+    (one per visible (query, key, head); 16 per clock per SM at the sampled
+    SM clock) and HBM (q, k, v read, out and lse written once). The binding
+    one is the slowest at its peak; frac = achieved / peak for it."""
+    mhz = float((clk or {}).get("sm_mhz") or (clk or {}).get("sm_max_mhz") or 1965.0)
+    t = kernel_ms * 1e-3
+    cands = {
+        "tensor": (w.flops() / 1e12, float(peaks["bf16_tflops"]), "TFLOP/s", f"{src} bf16_tflops (burst)"),
+        "alu": (w.exps() / 1e9, SFU_EXP_PER_CLK_PER_SM * sm_count * mhz * 1e-3, "Gexp/s",
+                f"SFU ex2 {SFU_EXP_PER_CLK_PER_SM}/clk/SM x {sm_count} SMs x {mhz:.0f} MHz"),
+        "hbm": (w.io_bytes() / 1e9, float(peaks["hbm_gbs"]), "GB/s", f"{src} hbm_gbs"),
+    }
+    bound = max(cands, key=lambda k: cands[k][0] / cands[k][1])
+    work, pk, unit, psrc = cands[bound]
+    return {"bound": bound, "achieved": round(work / t, 2), "peak": round(pk, 1), "unit": unit,
+            "frac": round(work / t / pk, 4), "peak_source": psrc,
+            "others": {k: {"achieved": round(v[0] / t, 2), "peak": round(v[1], 1), "unit": v[2],
+                           "frac": round(v[0] / t / v[1], 4)} for k, v in cands.items() if k != bound}}
+
+
 # The forward on already rotated q and k (gqa_rope_attn_fwd_rotated): a
 # forward workload's shape, its seeded N(0, 1) q and k taken as the rotated
 # operands (a rotation keeps that distribution), the forward's FLOP count.
@@ -1006,17 +1031,15 @@ def run_ours(args, rank, world, local_rank, rotated=False):
     value = flops * world / (ms_per_step * 1e-3) / 1e12
     peaks, src = load_peaks()
     peak = float(peaks["bf16_tflops"])
-    achieved = flops / (attn_ms * 1e-3) / 1e12
+    roof = fwd_roofline(w, attn_ms, peaks, src, clk, torch.cuda.get_device_properties(dev).multi_processor_count)
     res = {
         "metric": ROT_METRIC if rotated else METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": fwd_config(w, world, args.workload if rotated else None),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None if rotated else recorded_traffic(w.name),
-                     "peak_source": f"{src} bf16_tflops (burst)", "kernel": "gqa_attn_fwd_kernel",
-                     "kernel_ms": round(attn_ms, 4), "prologue_ms": round(prep_ms, 4)},
+        "roofline": dict(roof, traffic=None if rotated or roof["bound"] != "tensor" else recorded_traffic(w.name),
+                         kernel="gqa_attn_fwd_kernel", kernel_ms=round(attn_ms, 4), prologue_ms=round(prep_ms, 4)),
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
                 "streams": 2, "note": "independent batches on two alternating streams: a step's host-to-device "

@@ -47,3 +47,22 @@ def _gpu_arm_config(workload):
     if workload in bench.ROT_WORKLOADS:
         return bench.fwd_config(wl.WORKLOADS[bench.ROT_WORKLOADS[workload]], 1, workload)
     return bench.fwd_config(wl.WORKLOADS[workload], 1)
+
+
+def test_forward_roofline_picks_the_binding_unit():
+    """Long sequences at d = 128 are bound by the tensor cores; at d = 64 the
+    exponentials (one per visible pair and head, on the special-function
+    unit) take longer than the products."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from transformer_attention_gqa_b200 import workloads as wl
+
+    peaks = {"bf16_tflops": 1628.3, "hbm_gbs": 6535.0}
+    clk = {"sm_mhz": 1965.0}
+    llama = bench.fwd_roofline(wl.WORKLOADS["llama8b"], 0.5, peaks, "measured", clk, 148)
+    assert llama["bound"] == "tensor" and llama["unit"] == "TFLOP/s"
+    assert abs(llama["achieved"] - wl.WORKLOADS["llama8b"].flops() / 0.5e-3 / 1e12) < 0.01
+    qwen = bench.fwd_roofline(wl.WORKLOADS["qwen05b"], 0.08, peaks, "measured", clk, 148)
+    assert qwen["bound"] == "alu" and qwen["unit"] == "Gexp/s"
+    assert abs(qwen["peak"] - 16 * 148 * 1.965) < 0.1
+    assert set(qwen["others"]) == {"tensor", "hbm"}

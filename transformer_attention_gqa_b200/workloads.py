@@ -97,6 +97,15 @@ class Workload:
             tot += f / 2.0 if self.causal else f
         return tot
 
+    def exps(self) -> float:
+        """Exponentials by the same convention: one per (query, key, head)
+        pair, T^2/2 pairs per head when causal (summed per sequence)."""
+        tot = 0.0
+        for L in self.seq_lens:
+            e = float(L) * L * self.n_q_heads
+            tot += e / 2.0 if self.causal else e
+        return tot
+
     def io_bytes(self) -> int:
         """Algorithmic HBM bytes: read q, k, v once; write out once, lse once."""
         el = 4 if self.io_dtype == "fp32" else 2
