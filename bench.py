@@ -890,7 +890,7 @@ def run_ours(args, rank, world, local_rank, rotated=False):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = wl.WORKLOADS[args.workload]
+    w = wl.WORKLOADS[ROT_WORKLOADS[args.workload] if rotated else args.workload]
     # every rank runs its own batch of the same shape (weak scaling)
     inp = wl.make_inputs(w, seed=w.seed if rank == 0 else replicas.replica_seed(w.seed, rank))
     dt = torch.float32 if w.io_dtype == "fp32" else torch.bfloat16

@@ -10,28 +10,28 @@
 // is the causal mask's last row of the prefill computation.
 //
 // The step reads every cached K and V row once, so it is bound by HBM
-// bandwidth, not by arithmetic: the scores and the weighted sum run on the
-// FP32 pipes, and the cache streams through shared memory in TMA tiles.
+// bandwidth; the G heads that share a KV head make G multiply-adds per
+// cached value, which the tensor cores take (see gqa_decode_tc_kernel).
 //
-// Kernel 1 (split): one CTA per (key range, KV head, sequence). It rotates
-// the G queries of the KV head at p (and the new key, in the CTA whose range
-// holds p), then walks its key range in tiles of 64 keys (2-stage TMA ring
-// for K and V): scores of the tile for the G heads, an online softmax, and
-// the weighted sum of V. It leaves (running max, sum, un-normalised output)
-// per head in the workspace.
+// Kernel 1 (key ranges): one CTA per (key range, KV head, sequence). It
+// rotates the G queries of the KV head at p (and the new key, in the CTA
+// whose range holds p), then walks its key range in tiles of 64 keys through
+// a TMA ring: scores of the tile for the G heads, an online softmax, and the
+// weighted sum of V. It leaves (running max, sum, un-normalised output) per
+// head in the workspace.
 // Kernel 2 (combine): per (sequence, KV head) merges the ranges: out =
 // sum_s o_s 2^(m_s - M) / sum_s l_s 2^(m_s - M), lse = (M + log2 L) ln 2.
 #pragma once
 
+#include "attn_kernel.cuh"
 #include "common.cuh"
 #include "ptx.cuh"
 #include "rope_round.cuh"
 
 namespace gqa {
 
-constexpr int DEC_THREADS = 256;
-constexpr int DEC_KT = 64;      // keys per tile
-constexpr int DEC_STAGES = 2;
+constexpr int DEC_COMBINE_THREADS = 256;
+constexpr int DEC_KT = 64;      // keys per tile (the cache maps' box height)
 constexpr int DEC_GMAX = 16;    // query heads per KV head
 // The split count aims at about this many CTAs over the batch (measured:
 // fewer, longer CTAs amortise the per-CTA RoPE setup).
@@ -55,354 +55,373 @@ struct DecodeParams {
   float scale_log2;              // log2(e) / sqrt(d)
 };
 
-template <int D_, int GM_>
-struct DecCfg {
+// ---------------------------------------------------------------- key ranges on the tensor cores
+//
+// Both products on the tensor cores (tcgen05): the G rotated query heads of KV head
+// h fill G rows of a 128-row operand tile (the other rows are zero), so
+// S = Q K^T over a 64-key tile is one M = 128, N = 64 MMA into tensor memory
+// and O += P V one M = 128, N = d MMA with P read from tensor memory, the
+// operand forms of the prefill kernel. Head g sits at tile row
+// 32 (g % 4) + g / 4, so each of the four softmax warps (one TMEM lane
+// quadrant each) holds a share of the heads. Per CTA: one key range of one
+// (sequence, KV head), its partial (max, sum, un-normalised output) per head
+// for the combine kernel. (A CUDA-core version of this kernel, scores and
+// weighted sum on the FP32 pipes, reached 3.5 TB/s at G = 4 and 2.1 TB/s at
+// G = 8 on B200; this one 4.2 and 4.0.)
+//
+// Warps 0-3: RoPE of the queries and the new key, then the online softmax
+// (one row per thread; rows that hold no head compute zeros) and the partial
+// results. Warp 4: TMA of the K/V tiles through a two-stage ring, the
+// fix-up of the range's last tile (the new token's row from this CTA, rows
+// past the range zeroed in V so that their zero weights meet finite values)
+// and the appended cache row. Warp 5: tensor memory and the MMAs.
+// One CTA per SM with a four-stage ring (measured: two stages with two CTAs
+// per SM reached 2.7 TB/s, three 3.7, four to six 4.1-4.2).
+constexpr int DTC_KT = DEC_KT;   // keys per tile
+constexpr int DTC_STAGES = 4;
+constexpr int DTC_THREADS = 192;
+
+template <int D_>
+struct DtcCfg {
+  using A = AttnCfg<D_>;
   static constexpr int D = D_;
-  static constexpr int GM = GM_;                   // query heads per KV head, at most
-  static constexpr int BOXC = D >= 64 ? 64 : 32;   // columns per TMA box
-  static constexpr int NBOX = D / BOXC;
-  static constexpr int ROWB = BOXC * 2;            // bytes per box row (swizzle span)
-  static constexpr int SWZ_MASK = ROWB == 128 ? 7 : 3;
-  static constexpr int BOX_BYTES = DEC_KT * ROWB;
-  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one K or V tile
-  // Score phase: 4 lanes per key (a quarter of d each: CPQ 16-byte chunks),
-  // 8 keys per warp. Weighted-sum phase: thread = (4 output columns, key
-  // group of KPG keys), all heads.
-  static constexpr int CPQ = D / 32;
-  // Query chunk c (8 features) is stored at slot (c % CPQ) * 4 + c / CPQ, so
-  // the four lanes of a key, reading chunk i of their quarters at once, hit
-  // four different bank groups.
-  static __device__ __forceinline__ int qslot(int c) { return (c % CPQ) * 4 + c / CPQ; }
-  static constexpr int KGROUPS = DEC_THREADS / (D / 4);
-  static constexpr int KPG = DEC_KT / KGROUPS;
-  static constexpr int OFF_KV = 0;                                 // [stage][K tile, V tile]
-  static constexpr int OFF_Q = OFF_KV + DEC_STAGES * 2 * TILE_BYTES;  // float [GM][D]
-  static constexpr int OFF_S = OFF_Q + GM * D * 4;                    // float [KT][GM]
-  static constexpr int OFF_CS = OFF_S + GM * DEC_KT * 4;              // float2 [D/2] (cos, sin)
-  static constexpr int OFF_ML = OFF_CS + (D / 2) * 8;                 // float2 [GM] running (max, sum)
-  static constexpr int OFF_A = OFF_ML + GM * 8;                       // float [GM] rescale of the tile
-  static constexpr int OFF_NEW = OFF_A + GM * 4;                      // bf16 [2][D]: rotated new key, value
-  static constexpr int OFF_BAR = OFF_NEW + 2 * D * 2;                 // mbarriers [STAGES]
-  static constexpr int SMEM_BYTES = ((OFF_BAR + DEC_STAGES * 8 + 15) / 16) * 16 + 1024;  // + alignment slack
-  static_assert(DEC_THREADS == 4 * DEC_KT, "score phase: four lanes per key");
-  static_assert(KPG * KGROUPS == DEC_KT, "weighted-sum key groups");
-  static_assert(GM * D * 4 <= DEC_STAGES * 2 * TILE_BYTES, "final reduction buffer in the stage area");
-  static_assert(SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
+  static constexpr int KV_BOX_BYTES = DTC_KT * A::ROWB;      // one box of a 64-key tile
+  static constexpr int TILE_BYTES = A::NBOX * KV_BOX_BYTES;  // one K or V tile
+  static constexpr int OFF_Q = 0;                            // 128-row query tile
+  static constexpr int OFF_K = A::Q_BYTES;                   // [stage] K tiles
+  static constexpr int OFF_V = OFF_K + DTC_STAGES * TILE_BYTES;  // [stage] V tiles
+  static constexpr int OFF_CS = OFF_V + DTC_STAGES * TILE_BYTES;  // float2 [D/2] (cos, sin) at pos
+  static constexpr int OFF_NEW = OFF_CS + (D / 2) * 8;           // bf16 [2][D]: rotated new key, value
+  static constexpr int OFF_BAR = OFF_NEW + 2 * D * 2;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;       // + barriers + alignment slack
+  static constexpr uint32_t S_COL = 0;                          // two 64-column S/P buffers
+  static constexpr uint32_t O_COL = 2 * DTC_KT;
+  static constexpr uint32_t TMEM_COLS = 256;
+  // bf16 x bf16 -> fp32, both K-major, M = 128, N = 64 keys
+  static constexpr uint32_t IDESC_S =
+      (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(DTC_KT >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && TILE_BYTES % 1024 == 0, "swizzle atoms 1024-aligned");
+  static_assert(O_COL + D <= TMEM_COLS, "tensor memory budget");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
-__device__ __forceinline__ uint32_t dswz(uint32_t lin, int mask) { return lin ^ (((lin >> 7) & mask) << 4); }
+struct DtcBarriers {
+  uint64_t full[DTC_STAGES], empty[DTC_STAGES];
+  uint64_t fixed;     // the range's last tile patched in shared memory
+  uint64_t q_ready;   // query tile, new key and value written (128 arrivals)
+  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t o_full, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(DtcBarriers) <= 256, "barrier area");
 
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ void dtc_softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-// Bounded wait (2 s) for one mbarrier phase; false (and the device status
-// word set) when it runs out.
-__device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = ptx::globaltimer();
-  while (!ptx::mbar_try_wait(bar, parity)) {
-    if (ptx::globaltimer() - t0 > WAIT_TIMEOUT_NS) {
-      atomicCAS(&g_status, 0, kStatusTimeout);
-      return false;
-    }
-  }
-  return true;
-}
-
-// d = a * b + c on pairs of fp32 (one packed .f32x2 instruction).
-__device__ __forceinline__ float2 dec_ffma2(float2 a, float2 b, float2 c) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return d;
-}
-
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-template <int D, int GM>
-__global__ void __launch_bounds__(DEC_THREADS, 2)
-    gqa_decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                            const DecodeParams p) {
-  using C = DecCfg<D, GM>;
-  extern __shared__ uint8_t dec_smem_raw[];
-  // 1024-byte aligned base, derived from the shared array by pointer
-  // arithmetic so that accesses through it stay shared-memory accesses
-  uint8_t* sm = dec_smem_raw + ((1024u - (ptx::smem_u32(dec_smem_raw) & 1023u)) & 1023u);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+template <int D>
+__global__ void __launch_bounds__(DTC_THREADS, 1)
+    gqa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                         const DecodeParams p) {
+  using C = DtcCfg<D>;
+  using A = AttnCfg<D>;
+  constexpr int HALF = D / 2;
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int G = p.G;
   const int pos = __ldg(p.cache_seqlens + b);
   if (pos < 0 || pos >= p.Lmax) {  // the combine kernel skips this sequence too
-    if (tid == 0 && split == 0 && h == 0) atomicCAS(&g_status, 0, kStatusBadSeqlens);
+    if (threadIdx.x == 0 && split == 0 && h == 0) atomicCAS(&g_status, 0, kStatusBadSeqlens);
     return;
   }
   const int k0 = split * p.kps;
   const int k1 = min(k0 + p.kps, pos + 1);
   const size_t part = ((size_t)b * p.nkv + h) * p.splits + split;
-  float2* pml = p.part_ml + part * G;
-  float* po = p.part_o + part * G * D;
-  if (k0 >= k1) {  // no visible key in this range
-    for (int i = tid; i < G; i += DEC_THREADS) pml[i] = make_float2(-INFINITY, 0.f);
+  if (k0 >= k1) {  // no visible key in this range (the whole CTA, before any barrier or TMEM use)
+    for (int i = threadIdx.x; i < G; i += DTC_THREADS) p.part_ml[part * G + i] = make_float2(-INFINITY, 0.f);
     return;
   }
-  const int ntiles = (k1 - k0 + DEC_KT - 1) / DEC_KT;
+  const int ntiles = (k1 - k0 + DTC_KT - 1) / DTC_KT;
   const bool has_new = pos >= k0 && pos < k1;
+  const int last_start = k0 + (ntiles - 1) * DTC_KT;
+  const int last_valid = k1 - last_start;  // keys of the last tile inside the range, 1..64
+  const bool fix_last = has_new || last_valid < DTC_KT;
 
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
-  if (tid == 0) {
-    for (int i = 0; i < DEC_STAGES; ++i) ptx::mbar_init(ptx::smem_u32(&full[i]), 1);
+  extern __shared__ uint8_t dtc_smem_raw[];
+  uint8_t* smem = dtc_smem_raw + ((1024u - (ptx::smem_u32(dtc_smem_raw) & 1023u)) & 1023u);
+  DtcBarriers* bars = reinterpret_cast<DtcBarriers*>(smem + C::OFF_BAR);
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &bars->abort_flag;
+  auto B = [&](uint64_t& x) { return ptx::smem_u32(&x); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < DTC_STAGES; ++s) {
+      ptx::mbar_init(B(bars->full[s]), 1);
+      ptx::mbar_init(B(bars->empty[s]), 1);
+    }
+    ptx::mbar_init(B(bars->fixed), 1);
+    ptx::mbar_init(B(bars->q_ready), 128);
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(B(bars->s_full[s]), 1);
+      ptx::mbar_init(B(bars->p_full[s]), 128);
+      ptx::mbar_init(B(bars->pv_done[s]), 1);
+    }
+    ptx::mbar_init(B(bars->o_full), 1);
+    ptx::mbar_init(B(bars->drain), 1);
+    bars->abort_flag = 0;
     ptx::fence_mbar_init();
   }
+  if (warp == 4 && lane == 0) {
+    ptx::prefetch_tmap(&tmK);
+    ptx::prefetch_tmap(&tmV);
+  }
+  if (warp == 5) {
+    ptx::tmem_alloc(ptx::smem_u32(&bars->tmem_base), C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
   __syncthreads();
-
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
   const int row0 = b * p.Lmax + k0;  // key coordinate of the range's first row in the maps
-  auto issue = [&](int t) {
-    const int st = t % DEC_STAGES;
-    const uint32_t bar = ptx::smem_u32(&full[st]);
-    const uint32_t dk = ptx::smem_u32(sm + C::OFF_KV + st * 2 * C::TILE_BYTES);
-    ptx::mbar_arrive_expect_tx(bar, 2u * C::TILE_BYTES);
-#pragma unroll
-    for (int bx = 0; bx < C::NBOX; ++bx) {
-      ptx::tma_load_3d(dk + bx * C::BOX_BYTES, &tmK, bar, bx * C::BOXC, h, row0 + t * DEC_KT);
-      ptx::tma_load_3d(dk + C::TILE_BYTES + bx * C::BOX_BYTES, &tmV, bar, bx * C::BOXC, h, row0 + t * DEC_KT);
-    }
-  };
-  if (tid == 0)
-    for (int t = 0; t < min(DEC_STAGES, ntiles); ++t)
-      if (!(p.test_drop_first_load && t == 0)) issue(t);
 
-  // ---- RoPE at position pos: cos/sin (float64 angle, fp32 values, as in the
-  // prefill), the G queries of KV head h, and the new key if this range
-  // holds pos. The rotated values are rounded once to bf16.
-  float* qs = reinterpret_cast<float*>(sm + C::OFF_Q);
-  float2* cs = reinterpret_cast<float2*>(sm + C::OFF_CS);
-  __nv_bfloat16* knew = reinterpret_cast<__nv_bfloat16*>(sm + C::OFF_NEW);
-  __nv_bfloat16* vnew = knew + D;
-  for (int i = tid; i < D / 2; i += DEC_THREADS) {
-    double sd, cd;
-    sincos((double)pos * p.inv_freq[i], &sd, &cd);
-    cs[i] = make_float2((float)cd, (float)sd);
-  }
-  __syncthreads();
-  const int nrot = (G + (has_new ? 1 : 0)) * (D / 2);
-  for (int it = tid; it < nrot; it += DEC_THREADS) {
-    const int row = it / (D / 2), i = it - row * (D / 2);
-    const float2 c = cs[i];
-    const __nv_bfloat16* src =
-        row < G ? p.q + ((size_t)b * p.nq + h * G + row) * D : p.k_new + ((size_t)b * p.nkv + h) * D;
-    const float xl = __bfloat162float(src[i]), xh = __bfloat162float(src[i + D / 2]);
-    const uint16_t lo = rope_round_bf16(xl, c.x, xh, -c.y), hi = rope_round_bf16(xh, c.x, xl, c.y);
-    if (row < G) {
-      qs[row * D + C::qslot(i / 8) * 8 + i % 8] = __uint_as_float((uint32_t)lo << 16);
-      qs[row * D + C::qslot((i + D / 2) / 8) * 8 + i % 8] = __uint_as_float((uint32_t)hi << 16);
-    } else {
-      knew[i] = __ushort_as_bfloat16(lo);
-      knew[i + D / 2] = __ushort_as_bfloat16(hi);
-    }
-  }
-  if (has_new)
-    for (int i = tid; i < D; i += DEC_THREADS) vnew[i] = p.v_new[((size_t)b * p.nkv + h) * D + i];
-  float* sp = reinterpret_cast<float*>(sm + C::OFF_S);
-  float2* mls = reinterpret_cast<float2*>(sm + C::OFF_ML);
-  float* alpha_s = reinterpret_cast<float*>(sm + C::OFF_A);
-  if (tid < GM) mls[tid] = make_float2(-INFINITY, 0.f);
-  __syncthreads();
-
-  // weighted-sum phase: this thread's columns and key group
-  const int cq = tid % (D / 4);
-  const int kg = tid / (D / 4);
-  const int col = cq * 4;
-  const uint32_t vcol_off = (col / C::BOXC) * C::BOX_BYTES;
-  const uint32_t vcol_in = (col % C::BOXC) * 2;
-  float2 o[GM][2];  // columns (col, col + 1), (col + 2, col + 3) per head
-#pragma unroll
-  for (int g = 0; g < GM; ++g) o[g][0] = o[g][1] = make_float2(0.f, 0.f);
-
-  int t_fail = -1;
-  for (int t = 0; t < ntiles; ++t) {
-    const int st = t % DEC_STAGES;
-    uint8_t* kt = sm + C::OFF_KV + st * 2 * C::TILE_BYTES;
-    uint8_t* vt = kt + C::TILE_BYTES;
-    const bool landed = dec_wait(ptx::smem_u32(&full[st]), (t / DEC_STAGES) & 1);
-    if (__syncthreads_or(!landed)) {
-      t_fail = t;
-      break;
-    }
-    const int tstart = k0 + t * DEC_KT;
-    const int nvalid = min(DEC_KT, k1 - tstart);
-    if (has_new && pos >= tstart && pos < tstart + DEC_KT) {
-      // the new token's row comes from this CTA, not from the cache
-      const int r = pos - tstart;
-      for (int c = tid; c < D / 8; c += DEC_THREADS) {
-        const int bx = c / (C::BOXC / 8), ch = c % (C::BOXC / 8);
-        const uint32_t off = bx * C::BOX_BYTES + dswz(r * C::ROWB + ch * 16, C::SWZ_MASK);
-        *reinterpret_cast<uint4*>(kt + off) = *reinterpret_cast<const uint4*>(knew + c * 8);
-        *reinterpret_cast<uint4*>(vt + off) = *reinterpret_cast<const uint4*>(vnew + c * 8);
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA, last-tile fix-up, appended row
+    int issued = 0;
+    bool ok = true;
+    if (lane == 0) {
+      for (int t = 0; t < ntiles; ++t) {
+        const int st = t % DTC_STAGES;
+        if (!(ok = bwait_lazy(B(bars->empty[st]), ((t / DTC_STAGES) & 1) ^ 1, abort_flag))) break;
+        ptx::mbar_arrive_expect_tx(B(bars->full[st]), 2u * C::TILE_BYTES);
+        if (!(p.test_drop_first_load && t == 0)) {
+          for (int bx = 0; bx < A::NBOX; ++bx) {
+            ptx::tma_load_3d(sbase + C::OFF_K + st * C::TILE_BYTES + bx * C::KV_BOX_BYTES, &tmK, B(bars->full[st]),
+                             bx * A::BOXC, h, row0 + t * DTC_KT);
+            ptx::tma_load_3d(sbase + C::OFF_V + st * C::TILE_BYTES + bx * C::KV_BOX_BYTES, &tmV, B(bars->full[st]),
+                             bx * A::BOXC, h, row0 + t * DTC_KT);
+          }
+          ++issued;
+        }
       }
-      ptx::fence_proxy_async_smem();
-      __syncthreads();
     }
-
-    // ---- scores, log2 units: lanes (key, d quarter), all heads
-    {
-      const int key = warp * 8 + (lane & 7);
-      const int dq = lane >> 3;
-      float2 acc2[GM];  // two partial sums per head (even / odd features)
-#pragma unroll
-      for (int g = 0; g < GM; ++g) acc2[g] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int i = 0; i < C::CPQ; ++i) {
-        const int c = dq * C::CPQ + i;
-        const int bx = c / (C::BOXC / 8), ch = c % (C::BOXC / 8);
-        const uint4 kw = *reinterpret_cast<const uint4*>(kt + bx * C::BOX_BYTES +
-                                                         dswz(key * C::ROWB + ch * 16, C::SWZ_MASK));
-        const float2 k01 = make_float2(bf_lo(kw.x), bf_hi(kw.x)), k23 = make_float2(bf_lo(kw.y), bf_hi(kw.y));
-        const float2 k45 = make_float2(bf_lo(kw.z), bf_hi(kw.z)), k67 = make_float2(bf_lo(kw.w), bf_hi(kw.w));
-#pragma unroll
-        for (int g = 0; g < GM; ++g) {
-          if (g < G) {
-            const float4 qa = *reinterpret_cast<const float4*>(qs + g * D + (i * 4 + dq) * 8);
-            const float4 qb = *reinterpret_cast<const float4*>(qs + g * D + (i * 4 + dq) * 8 + 4);
-            float2 a = acc2[g];
-            a = dec_ffma2(make_float2(qa.x, qa.y), k01, a);
-            a = dec_ffma2(make_float2(qa.z, qa.w), k23, a);
-            a = dec_ffma2(make_float2(qb.x, qb.y), k45, a);
-            a = dec_ffma2(make_float2(qb.z, qb.w), k67, a);
-            acc2[g] = a;
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    const int tl = ntiles - 1, stl = tl % DTC_STAGES;
+    if (ok && fix_last) {
+      // the last tile: the new token's rotated key and value in row pos, and
+      // V rows past the range zero (their weights are zero; the cache rows
+      // there may hold anything)
+      ok = __all_sync(0xffffffffu, bwait(B(bars->full[stl]), (tl / DTC_STAGES) & 1, abort_flag) &&
+                                       bwait(B(bars->q_ready), 0, abort_flag));
+      if (ok) {
+        uint8_t* kt = smem + C::OFF_K + stl * C::TILE_BYTES;
+        uint8_t* vt = smem + C::OFF_V + stl * C::TILE_BYTES;
+        const __nv_bfloat16* knew = reinterpret_cast<const __nv_bfloat16*>(smem + C::OFF_NEW);
+        constexpr int CPR = D / 8;  // 16-byte chunks per row
+        if (has_new) {
+          const int r = pos - last_start;
+          for (int c = lane; c < CPR; c += 32) {
+            const int bx = c / (A::BOXC / 8), ch = c % (A::BOXC / 8);
+            const uint32_t off = bx * C::KV_BOX_BYTES + swz(r * A::ROWB + ch * 16, A::SWZ_MASK);
+            *reinterpret_cast<uint4*>(kt + off) = *reinterpret_cast<const uint4*>(knew + c * 8);
+            *reinterpret_cast<uint4*>(vt + off) = *reinterpret_cast<const uint4*>(knew + D + c * 8);
           }
         }
-      }
-      float acc[GM];
-#pragma unroll
-      for (int g = 0; g < GM; ++g) acc[g] = acc2[g].x + acc2[g].y;
-#pragma unroll
-      for (int g = 0; g < GM; ++g) {
-        acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 8);
-        acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 16);
-        if (g < G && (g & 3) == dq) sp[key * GM + g] = key < nvalid ? acc[g] * p.scale_log2 : -INFINITY;
-      }
-    }
-    __syncthreads();
-
-    // ---- online softmax: warp w takes heads w, w + 8
-    for (int g = warp; g < G; g += DEC_THREADS / 32) {
-      const float s0 = sp[lane * GM + g], s1 = sp[(lane + 32) * GM + g];
-      const float2 ml = mls[g];
-      const float mnew = fmaxf(ml.x, warp_max(fmaxf(s0, s1)));  // finite: key tstart is visible
-      const float p0 = ptx::ex2(s0 - mnew), p1 = ptx::ex2(s1 - mnew);
-      const float sum = warp_sum(p0 + p1);
-      const float a = ptx::ex2(ml.x - mnew);
-      sp[lane * GM + g] = p0;
-      sp[(lane + 32) * GM + g] = p1;
-      __syncwarp();
-      if (lane == 0) {
-        mls[g] = make_float2(mnew, ml.y * a + sum);
-        alpha_s[g] = a;
-      }
-    }
-    __syncthreads();
-
-    // ---- O = O * a + P V: this thread's 4 columns, its key group, all heads
-    {
-#pragma unroll
-      for (int g = 0; g < GM; ++g) {
-        if (g < G) {
-          const float a = alpha_s[g];
-          o[g][0].x *= a; o[g][0].y *= a; o[g][1].x *= a; o[g][1].y *= a;
+        for (int i = lane; i < (DTC_KT - last_valid) * CPR; i += 32) {
+          const int r = last_valid + i / CPR, c = i % CPR;
+          const int bx = c / (A::BOXC / 8), ch = c % (A::BOXC / 8);
+          *reinterpret_cast<uint4*>(vt + bx * C::KV_BOX_BYTES + swz(r * A::ROWB + ch * 16, A::SWZ_MASK)) =
+              make_uint4(0, 0, 0, 0);
         }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(B(bars->fixed));
       }
-#pragma unroll 2
-      for (int j = 0; j < C::KPG; ++j) {
-        const int k = kg * C::KPG + j;
-        if (k < nvalid) {  // uniform across the warp
-          const uint2 vw = *reinterpret_cast<const uint2*>(vt + vcol_off + dswz(k * C::ROWB + vcol_in, C::SWZ_MASK));
-          const float2 v01 = make_float2(bf_lo(vw.x), bf_hi(vw.x)), v23 = make_float2(bf_lo(vw.y), bf_hi(vw.y));
-#pragma unroll
-          for (int g4 = 0; g4 < GM / 4; ++g4) {
-            if (4 * g4 < G) {
-              const float4 pk = *reinterpret_cast<const float4*>(sp + k * GM + 4 * g4);
-              const float pv[4] = {pk.x, pk.y, pk.z, pk.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int g = 4 * g4 + e;
-                if (g < G) {
-                  const float2 pp = make_float2(pv[e], pv[e]);
-                  o[g][0] = dec_ffma2(pp, v01, o[g][0]);
-                  o[g][1] = dec_ffma2(pp, v23, o[g][1]);
-                }
-              }
-            }
-          }
+    }
+    if (ok) {
+      // all MMAs done: every load of this CTA has landed; append the new row
+      ok = __all_sync(0xffffffffu, bwait_lazy(B(bars->o_full), 0, abort_flag));
+      if (ok && has_new) {
+        const size_t row = (((size_t)b * p.Lmax + pos) * p.nkv + h) * D;
+        const uint4* kv4 = reinterpret_cast<const uint4*>(smem + C::OFF_NEW);
+        for (int i = lane; i < D / 8; i += 32) {
+          reinterpret_cast<uint4*>(p.k_cache + row)[i] = kv4[i];
+          reinterpret_cast<uint4*>(p.v_cache + row)[i] = kv4[D / 8 + i];
         }
       }
     }
-    __syncthreads();  // stage and scores free
-    if (tid == 0 && t + DEC_STAGES < ntiles) issue(t + DEC_STAGES);
+    if (!ok && lane == 0) {  // every copy issued lands before the CTA exits
+      const int first = p.test_drop_first_load ? 1 : 0;
+      for (int t = first; t < first + issued; ++t)
+        drain_wait(B(bars->full[t % DTC_STAGES]), (t / DTC_STAGES) & 1);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint64_t dq = umma_desc(sbase + C::OFF_Q, 16, A::SBO, A::UMMA_LAYOUT);
+      const uint64_t dk0 = umma_desc(sbase + C::OFF_K, 16, A::SBO, A::UMMA_LAYOUT);
+      const uint64_t dv0 = umma_desc(sbase + C::OFF_V, C::KV_BOX_BYTES, A::SBO, A::UMMA_LAYOUT);
+      const uint64_t stage = (uint64_t)(C::TILE_BYTES >> 4);
+      // S(j) into S buffer j & 1 once K(j) is in place and P V(j - 2), which
+      // read P from that buffer, is done
+      auto issue_s = [&](int j) -> bool {
+        const int sb = j & 1, st = j % DTC_STAGES;
+        if (j >= 2 && !bwait(B(bars->pv_done[sb]), ((j - 2) >> 1) & 1, abort_flag)) return false;
+        const bool w = (j == ntiles - 1 && fix_last) ? bwait(B(bars->fixed), 0, abort_flag)
+                                                     : bwait(B(bars->full[st]), (j / DTC_STAGES) & 1, abort_flag);
+        if (!w) return false;
+        ptx::tc_fence_after();
+        const uint64_t dk = dk0 + st * stage;
+#pragma unroll
+        for (int kk = 0; kk < A::KSTEPS_S; ++kk) {
+          const uint32_t off_q = (kk / A::STEPS_PER_BOX) * A::Q_BOX_BYTES + (kk % A::STEPS_PER_BOX) * 32;
+          const uint32_t off_k = (kk / A::STEPS_PER_BOX) * C::KV_BOX_BYTES + (kk % A::STEPS_PER_BOX) * 32;
+          ptx::mma_ss(tmem + C::S_COL + sb * DTC_KT, dq + (uint64_t)(off_q >> 4), dk + (uint64_t)(off_k >> 4),
+                      C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(B(bars->s_full[sb]));
+        return true;
+      };
+      bool ok = bwait(B(bars->q_ready), 0, abort_flag) && issue_s(0);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        const int sb = j & 1, st = j % DTC_STAGES;
+        if (j + 1 < ntiles && !(ok = issue_s(j + 1))) break;
+        if (!(ok = bwait(B(bars->p_full[sb]), (j >> 1) & 1, abort_flag))) break;
+        ptx::tc_fence_after();
+        // O (+)= P V: 64 keys in 4 K-steps of 16, P from the S buffer's first 32 columns
+#pragma unroll
+        for (int kk = 0; kk < DTC_KT / 16; ++kk)
+          ptx::mma_ts(tmem + C::O_COL, tmem + C::S_COL + sb * DTC_KT + kk * 8,
+                      dv0 + st * stage + (uint64_t)((kk * 16 * A::ROWB) >> 4), A::IDESC_O,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(B(bars->pv_done[sb]));
+        ptx::mma_commit(B(bars->empty[st]));
+      }
+      if (ok) ptx::mma_commit(B(bars->o_full));
+      // all tensor-core work issued here has finished before TMEM is freed
+      ptx::mma_commit(B(bars->drain));
+      drain_wait(B(bars->drain), 0);
+    }
+  } else {
+    // ------------------------------------------------------------ RoPE, softmax, partial results
+    const int tid = threadIdx.x;  // 0..127 == tile row == TMEM lane
+    const int g = 4 * lane + warp;  // the head of this row (a row past G holds none)
+    const bool active = g < G;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    float2* cs = reinterpret_cast<float2*>(smem + C::OFF_CS);
+    __nv_bfloat16* knew = reinterpret_cast<__nv_bfloat16*>(smem + C::OFF_NEW);
+    // zero query tile; (cos, sin) at pos (float64 angle, fp32 values)
+    for (int i = tid; i < A::Q_BYTES / 16; i += 128)
+      reinterpret_cast<uint4*>(smem + C::OFF_Q)[i] = make_uint4(0, 0, 0, 0);
+    for (int i = tid; i < HALF; i += 128) {
+      double sd, cd;
+      sincos((double)pos * p.inv_freq[i], &sd, &cd);
+      cs[i] = make_float2((float)cd, (float)sd);
+    }
+    dtc_softmax_sync();
+    // rotated queries into their tile rows, and the new key (if this range
+    // holds pos); each rotated value rounded once to bf16, as in the prefill
+    const int nrot = (G + (has_new ? 1 : 0)) * HALF;
+    for (int it = tid; it < nrot; it += 128) {
+      const int hg = it / HALF, i = it - hg * HALF;
+      const float2 c = cs[i];
+      const __nv_bfloat16* src =
+          hg < G ? p.q + ((size_t)b * p.nq + h * G + hg) * D : p.k_new + ((size_t)b * p.nkv + h) * D;
+      const float xl = __bfloat162float(src[i]), xh = __bfloat162float(src[i + HALF]);
+      const uint16_t lo = rope_round_bf16(xl, c.x, xh, -c.y), hi = rope_round_bf16(xh, c.x, xl, c.y);
+      if (hg < G) {
+        const int row = 32 * (hg % 4) + hg / 4;
+        const int cl = i, chh = i + HALF;
+        *reinterpret_cast<uint16_t*>(smem + C::OFF_Q + (cl / A::BOXC) * A::Q_BOX_BYTES +
+                                     swz(row * A::ROWB + (cl % A::BOXC) * 2, A::SWZ_MASK)) = lo;
+        *reinterpret_cast<uint16_t*>(smem + C::OFF_Q + (chh / A::BOXC) * A::Q_BOX_BYTES +
+                                     swz(row * A::ROWB + (chh % A::BOXC) * 2, A::SWZ_MASK)) = hi;
+      } else {
+        knew[i] = __ushort_as_bfloat16(lo);
+        knew[i + HALF] = __ushort_as_bfloat16(hi);
+      }
+    }
+    if (has_new)
+      for (int i = tid; i < D; i += 128) knew[D + i] = p.v_new[((size_t)b * p.nkv + h) * D + i];
+    ptx::fence_proxy_async_smem();
+    ptx::mbar_arrive(B(bars->q_ready));
+
+    const float sl2 = p.scale_log2;
+    const float thr = 8.f / sl2;  // raw-score growth that forces an O rescale (2^8 in p)
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    uint32_t sr[DTC_KT];
+    uint32_t ob[32];  // scratch of the O rescale
+    for (int j = 0; j < ntiles; ++j) {
+      const int sb = j & 1;
+      ok = __all_sync(0xffffffffu, bwait(B(bars->s_full[sb]), (j >> 1) & 1, abort_flag));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      load_s_cols<DTC_KT>(trow + C::S_COL + sb * DTC_KT, sr);
+      const int nvalid = min(DTC_KT, k1 - (k0 + j * DTC_KT));
+      if (nvalid < DTC_KT) mask_cols<DTC_KT>(sr, nvalid - 1);
+      const float mx = cols_max<DTC_KT>(sr);
+      // exponentials against the running max; it moves only when a score
+      // exceeds it by more than the threshold (the first tile sets it)
+      const bool need = mx > m + thr;
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = need ? mx : m;
+        if (j > 0) {
+          const float alpha = need ? ptx::ex2((m - m_new) * sl2) : 1.f;
+          const int jp = j - 1;
+          ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[jp & 1]), (jp >> 1) & 1, abort_flag));
+          if (!ok) break;
+          ptx::tc_fence_after();
+          scale_o_cols<D>(trow + C::O_COL, alpha, ob);
+          l *= alpha;
+        }
+        m = m_new;
+      }
+      l += exp_pack<DTC_KT, emu_period(D)>(sr, -m * sl2, sl2, nullptr);
+      ptx::tmem_st32(trow + C::S_COL + sb * DTC_KT, sr);  // P (bf16 pairs) in the buffer's first 32 columns
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(B(bars->p_full[sb]));
+    }
+    if (ok) ok = __all_sync(0xffffffffu, bwait(B(bars->o_full), 0, abort_flag));
+    if (ok) {
+      ptx::tc_fence_after();
+      float* po = p.part_o + (part * G + (active ? g : 0)) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        ptx::tmem_ld32(trow + C::O_COL + c * 32, sr);
+        ptx::tmem_wait_ld();
+        ptx::reg_fence32(sr);
+        if (active) {
+          float4* dst = reinterpret_cast<float4*>(po + c * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(sr[4 * e]), __uint_as_float(sr[4 * e + 1]),
+                                 __uint_as_float(sr[4 * e + 2]), __uint_as_float(sr[4 * e + 3]));
+        }
+      }
+      if (active) p.part_ml[part * G + g] = make_float2(m * sl2, l);
+    }
   }
 
-  if (t_fail >= 0) {
-    // tiles t_fail .. t_fail + STAGES - 1 may still be in flight: let them
-    // land (bounded waits) before the CTA exits
-    if (tid == 0)
-      for (int t = t_fail; t < min(ntiles, t_fail + DEC_STAGES); ++t)
-        dec_wait(ptx::smem_u32(&full[t % DEC_STAGES]), (t / DEC_STAGES) & 1);
-    __syncthreads();
-    return;
-  }
-
-  // ---- this range's partial results: the key groups' sums, added in a
-  // fixed order (group 0 first) in shared memory (the stage area is free)
-  float* red = reinterpret_cast<float*>(sm + C::OFF_KV);  // [G][D]
-  for (int i = tid; i < G * D; i += DEC_THREADS) red[i] = 0.f;
+  ptx::tc_fence_before();
   __syncthreads();
-  for (int r = 0; r < C::KGROUPS; ++r) {
-    if (kg == r) {
-#pragma unroll
-      for (int g = 0; g < GM; ++g) {
-        if (g < G) {
-          float4* dst = reinterpret_cast<float4*>(red + g * D + col);
-          const float4 cur = *dst;
-          *dst = make_float4(cur.x + o[g][0].x, cur.y + o[g][0].y, cur.z + o[g][1].x, cur.w + o[g][1].y);
-        }
-      }
-    }
-    __syncthreads();
-  }
-  for (int i = tid; i < G * D / 4; i += DEC_THREADS)
-    reinterpret_cast<float4*>(po)[i] = reinterpret_cast<const float4*>(red)[i];
-  for (int i = tid; i < G; i += DEC_THREADS) pml[i] = mls[i];
-  // the appended cache row (after every load of this CTA has landed)
-  if (has_new) {
-    const size_t row = (((size_t)b * p.Lmax + pos) * p.nkv + h) * D;
-    for (int i = tid; i < D / 8; i += DEC_THREADS) {
-      reinterpret_cast<uint4*>(p.k_cache + row)[i] = reinterpret_cast<const uint4*>(knew)[i];
-      reinterpret_cast<uint4*>(p.v_cache + row)[i] = reinterpret_cast<const uint4*>(vnew)[i];
-    }
+  if (warp == 5) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
 // Merge of the key ranges of one (sequence, KV head); threads over
 // (head, column).
-__global__ void __launch_bounds__(DEC_THREADS) gqa_decode_combine_kernel(const DecodeParams p, int D) {
+__global__ void __launch_bounds__(DEC_COMBINE_THREADS) gqa_decode_combine_kernel(const DecodeParams p, int D) {
   const int h = blockIdx.x, b = blockIdx.y;
   const int G = p.G;
   const int pos = __ldg(p.cache_seqlens + b);
   if (pos < 0 || pos >= p.Lmax) return;
   const int used = min(p.splits, pos / p.kps + 1);  // ranges holding a visible key
   const size_t part0 = ((size_t)b * p.nkv + h) * p.splits;
-  for (int u = threadIdx.x; u < G * D; u += DEC_THREADS) {
+  for (int u = threadIdx.x; u < G * D; u += DEC_COMBINE_THREADS) {
     const int g = u / D, d = u - g * D;
     float M = -INFINITY;
     for (int s = 0; s < used; ++s) M = fmaxf(M, p.part_ml[(part0 + s) * G + g].x);

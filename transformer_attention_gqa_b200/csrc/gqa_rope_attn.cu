@@ -33,10 +33,10 @@ struct DeviceState {
   bool init = false;
   int sm_count = 0;
   bool attr_set[3][2] = {};
-  bool dec_attr_set[3][3] = {};
   bool bwd_attr_set[3] = {};
   bool proj_attr_set[3] = {};
   bool masked_attr_set[3] = {};
+  bool dtc_attr_set[3] = {};
 };
 
 std::mutex g_mu;
@@ -284,28 +284,27 @@ DecLayout dec_layout(int B, int Lmax, int nq, int nkv, int d) {
   return L;
 }
 
-template <int D, int GM>
+template <int D>
 int launch_decode(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
                   const int32_t* lens, double theta, int B, int Lmax, int nq, int nkv, void* out, float* lse,
                   uint8_t* ws, const DecLayout& lay, cudaStream_t stream, int device) {
-  using C = DecCfg<D, GM>;
-  constexpr int gi = GM == 4 ? 0 : (GM == 8 ? 1 : 2);
+  using C = DtcCfg<D>;
   {  // caller holds g_mu
     DeviceState& ds = g_dev[device];
-    if (!ds.dec_attr_set[dim_index(D)][gi]) {
-      if (cudaFuncSetAttribute(gqa_decode_split_kernel<D, GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (!ds.dtc_attr_set[dim_index(D)]) {
+      if (cudaFuncSetAttribute(gqa_decode_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_BYTES) != cudaSuccess)
         return GQA_ERR_CUDA;
-      ds.dec_attr_set[dim_index(D)][gi] = true;
+      ds.dtc_attr_set[dim_index(D)] = true;
     }
   }
   // Cache maps: [B*Lmax rows][nkv][d], box (BOXC columns, 1 head, 64 rows).
   CUtensorMap tmK, tmV;
   const uint64_t dims[3] = {(uint64_t)D, (uint64_t)nkv, (uint64_t)B * (uint64_t)Lmax};
   const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)nkv * D * 2};
-  const uint32_t box[3] = {(uint32_t)C::BOXC, 1u, (uint32_t)DEC_KT};
-  if (!make_tmap(device, k_cache, dims, str, box, C::ROWB, &tmK)) return GQA_ERR_CUDA;
-  if (!make_tmap(device, v_cache, dims, str, box, C::ROWB, &tmV)) return GQA_ERR_CUDA;
+  const uint32_t box[3] = {(uint32_t)C::A::BOXC, 1u, (uint32_t)DEC_KT};
+  if (!make_tmap(device, k_cache, dims, str, box, C::A::ROWB, &tmK)) return GQA_ERR_CUDA;
+  if (!make_tmap(device, v_cache, dims, str, box, C::A::ROWB, &tmV)) return GQA_ERR_CUDA;
 
   DecodeParams dp{};
   dp.q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -335,10 +334,10 @@ int launch_decode(const void* q, const void* k_new, const void* v_new, void* k_c
   dp.test_drop_first_load = (drop && drop[0] == '1' && drop[1] == '\0') ? 1 : 0;
 
   if (t_prof_ev[0] && cudaEventRecord(t_prof_ev[0], stream) != cudaSuccess) return GQA_ERR_CUDA;
-  gqa_decode_split_kernel<D, GM><<<dim3(lay.splits, nkv, B), DEC_THREADS, C::SMEM_BYTES, stream>>>(tmK, tmV, dp);
+  gqa_decode_tc_kernel<D><<<dim3(lay.splits, nkv, B), DTC_THREADS, C::SMEM_BYTES, stream>>>(tmK, tmV, dp);
   if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   if (t_prof_ev[1] && cudaEventRecord(t_prof_ev[1], stream) != cudaSuccess) return GQA_ERR_CUDA;
-  gqa_decode_combine_kernel<<<dim3(nkv, B), DEC_THREADS, 0, stream>>>(dp, D);
+  gqa_decode_combine_kernel<<<dim3(nkv, B), DEC_COMBINE_THREADS, 0, stream>>>(dp, D);
   if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;
   t_last_launches = 2;
@@ -679,15 +678,11 @@ extern "C" int gqa_rope_attn_decode(const void* q, const void* k_new, const void
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   std::lock_guard<std::mutex> lk(g_mu);  // descriptor cache
-  const int G = n_q_heads / n_kv_heads;
-  const int gb = G <= 4 ? 4 : (G <= 8 ? 8 : 16);
-#define GQA_DEC_CASE(DD, GG)                                                                                  \
-  if (head_dim == DD && gb == GG)                                                                             \
-    return launch_decode<DD, GG>(q, k_new, v_new, k_cache, v_cache, cache_seqlens, rope_theta, batch,         \
-                                 max_cache_len, n_q_heads, n_kv_heads, out, lse, ws, lay, st, device);
-  GQA_DEC_CASE(32, 4) GQA_DEC_CASE(32, 8) GQA_DEC_CASE(32, 16)
-  GQA_DEC_CASE(64, 4) GQA_DEC_CASE(64, 8) GQA_DEC_CASE(64, 16)
-  GQA_DEC_CASE(128, 4) GQA_DEC_CASE(128, 8) GQA_DEC_CASE(128, 16)
+#define GQA_DEC_CASE(DD)                                                                                      \
+  if (head_dim == DD)                                                                                         \
+    return launch_decode<DD>(q, k_new, v_new, k_cache, v_cache, cache_seqlens, rope_theta, batch, max_cache_len, \
+                             n_q_heads, n_kv_heads, out, lse, ws, lay, st, device);
+  GQA_DEC_CASE(32) GQA_DEC_CASE(64) GQA_DEC_CASE(128)
 #undef GQA_DEC_CASE
   return GQA_ERR_UNSUPPORTED;
 }
