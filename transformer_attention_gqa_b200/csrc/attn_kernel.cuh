@@ -438,7 +438,7 @@ __device__ __forceinline__ bool rope_q_tile(const AttnParams& p, uint8_t* smem, 
   if (w < 0) return true;
   const WorkItem wi = decode_item(p, w);
   uint8_t* qbuf = smem + qb * C::Q_BYTES;
-  const int items = p.prerotated ? 0 : p.tq * NCH;  // rotated inputs: Q is used as loaded
+  const int items = p.q_rotated ? 0 : p.tq * NCH;  // rotated Q tiles are used as loaded
   for (int item = tid; item < items; item += 128) {
     const int tt = item / NCH;
     const int ch = item - tt * NCH;
@@ -668,8 +668,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           ptx::mbar_arrive_expect_tx(B(bars->k_full[ks]), (uint32_t)C::KV_BYTES);
           // K' head-major (token, head) or, for rotated inputs, the caller's
           // token-major K (head, token): the same 128-byte rows in shared memory
-          const int c1 = p.prerotated ? wi.kvh : wi.seq_start + j * BN;
-          const int c2 = p.prerotated ? wi.seq_start + j * BN : wi.kvh;
+          const int c1 = p.k_token_major ? wi.kvh : wi.seq_start + j * BN;
+          const int c2 = p.k_token_major ? wi.seq_start + j * BN : wi.kvh;
           for (int b = 0; b < C::NBOX; ++b)
             ptx::tma_load_3d(sbase + C::OFF_K + ks * C::KV_BYTES + b * C::KV_BOX_BYTES, &tmK,
                              B(bars->k_full[ks]), b * C::BOXC, c1, c2);

@@ -19,6 +19,9 @@ constexpr int ATTN_THREADS = 512;   // 16 warps (roles: attention kernel)
 constexpr int PREP_THREADS = 256;
 constexpr int SCHED_BINS = 2048;    // cost histogram bins of the tile scheduler
 constexpr unsigned long long WAIT_TIMEOUT_NS = 2000000000ull;  // bounded waits: 2 s
+// bf16 inputs with at most this many tokens per sequence on average have Q
+// rotated by the prologue instead of the attention kernel (0: never).
+constexpr int kQPrologueMaxTokensPerSeq = 0;
 
 // Device status word: first device-detected error since the host last read
 // it. The library is a single translation unit, so it is defined here.
@@ -40,11 +43,20 @@ struct WsLayout {
   size_t pairs;    // int2[max_pairs]: (sequence, q-tile) in decreasing cost order
   size_t table;    // float2[N * d/2]: (cos, sin) of each token's angles
   size_t kws;      // bf16[n_kv][N][d]: RoPE'd K, head-major
-  size_t qws;      // bf16[N][n_q][d]: q rounded to bf16 (fp32 inputs only)
+  size_t qws;      // bf16[N][n_q][d]: rotated q (when the prologue rotates it)
   size_t vws;      // bf16[N][n_kv][d]: v rounded to bf16 (fp32 inputs only)
   size_t total;
   long long max_pairs;
 };
+
+// Whether the prologue writes the rotated queries Q' (bf16, [N][n_q][d]) into
+// the workspace, so that the attention kernel uses the Q tiles as loaded:
+// always for fp32 inputs (the prologue writes a bf16 copy of q anyway), and
+// for bf16 inputs when the work items are short (see the forward's launch).
+__host__ inline bool q_rotated_in_prologue(int num_seqs, int N, bool fp32_in) {
+  return fp32_in || (kQPrologueMaxTokensPerSeq > 0 && num_seqs > 0 &&
+                     (long long)N <= (long long)kQPrologueMaxTokensPerSeq * num_seqs);
+}
 
 __host__ inline WsLayout ws_layout(int num_seqs, int N, int nq, int nkv, int d, bool fp32_in) {
   WsLayout w{};
@@ -62,20 +74,21 @@ __host__ inline WsLayout ws_layout(int num_seqs, int N, int nq, int nkv, int d, 
   off = align_up(off + (size_t)N * (d / 2) * 8, 256);
   w.kws = off;
   off = align_up(off + (size_t)nkv * N * d * 2, 256);
-  if (fp32_in) {
+  w.qws = w.vws = 0;
+  if (q_rotated_in_prologue(num_seqs, N, fp32_in)) {
     w.qws = off;
     off = align_up(off + (size_t)N * nq * d * 2, 256);
+  }
+  if (fp32_in) {
     w.vws = off;
     off = align_up(off + (size_t)N * nkv * d * 2, 256);
-  } else {
-    w.qws = w.vws = 0;
   }
   w.total = off;
   return w;
 }
 
 struct PrepParams {
-  const void* q;  // fp32 inputs only
+  const void* q;  // read when the prologue rotates q
   const void* k;
   const void* v;  // fp32 inputs only
   const int* positions;
@@ -104,8 +117,9 @@ struct AttnParams {
   int sched_dynamic;    // 1: items beyond the first from item_counter; 0: static alternating deal
   float scale_log2;     // log2(e) / sqrt(d)
   float rescale_thr;    // raw-score growth that triggers an O rescale
-  int prerotated;       // 1: q and k arrive rotated; K is read token-major [N][n_kv][d] from the
-                        // caller's tensor and Q is not rotated again; 0: K' head-major from the prologue
+  int q_rotated;        // 1: the Q tiles arrive rotated (the caller's, or the prologue's Q'); 0: rotate them
+  int k_token_major;    // 1: K is the caller's rotated token-major [N][n_kv][d] tensor; 0: K' head-major
+                        // from the prologue
 };
 
 }  // namespace gqa

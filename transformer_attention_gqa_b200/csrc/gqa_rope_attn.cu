@@ -170,13 +170,17 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
   pp.pairs = reinterpret_cast<int2*>(ws + lay.pairs);
   pp.table = reinterpret_cast<float2*>(ws + lay.table);
   pp.kws = reinterpret_cast<__nv_bfloat16*>(ws + lay.kws);
-  pp.qws = FP32 ? reinterpret_cast<__nv_bfloat16*>(ws + lay.qws) : nullptr;
+  // the prologue rotates Q into the workspace when the layout has room for it
+  // (fp32 inputs, or short work items), never for inputs already rotated
+  const bool q_in_ws = !prerotated && lay.qws != 0;
+  pp.qws = q_in_ws ? reinterpret_cast<__nv_bfloat16*>(ws + lay.qws) : nullptr;
   pp.vws = FP32 ? reinterpret_cast<__nv_bfloat16*>(ws + lay.vws) : nullptr;
 
-  // Tensor maps. Q: [N][nq][d] (caller's, or its bf16 copy); K: RoPE'd,
-  // head-major [nkv][N][d]; V: [N][nkv][d] (caller's, or its bf16 copy).
+  // Tensor maps. Q: [N][nq][d] (caller's, or the prologue's rotated Q');
+  // K: RoPE'd, head-major [nkv][N][d] (or the caller's rotated K,
+  // token-major); V: [N][nkv][d] (caller's, or its bf16 copy).
   CUtensorMap tmQ, tmK, tmV;
-  const void* qsrc = FP32 ? (const void*)(ws + lay.qws) : q;
+  const void* qsrc = q_in_ws ? (const void*)(ws + lay.qws) : q;
   const void* vsrc = FP32 ? (const void*)(ws + lay.vws) : v;
   const uint64_t es = 2;
   {
@@ -232,7 +236,8 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
   ap.causal = causal;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   ap.rescale_thr = (float)(8.0 / (1.4426950408889634 / std::sqrt((double)D)));
-  ap.prerotated = prerotated ? 1 : 0;
+  ap.q_rotated = (prerotated || q_in_ws) ? 1 : 0;
+  ap.k_token_major = prerotated ? 1 : 0;
 
   const long long max_items = lay.max_pairs * (long long)nkv;
   const unsigned grid = (unsigned)(max_items < sm_count ? max_items : sm_count);

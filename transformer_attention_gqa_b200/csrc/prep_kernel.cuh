@@ -8,7 +8,8 @@
 //  * the other blocks compute each token's RoPE (cos, sin) table row and
 //    write the RoPE'd K once, head-major, into the workspace. K is shared by
 //    every query tile that attends to it, so it is rotated once per
-//    (token, KV head) instead of once per visiting tile.
+//    (token, KV head) instead of once per visiting tile. When asked (short
+//    work items, or fp32 inputs) they also write the rotated Q.
 //
 // RoPE ("Embeddings & the Residual Stream", section "Positional information:
 // RoPE, not a learned table"): inv_freq[i] = theta^(-2i/d); angle =
@@ -238,15 +239,35 @@ __device__ void rope_k_and_table(const PrepParams& p, int block, int nblocks) {
       }
     }
 
-    if constexpr (FP32_IN) {
-      // bf16 copies of q (rotated later, in the attention kernel) and v.
+    if (p.qws) {
+      // rotated queries Q' (inputs rounded to bf16 first, as for K)
       for (int h = 0; h < p.nq; ++h) {
         const size_t o = ((size_t)t * p.nq + h) * D;
-        const float2 a = *reinterpret_cast<const float2*>((const float*)p.q + o + i);
-        const float2 b = *reinterpret_cast<const float2*>((const float*)p.q + o + i + HALF);
-        *reinterpret_cast<__nv_bfloat162*>(p.qws + o + i) = __floats2bfloat162_rn(a.x, a.y);
-        *reinterpret_cast<__nv_bfloat162*>(p.qws + o + i + HALF) = __floats2bfloat162_rn(b.x, b.y);
+        float xl[2], xh[2];
+        if constexpr (FP32_IN) {
+          const float2 a = *reinterpret_cast<const float2*>((const float*)p.q + o + i);
+          const float2 b = *reinterpret_cast<const float2*>((const float*)p.q + o + i + HALF);
+          xl[0] = __bfloat162float(__float2bfloat16_rn(a.x));
+          xl[1] = __bfloat162float(__float2bfloat16_rn(a.y));
+          xh[0] = __bfloat162float(__float2bfloat16_rn(b.x));
+          xh[1] = __bfloat162float(__float2bfloat16_rn(b.y));
+        } else {
+          const uint32_t wa = *reinterpret_cast<const uint32_t*>((const __nv_bfloat16*)p.q + o + i);
+          const uint32_t wb = *reinterpret_cast<const uint32_t*>((const __nv_bfloat16*)p.q + o + i + HALF);
+          xl[0] = __uint_as_float(wa << 16);
+          xl[1] = __uint_as_float(wa & 0xFFFF0000u);
+          xh[0] = __uint_as_float(wb << 16);
+          xh[1] = __uint_as_float(wb & 0xFFFF0000u);
+        }
+        __nv_bfloat16 lo[2], hi[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) rope_pair(xl[e], xh[e], c[e], sn[e], lo[e], hi[e]);
+        *reinterpret_cast<__nv_bfloat162*>(p.qws + o + i) = __halves2bfloat162(lo[0], lo[1]);
+        *reinterpret_cast<__nv_bfloat162*>(p.qws + o + i + HALF) = __halves2bfloat162(hi[0], hi[1]);
       }
+    }
+    if constexpr (FP32_IN) {
+      // bf16 copy of v
       for (int h = 0; h < p.nkv; ++h) {
         const size_t o = ((size_t)t * p.nkv + h) * D;
         const float2 a = *reinterpret_cast<const float2*>((const float*)p.v + o + i);
