@@ -13,7 +13,7 @@ import pytest
 from transformer_attention_gqa_b200 import build as B
 
 # kernel name -> registers per thread at launch (threads x registers = the split's total)
-EXPECTED = {"gqa_attn_fwd_kernel": 128, "gqa_attn_bwd_kernel": 168}
+EXPECTED = {"gqa_attn_fwd_kernel": 128, "gqa_attn_bwd_kernel": 128}
 
 
 @pytest.fixture(scope="module")

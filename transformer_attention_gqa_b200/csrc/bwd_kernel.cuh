@@ -32,15 +32,18 @@
 //    atomics (several key tiles contribute to one query tile).
 //  * gqa_bwd_dq_kernel: dq = rope^T(dQ' / sqrt(d)) -> bf16.
 //
-// Warp roles of the attention-backward kernel (384 threads):
+// Warp roles of the attention-backward kernel (512 threads):
 //   warp 0      TMA: K', V once; Q', dO per query tile (two stages each);
 //               lse * log2(e) and Delta of the tile's 128 rows into shared
 //               memory (all 32 lanes)
 //   warp 1      TMEM allocator; one thread issues every MMA
-//   warps 4-7   P^T and dS^T, one key row per thread
-//   warps 8-11  dQ' tile -> fp32 atomics; at the end dV and dK' -> bf16
-// Tensor memory (512 columns): [0,128) S^T, then P^T (bf16 pairs, first 64
-// columns); [128,256) dP^T, then the dQ' tile; [256, 256+d) dV;
+//   warps 4-11  P^T and dS^T, one key row per thread: warps 4-7 the packed
+//               query columns [0, 64), warps 8-11 [64, 128)
+//   warps 12-15 dQ' tile -> fp32 atomics; at the end dV and dK' -> bf16
+// Tensor memory (512 columns): [0,128) S^T, then P^T (bf16 pairs: packed
+// columns [0, 64) over S columns [0, 32), [64, 128) over [64, 96), so each
+// warpgroup overwrites only S columns it has read); [128,256) dP^T, then the
+// dQ' tile; [256, 256+d) dV;
 // [256+d, 256+2d) dK'.
 #pragma once
 
@@ -52,14 +55,15 @@
 
 namespace gqa {
 
-constexpr int BWD_THREADS = 384;
-// Register split (launch: 384 threads x 168, the most __launch_bounds__(384, 1)
-// allows): loaders and MMA issuer 104, P^T/dS^T rows 232, dQ'/dK'/dV
-// epilogue 168 (the launch value).
-constexpr int BWD_LAUNCH_REGS = 168;
+constexpr int BWD_THREADS = 512;
+// Register split (launch: 512 threads x 128, the most __launch_bounds__(512, 1)
+// allows): loaders and MMA issuer 104, the two P^T/dS^T warpgroups (half of
+// the packed query columns each) 136, dQ'/dK'/dV epilogue 136.
+constexpr int BWD_LAUNCH_REGS = 128;
 constexpr int BWD_REG_PRODUCER = 104;
-constexpr int BWD_REG_SOFTMAX = 232;
-static_assert(BWD_REG_PRODUCER * 128 + BWD_REG_SOFTMAX * 128 + BWD_LAUNCH_REGS * 128 <= BWD_LAUNCH_REGS * BWD_THREADS,
+constexpr int BWD_REG_SOFTMAX = 136;
+constexpr int BWD_REG_READOUT = 136;
+static_assert(BWD_REG_PRODUCER * 128 + 2 * BWD_REG_SOFTMAX * 128 + BWD_REG_READOUT * 128 <= BWD_LAUNCH_REGS * BWD_THREADS,
               "register split exceeds the launch's registers");
 
 // Workspace regions of the backward (byte offsets from the 256-byte aligned base).
@@ -419,9 +423,9 @@ __device__ __forceinline__ void bwd_mma_rows(uint32_t d_tmem, uint64_t da, uint6
 template <class C>
 __device__ __forceinline__ void bwd_mma_dv(uint32_t d_tmem, uint32_t p_tmem, uint64_t db, bool acc) {
 #pragma unroll
-  for (int kk = 0; kk < BM / 16; ++kk)
-    ptx::mma_ts(d_tmem, p_tmem + kk * 8, db + (uint64_t)((kk * 16 * C::ROWB) >> 4), C::IDESC_D,
-                (acc || kk > 0) ? 1u : 0u);
+  for (int kk = 0; kk < BM / 16; ++kk)  // packed columns [0, 64) at p_tmem, [64, 128) at p_tmem + 64
+    ptx::mma_ts(d_tmem, p_tmem + (kk >> 2) * 64 + (kk & 3) * 8, db + (uint64_t)((kk * 16 * C::ROWB) >> 4),
+                C::IDESC_D, (acc || kk > 0) ? 1u : 0u);
 }
 
 // dK' (+)= dS^T Q': A = dS^T (K-major SW128, 64 columns per box), B = Q' (MN-major).
@@ -477,13 +481,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       ptx::mbar_init(B(bars->st_full[s]), 32);
       ptx::mbar_init(B(bars->q_empty[s]), 1);
       ptx::mbar_init(B(bars->do_empty[s]), 1);
-      ptx::mbar_init(B(bars->st_empty[s]), 4);
+      ptx::mbar_init(B(bars->st_empty[s]), 8);
     }
     ptx::mbar_init(B(bars->s_full), 1);
     ptx::mbar_init(B(bars->dp_full), 1);
-    ptx::mbar_init(B(bars->p_full), 128);
+    ptx::mbar_init(B(bars->p_full), 256);
     ptx::mbar_init(B(bars->dv_done), 1);
-    ptx::mbar_init(B(bars->ds_full), 128);
+    ptx::mbar_init(B(bars->ds_full), 256);
     ptx::mbar_init(B(bars->dq_full), 1);
     ptx::mbar_init(B(bars->dq_free), 128);
     ptx::mbar_init(B(bars->acc_done), 1);
@@ -658,16 +662,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       drain_wait(B(bars->drain), 0);
     }
    }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     ptx::setmaxnreg_inc<BWD_REG_SOFTMAX>();
     // ------------------------------------------------------------ P^T, dS^T
-    const int quad = warp - 4;
+    // Two warpgroups: warps 4-7 the packed query columns [0, 64), warps 8-11
+    // [64, 128), of the same key rows (one per thread, TMEM lane quadrant
+    // warp % 4).
+    const int quad = warp & 3;
+    const int half = (warp - 4) >> 2;
+    constexpr int HC = BM / 2;        // columns per warpgroup
+    const int c_lo = half * (HC / 32);  // first 32-column chunk of this half
     const int j = quad * 32 + lane;  // key row of the tile == TMEM lane
     const int key = it.k0 + j;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
     const float sl2 = p.scale_log2;
     bool ok = true;
-    uint32_t pw[BM / 2];  // P^T row, bf16 pairs
+    uint32_t pw[HC / 2];  // this half of the P^T row, bf16 pairs
     uint32_t v[32];
     for (int i = 0; i < it.nt; ++i) {
       const int s = i & 1;
@@ -685,7 +695,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (!ok) break;
       ptx::tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < BM / 32; ++c) {
+      for (int cc = 0; cc < HC / 32; ++cc) {
+        const int c = c_lo + cc;
         ptx::tmem_ld32(trow + C::S_COL + c * 32, v);
         ptx::tmem_wait_ld();
         ptx::reg_fence32(v);
@@ -696,11 +707,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           const float x1 = fmaf(__uint_as_float(v[e + 1]), sl2, -st[col + 1]);
           const float p0 = col >= r_lo ? ptx::ex2(x0) : 0.f;
           const float p1 = col + 1 >= r_lo ? ptx::ex2(x1) : 0.f;
-          pw[col >> 1] = pack_bf16x2(p0, p1);
+          pw[(cc * 32 + e) >> 1] = pack_bf16x2(p0, p1);
         }
       }
-      ptx::tmem_st32(trow + C::S_COL, pw);
-      ptx::tmem_st32(trow + C::S_COL + 32, pw + 32);
+      // P^T of packed columns [64 half, 64 half + 64) as bf16 pairs over the
+      // first 32 of the S columns this warpgroup has just read
+      ptx::tmem_st32(trow + C::S_COL + half * 64, pw);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(B(bars->p_full));
@@ -714,7 +726,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       ptx::tc_fence_after();
       uint8_t* ds = smem + C::ds_off(s);
 #pragma unroll
-      for (int c = 0; c < BM / 32; ++c) {
+      for (int cc = 0; cc < HC / 32; ++cc) {
+        const int c = c_lo + cc;
         ptx::tmem_ld32(trow + C::DP_COL + c * 32, v);
         ptx::tmem_wait_ld();
         ptx::reg_fence32(v);
@@ -727,7 +740,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           for (int e = 0; e < 8; e += 2) {
             const int ce = q4 * 8 + e;  // column inside the chunk of 32
             const int col = c * 32 + ce;
-            const uint32_t pp = pw[col >> 1];
+            const uint32_t pp = pw[(cc * 32 + ce) >> 1];
             const float p0 = __uint_as_float(pp << 16);
             const float p1 = __uint_as_float(pp & 0xFFFF0000u);
             const float d0 = p0 * (__uint_as_float(v[ce]) - st[BM + col]);
@@ -745,9 +758,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (lane == 0) ptx::mbar_arrive(B(bars->st_empty[s]));
     }
   } else {
-    // (runs with the launch's BWD_LAUNCH_REGS registers)
+    ptx::setmaxnreg_inc<BWD_REG_READOUT>();
     // ------------------------------------------------------------ dQ' tiles; dV, dK' at the end
-    const int quad = warp - 8;
+    const int quad = warp - 12;
     const int r = quad * 32 + lane;  // packed q row (dQ' tile) or key row (dV, dK') == TMEM lane
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
     const int tt = r / G;
