@@ -774,22 +774,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (!ok) break;
       ptx::tc_fence_after();
       float* dst = valid ? p.dq_acc + ((size_t)(it.seq_start + tok) * p.nq + it.kvh * G + hin) * D : nullptr;
+      // the whole dQ' row into registers first, so that the next dP may
+      // overwrite these columns before the atomics are issued
+      uint32_t dqr[D];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        ptx::tmem_ld32(trow + C::DP_COL + c * 32, v);
-        ptx::tmem_wait_ld();
-        ptx::reg_fence32(v);
-        if (c == D / 32 - 1) {  // tile read: the next dP may overwrite these columns
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(B(bars->dq_free));
-        }
-        if (valid) {
+      for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(trow + C::DP_COL + c * 32, dqr + c * 32);
+      ptx::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            atomicAdd(reinterpret_cast<float4*>(dst + c * 32) + e,
-                      make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                  __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
-        }
+      for (int c = 0; c < D / 32; ++c) ptx::reg_fence32(dqr + c * 32);
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(B(bars->dq_free));
+      if (valid) {
+#pragma unroll
+        for (int e = 0; e < D / 4; ++e)
+          atomicAdd(reinterpret_cast<float4*>(dst) + e,
+                    make_float4(__uint_as_float(dqr[4 * e]), __uint_as_float(dqr[4 * e + 1]),
+                                __uint_as_float(dqr[4 * e + 2]), __uint_as_float(dqr[4 * e + 3])));
       }
     }
     if (ok) ok = __all_sync(0xffffffffu, bwait(B(bars->acc_done), 0, abort_flag));
