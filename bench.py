@@ -783,7 +783,7 @@ def run_masked(args, rank, world, local_rank, inp, mask_np):
     value = flops * world / (ms_per_step * 1e-3) / 1e12
     peaks, src = load_peaks()
     peak = float(peaks["bf16_tflops"])
-    roof = fwd_roofline(w, attn_ms, peaks, src, clk, torch.cuda.get_device_properties(dev).multi_processor_count)
+    achieved = flops / (attn_ms * 1e-3) / 1e12
     res = {
         "metric": MASKED_METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
