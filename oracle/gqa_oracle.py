@@ -35,13 +35,14 @@ positions default to 0..L-1 ("Kohaku-TT" page, Highlights: flash attention with
 packed variable-length batches).
 
 Precision. Everything is float64. One quantisation is part of the method and
-is modelled on purpose: the rotated Q and K are tensors of the input dtype
-(the RoPE page's ``apply_rope`` returns ``x.dtype``; for bf16 inputs that is
-bf16, which is also what the tensor-core operands are). With
-``operand_rounding=True`` the rotation uses the fp32 cos/sin table the RoPE
-page builds (here: the float64 cos/sin of the float64 angle, rounded once to
-fp32), evaluates x*cos - y*sin in float64 and rounds that once to bf16 (round
-to nearest, ties to even). With ``operand_rounding=False`` the rotation is
+is modelled on purpose: the rotated Q and K are tensors of the input dtype.
+The RoPE page's ``apply_rope`` casts the fp32 cos/sin table to ``x.dtype``
+and evaluates ``x * cos + rotate_half(x) * sin`` in that dtype; for bf16
+inputs (also the tensor-core operands' type) that is: cos and sin rounded to
+bf16, each product rounded to bf16, the sum rounded to bf16, all to nearest
+even. With ``operand_rounding=True`` the rotation is evaluated that way, on
+the fp32 table the page builds (here: the float64 cos/sin of the float64
+angle, rounded once to fp32). With ``operand_rounding=False`` the rotation is
 exact float64 and nothing is rounded; the RoPE pins use that form.
 
 Decoding (``gqa_rope_decode``): one new token per sequence against a cache of
@@ -87,6 +88,7 @@ __all__ = [
     "rope_cos_sin",
     "rotate_half",
     "apply_rope",
+    "rope_exact_rounded_once",
     "share_kv_heads",
     "score",
     "causal_mask",
@@ -168,7 +170,16 @@ def rotate_half(x: np.ndarray) -> np.ndarray:
 
 def apply_rope(x: np.ndarray, positions, theta: float, operand_rounding: bool = False) -> np.ndarray:
     """x: [T, H, d] (token-major). Returns x*cos + rotate_half(x)*sin with the
-    cos/sin row of each token's position broadcast over heads."""
+    cos/sin row of each token's position broadcast over heads.
+
+    With ``operand_rounding`` the page's bf16 evaluation: x taken as bf16
+    (rounded first; a no-op for bf16 inputs), the fp32 table cast to bf16,
+    then x*cos and rotate_half(x)*sin each rounded to bf16 and their sum
+    rounded to bf16. A product of two bf16 values has at most 16 significant
+    bits, so it is exact in float64 and rounding it here is the page's fp32
+    product cast to bf16; a sum of two bf16 values is exact in float64 unless
+    the addends' exponents differ by more than 44, and then the sum rounds to
+    the larger addend either way."""
     x = np.asarray(x, dtype=np.float64)
     d = x.shape[-1]
     c, s = rope_cos_sin(positions, d, theta, table_fp32=operand_rounding)
@@ -176,10 +187,22 @@ def apply_rope(x: np.ndarray, positions, theta: float, operand_rounding: bool = 
     s = s[:, None, :]
     if not operand_rounding:
         return x * c + rotate_half(x) * s
-    # Each product below is exact in float64 (8-bit by 24-bit significands);
-    # the sum is rounded once to float64, then once to bf16.
-    y = x * c + rotate_half(x) * s
-    return round_to_bf16(y)
+    xb = round_to_bf16(x)
+    cb, sb = round_to_bf16(c), round_to_bf16(s)
+    a = round_to_bf16(xb * cb)
+    b = round_to_bf16(rotate_half(xb) * sb)
+    return round_to_bf16(a + b)
+
+
+def rope_exact_rounded_once(x: np.ndarray, positions, theta: float) -> np.ndarray:
+    """The rotation of a fused projection epilogue: x (float64, e.g. a
+    projection before any rounding) rotated exactly with the fp32 cos/sin
+    table and rounded once, to nearest even, to bf16. Each product of a
+    float64 value with an fp32 table entry is formed in float64, the sum
+    rounded once to float64, then once to bf16."""
+    x = np.asarray(x, dtype=np.float64)
+    c, s = rope_cos_sin(positions, x.shape[-1], theta, table_fp32=True)
+    return round_to_bf16(x * c[:, None, :] + rotate_half(x) * s[:, None, :])
 
 
 # ---------------------------------------------------------------------------
@@ -488,9 +511,10 @@ def qkv_rope_projection(x, w_q, w_k, w_v, n_q_heads: int, n_kv_heads: int, rope_
     column c of head h. Each token is rotated by positions[t] if given, else
     by its index inside its sequence of ``cu_seqlens`` if given, else by t.
     Returns q [N, n_q, d], k [N, n_kv, d], v [N, n_kv, d] in float64. With
-    ``operand_rounding`` the rotation takes the fp32 cos/sin table and every
-    output is rounded once, to bf16, from its float64 value (no rounding
-    between the projection and the rotation)."""
+    ``operand_rounding`` the outputs are those of a fused epilogue: the
+    rotation takes the fp32 cos/sin table and every output is rounded once,
+    to bf16, from its float64 value (no rounding between the projection and
+    the rotation; ``rope_exact_rounded_once``)."""
     x = np.asarray(x, dtype=np.float64)
     w_q = np.asarray(w_q, dtype=np.float64)
     w_k = np.asarray(w_k, dtype=np.float64)
@@ -513,9 +537,14 @@ def qkv_rope_projection(x, w_q, w_k, w_v, n_q_heads: int, n_kv_heads: int, rope_
     yk = np.matmul(x, w_k.T).reshape(N, n_kv_heads, d)
     yv = np.matmul(x, w_v.T).reshape(N, n_kv_heads, d)
     # 2. Rotate Q and K, never V.
-    q = apply_rope(yq, pos, rope_theta, operand_rounding)
-    k = apply_rope(yk, pos, rope_theta, operand_rounding)
+    if operand_rounding:
+        rope = lambda y: rope_exact_rounded_once(y, pos, rope_theta)  # noqa: E731
+    else:
+        rope = lambda y: apply_rope(y, pos, rope_theta)  # noqa: E731
+    q = rope(yq)
+    k = rope(yk)
     v = round_to_bf16(yv) if operand_rounding else yv
+    return q, k, v
     return q, k, v
 
 

@@ -29,6 +29,8 @@ def _all_pins(m, golden):
         lambda: pins.pin_rope_identity_at_zero(m),
         lambda: pins.pin_rope_relative(m),
         lambda: pins.pin_rope_basis_closed_form(m),
+        lambda: pins.pin_rope_operand_rounding(m),
+        lambda: pins.pin_rope_bf16_matches_torch(m),
         lambda: pins.pin_worked_attention(golden, m),
         lambda: pins.pin_first_row(m),
         lambda: pins.pin_identical_keys(m),
@@ -138,6 +140,31 @@ MUTATIONS = {
     "rope on V": _mut_rope_on_v,
     "softmax not normalised": _mut_no_normalise,
 }
+
+
+# Planted mistakes in the rounded rotation, made in the oracle's source text.
+SOURCE_MUTATIONS = {
+    "cos/sin left in fp32": ("cb, sb = round_to_bf16(c), round_to_bf16(s)", "cb, sb = c, s"),
+    "products not rounded": ("a = round_to_bf16(xb * cb)", "a = xb * cb"),
+    "one rounding of the whole rotation": ("return round_to_bf16(a + b)",
+                                           "return round_to_bf16(xb * c + rotate_half(xb) * s)"),
+    "sum left unrounded": ("return round_to_bf16(a + b)", "return a + b"),
+}
+
+
+def _source_mutant(old, new):
+    src = open(os.path.join(ROOT, "oracle", "gqa_oracle.py")).read()
+    assert src.count(old) == 1, old
+    spec = importlib.util.spec_from_loader("_oracle_src_mut", loader=None)
+    m = importlib.util.module_from_spec(spec)
+    exec(compile(src.replace(old, new), "_oracle_src_mut", "exec"), m.__dict__)
+    return m
+
+
+@pytest.mark.parametrize("name", sorted(SOURCE_MUTATIONS))
+def test_planted_rounding_mistake_is_caught(name, golden):
+    m = _source_mutant(*SOURCE_MUTATIONS[name])
+    assert _all_pins(m, golden) >= 1, f"no pin caught the planted mistake: {name}"
 
 
 def test_unmutated_copy_passes_all_pins(golden):

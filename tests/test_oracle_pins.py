@@ -158,18 +158,59 @@ def test_rope_basis_closed_form():
     pin_rope_basis_closed_form()
 
 
+def _table(pos, d, theta):
+    """fp32 cos/sin of the float64 angle pos * theta^(-2i/d), duplicated over
+    the two halves (the RoPE page's table), written out here on its own."""
+    i = np.arange(d // 2, dtype=np.float64)
+    ang = np.asarray(pos, np.float64)[:, None] * theta ** (-2.0 * i / d)
+    ang = np.concatenate([ang, ang], axis=-1)
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
 def pin_rope_operand_rounding(m=orc):
-    """Rounded rotation: bf16-representable and within half a bf16 ulp (2^-8
-    relative, 8 significant bits) plus the fp32-table error of the exact rotation."""
+    """Rounded rotation: bf16-representable and within the error of its
+    roundings of the exact rotation: cos/sin and the two products each to
+    bf16 (unit roundoff u = 2^-8), the sum to bf16 (u of the result), plus
+    the fp32 table's error."""
     r = _rng(5)
     x = _bf16(r.standard_normal((300, 2, 128)))
     pos = r.integers(0, 8192, 300)
     ex = m.apply_rope(x, pos, 5e5, operand_rounding=False)
     ro = m.apply_rope(x, pos, 5e5, operand_rounding=True)
     assert np.array_equal(ro, _bf16(ro))
+    c, s = (t.astype(np.float64)[:, None, :] for t in _table(pos, 128, 5e5))
+    u = 2.0 ** -8
+    y = orc.rotate_half(x)
     err = np.abs(ro - ex)
-    bound = np.abs(ex) * 2.0 ** -8 + 4e-7 * (np.abs(x) + np.abs(orc.rotate_half(x)))
+    bound = u * np.abs(ex) + 2.1 * u * (np.abs(x * c) + np.abs(y * s)) + 4e-7 * (np.abs(x) + np.abs(y))
     assert np.all(err <= bound + 1e-30)
+
+
+def pin_rope_bf16_matches_torch(m=orc):
+    """The rounded rotation is, bit for bit, the RoPE page's apply_rope run by
+    torch on bf16 CPU tensors (cos and sin cast to bf16, x * cos +
+    rotate_half(x) * sin in bf16): inputs over a wide range of scales, with
+    cancelling pairs, zeros and position 0."""
+    import torch
+
+    r = _rng(6)
+    T, H, d, theta = 400, 3, 64, 5e5
+    x = r.standard_normal((T, H, d)) * np.exp2(r.integers(-20, 21, (T, H, d)))
+    x[:5] = 0.0
+    x[5:40, :, d // 2:] = x[5:40, :, : d // 2]  # pairs (v, v): x*cos and x*sin cancel near 45 degrees
+    x = _bf16(x)
+    pos = r.integers(0, 100000, T)
+    pos[:10] = 0
+    cos, sin = (torch.from_numpy(t)[:, None, :].to(torch.bfloat16) for t in _table(pos, d, theta))
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    rot = torch.cat((-xt[..., d // 2:], xt[..., : d // 2]), dim=-1)
+    ref = (xt * cos + rot * sin).double().numpy()
+    got = m.apply_rope(x, pos, theta, operand_rounding=True)
+    assert np.array_equal(got, ref)
+
+
+def test_rope_bf16_matches_torch():
+    pin_rope_bf16_matches_torch()
 
 
 def test_rope_operand_rounding_bound():

@@ -136,8 +136,8 @@ MUTATIONS = {
     "head_split_transposed": ("np.matmul(x, w_k.T).reshape(N, n_kv_heads, d)",
                               "np.matmul(x, w_k.T).reshape(N, d, n_kv_heads).transpose(0, 2, 1)"),
     "v_rotated": ("v = round_to_bf16(yv) if operand_rounding else yv",
-                  "v = apply_rope(yv, pos, rope_theta, operand_rounding)"),
-    "k_not_rotated": ("k = apply_rope(yk, pos, rope_theta, operand_rounding)", "k = yk"),
+                  "v = rope(yv)"),
+    "k_not_rotated": ("k = rope(yk)", "k = yk"),
     "positions_ignored": ("pos = np.asarray(positions, dtype=np.int64).reshape(-1)\n    elif",
                           "pos = np.arange(N)\n    elif"),
 }
