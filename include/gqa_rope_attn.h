@@ -30,11 +30,13 @@
  * (gqa_rope_attn_qkv_proj) are declared further down.
  *
  * Precision: q, k, v, out are bf16 (or fp32 with dtype GQA_DTYPE_FP32; then
- * q, k, v are rounded to bf16 on load and out is written as fp32). cos/sin
- * are the fp32 values of the float64 angle's cos/sin; the rotated q and k are
- * rounded once, to nearest even, to bf16 (the tensor-core operands). Scores
- * and the output accumulate in fp32; the softmax weights enter P.V as bf16.
- * lse is fp32.
+ * q, k, v are rounded to bf16 on load and out is written as fp32). RoPE is
+ * evaluated in bf16, as the RoPE page's apply_rope evaluates it on bf16
+ * tensors: cos/sin are the fp32 values of the float64 angle's cos/sin cast to
+ * bf16, and x*cos and rotate_half(x)*sin are each rounded to bf16, then their
+ * sum (round to nearest even throughout); the rotated q and k are the
+ * tensor-core operands. Scores and the output accumulate in fp32; the softmax
+ * weights enter P.V as bf16. lse is fp32.
  *
  * Memory layout ("THD", all row-major, contiguous, device memory):
  *   q          [total_tokens, n_q_heads,  head_dim]
@@ -232,7 +234,7 @@ int gqa_rope_attn_fwd_masked(const void* q, const void* k, const void* v, const 
  * K and one V vector per token and KV head is kept for every token so far.
  * For sequence b the new token sits at position p = cache_seqlens[b]:
  *
- *   k_cache[b, p, kv, :] = rope(k_new[b, kv], p)   (rounded once to bf16)
+ *   k_cache[b, p, kv, :] = rope(k_new[b, kv], p)   (bf16, the prefill's rotation)
  *   v_cache[b, p, kv, :] = v_new[b, kv]
  *   out[b, h, :] = softmax_j( rope(q[b, h], p) . k_cache[b, j, kv] / sqrt(d) ) v_cache[b, j, kv],
  *                  j = 0 .. p, kv = h / G
@@ -281,8 +283,9 @@ int gqa_rope_attn_decode(const void* q, const void* k_new, const void* v_new, vo
  * where rope^T rotates each pair (i, i + d/2) by the negative angle (the
  * transpose of the rotation). lse and out are the forward's outputs for the
  * same q, k, v (lse is required: P is recomputed from it, not stored). The
- * rotated q and k are rounded to bf16 exactly as the forward rounds them; the
- * gradient passes that rounding unchanged. P and dS enter their products as
+ * rotated q and k are computed exactly as the forward computes them; the
+ * gradient passes the rotation's roundings unchanged (rope^T uses the fp32
+ * cos/sin). P and dS enter their products as
  * bf16; every product accumulates in fp32; dq accumulates over key tiles in
  * fp32 in the workspace.
  *

@@ -51,8 +51,8 @@ def test_abi_version_and_strerror():
 
 def test_workspace_size():
     ws = _abi.workspace_size(1, 8192, 32, 8, 128)
-    # at least the RoPE'd K (n_kv * N * d * 2) and the cos/sin table (N * d/2 * 8)
-    assert ws >= 8 * 8192 * 128 * 2 + 8192 * 64 * 8
+    # at least the RoPE'd K (n_kv * N * d * 2) and the bf16 cos/sin table (N * d/2 * 4)
+    assert ws >= 8 * 8192 * 128 * 2 + 8192 * 64 * 4
     assert ws % 256 == 0
     assert _abi.workspace_size(1, 8192, 32, 8, 128, _abi.GQA_DTYPE_FP32) > ws
     assert _abi.workspace_size(1, 8192, 32, 8, 96) == 0

@@ -444,16 +444,11 @@ __device__ __forceinline__ bool rope_q_tile(const AttnParams& p, uint8_t* smem, 
     const int ch = item - tt * NCH;
     const int tok = wi.t0 + tt;
     if (tok >= wi.L) continue;
-    const float4* tab = reinterpret_cast<const float4*>(p.table + (size_t)(wi.seq_start + tok) * HALF + ch * 8);
-    float cs[8], sn[8];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float4 t4 = ptx::ld_cg_v4f32(tab + e);
-      cs[2 * e] = t4.x;
-      sn[2 * e] = t4.y;
-      cs[2 * e + 1] = t4.z;
-      sn[2 * e + 1] = t4.w;
-    }
+    // bf16 cos and sin of frequencies ch*8 .. ch*8+7 (table_word layout)
+    const float4* tab = reinterpret_cast<const float4*>(p.table + table_word(wi.seq_start + tok, HALF, ch * 8));
+    const float4 cf = ptx::ld_cg_v4f32(tab), sf = ptx::ld_cg_v4f32(tab + 1);
+    const uint32_t cw[4] = {__float_as_uint(cf.x), __float_as_uint(cf.y), __float_as_uint(cf.z), __float_as_uint(cf.w)};
+    const uint32_t sw[4] = {__float_as_uint(sf.x), __float_as_uint(sf.y), __float_as_uint(sf.z), __float_as_uint(sf.w)};
     const int col_lo = ch * 8, col_hi = ch * 8 + HALF;
     const int bx_lo = col_lo / C::BOXC, bx_hi = col_hi / C::BOXC;
     for (int hh = 0; hh < G; ++hh) {
@@ -463,14 +458,10 @@ __device__ __forceinline__ bool rope_q_tile(const AttnParams& p, uint8_t* smem, 
       uint4* phi = reinterpret_cast<uint4*>(qbuf + bx_hi * C::Q_BOX_BYTES +
                                             swz(row * C::ROWB + (col_hi % C::BOXC) * 2, C::SWZ_MASK));
       uint4 vlo = *plo, vhi = *phi;
-      __nv_bfloat16* xl = reinterpret_cast<__nv_bfloat16*>(&vlo);
-      __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(&vhi);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float fl = __bfloat162float(xl[e]), fh = __bfloat162float(xh[e]);
-        xl[e] = __ushort_as_bfloat16(rope_round_bf16(fl, cs[e], fh, -sn[e]));
-        xh[e] = __ushort_as_bfloat16(rope_round_bf16(fh, cs[e], fl, sn[e]));
-      }
+      rope_bf16x2(vlo.x, vhi.x, cw[0], sw[0], vlo.x, vhi.x);
+      rope_bf16x2(vlo.y, vhi.y, cw[1], sw[1], vlo.y, vhi.y);
+      rope_bf16x2(vlo.z, vhi.z, cw[2], sw[2], vlo.z, vhi.z);
+      rope_bf16x2(vlo.w, vhi.w, cw[3], sw[3], vlo.w, vhi.w);
       *plo = vlo;
       *phi = vhi;
     }

@@ -222,9 +222,10 @@ __device__ void build_kv_schedule(const BwdPrepParams& p) {
   if (tid == 0) p.header[0] = P;
 }
 
-// (cos, sin) row of every token, K' head-major and Q' token-major, rounded
-// exactly as the forward rounds them (rope_round.cuh). One thread per
-// (token, pair of frequencies).
+// (cos, sin) row of every token (fp32, for the transposed rotations of dq
+// and dk), K' head-major and Q' token-major in the forward's bf16 rotation
+// (rope_bf16x2 in rope_round.cuh), so that the recomputed scores are the
+// forward's. One thread per (token, pair of frequencies).
 template <int D>
 __device__ void bwd_rope_rows(const BwdPrepParams& p, int block, int nblocks) {
   constexpr int HALF = D / 2;
@@ -250,20 +251,13 @@ __device__ void bwd_rope_rows(const BwdPrepParams& p, int block, int nblocks) {
       sn[e] = (float)sd;
     }
     *reinterpret_cast<float4*>(p.table + (size_t)t * HALF + i) = make_float4(c[0], sn[0], c[1], sn[1]);
+    const uint32_t c2 = bf16x2_rn(c[0], c[1]), s2 = bf16x2_rn(sn[0], sn[1]);
     auto rotate = [&](const __nv_bfloat16* src, __nv_bfloat16* dst) {
-      const uint32_t wl = *reinterpret_cast<const uint32_t*>(src + i);
-      const uint32_t wh = *reinterpret_cast<const uint32_t*>(src + i + HALF);
-      uint32_t ol[2], oh[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        __nv_bfloat16 lo, hi;
-        rope_pair(__uint_as_float(((wl >> (16 * e)) & 0xFFFFu) << 16),
-                  __uint_as_float(((wh >> (16 * e)) & 0xFFFFu) << 16), c[e], sn[e], lo, hi);
-        ol[e] = __bfloat16_as_ushort(lo);
-        oh[e] = __bfloat16_as_ushort(hi);
-      }
-      *reinterpret_cast<uint32_t*>(dst + i) = ol[0] | (ol[1] << 16);
-      *reinterpret_cast<uint32_t*>(dst + i + HALF) = oh[0] | (oh[1] << 16);
+      uint32_t ol, oh;
+      rope_bf16x2(*reinterpret_cast<const uint32_t*>(src + i), *reinterpret_cast<const uint32_t*>(src + i + HALF), c2,
+                  s2, ol, oh);
+      *reinterpret_cast<uint32_t*>(dst + i) = ol;
+      *reinterpret_cast<uint32_t*>(dst + i + HALF) = oh;
     };
     for (int h = 0; h < p.nkv; ++h)
       rotate(p.k + ((size_t)t * p.nkv + h) * D, p.kws + ((size_t)h * p.N + t) * D);

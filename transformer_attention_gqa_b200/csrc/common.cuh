@@ -41,7 +41,7 @@ struct WsLayout {
   size_t header;   // int[16]: [0] number of (sequence, q-tile) pairs, [8] work-item counter
   size_t seq_pfx;  // int[num_seqs + 1]: first pair index of each sequence
   size_t pairs;    // int2[max_pairs]: (sequence, q-tile) in decreasing cost order
-  size_t table;    // float2[N * d/2]: (cos, sin) of each token's angles
+  size_t table;    // uint32[N * d/2]: bf16 (cos, sin) of each token's angles (table_word)
   size_t kws;      // bf16[n_kv][N][d]: RoPE'd K, head-major
   size_t qws;      // bf16[N][n_q][d]: rotated q (when the prologue rotates it)
   size_t vws;      // bf16[N][n_kv][d]: v rounded to bf16 (fp32 inputs only)
@@ -71,7 +71,7 @@ __host__ inline WsLayout ws_layout(int num_seqs, int N, int nq, int nkv, int d, 
   w.pairs = off;
   off = align_up(off + (size_t)w.max_pairs * 8, 256);
   w.table = off;
-  off = align_up(off + (size_t)N * (d / 2) * 8, 256);
+  off = align_up(off + (size_t)N * (d / 2) * 4, 256);
   w.kws = off;
   off = align_up(off + (size_t)nkv * N * d * 2, 256);
   w.qws = w.vws = 0;
@@ -87,6 +87,14 @@ __host__ inline WsLayout ws_layout(int num_seqs, int N, int nq, int nkv, int d, 
   return w;
 }
 
+// The forward's RoPE table holds, for each token, d/16 chunks of 8
+// frequencies: the chunk's bf16 cos values as 4 bf16x2 words, then its bf16
+// sin values as 4 words (d/2 words per token). Word of the cos of the even
+// frequency i and i + 1 (the sin word follows 4 words later):
+__host__ __device__ constexpr size_t table_word(int t, int half, int i) {
+  return (size_t)t * half + (size_t)(i / 8) * 8 + (i % 8) / 2;
+}
+
 struct PrepParams {
   const void* q;  // read when the prologue rotates q
   const void* k;
@@ -99,7 +107,7 @@ struct PrepParams {
   int* header;
   int* seq_pfx;
   int2* pairs;
-  float2* table;
+  uint32_t* table;  // table_word layout
   __nv_bfloat16* kws;
   __nv_bfloat16* qws;
   __nv_bfloat16* vws;
@@ -110,7 +118,7 @@ struct AttnParams {
   const int* header;
   int* item_counter;    // work items taken so far beyond the first of each CTA (zeroed by the prologue)
   const int2* pairs;
-  const float2* table;
+  const uint32_t* table;  // table_word layout
   void* out;
   float* lse;
   int N, nq, nkv, G, tq, causal;

@@ -90,7 +90,7 @@ struct DtcCfg {
   static constexpr int OFF_Q = 0;                            // 128-row query tile
   static constexpr int OFF_K = A::Q_BYTES;                   // [stage] K tiles
   static constexpr int OFF_V = OFF_K + DTC_STAGES * TILE_BYTES;  // [stage] V tiles
-  static constexpr int OFF_CS = OFF_V + DTC_STAGES * TILE_BYTES;  // float2 [D/2] (cos, sin) at pos
+  static constexpr int OFF_CS = OFF_V + DTC_STAGES * TILE_BYTES;  // uint2 [D/4]: bf16x2 (cos, sin) at pos
   static constexpr int OFF_NEW = OFF_CS + (D / 2) * 8;           // bf16 [2][D]: rotated new key, value
   static constexpr int OFF_BAR = OFF_NEW + 2 * D * 2;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;       // + barriers + alignment slack
@@ -307,37 +307,46 @@ __global__ void __launch_bounds__(DTC_THREADS, 1)
     const int g = 4 * lane + warp;  // the head of this row (a row past G holds none)
     const bool active = g < G;
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-    float2* cs = reinterpret_cast<float2*>(smem + C::OFF_CS);
+    uint2* cs = reinterpret_cast<uint2*>(smem + C::OFF_CS);
     __nv_bfloat16* knew = reinterpret_cast<__nv_bfloat16*>(smem + C::OFF_NEW);
-    // zero query tile; (cos, sin) at pos (float64 angle, fp32 values)
+    // zero query tile; bf16x2 (cos, sin) words of frequencies (2j, 2j + 1) at
+    // pos (float64 angle, rounded to fp32, then to bf16 as in the prefill)
     for (int i = tid; i < A::Q_BYTES / 16; i += 128)
       reinterpret_cast<uint4*>(smem + C::OFF_Q)[i] = make_uint4(0, 0, 0, 0);
-    for (int i = tid; i < HALF; i += 128) {
-      double sd, cd;
-      sincos((double)pos * p.inv_freq[i], &sd, &cd);
-      cs[i] = make_float2((float)cd, (float)sd);
+    for (int j = tid; j < HALF / 2; j += 128) {
+      float c[2], sn[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        double sd, cd;
+        sincos((double)pos * p.inv_freq[2 * j + e], &sd, &cd);
+        c[e] = (float)cd;
+        sn[e] = (float)sd;
+      }
+      cs[j] = make_uint2(bf16x2_rn(c[0], c[1]), bf16x2_rn(sn[0], sn[1]));
     }
     dtc_softmax_sync();
     // rotated queries into their tile rows, and the new key (if this range
-    // holds pos); each rotated value rounded once to bf16, as in the prefill
-    const int nrot = (G + (has_new ? 1 : 0)) * HALF;
+    // holds pos), two frequencies per item, in the prefill's bf16 rotation
+    constexpr int NPAIR = HALF / 2;
+    const int nrot = (G + (has_new ? 1 : 0)) * NPAIR;
     for (int it = tid; it < nrot; it += 128) {
-      const int hg = it / HALF, i = it - hg * HALF;
-      const float2 c = cs[i];
+      const int hg = it / NPAIR, i = 2 * (it - hg * NPAIR);
+      const uint2 c = cs[i / 2];
       const __nv_bfloat16* src =
           hg < G ? p.q + ((size_t)b * p.nq + h * G + hg) * D : p.k_new + ((size_t)b * p.nkv + h) * D;
-      const float xl = __bfloat162float(src[i]), xh = __bfloat162float(src[i + HALF]);
-      const uint16_t lo = rope_round_bf16(xl, c.x, xh, -c.y), hi = rope_round_bf16(xh, c.x, xl, c.y);
+      uint32_t lo, hi;
+      rope_bf16x2(*reinterpret_cast<const uint32_t*>(src + i), *reinterpret_cast<const uint32_t*>(src + i + HALF),
+                  c.x, c.y, lo, hi);
       if (hg < G) {
         const int row = 32 * (hg % 4) + hg / 4;
         const int cl = i, chh = i + HALF;
-        *reinterpret_cast<uint16_t*>(smem + C::OFF_Q + (cl / A::BOXC) * A::Q_BOX_BYTES +
+        *reinterpret_cast<uint32_t*>(smem + C::OFF_Q + (cl / A::BOXC) * A::Q_BOX_BYTES +
                                      swz(row * A::ROWB + (cl % A::BOXC) * 2, A::SWZ_MASK)) = lo;
-        *reinterpret_cast<uint16_t*>(smem + C::OFF_Q + (chh / A::BOXC) * A::Q_BOX_BYTES +
+        *reinterpret_cast<uint32_t*>(smem + C::OFF_Q + (chh / A::BOXC) * A::Q_BOX_BYTES +
                                      swz(row * A::ROWB + (chh % A::BOXC) * 2, A::SWZ_MASK)) = hi;
       } else {
-        knew[i] = __ushort_as_bfloat16(lo);
-        knew[i + HALF] = __ushort_as_bfloat16(hi);
+        *reinterpret_cast<uint32_t*>(knew + i) = lo;
+        *reinterpret_cast<uint32_t*>(knew + i + HALF) = hi;
       }
     }
     if (has_new)

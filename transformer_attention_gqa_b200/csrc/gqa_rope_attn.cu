@@ -168,7 +168,7 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
   pp.header = reinterpret_cast<int*>(ws + lay.header);
   pp.seq_pfx = reinterpret_cast<int*>(ws + lay.seq_pfx);
   pp.pairs = reinterpret_cast<int2*>(ws + lay.pairs);
-  pp.table = reinterpret_cast<float2*>(ws + lay.table);
+  pp.table = reinterpret_cast<uint32_t*>(ws + lay.table);
   pp.kws = reinterpret_cast<__nv_bfloat16*>(ws + lay.kws);
   // the prologue rotates Q into the workspace when the layout has room for it
   // (fp32 inputs, or short work items), never for inputs already rotated
@@ -563,7 +563,7 @@ int launch_masked(const void* q, const void* k, const void* v, const int32_t* po
   pp.header = reinterpret_cast<int*>(ws + lay.header);
   pp.seq_pfx = reinterpret_cast<int*>(ws + lay.seq_pfx);
   pp.pairs = reinterpret_cast<int2*>(ws + lay.pairs);
-  pp.table = reinterpret_cast<float2*>(ws + lay.table);
+  pp.table = reinterpret_cast<uint32_t*>(ws + lay.table);
   pp.kws = reinterpret_cast<__nv_bfloat16*>(ws + lay.kws);
   pp.qws = nullptr;
   pp.vws = nullptr;

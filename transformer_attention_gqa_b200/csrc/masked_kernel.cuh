@@ -240,23 +240,19 @@ __global__ void __launch_bounds__(MK_THREADS, 1)
     const bool row_valid = r < rows && tok < wi.L;
     bool ok = __all_sync(0xffffffffu, bwait(B(bars->q_loaded), 0, abort_flag));
     if (ok) {
-      // rotate the Q tile in shared memory (the forward's exact rounding)
+      // rotate the Q tile in shared memory (the forward's bf16 rotation)
       uint8_t* qbuf = smem + C::OFF_Q;
       for (int item = tid; item < p.tq * NCH; item += 128) {
         const int it_t = item / NCH;
         const int ch = item - it_t * NCH;
         const int qt = wi.t0 + it_t;
         if (qt >= wi.L) continue;
-        const float4* tab = reinterpret_cast<const float4*>(p.table + (size_t)(wi.seq_start + qt) * HALF + ch * 8);
-        float cs[8], sn[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float4 t4 = ptx::ld_cg_v4f32(tab + e);
-          cs[2 * e] = t4.x;
-          sn[2 * e] = t4.y;
-          cs[2 * e + 1] = t4.z;
-          sn[2 * e + 1] = t4.w;
-        }
+        const float4* tab = reinterpret_cast<const float4*>(p.table + table_word(wi.seq_start + qt, HALF, ch * 8));
+        const float4 cf = ptx::ld_cg_v4f32(tab), sf = ptx::ld_cg_v4f32(tab + 1);
+        const uint32_t cw[4] = {__float_as_uint(cf.x), __float_as_uint(cf.y), __float_as_uint(cf.z),
+                                __float_as_uint(cf.w)};
+        const uint32_t sw[4] = {__float_as_uint(sf.x), __float_as_uint(sf.y), __float_as_uint(sf.z),
+                                __float_as_uint(sf.w)};
         const int col_lo = ch * 8, col_hi = ch * 8 + HALF;
         for (int hh = 0; hh < G; ++hh) {
           const int row = it_t * G + hh;
@@ -265,14 +261,10 @@ __global__ void __launch_bounds__(MK_THREADS, 1)
           uint4* phi = reinterpret_cast<uint4*>(qbuf + (col_hi / A::BOXC) * A::Q_BOX_BYTES +
                                                 swz(row * A::ROWB + (col_hi % A::BOXC) * 2, A::SWZ_MASK));
           uint4 vlo = *plo, vhi = *phi;
-          __nv_bfloat16* xl = reinterpret_cast<__nv_bfloat16*>(&vlo);
-          __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(&vhi);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float fl = __bfloat162float(xl[e]), fh = __bfloat162float(xh[e]);
-            xl[e] = __ushort_as_bfloat16(rope_round_bf16(fl, cs[e], fh, -sn[e]));
-            xh[e] = __ushort_as_bfloat16(rope_round_bf16(fh, cs[e], fl, sn[e]));
-          }
+          rope_bf16x2(vlo.x, vhi.x, cw[0], sw[0], vlo.x, vhi.x);
+          rope_bf16x2(vlo.y, vhi.y, cw[1], sw[1], vlo.y, vhi.y);
+          rope_bf16x2(vlo.z, vhi.z, cw[2], sw[2], vlo.z, vhi.z);
+          rope_bf16x2(vlo.w, vhi.w, cw[3], sw[3], vlo.w, vhi.w);
           *plo = vlo;
           *phi = vhi;
         }

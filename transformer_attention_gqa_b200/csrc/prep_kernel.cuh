@@ -16,9 +16,10 @@
 // position * inv_freq[i]; feature i is rotated with feature i + d/2:
 //   out[i]       = x[i]       * cos - x[i + d/2] * sin
 //   out[i + d/2] = x[i + d/2] * cos + x[i]       * sin
-// The angle and cos/sin are evaluated in float64 and stored as fp32; the
-// rotated value is rounded once, to nearest even, to bf16 from its exact
-// value (rope_round.cuh).
+// The angle and cos/sin are evaluated in float64 and rounded to fp32 (the
+// page's table is fp32), then cast to bf16 as the page's apply_rope casts
+// them to the bf16 inputs' dtype; the rotation is evaluated in bf16
+// arithmetic (rope_bf16x2 in rope_round.cuh).
 #pragma once
 
 #include "common.cuh"
@@ -29,12 +30,6 @@ namespace gqa {
 
 
 __device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
-
-__device__ __forceinline__ void rope_pair(float xl, float xh, float c, float s, __nv_bfloat16& ol,
-                                          __nv_bfloat16& oh) {
-  ol = __ushort_as_bfloat16(rope_round_bf16(xl, c, xh, -s));
-  oh = __ushort_as_bfloat16(rope_round_bf16(xh, c, xl, s));
-}
 
 // largest s in [0, n) with a[s] <= x (a nondecreasing, a[0] <= x)
 __device__ __forceinline__ int upper_index(const int* a, int n, int x) {
@@ -191,9 +186,8 @@ __device__ void rope_k_and_table(const PrepParams& p, int block, int nblocks) {
           // inputs are rounded to bf16 before anything else
           const float2 a = *reinterpret_cast<const float2*>((const float*)p.k + src + i);
           const float2 b = *reinterpret_cast<const float2*>((const float*)p.k + src + i + HALF);
-          const __nv_bfloat162 ra = __floats2bfloat162_rn(a.x, a.y), rb = __floats2bfloat162_rn(b.x, b.y);
-          wl[u] = *reinterpret_cast<const uint32_t*>(&ra);
-          wh[u] = *reinterpret_cast<const uint32_t*>(&rb);
+          wl[u] = bf16x2_rn(a.x, a.y);
+          wh[u] = bf16x2_rn(b.x, b.y);
         } else {
           wl[u] = *reinterpret_cast<const uint32_t*>((const __nv_bfloat16*)p.k + src + i);
           wh[u] = *reinterpret_cast<const uint32_t*>((const __nv_bfloat16*)p.k + src + i + HALF);
@@ -217,25 +211,21 @@ __device__ void rope_k_and_table(const PrepParams& p, int block, int nblocks) {
       c[e] = (float)cd;
       sn[e] = (float)sd;
     }
-    *reinterpret_cast<float4*>(p.table + (size_t)t * HALF + i) = make_float4(c[0], sn[0], c[1], sn[1]);
+    const uint32_t c2 = bf16x2_rn(c[0], c[1]), s2 = bf16x2_rn(sn[0], sn[1]);
+    const size_t tw = table_word(t, HALF, i);
+    p.table[tw] = c2;
+    p.table[tw + 4] = s2;
 
     for (int h0 = 0; h0 < p.nkv; h0 += HB) {
       if (h0 > 0) load_heads(h0);
 #pragma unroll
       for (int u = 0; u < HB; ++u) {
         if (h0 + u >= p.nkv) break;
-        uint32_t ol[2], oh[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          __nv_bfloat16 lo, hi;
-          rope_pair(__uint_as_float(((wl[u] >> (16 * e)) & 0xFFFFu) << 16),
-                    __uint_as_float(((wh[u] >> (16 * e)) & 0xFFFFu) << 16), c[e], sn[e], lo, hi);
-          ol[e] = __bfloat16_as_ushort(lo);
-          oh[e] = __bfloat16_as_ushort(hi);
-        }
+        uint32_t ol, oh;
+        rope_bf16x2(wl[u], wh[u], c2, s2, ol, oh);
         const size_t dst = ((size_t)(h0 + u) * p.N + t) * D;
-        *reinterpret_cast<uint32_t*>(p.kws + dst + i) = ol[0] | (ol[1] << 16);
-        *reinterpret_cast<uint32_t*>(p.kws + dst + i + HALF) = oh[0] | (oh[1] << 16);
+        *reinterpret_cast<uint32_t*>(p.kws + dst + i) = ol;
+        *reinterpret_cast<uint32_t*>(p.kws + dst + i + HALF) = oh;
       }
     }
 
@@ -243,27 +233,20 @@ __device__ void rope_k_and_table(const PrepParams& p, int block, int nblocks) {
       // rotated queries Q' (inputs rounded to bf16 first, as for K)
       for (int h = 0; h < p.nq; ++h) {
         const size_t o = ((size_t)t * p.nq + h) * D;
-        float xl[2], xh[2];
+        uint32_t wa, wb;
         if constexpr (FP32_IN) {
           const float2 a = *reinterpret_cast<const float2*>((const float*)p.q + o + i);
           const float2 b = *reinterpret_cast<const float2*>((const float*)p.q + o + i + HALF);
-          xl[0] = __bfloat162float(__float2bfloat16_rn(a.x));
-          xl[1] = __bfloat162float(__float2bfloat16_rn(a.y));
-          xh[0] = __bfloat162float(__float2bfloat16_rn(b.x));
-          xh[1] = __bfloat162float(__float2bfloat16_rn(b.y));
+          wa = bf16x2_rn(a.x, a.y);
+          wb = bf16x2_rn(b.x, b.y);
         } else {
-          const uint32_t wa = *reinterpret_cast<const uint32_t*>((const __nv_bfloat16*)p.q + o + i);
-          const uint32_t wb = *reinterpret_cast<const uint32_t*>((const __nv_bfloat16*)p.q + o + i + HALF);
-          xl[0] = __uint_as_float(wa << 16);
-          xl[1] = __uint_as_float(wa & 0xFFFF0000u);
-          xh[0] = __uint_as_float(wb << 16);
-          xh[1] = __uint_as_float(wb & 0xFFFF0000u);
+          wa = *reinterpret_cast<const uint32_t*>((const __nv_bfloat16*)p.q + o + i);
+          wb = *reinterpret_cast<const uint32_t*>((const __nv_bfloat16*)p.q + o + i + HALF);
         }
-        __nv_bfloat16 lo[2], hi[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) rope_pair(xl[e], xh[e], c[e], sn[e], lo[e], hi[e]);
-        *reinterpret_cast<__nv_bfloat162*>(p.qws + o + i) = __halves2bfloat162(lo[0], lo[1]);
-        *reinterpret_cast<__nv_bfloat162*>(p.qws + o + i + HALF) = __halves2bfloat162(hi[0], hi[1]);
+        uint32_t ol, oh;
+        rope_bf16x2(wa, wb, c2, s2, ol, oh);
+        *reinterpret_cast<uint32_t*>(p.qws + o + i) = ol;
+        *reinterpret_cast<uint32_t*>(p.qws + o + i + HALF) = oh;
       }
     }
     if constexpr (FP32_IN) {
