@@ -2,13 +2,16 @@
 update rules and checked against the oracle (``gqa_rope_decode``) before
 the kernel runs on a GPU:
 
-* key ranges of kps keys (whole 64-key tiles, about 256 ranges over the
+* key ranges of kps keys (whole 128-key tiles, about 256 ranges over the
   batch), one per CTA, merged by the combine kernel's rule;
-* the G heads of a KV head in rows 32 (g % 4) + g / 4 of a 128-row tile,
-  the other rows zero (they must not disturb the real rows);
-* per 64-key tile: scores masked past the range, the running max set by the
-  first tile and moved only when a score exceeds it by more than 2^8 in p
-  (O and l then rescaled), p = 2^((s - m) log2(e) / sqrt(d));
+* keys in the rows of the products: per tile S^T = K Q^T (128 keys x the G
+  heads) and O^T += V^T P^T (features x heads), so the G heads of a KV head
+  are columns and no row is padding;
+* per 128-key tile and head: scores masked past the range (selected to
+  -inf, so NaN cache rows there never count), the head's max over the
+  tile's keys, the running max set by the first tile and moved only when a
+  score exceeds it by more than 2^8 in p (O and l then rescaled),
+  p = 2^((s - m) log2(e) / sqrt(d));
 * the range's last tile fixed up in shared memory: the new token's rotated
   key and value in row pos, V rows past the range zeroed, so that the cache
   rows there (NaN in the tests) never reach a product with a nonzero weight.
@@ -20,7 +23,7 @@ import pytest
 
 import oracle.gqa_oracle as orc
 
-KT = 64
+KT = 128
 
 
 def layout(B, Lmax, nkv, target=256):
@@ -40,17 +43,14 @@ def kernel_model(q, k_new, v_new, k_cache, v_cache, lens, nq, nkv, theta):
     out = np.zeros((B, nq, d))
     lse = np.zeros((nq, B))
     kc, vc = k_cache.copy(), v_cache.copy()
+    flat_k = k_cache.reshape(-1, nkv, d)
+    flat_v = v_cache.reshape(-1, nkv, d)
     for b in range(B):
         pos = int(lens[b])
         qr = orc.apply_rope(q[b][None], [pos], theta, operand_rounding=True)[0]
         kr = orc.apply_rope(k_new[b][None], [pos], theta, operand_rounding=True)[0]
         for h in range(nkv):
-            # the 128-row query tile: head g at row 32 (g % 4) + g / 4
-            qt = np.zeros((128, d))
-            rows = [32 * (g % 4) + g // 4 for g in range(G)]
-            assert len(set(rows)) == G and max(rows) < 128
-            for g in range(G):
-                qt[rows[g]] = qr[h * G + g]
+            Q = qr[h * G:(h + 1) * G]  # [G, d]: the heads are the MMA's N
             parts = []
             for split in range(splits):
                 k0 = split * kps
@@ -59,15 +59,13 @@ def kernel_model(q, k_new, v_new, k_cache, v_cache, lens, nq, nkv, theta):
                     parts.append(None)
                     continue
                 ntiles = -(-(k1 - k0) // KT)
-                m = np.full(128, -np.inf)
-                l = np.zeros(128)
-                o = np.zeros((128, d))
+                m = np.full(G, -np.inf)
+                l = np.zeros(G)
+                oT = np.zeros((d, G))
                 for j in range(ntiles):
                     t0 = k0 + j * KT
                     idx = b * Lmax + t0 + np.arange(KT)  # rows of the cache maps (may run into b + 1)
-                    flat_k = k_cache.reshape(-1, nkv, d)
-                    flat_v = v_cache.reshape(-1, nkv, d)
-                    ok_rows = idx < flat_k.shape[0]
+                    ok_rows = idx < flat_k.shape[0]      # past the cache's end: zero fill
                     K = np.where(ok_rows[:, None], flat_k[np.minimum(idx, flat_k.shape[0] - 1), h], 0.0)
                     V = np.where(ok_rows[:, None], flat_v[np.minimum(idx, flat_v.shape[0] - 1), h], 0.0)
                     nvalid = min(KT, k1 - t0)
@@ -77,28 +75,28 @@ def kernel_model(q, k_new, v_new, k_cache, v_cache, lens, nq, nkv, theta):
                             V[pos - t0] = v_new[b, h]
                         V[nvalid:] = 0.0
                     with np.errstate(invalid="ignore"):
-                        S = qt @ K.T  # NaN in K rows past the range stays in masked columns
-                    S[:, nvalid:] = -np.inf
-                    mx = S.max(axis=1)
+                        ST = K @ Q.T  # [KT, G]; NaN in K rows past the range
+                    valid = np.arange(KT) < nvalid
+                    ST = np.where(valid[:, None], ST, -np.inf)
+                    mx = ST.max(axis=0)  # per head, over the tile's keys
                     need = mx > m + thr
                     if need.any():
                         m_new = np.where(need, mx, m)
                         if j > 0:
                             alpha = np.where(need, np.exp2((m - m_new) * sl2), 1.0)
-                            o *= alpha[:, None]
+                            oT *= alpha[None, :]
                             l *= alpha
                         m = m_new
-                    P = np.exp2(S * sl2 - (m * sl2)[:, None])
-                    l += P.sum(axis=1)
-                    o += P @ V
-                parts.append((m * sl2, l, o))
+                    PT = np.exp2(ST * sl2 - (m * sl2)[None, :])  # [KT, G]
+                    l += PT.sum(axis=0)
+                    oT += V.T @ PT
+                parts.append((m * sl2, l, oT.T))
             # combine: per head, over the ranges holding a visible key
+            used = [pt for pt in parts if pt is not None]
             for g in range(G):
-                r = rows[g]
-                used = [pt for pt in parts if pt is not None]
-                M = max(pt[0][r] for pt in used)
-                L = sum(pt[1][r] * 2.0 ** (pt[0][r] - M) for pt in used)
-                acc = sum(pt[2][r] * 2.0 ** (pt[0][r] - M) for pt in used)
+                M = max(pt[0][g] for pt in used)
+                L = sum(pt[1][g] * 2.0 ** (pt[0][g] - M) for pt in used)
+                acc = sum(pt[2][g] * 2.0 ** (pt[0][g] - M) for pt in used)
                 out[b, h * G + g] = acc / L
                 lse[h * G + g, b] = (M + math.log2(L)) * math.log(2.0)
             kc[b, pos, h] = kr[h]
@@ -122,10 +120,10 @@ def _inputs(lens, Lmax, nq, nkv, d, seed):
 
 
 @pytest.mark.parametrize("lens, Lmax, nq, nkv, d", [
-    ((0, 1, 63, 64, 65, 190), 200, 12, 4, 32),   # G = 3; an empty cache, tile edges
-    ((300, 1023, 5), 1100, 16, 2, 64),           # G = 8; several ranges per sequence
-    ((129, 400), 513, 16, 1, 32),                # G = 16
-    ((77,), 128, 4, 4, 64),                      # G = 1
+    ((0, 1, 127, 128, 129, 300), 310, 12, 4, 32),  # G = 3; an empty cache, tile edges
+    ((300, 2047, 5), 2100, 16, 2, 64),             # G = 8; several ranges per sequence
+    ((129, 400), 513, 16, 1, 32),                  # G = 16
+    ((77,), 128, 4, 4, 64),                        # G = 1
 ])
 def test_kernel_model_matches_the_oracle(lens, Lmax, nq, nkv, d):
     theta = 1e4
@@ -159,6 +157,6 @@ def test_planted_mistake_is_caught():
     lens, Lmax, nq, nkv, d = (70,), 128, 4, 2, 32
     q, kn, vn, kc, vc, L = _inputs(lens, Lmax, nq, nkv, d, seed=9)
     with np.errstate(invalid="ignore"):
-        P = np.zeros((1, KT))
-        V = vc[0, 64:128, 0]  # rows 70.. are NaN
-        assert np.isnan(P @ V).any()
+        PT = np.zeros((KT, 1))
+        V = vc[0, 0:128, 0]  # rows 70.. are NaN
+        assert np.isnan(V.T @ PT).any()

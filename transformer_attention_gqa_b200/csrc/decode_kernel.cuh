@@ -15,7 +15,7 @@
 //
 // Kernel 1 (key ranges): one CTA per (key range, KV head, sequence). It
 // rotates the G queries of the KV head at p (and the new key, in the CTA
-// whose range holds p), then walks its key range in tiles of 64 keys through
+// whose range holds p), then walks its key range in tiles of 128 keys through
 // a TMA ring: scores of the tile for the G heads, an online softmax, and the
 // weighted sum of V. It leaves (running max, sum, un-normalised output) per
 // head in the workspace.
@@ -31,7 +31,7 @@
 namespace gqa {
 
 constexpr int DEC_COMBINE_THREADS = 256;
-constexpr int DEC_KT = 64;      // keys per tile (the cache maps' box height)
+constexpr int DEC_KT = 128;     // keys per tile (the cache maps' box height)
 constexpr int DEC_GMAX = 16;    // query heads per KV head
 // The split count aims at about this many CTAs over the batch (measured:
 // fewer, longer CTAs amortise the per-CTA RoPE setup).
@@ -57,60 +57,89 @@ struct DecodeParams {
 
 // ---------------------------------------------------------------- key ranges on the tensor cores
 //
-// Both products on the tensor cores (tcgen05): the G rotated query heads of KV head
-// h fill G rows of a 128-row operand tile (the other rows are zero), so
-// S = Q K^T over a 64-key tile is one M = 128, N = 64 MMA into tensor memory
-// and O += P V one M = 128, N = d MMA with P read from tensor memory, the
-// operand forms of the prefill kernel. Head g sits at tile row
-// 32 (g % 4) + g / 4, so each of the four softmax warps (one TMEM lane
-// quadrant each) holds a share of the heads. Per CTA: one key range of one
-// (sequence, KV head), its partial (max, sum, un-normalised output) per head
-// for the combine kernel. (A CUDA-core version of this kernel, scores and
-// weighted sum on the FP32 pipes, reached 3.5 TB/s at G = 4 and 2.1 TB/s at
-// G = 8 on B200; this one 4.2 and 4.0.)
+// Keys in the rows of the products. Per 128-key tile of one (sequence, KV
+// head) key range:
+//   S^T = K Q^T    one M = 128 (keys) x N = 16 (heads) x K = d MMA,
+//                  A = the K tile as loaded (K-major), B = the G rotated
+//                  query heads in rows 0..G-1 of a 16-row tile (rows past
+//                  G zero), scores into tensor memory (lane = key);
+//   O^T += V^T P^T one M = 128 (features) x N = 16 x K = 128 (keys) MMA,
+//                  A = the V tile read feature-major (MN-major), B = the
+//                  bf16 weights P^T (row = head) that the softmax threads
+//                  write to shared memory; O^T in tensor memory
+//                  (lane = feature; for d < 128 the upper lanes repeat the
+//                  lower ones and are not read).
+// The G heads of a KV head are the N dimension, so no tensor-core row or
+// softmax thread is spent on padding: per tile the tensor core does
+// 2 * 128 * 16 * 128 multiply-adds and each softmax thread (one key) G
+// exponentials. (The previous form, heads in the rows of an M = 128 tile
+// and 64 keys in N, did 32 times the tensor work at G = 4 and ran the
+// exponentials of 128 rows, G of them real: 4.2 TB/s at G = 4.)
 //
-// Warps 0-3: RoPE of the queries and the new key, then the online softmax
-// (one row per thread; rows that hold no head compute zeros) and the partial
-// results. Warp 4: TMA of the K/V tiles through a two-stage ring, the
-// fix-up of the range's last tile (the new token's row from this CTA, rows
-// past the range zeroed in V so that their zero weights meet finite values)
-// and the appended cache row. Warp 5: tensor memory and the MMAs.
-// One CTA per SM with a four-stage ring (measured: two stages with two CTAs
-// per SM reached 2.7 TB/s, three 3.7, four to six 4.1-4.2).
+// Online softmax per head over the range's tiles: the tile's max over its
+// keys (warp shuffles, then the four warps through shared memory); the
+// running max moves only when a score exceeds it by more than 2^8 in p
+// (then O^T's column and the thread's partial sum are rescaled); the row
+// sum is kept per thread and summed over the keys at the end.
+//
+// Warps 0-3: RoPE of the queries and the new key, the softmax (one key of
+// the tile per thread), the partial results. Warp 4: TMA of the K/V tiles
+// through a ring of 192 KB, the fix-up of the range's last tile (the new
+// token's row from this CTA, rows past the range zeroed in V so that their
+// zero weights meet finite values) and the appended cache row. Warp 5:
+// tensor memory and the S^T MMAs; warp 6: the O^T MMAs. (A tcgen05.mma
+// issue or a wait blocks its thread: with one issuing thread, O^T(j) and
+// the release of tile j's stage waited for tile j + 1 to land, which cost
+// the ring a stage.)
 constexpr int DTC_KT = DEC_KT;   // keys per tile
-constexpr int DTC_STAGES = 4;
-constexpr int DTC_THREADS = 192;
+constexpr int DTC_N = DEC_GMAX;  // heads per MMA
+constexpr int DTC_THREADS = 224;
 
 template <int D_>
 struct DtcCfg {
   using A = AttnCfg<D_>;
   static constexpr int D = D_;
-  static constexpr int KV_BOX_BYTES = DTC_KT * A::ROWB;      // one box of a 64-key tile
+  static constexpr int KV_BOX_BYTES = DTC_KT * A::ROWB;      // one box (BOXC features) of a tile
   static constexpr int TILE_BYTES = A::NBOX * KV_BOX_BYTES;  // one K or V tile
-  static constexpr int OFF_Q = 0;                            // 128-row query tile
-  static constexpr int OFF_K = A::Q_BYTES;                   // [stage] K tiles
-  static constexpr int OFF_V = OFF_K + DTC_STAGES * TILE_BYTES;  // [stage] V tiles
-  static constexpr int OFF_CS = OFF_V + DTC_STAGES * TILE_BYTES;  // uint2 [D/4]: bf16x2 (cos, sin) at pos
-  static constexpr int OFF_NEW = OFF_CS + (D / 2) * 8;           // bf16 [2][D]: rotated new key, value
-  static constexpr int OFF_BAR = OFF_NEW + 2 * D * 2;
-  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;       // + barriers + alignment slack
-  static constexpr uint32_t S_COL = 0;                          // two 64-column S/P buffers
-  static constexpr uint32_t O_COL = 2 * DTC_KT;
-  static constexpr uint32_t TMEM_COLS = 256;
-  // bf16 x bf16 -> fp32, both K-major, M = 128, N = 64 keys
+  static constexpr int STAGES = 2 * 3 * 32768 / (2 * TILE_BYTES) < 8 ? 2 * 3 * 32768 / (2 * TILE_BYTES) : 8;
+  static constexpr int Q_BOX_BYTES = DTC_N * A::ROWB;        // query tile: 16 rows per box
+  static constexpr int Q_BYTES = A::NBOX * Q_BOX_BYTES;
+  static constexpr int P_BOX_BYTES = DTC_N * 128;            // P^T: 16 rows x 64 keys (128-byte swizzle)
+  static constexpr int P_BYTES = 2 * P_BOX_BYTES;            // 128 keys
+  static constexpr int OFF_K = 0;                            // [stage] K tiles
+  static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;  // [stage] V tiles
+  static constexpr int OFF_Q = OFF_V + STAGES * TILE_BYTES;
+  static constexpr int OFF_P = OFF_Q + Q_BYTES;              // [2] P^T buffers
+  static constexpr int OFF_CS = OFF_P + 2 * P_BYTES;         // uint2 [D/4]: bf16x2 (cos, sin) at pos
+  static constexpr int OFF_NEW = OFF_CS + D * 2;             // bf16 [2][D]: rotated new key, value
+  static constexpr int OFF_RED = OFF_NEW + 2 * D * 2;        // float [3][4 warps][16]: maxima x2, sums
+  static constexpr int OFF_BAR = OFF_RED + 3 * 4 * DTC_N * 4;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;    // + barriers + alignment slack
+  static constexpr uint32_t S_COL = 0;                       // two 16-column S^T buffers
+  static constexpr uint32_t O_COL = 2 * DTC_N;               // O^T
+  static constexpr uint32_t TMEM_COLS = 64;
+  // bf16 x bf16 -> fp32, M = 128, N = 16; S^T: A and B K-major; O^T: A MN-major
   static constexpr uint32_t IDESC_S =
-      (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(DTC_KT >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && TILE_BYTES % 1024 == 0, "swizzle atoms 1024-aligned");
-  static_assert(O_COL + D <= TMEM_COLS, "tensor memory budget");
+      (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(DTC_N >> 3) << 17) | ((uint32_t)(DTC_KT >> 4) << 24);
+  static constexpr uint32_t IDESC_O = IDESC_S | (1u << 15);
+  // V^T's M = 128 features span 128 / BOXC swizzle atoms; for d < 128 they
+  // all start at the same box (stride 0), so the upper lanes repeat d.
+  static constexpr uint32_t V_LBO = D == 128 ? (uint32_t)KV_BOX_BYTES : 0u;
+  static_assert(DTC_KT == 128 && DTC_N == 16, "MMA shape M = 128, N = 16");
+  static_assert(OFF_V % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_P % 1024 == 0 && TILE_BYTES % 1024 == 0,
+                "swizzle atoms 1024-aligned");
+  static_assert(O_COL + DTC_N <= TMEM_COLS, "tensor memory budget");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
 struct DtcBarriers {
-  uint64_t full[DTC_STAGES], empty[DTC_STAGES];
+  uint64_t full[8], empty[8];
   uint64_t fixed;     // the range's last tile patched in shared memory
   uint64_t q_ready;   // query tile, new key and value written (128 arrivals)
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t o_full, drain;
+  uint64_t xchg[2];   // per-head tile maxima of the four softmax warps published (by tile parity)
+  uint64_t lsum;      // per-head partial sums of the four softmax warps published
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -118,15 +147,29 @@ static_assert(sizeof(DtcBarriers) <= 256, "barrier area");
 
 __device__ __forceinline__ void dtc_softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-template <int D>
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int D, int NH>
 __global__ void __launch_bounds__(DTC_THREADS, 1)
     gqa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const DecodeParams p) {
   using C = DtcCfg<D>;
   using A = AttnCfg<D>;
   constexpr int HALF = D / 2;
+  constexpr int ST = C::STAGES;
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int G = p.G;
+  const int G = p.G;  // <= NH
+  static_assert(NH % 4 == 0 && NH <= DTC_N, "heads per thread");
   const int pos = __ldg(p.cache_seqlens + b);
   if (pos < 0 || pos >= p.Lmax) {  // the combine kernel skips this sequence too
     if (threadIdx.x == 0 && split == 0 && h == 0) atomicCAS(&g_status, 0, kStatusBadSeqlens);
@@ -142,7 +185,7 @@ __global__ void __launch_bounds__(DTC_THREADS, 1)
   const int ntiles = (k1 - k0 + DTC_KT - 1) / DTC_KT;
   const bool has_new = pos >= k0 && pos < k1;
   const int last_start = k0 + (ntiles - 1) * DTC_KT;
-  const int last_valid = k1 - last_start;  // keys of the last tile inside the range, 1..64
+  const int last_valid = k1 - last_start;  // keys of the last tile inside the range, 1..128
   const bool fix_last = has_new || last_valid < DTC_KT;
 
   extern __shared__ uint8_t dtc_smem_raw[];
@@ -154,7 +197,7 @@ __global__ void __launch_bounds__(DTC_THREADS, 1)
   auto B = [&](uint64_t& x) { return ptx::smem_u32(&x); };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < DTC_STAGES; ++s) {
+    for (int s = 0; s < ST; ++s) {
       ptx::mbar_init(B(bars->full[s]), 1);
       ptx::mbar_init(B(bars->empty[s]), 1);
     }
@@ -166,7 +209,9 @@ __global__ void __launch_bounds__(DTC_THREADS, 1)
       ptx::mbar_init(B(bars->pv_done[s]), 1);
     }
     ptx::mbar_init(B(bars->o_full), 1);
-    ptx::mbar_init(B(bars->drain), 1);
+    ptx::mbar_init(B(bars->drain), 2);  // one commit per MMA-issuing thread
+    for (int s = 0; s < 2; ++s) ptx::mbar_init(B(bars->xchg[s]), 4);
+    ptx::mbar_init(B(bars->lsum), 4);
     bars->abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -190,8 +235,10 @@ __global__ void __launch_bounds__(DTC_THREADS, 1)
     bool ok = true;
     if (lane == 0) {
       for (int t = 0; t < ntiles; ++t) {
-        const int st = t % DTC_STAGES;
-        if (!(ok = bwait_lazy(B(bars->empty[st]), ((t / DTC_STAGES) & 1) ^ 1, abort_flag))) break;
+        const int st = t % ST;
+        // (a spinning wait: the ring is three tiles deep, so a sleeping
+        // producer's late refill would stall the stream)
+        if (!(ok = bwait(B(bars->empty[st]), ((t / ST) & 1) ^ 1, abort_flag))) break;
         ptx::mbar_arrive_expect_tx(B(bars->full[st]), 2u * C::TILE_BYTES);
         if (!(p.test_drop_first_load && t == 0)) {
           for (int bx = 0; bx < A::NBOX; ++bx) {
@@ -205,12 +252,12 @@ __global__ void __launch_bounds__(DTC_THREADS, 1)
       }
     }
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    const int tl = ntiles - 1, stl = tl % DTC_STAGES;
+    const int tl = ntiles - 1, stl = tl % ST;
     if (ok && fix_last) {
       // the last tile: the new token's rotated key and value in row pos, and
       // V rows past the range zero (their weights are zero; the cache rows
       // there may hold anything)
-      ok = __all_sync(0xffffffffu, bwait(B(bars->full[stl]), (tl / DTC_STAGES) & 1, abort_flag) &&
+      ok = __all_sync(0xffffffffu, bwait(B(bars->full[stl]), (tl / ST) & 1, abort_flag) &&
                                        bwait(B(bars->q_ready), 0, abort_flag));
       if (ok) {
         uint8_t* kt = smem + C::OFF_K + stl * C::TILE_BYTES;
@@ -251,67 +298,74 @@ __global__ void __launch_bounds__(DTC_THREADS, 1)
     }
     if (!ok && lane == 0) {  // every copy issued lands before the CTA exits
       const int first = p.test_drop_first_load ? 1 : 0;
-      for (int t = first; t < first + issued; ++t)
-        drain_wait(B(bars->full[t % DTC_STAGES]), (t / DTC_STAGES) & 1);
+      for (int t = first; t < first + issued; ++t) drain_wait(B(bars->full[t % ST]), (t / ST) & 1);
     }
   } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S^T issuer
     if (lane == 0) {
       const uint64_t dq = umma_desc(sbase + C::OFF_Q, 16, A::SBO, A::UMMA_LAYOUT);
       const uint64_t dk0 = umma_desc(sbase + C::OFF_K, 16, A::SBO, A::UMMA_LAYOUT);
-      const uint64_t dv0 = umma_desc(sbase + C::OFF_V, C::KV_BOX_BYTES, A::SBO, A::UMMA_LAYOUT);
       const uint64_t stage = (uint64_t)(C::TILE_BYTES >> 4);
-      // S(j) into S buffer j & 1 once K(j) is in place and P V(j - 2), which
-      // read P from that buffer, is done
-      auto issue_s = [&](int j) -> bool {
-        const int sb = j & 1, st = j % DTC_STAGES;
-        if (j >= 2 && !bwait(B(bars->pv_done[sb]), ((j - 2) >> 1) & 1, abort_flag)) return false;
-        const bool w = (j == ntiles - 1 && fix_last) ? bwait(B(bars->fixed), 0, abort_flag)
-                                                     : bwait(B(bars->full[st]), (j / DTC_STAGES) & 1, abort_flag);
-        if (!w) return false;
+      bool ok = bwait(B(bars->q_ready), 0, abort_flag);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        const int sb = j & 1, st = j % ST;
+        // S buffer sb held S^T(j - 2): the softmax read it before releasing P^T(j - 2)
+        if (j >= 2 && !(ok = bwait(B(bars->p_full[sb]), ((j - 2) >> 1) & 1, abort_flag))) break;
+        if (!(ok = (j == ntiles - 1 && fix_last) ? bwait(B(bars->fixed), 0, abort_flag)
+                                                 : bwait(B(bars->full[st]), (j / ST) & 1, abort_flag)))
+          break;
         ptx::tc_fence_after();
         const uint64_t dk = dk0 + st * stage;
 #pragma unroll
         for (int kk = 0; kk < A::KSTEPS_S; ++kk) {
-          const uint32_t off_q = (kk / A::STEPS_PER_BOX) * A::Q_BOX_BYTES + (kk % A::STEPS_PER_BOX) * 32;
           const uint32_t off_k = (kk / A::STEPS_PER_BOX) * C::KV_BOX_BYTES + (kk % A::STEPS_PER_BOX) * 32;
-          ptx::mma_ss(tmem + C::S_COL + sb * DTC_KT, dq + (uint64_t)(off_q >> 4), dk + (uint64_t)(off_k >> 4),
+          const uint32_t off_q = (kk / A::STEPS_PER_BOX) * C::Q_BOX_BYTES + (kk % A::STEPS_PER_BOX) * 32;
+          ptx::mma_ss(tmem + C::S_COL + sb * DTC_N, dk + (uint64_t)(off_k >> 4), dq + (uint64_t)(off_q >> 4),
                       C::IDESC_S, kk > 0 ? 1u : 0u);
         }
         ptx::mma_commit(B(bars->s_full[sb]));
-        return true;
-      };
-      bool ok = bwait(B(bars->q_ready), 0, abort_flag) && issue_s(0);
+      }
+      // all tensor-core work issued here has finished before TMEM is freed
+      ptx::mma_commit(B(bars->drain));
+      drain_wait(B(bars->drain), 0);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ O^T issuer
+    if (lane == 0) {
+      const uint64_t dv0 = umma_desc(sbase + C::OFF_V, C::V_LBO, A::SBO, A::UMMA_LAYOUT);
+      const uint64_t dp0 = umma_desc(sbase + C::OFF_P, 16, 1024, 2);  // P^T: 128-byte swizzle
+      const uint64_t stage = (uint64_t)(C::TILE_BYTES >> 4);
+      bool ok = true;
       for (int j = 0; ok && j < ntiles; ++j) {
-        const int sb = j & 1, st = j % DTC_STAGES;
-        if (j + 1 < ntiles && !(ok = issue_s(j + 1))) break;
+        const int sb = j & 1, st = j % ST;
         if (!(ok = bwait(B(bars->p_full[sb]), (j >> 1) & 1, abort_flag))) break;
         ptx::tc_fence_after();
-        // O (+)= P V: 64 keys in 4 K-steps of 16, P from the S buffer's first 32 columns
+        // O^T (+)= V^T P^T: 128 keys in 8 K-steps of 16
 #pragma unroll
-        for (int kk = 0; kk < DTC_KT / 16; ++kk)
-          ptx::mma_ts(tmem + C::O_COL, tmem + C::S_COL + sb * DTC_KT + kk * 8,
-                      dv0 + st * stage + (uint64_t)((kk * 16 * A::ROWB) >> 4), A::IDESC_O,
-                      (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < DTC_KT / 16; ++kk) {
+          const uint32_t off_p = sb * C::P_BYTES + (kk / 4) * C::P_BOX_BYTES + (kk % 4) * 32;
+          ptx::mma_ss(tmem + C::O_COL, dv0 + st * stage + (uint64_t)((kk * 16 * A::ROWB) >> 4),
+                      dp0 + (uint64_t)(off_p >> 4), C::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+        }
         ptx::mma_commit(B(bars->pv_done[sb]));
+        // the stage's K was read by S^T(j), issued and finished before P^T(j) existed
         ptx::mma_commit(B(bars->empty[st]));
       }
       if (ok) ptx::mma_commit(B(bars->o_full));
-      // all tensor-core work issued here has finished before TMEM is freed
       ptx::mma_commit(B(bars->drain));
       drain_wait(B(bars->drain), 0);
     }
   } else {
     // ------------------------------------------------------------ RoPE, softmax, partial results
-    const int tid = threadIdx.x;  // 0..127 == tile row == TMEM lane
-    const int g = 4 * lane + warp;  // the head of this row (a row past G holds none)
-    const bool active = g < G;
+    const int tid = threadIdx.x;  // 0..127 == tile row (key, then feature) == TMEM lane
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     uint2* cs = reinterpret_cast<uint2*>(smem + C::OFF_CS);
     __nv_bfloat16* knew = reinterpret_cast<__nv_bfloat16*>(smem + C::OFF_NEW);
-    // zero query tile; bf16x2 (cos, sin) words of frequencies (2j, 2j + 1) at
-    // pos (float64 angle, rounded to fp32, then to bf16 as in the prefill)
-    for (int i = tid; i < A::Q_BYTES / 16; i += 128)
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);  // [3][4][16], 16-byte aligned
+    // zero query tile and both P^T buffers (rows past G stay zero); bf16x2
+    // (cos, sin) words of frequencies (2j, 2j + 1) at pos (float64 angle,
+    // rounded to fp32, then to bf16 as in the prefill)
+    for (int i = tid; i < (C::Q_BYTES + 2 * C::P_BYTES) / 16; i += 128)
       reinterpret_cast<uint4*>(smem + C::OFF_Q)[i] = make_uint4(0, 0, 0, 0);
     for (int j = tid; j < HALF / 2; j += 128) {
       float c[2], sn[2];
@@ -325,8 +379,9 @@ __global__ void __launch_bounds__(DTC_THREADS, 1)
       cs[j] = make_uint2(bf16x2_rn(c[0], c[1]), bf16x2_rn(sn[0], sn[1]));
     }
     dtc_softmax_sync();
-    // rotated queries into their tile rows, and the new key (if this range
-    // holds pos), two frequencies per item, in the prefill's bf16 rotation
+    // rotated queries into rows 0..G-1 of the query tile, and the new key (if
+    // this range holds pos), two frequencies per item, in the prefill's bf16
+    // rotation
     constexpr int NPAIR = HALF / 2;
     const int nrot = (G + (has_new ? 1 : 0)) * NPAIR;
     for (int it = tid; it < nrot; it += 128) {
@@ -338,12 +393,11 @@ __global__ void __launch_bounds__(DTC_THREADS, 1)
       rope_bf16x2(*reinterpret_cast<const uint32_t*>(src + i), *reinterpret_cast<const uint32_t*>(src + i + HALF),
                   c.x, c.y, lo, hi);
       if (hg < G) {
-        const int row = 32 * (hg % 4) + hg / 4;
         const int cl = i, chh = i + HALF;
-        *reinterpret_cast<uint32_t*>(smem + C::OFF_Q + (cl / A::BOXC) * A::Q_BOX_BYTES +
-                                     swz(row * A::ROWB + (cl % A::BOXC) * 2, A::SWZ_MASK)) = lo;
-        *reinterpret_cast<uint32_t*>(smem + C::OFF_Q + (chh / A::BOXC) * A::Q_BOX_BYTES +
-                                     swz(row * A::ROWB + (chh % A::BOXC) * 2, A::SWZ_MASK)) = hi;
+        *reinterpret_cast<uint32_t*>(smem + C::OFF_Q + (cl / A::BOXC) * C::Q_BOX_BYTES +
+                                     swz(hg * A::ROWB + (cl % A::BOXC) * 2, A::SWZ_MASK)) = lo;
+        *reinterpret_cast<uint32_t*>(smem + C::OFF_Q + (chh / A::BOXC) * C::Q_BOX_BYTES +
+                                     swz(hg * A::ROWB + (chh % A::BOXC) * 2, A::SWZ_MASK)) = hi;
       } else {
         *reinterpret_cast<uint32_t*>(knew + i) = lo;
         *reinterpret_cast<uint32_t*>(knew + i + HALF) = hi;
@@ -356,59 +410,144 @@ __global__ void __launch_bounds__(DTC_THREADS, 1)
 
     const float sl2 = p.scale_log2;
     const float thr = 8.f / sl2;  // raw-score growth that forces an O rescale (2^8 in p)
-    float m = -INFINITY, l = 0.f;
+    // NH >= G heads per thread, without branches on G: the query rows past G
+    // are zero, so those heads' scores are 0, their weights land in P^T rows
+    // and O^T columns that nothing reads, and their max never moves
+    float m[NH], l[NH];
+#pragma unroll
+    for (int g = 0; g < NH; ++g) {
+      m[g] = -INFINITY;
+      l[g] = 0.f;
+    }
+    // this thread's key in the P^T tile: box, and byte offset in row 0
+    uint8_t* const p_base = smem + C::OFF_P + (tid / 64) * C::P_BOX_BYTES;
+    const uint32_t p_col = (uint32_t)(tid % 64) * 2;
     bool ok = true;
-    uint32_t sr[DTC_KT];
-    uint32_t ob[32];  // scratch of the O rescale
+    uint32_t sv[DTC_N];
     for (int j = 0; j < ntiles; ++j) {
       const int sb = j & 1;
       ok = __all_sync(0xffffffffu, bwait(B(bars->s_full[sb]), (j >> 1) & 1, abort_flag));
       if (!ok) break;
       ptx::tc_fence_after();
-      load_s_cols<DTC_KT>(trow + C::S_COL + sb * DTC_KT, sr);
-      const int nvalid = min(DTC_KT, k1 - (k0 + j * DTC_KT));
-      if (nvalid < DTC_KT) mask_cols<DTC_KT>(sr, nvalid - 1);
-      const float mx = cols_max<DTC_KT>(sr);
-      // exponentials against the running max; it moves only when a score
-      // exceeds it by more than the threshold (the first tile sets it)
-      const bool need = mx > m + thr;
-      if (__any_sync(0xffffffffu, need)) {
-        const float m_new = need ? mx : m;
-        if (j > 0) {
-          const float alpha = need ? ptx::ex2((m - m_new) * sl2) : 1.f;
-          const int jp = j - 1;
-          ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[jp & 1]), (jp >> 1) & 1, abort_flag));
-          if (!ok) break;
-          ptx::tc_fence_after();
-          scale_o_cols<D>(trow + C::O_COL, alpha, ob);
-          l *= alpha;
-        }
-        m = m_new;
+      ptx::tmem_ld16(trow + C::S_COL + sb * DTC_N, sv);
+      ptx::tmem_wait_ld();
+      float s[NH], mx[NH];
+#pragma unroll
+      for (int g = 0; g < NH; ++g) s[g] = __uint_as_float(sv[g]);
+      if (j == ntiles - 1 && k0 + j * DTC_KT + tid >= k1) {  // keys past the range (last tile only)
+#pragma unroll
+        for (int g = 0; g < NH; ++g) s[g] = -INFINITY;
       }
-      l += exp_pack<DTC_KT, emu_period(D)>(sr, -m * sl2, sl2, nullptr);
-      ptx::tmem_st32(trow + C::S_COL + sb * DTC_KT, sr);  // P (bf16 pairs) in the buffer's first 32 columns
-      ptx::tmem_wait_st();
+      // the tile's max per head over its 128 keys: shuffles interleaved over
+      // the heads, then each warp publishes its maxima and waits (bounded)
+      // for the other three
+#pragma unroll
+      for (int g = 0; g < NH; ++g) mx[g] = s[g];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+        for (int g = 0; g < NH; ++g) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], o));
+      }
+      float4* rx = reinterpret_cast<float4*>(red + sb * 4 * DTC_N);
+      if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < NH; g += 4) rx[(warp * DTC_N + g) / 4] = make_float4(mx[g], mx[g + 1], mx[g + 2], mx[g + 3]);
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(B(bars->xchg[sb]));
+      ok = __all_sync(0xffffffffu, bwait(B(bars->xchg[sb]), (j >> 1) & 1, abort_flag));
+      if (!ok) break;
+#pragma unroll
+      for (int g = 0; g < NH; g += 4) {
+        const float4 a = rx[g / 4], b2 = rx[(DTC_N + g) / 4], c = rx[(2 * DTC_N + g) / 4], d4 = rx[(3 * DTC_N + g) / 4];
+        mx[g] = fmaxf(fmaxf(a.x, b2.x), fmaxf(c.x, d4.x));
+        mx[g + 1] = fmaxf(fmaxf(a.y, b2.y), fmaxf(c.y, d4.y));
+        mx[g + 2] = fmaxf(fmaxf(a.z, b2.z), fmaxf(c.z, d4.z));
+        mx[g + 3] = fmaxf(fmaxf(a.w, b2.w), fmaxf(c.w, d4.w));
+      }
+      // the running max moves when a head's tile max exceeds it by more than
+      // the threshold (every thread sees the same maxima: uniform branches)
+      bool need_any = false;
+      float alpha[NH];
+#pragma unroll
+      for (int g = 0; g < NH; ++g) {
+        alpha[g] = 1.f;
+        if (mx[g] > m[g] + thr) {
+          if (j > 0) {
+            alpha[g] = ptx::ex2((m[g] - mx[g]) * sl2);
+            need_any = true;
+          }
+          m[g] = mx[g];
+        }
+      }
+      if (need_any) {
+        // O^T holds the sum up to the previous tile: wait for PV(j - 1), then
+        // scale the heads' columns of this thread's feature row
+        const int jp = j - 1;
+        ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[jp & 1]), (jp >> 1) & 1, abort_flag));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        uint32_t ov[DTC_N];
+        ptx::tmem_ld16(trow + C::O_COL, ov);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int g = 0; g < NH; ++g) ov[g] = __float_as_uint(__uint_as_float(ov[g]) * alpha[g]);
+        ptx::tmem_st16(trow + C::O_COL, ov);
+        ptx::tmem_wait_st();
+#pragma unroll
+        for (int g = 0; g < NH; ++g) l[g] *= alpha[g];
+      }
+      // P^T buffer sb was read by PV(j - 2)
+      if (j >= 2) {
+        const int jq = j - 2;
+        ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[sb]), (jq >> 1) & 1, abort_flag));
+        if (!ok) break;
+      }
+      uint8_t* pt = p_base + sb * C::P_BYTES;
+#pragma unroll
+      for (int g = 0; g < NH; ++g) {
+        const float pg = ptx::ex2((s[g] - m[g]) * sl2);
+        l[g] += pg;
+        *reinterpret_cast<__nv_bfloat16*>(pt + swz(g * 128 + p_col, 7)) = __float2bfloat16_rn(pg);
+      }
+      ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       ptx::mbar_arrive(B(bars->p_full[sb]));
     }
     if (ok) ok = __all_sync(0xffffffffu, bwait(B(bars->o_full), 0, abort_flag));
     if (ok) {
       ptx::tc_fence_after();
-      float* po = p.part_o + (part * G + (active ? g : 0)) * D;
+      // partial sums per head over this range's keys
+      float* rl = red + 2 * 4 * DTC_N;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        ptx::tmem_ld32(trow + C::O_COL + c * 32, sr);
-        ptx::tmem_wait_ld();
-        ptx::reg_fence32(sr);
-        if (active) {
-          float4* dst = reinterpret_cast<float4*>(po + c * 32);
+      for (int o = 16; o > 0; o >>= 1) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(sr[4 * e]), __uint_as_float(sr[4 * e + 1]),
-                                 __uint_as_float(sr[4 * e + 2]), __uint_as_float(sr[4 * e + 3]));
-        }
+        for (int g = 0; g < NH; ++g) l[g] += __shfl_xor_sync(0xffffffffu, l[g], o);
       }
-      if (active) p.part_ml[part * G + g] = make_float2(m * sl2, l);
+      if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < NH; ++g) rl[warp * DTC_N + g] = l[g];
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(B(bars->lsum));
+      uint32_t ov[DTC_N];
+      ptx::tmem_ld16(trow + C::O_COL, ov);
+      ptx::tmem_wait_ld();
+      if (tid < D) {
+        float* po = p.part_o + part * G * D + tid;
+#pragma unroll
+        for (int g = 0; g < NH; ++g)
+          if (g < G) po[(size_t)g * D] = __uint_as_float(ov[g]);
+      }
+      ok = __all_sync(0xffffffffu, bwait(B(bars->lsum), 0, abort_flag));
+      if (ok && tid < G) {
+        float mg = 0.f;
+#pragma unroll
+        for (int g = 0; g < NH; ++g)
+          if (g == tid) mg = m[g];
+        const float lg = rl[tid] + rl[DTC_N + tid] + rl[2 * DTC_N + tid] + rl[3 * DTC_N + tid];
+        p.part_ml[part * G + tid] = make_float2(mg * sl2, lg);
+      }
     }
   }
 

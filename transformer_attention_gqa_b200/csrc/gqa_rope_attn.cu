@@ -294,10 +294,18 @@ int launch_decode(const void* q, const void* k_new, const void* v_new, void* k_c
                   const int32_t* lens, double theta, int B, int Lmax, int nq, int nkv, void* out, float* lse,
                   uint8_t* ws, const DecLayout& lay, cudaStream_t stream, int device) {
   using C = DtcCfg<D>;
+  // heads per softmax thread: G rounded up to 4, 8 or 16
+  const int G = nq / nkv;
+  void (*kern)(CUtensorMap, CUtensorMap, DecodeParams) =
+      G <= 4 ? gqa_decode_tc_kernel<D, 4> : (G <= 8 ? gqa_decode_tc_kernel<D, 8> : gqa_decode_tc_kernel<D, 16>);
   {  // caller holds g_mu
     DeviceState& ds = g_dev[device];
     if (!ds.dtc_attr_set[dim_index(D)]) {
-      if (cudaFuncSetAttribute(gqa_decode_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(gqa_decode_tc_kernel<D, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(gqa_decode_tc_kernel<D, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(gqa_decode_tc_kernel<D, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_BYTES) != cudaSuccess)
         return GQA_ERR_CUDA;
       ds.dtc_attr_set[dim_index(D)] = true;
@@ -328,7 +336,7 @@ int launch_decode(const void* q, const void* k_new, const void* v_new, void* k_c
   dp.Lmax = Lmax;
   dp.nq = nq;
   dp.nkv = nkv;
-  dp.G = nq / nkv;
+  dp.G = G;
   dp.splits = lay.splits;
   dp.kps = lay.kps;
   dp.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
@@ -339,7 +347,7 @@ int launch_decode(const void* q, const void* k_new, const void* v_new, void* k_c
   dp.test_drop_first_load = (drop && drop[0] == '1' && drop[1] == '\0') ? 1 : 0;
 
   if (t_prof_ev[0] && cudaEventRecord(t_prof_ev[0], stream) != cudaSuccess) return GQA_ERR_CUDA;
-  gqa_decode_tc_kernel<D><<<dim3(lay.splits, nkv, B), DTC_THREADS, C::SMEM_BYTES, stream>>>(tmK, tmV, dp);
+  kern<<<dim3(lay.splits, nkv, B), DTC_THREADS, C::SMEM_BYTES, stream>>>(tmK, tmV, dp);
   if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   if (t_prof_ev[1] && cudaEventRecord(t_prof_ev[1], stream) != cudaSuccess) return GQA_ERR_CUDA;
   gqa_decode_combine_kernel<<<dim3(nkv, B), DEC_COMBINE_THREADS, 0, stream>>>(dp, D);
