@@ -48,11 +48,11 @@ namespace gqa {
 
 
 // Work-item hand-off ring: the K producer takes item indices and publishes
-// them; every other role (V producer, S issuer, PV issuer: one thread each;
-// softmax warps: one arrival per warp; Q warps: their first thread, which
-// passes the index on with the tile's Q load) reads each slot once.
+// them, decoded; every other role (V producer, S issuer, PV issuer: one
+// thread each; softmax and Q warps: one arrival per warp) reads each slot
+// once.
 constexpr int ITEM_SLOTS = 8;
-constexpr int ITEM_READERS = 3 + 8 + 1;
+constexpr int ITEM_READERS = 3 + 8 + 4;
 
 // Register split (launch: 512 threads x 128): producers/MMA 56, softmax 160
 // (8 warps), Q rotation/epilogue 128 (the launch value).
@@ -61,6 +61,10 @@ constexpr int REG_SOFTMAX = 160;
 constexpr int REG_ROPE = 128;
 static_assert(REG_PRODUCER * 128 + REG_SOFTMAX * 256 + REG_ROPE * 128 <= 65536 / ATTN_THREADS * ATTN_THREADS,
               "register split exceeds the launch's register file share");
+
+struct WorkItem {
+  int seq_start, L, t0, nkv, kvh;
+};
 
 struct Barriers {
   uint64_t q_loaded[2], q_ready[2], q_empty[2];
@@ -71,7 +75,7 @@ struct Barriers {
   uint64_t xchg[2][4];  // row-max exchange of the two softmax halves: [tile parity][lane quadrant]
   uint64_t item_full[ITEM_SLOTS], item_empty[ITEM_SLOTS];
   int item[ITEM_SLOTS];  // work-item index, -1 = no more items
-  int q_item[2];         // work item whose Q is in Q buffer 0 / 1 (-1: none left)
+  WorkItem witem[ITEM_SLOTS];  // the item decoded (sequence, tile, KV head), by the publisher
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -119,10 +123,6 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (layout << 61);
 }
-
-struct WorkItem {
-  int seq_start, L, t0, nkv, kvh;
-};
 
 __device__ __forceinline__ WorkItem decode_item(const AttnParams& p, int w) {
   WorkItem it;
@@ -189,12 +189,34 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-// Work item k of this CTA from the hand-off ring (-1: none left), read by one
-// thread (take_item) or by a whole warp (take_item_warp, one arrival).
-__device__ __forceinline__ bool take_item(Barriers* bars, int k, int& w, volatile int* abort_flag) {
+__device__ __forceinline__ WorkItem load_witem(const WorkItem* src) {
+  const volatile int* v = reinterpret_cast<const volatile int*>(src);
+  WorkItem wi;
+  wi.seq_start = v[0];
+  wi.L = v[1];
+  wi.t0 = v[2];
+  wi.nkv = v[3];
+  wi.kvh = v[4];
+  return wi;
+}
+
+__device__ __forceinline__ void store_witem(WorkItem* dst, const WorkItem& wi) {
+  volatile int* v = reinterpret_cast<volatile int*>(dst);
+  v[0] = wi.seq_start;
+  v[1] = wi.L;
+  v[2] = wi.t0;
+  v[3] = wi.nkv;
+  v[4] = wi.kvh;
+}
+
+// Work item k of this CTA from the hand-off ring (-1: none left) with its
+// decoded fields, read by one thread (take_item) or by a whole warp
+// (take_item_warp, one arrival).
+__device__ __forceinline__ bool take_item(Barriers* bars, int k, int& w, WorkItem& wi, volatile int* abort_flag) {
   const int slot = k & (ITEM_SLOTS - 1);
   if (!bwait(ptx::smem_u32(&bars->item_full[slot]), (k / ITEM_SLOTS) & 1, abort_flag)) return false;
   w = *reinterpret_cast<volatile int*>(&bars->item[slot]);
+  wi = load_witem(&bars->witem[slot]);
   ptx::mbar_arrive(ptx::smem_u32(&bars->item_empty[slot]));
   return true;
 }
@@ -210,22 +232,29 @@ __device__ __forceinline__ int next_item_index(const AttnParams& p, int k) {
   return k * G + ((k & 1) ? G - 1 - b : b);
 }
 
-// Publishes work item k (index w, -1 = none left) once every reader has
-// taken item k - ITEM_SLOTS from the same slot.
-__device__ __forceinline__ bool publish_item(Barriers* bars, int k, int w, volatile int* abort_flag) {
+// Publishes work item k (index w, -1 = none left), decoded (its global
+// loads are paid here, by the producer that runs ahead, not by the roles
+// that start the item), once every reader has taken item k - ITEM_SLOTS
+// from the same slot.
+__device__ __forceinline__ bool publish_item(const AttnParams& p, Barriers* bars, int k, int w,
+                                             volatile int* abort_flag) {
   const int slot = k & (ITEM_SLOTS - 1);
+  WorkItem wi{};
+  if (w >= 0) wi = decode_item(p, w);
   if (k >= ITEM_SLOTS &&
       !bwait_lazy(ptx::smem_u32(&bars->item_empty[slot]), ((k / ITEM_SLOTS) - 1) & 1, abort_flag))
     return false;
   *reinterpret_cast<volatile int*>(&bars->item[slot]) = w;
+  store_witem(&bars->witem[slot], wi);
   ptx::mbar_arrive(ptx::smem_u32(&bars->item_full[slot]));
   return true;
 }
-__device__ __forceinline__ bool take_item_warp(Barriers* bars, int k, int& w, volatile int* abort_flag) {
+__device__ __forceinline__ bool take_item_warp(Barriers* bars, int k, int& w, WorkItem& wi, volatile int* abort_flag) {
   const int slot = k & (ITEM_SLOTS - 1);
   if (!__all_sync(0xffffffffu, bwait(ptx::smem_u32(&bars->item_full[slot]), (k / ITEM_SLOTS) & 1, abort_flag)))
     return false;
   w = *reinterpret_cast<volatile int*>(&bars->item[slot]);
+  wi = load_witem(&bars->witem[slot]);
   __syncwarp();
   if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(ptx::smem_u32(&bars->item_empty[slot]));
   return true;
@@ -398,83 +427,96 @@ __device__ __forceinline__ void scale_o_cols(uint32_t taddr, float alpha, uint32
 // Q-rotation/epilogue warpgroup; thread 0 takes the item and loads Q, and
 // the item index reaches the others with the load's barrier. Returns false
 // on abort; w_out = the item's index, or -1 when no items are left.
+// Q tile of work item `it` into Q buffer it & 1, rotated in shared memory by
+// the Q warpgroup (128 threads). Every warp takes the item from the hand-off
+// ring; thread 0 loads the tile once the buffer's previous item has finished
+// its S MMAs; each thread's first cos/sin words are loaded before the tile
+// lands and the next ones while it rotates the current ones.
 template <class C>
 __device__ __forceinline__ bool rope_q_tile(const AttnParams& p, uint8_t* smem, Barriers* bars,
                                             const CUtensorMap* tmQ, int it, int tid, volatile int* abort_flag,
-                                            int& w_out) {
+                                            int& w_out, WorkItem& wi_out) {
   constexpr int D = C::D;
   constexpr int NCH = D / 16;  // 16-byte chunks in the first half of a row
   constexpr int HALF = D / 2;
   const int qb = it & 1;
   const int G = p.G;
+  int w;
+  WorkItem wi;
+  if (!take_item_warp(bars, it, w, wi, abort_flag)) return false;
   bool issued = false;
-  if (tid == 0) {
-    int w;
-    if (take_item(bars, it, w, abort_flag) &&
-        // the buffer's previous tile has finished its S MMAs: load this tile's Q
-        bwait(ptx::smem_u32(&bars->q_empty[qb]), ((it >> 1) & 1) ^ 1, abort_flag)) {
-      const uint32_t bar = ptx::smem_u32(&bars->q_loaded[qb]);
-      *reinterpret_cast<volatile int*>(&bars->q_item[qb]) = w;
-      if (w >= 0) {
-        issued = true;
-        const WorkItem wi = decode_item(p, w);
-        ptx::mbar_arrive_expect_tx(bar, (uint32_t)(D * 2 * G * p.tq));
+  if (tid == 0 && bwait(ptx::smem_u32(&bars->q_empty[qb]), ((it >> 1) & 1) ^ 1, abort_flag)) {
+    // the buffer's previous tile has finished its S MMAs: load this tile's Q
+    const uint32_t bar = ptx::smem_u32(&bars->q_loaded[qb]);
+    if (w >= 0) {
+      issued = true;
+      ptx::mbar_arrive_expect_tx(bar, (uint32_t)(D * 2 * G * p.tq));
 #pragma unroll
-        for (int b = 0; b < C::NBOX; ++b)
-          ptx::tma_load_3d(ptx::smem_u32(smem + qb * C::Q_BYTES + b * C::Q_BOX_BYTES), tmQ, bar, b * C::BOXC,
-                           wi.kvh * G, wi.seq_start + wi.t0);
-      } else {
-        ptx::mbar_arrive(bar);
-      }
+      for (int b = 0; b < C::NBOX; ++b)
+        ptx::tma_load_3d(ptx::smem_u32(smem + qb * C::Q_BYTES + b * C::Q_BOX_BYTES), tmQ, bar, b * C::BOXC,
+                         wi.kvh * G, wi.seq_start + wi.t0);
+    } else {
+      ptx::mbar_arrive(bar);
     }
   }
+  // this thread's work: (token, 8-column chunk) pairs item = tid, tid + 128, ...
+  const int items = (w < 0 || p.q_rotated) ? 0 : p.tq * NCH;  // rotated Q tiles are used as loaded
+  auto load_tab = [&](int item, float4& cf, float4& sf) {
+    const int tt = item / NCH;
+    const int ch = item - tt * NCH;
+    if (wi.t0 + tt < wi.L) {
+      // bf16 cos and sin of frequencies ch*8 .. ch*8+7 (table_word layout)
+      const float4* tab = reinterpret_cast<const float4*>(p.table + table_word(wi.seq_start + wi.t0 + tt, HALF, ch * 8));
+      cf = ptx::ld_cg_v4f32(tab);
+      sf = ptx::ld_cg_v4f32(tab + 1);
+    }
+  };
+  float4 cf = make_float4(0.f, 0.f, 0.f, 0.f), sf = cf;
+  if (tid < items) load_tab(tid, cf, sf);
   const bool ok = __all_sync(0xffffffffu, bwait_lazy(ptx::smem_u32(&bars->q_loaded[qb]), (it >> 1) & 1, abort_flag));
   if (!ok) {  // a load issued above lands before the CTA may exit
     if (issued) drain_wait(ptx::smem_u32(&bars->q_loaded[qb]), (it >> 1) & 1);
     return false;
   }
-  const int w = *reinterpret_cast<volatile int*>(&bars->q_item[qb]);
   w_out = w;
+  wi_out = wi;
   if (w < 0) return true;
-  const WorkItem wi = decode_item(p, w);
   uint8_t* qbuf = smem + qb * C::Q_BYTES;
-  const int items = p.q_rotated ? 0 : p.tq * NCH;  // rotated Q tiles are used as loaded
   for (int item = tid; item < items; item += 128) {
+    float4 cfn = cf, sfn = sf;
+    if (item + 128 < items) load_tab(item + 128, cfn, sfn);
     const int tt = item / NCH;
     const int ch = item - tt * NCH;
-    const int tok = wi.t0 + tt;
-    if (tok >= wi.L) continue;
-    // bf16 cos and sin of frequencies ch*8 .. ch*8+7 (table_word layout)
-    const float4* tab = reinterpret_cast<const float4*>(p.table + table_word(wi.seq_start + tok, HALF, ch * 8));
-    const float4 cf = ptx::ld_cg_v4f32(tab), sf = ptx::ld_cg_v4f32(tab + 1);
-    const uint32_t cw[4] = {__float_as_uint(cf.x), __float_as_uint(cf.y), __float_as_uint(cf.z), __float_as_uint(cf.w)};
-    const uint32_t sw[4] = {__float_as_uint(sf.x), __float_as_uint(sf.y), __float_as_uint(sf.z), __float_as_uint(sf.w)};
-    const int col_lo = ch * 8, col_hi = ch * 8 + HALF;
-    const int bx_lo = col_lo / C::BOXC, bx_hi = col_hi / C::BOXC;
-    for (int hh = 0; hh < G; ++hh) {
-      const int row = tt * G + hh;
-      uint4* plo = reinterpret_cast<uint4*>(qbuf + bx_lo * C::Q_BOX_BYTES +
-                                            swz(row * C::ROWB + (col_lo % C::BOXC) * 2, C::SWZ_MASK));
-      uint4* phi = reinterpret_cast<uint4*>(qbuf + bx_hi * C::Q_BOX_BYTES +
-                                            swz(row * C::ROWB + (col_hi % C::BOXC) * 2, C::SWZ_MASK));
-      uint4 vlo = *plo, vhi = *phi;
-      rope_bf16x2(vlo.x, vhi.x, cw[0], sw[0], vlo.x, vhi.x);
-      rope_bf16x2(vlo.y, vhi.y, cw[1], sw[1], vlo.y, vhi.y);
-      rope_bf16x2(vlo.z, vhi.z, cw[2], sw[2], vlo.z, vhi.z);
-      rope_bf16x2(vlo.w, vhi.w, cw[3], sw[3], vlo.w, vhi.w);
-      *plo = vlo;
-      *phi = vhi;
+    if (wi.t0 + tt < wi.L) {
+      const uint32_t cw[4] = {__float_as_uint(cf.x), __float_as_uint(cf.y), __float_as_uint(cf.z),
+                              __float_as_uint(cf.w)};
+      const uint32_t sw[4] = {__float_as_uint(sf.x), __float_as_uint(sf.y), __float_as_uint(sf.z),
+                              __float_as_uint(sf.w)};
+      const int col_lo = ch * 8, col_hi = ch * 8 + HALF;
+      const int bx_lo = col_lo / C::BOXC, bx_hi = col_hi / C::BOXC;
+      for (int hh = 0; hh < G; ++hh) {
+        const int row = tt * G + hh;
+        uint4* plo = reinterpret_cast<uint4*>(qbuf + bx_lo * C::Q_BOX_BYTES +
+                                              swz(row * C::ROWB + (col_lo % C::BOXC) * 2, C::SWZ_MASK));
+        uint4* phi = reinterpret_cast<uint4*>(qbuf + bx_hi * C::Q_BOX_BYTES +
+                                              swz(row * C::ROWB + (col_hi % C::BOXC) * 2, C::SWZ_MASK));
+        uint4 vlo = *plo, vhi = *phi;
+        rope_bf16x2(vlo.x, vhi.x, cw[0], sw[0], vlo.x, vhi.x);
+        rope_bf16x2(vlo.y, vhi.y, cw[1], sw[1], vlo.y, vhi.y);
+        rope_bf16x2(vlo.z, vhi.z, cw[2], sw[2], vlo.z, vhi.z);
+        rope_bf16x2(vlo.w, vhi.w, cw[3], sw[3], vlo.w, vhi.w);
+        *plo = vlo;
+        *phi = vhi;
+      }
     }
+    cf = cfn;
+    sf = sfn;
   }
   ptx::fence_proxy_async_smem();
   ptx::mbar_arrive(ptx::smem_u32(&bars->q_ready[qb]));
   return true;
 }
 
-// Epilogue of work item `wi` (the CTA's it-th): out = O / l (bf16 or fp32),
-// lse = (m log2e/sqrt(d) + log2 l) ln 2. One thread per row (TMEM lane),
-// 16-byte stores of the row. (Staging the tile in shared memory for a TMA
-// store was measured slower: this runs off the softmax's critical path.)
 template <class C, bool OUT_FP32>
 __device__ __forceinline__ bool epilogue_tile(const AttnParams& p, const WorkItem& wi, uint8_t* smem, Barriers* bars,
                                               uint32_t tmem, int it, uint32_t g, int tid,
@@ -647,10 +689,10 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       bool ok = true;
       int w = (int)blockIdx.x < n_items ? (int)blockIdx.x : -1;  // first item of CTA b: item b
       int nxt = w >= 0 ? next_item_index(p, 1) : n_items;
-      ok = publish_item(bars, 0, w, abort_flag);
+      ok = publish_item(p, bars, 0, w, abort_flag);
       for (int k = 0; ok && w >= 0; ++k) {
         const int wn = nxt < n_items ? nxt : -1;
-        if (!(ok = publish_item(bars, k + 1, wn, abort_flag))) break;
+        if (!(ok = publish_item(p, bars, k + 1, wn, abort_flag))) break;
         if (wn >= 0) nxt = next_item_index(p, k + 2);
         const WorkItem wi = decode_item(p, w);
         for (int j = 0; j < wi.nkv; ++j, ++g) {
@@ -682,8 +724,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       bool ok = true;
       for (int k = 0; ok; ++k) {
         int w;
-        if (!(ok = take_item(bars, k, w, abort_flag)) || w < 0) break;
-        const WorkItem wi = decode_item(p, w);
+        WorkItem wi;
+        if (!(ok = take_item(bars, k, w, wi, abort_flag)) || w < 0) break;
         for (int j = 0; j < wi.nkv; ++j, ++g) {
           const int vs = g % C::VST;
           if (!(ok = bwait_lazy(B(bars->v_empty[vs]), ((g / C::VST) & 1) ^ 1, abort_flag))) break;
@@ -717,8 +759,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       bool ok = true;
       for (; ok; ++it) {
         int w;
-        if (!(ok = take_item(bars, it, w, abort_flag)) || w < 0) break;
-        const WorkItem wi = decode_item(p, w);
+        WorkItem wi;
+        if (!(ok = take_item(bars, it, w, wi, abort_flag)) || w < 0) break;
         const int qb = it & 1;
         if (!(ok = bwait(bar_qr0 + 8 * qb, (it >> 1) & 1, abort_flag))) break;
         const uint64_t dq = dq_base + (uint64_t)((qb * C::Q_BYTES) >> 4);
@@ -749,8 +791,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       bool ok = true;
       for (; ok; ++it) {
         int w;
-        if (!(ok = take_item(bars, it, w, abort_flag)) || w < 0) break;
-        const WorkItem wi = decode_item(p, w);
+        WorkItem wi;
+        if (!(ok = take_item(bars, it, w, wi, abort_flag)) || w < 0) break;
         for (int j = 0; j < wi.nkv; ++j, ++g) {
           const int b = g % NUM_S_BUF, vs = g % C::VST;
           if (!(ok = bwait(bar_vf0 + 8 * vs, (g / C::VST) & 1, abort_flag))) break;
@@ -785,8 +827,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     uint32_t sr[NC];
     for (; ok; ++it) {
       int w;
-      if (!(ok = take_item_warp(bars, it, w, abort_flag)) || w < 0) break;
-      const WorkItem wi = decode_item(p, w);
+      WorkItem wi;
+      if (!(ok = take_item_warp(bars, it, w, wi, abort_flag)) || w < 0) break;
       const int tok = wi.t0 + tok_off;  // index inside the sequence
       const int last_key = p.causal ? tok : wi.L - 1;
       float m = -INFINITY;
@@ -887,16 +929,18 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     // next tile's Q is rotated while tile t still runs; the epilogue of t
     // runs once its last P.V is done.
     int w;
-    bool ok = rope_q_tile<C>(p, smem, bars, &tmQ, 0, tid, abort_flag, w);
+    WorkItem wi{};
+    bool ok = rope_q_tile<C>(p, smem, bars, &tmQ, 0, tid, abort_flag, w, wi);
     int it = 0;
     uint32_t g = 0;
     while (ok && w >= 0) {
       int wn;
-      if (!(ok = rope_q_tile<C>(p, smem, bars, &tmQ, it + 1, tid, abort_flag, wn))) break;
-      const WorkItem wi = decode_item(p, w);
+      WorkItem win{};
+      if (!(ok = rope_q_tile<C>(p, smem, bars, &tmQ, it + 1, tid, abort_flag, wn, win))) break;
       ok = epilogue_tile<C, OUT_FP32>(p, wi, smem, bars, tmem, it, g, tid, abort_flag);
       g += wi.nkv;
       w = wn;
+      wi = win;
       ++it;
     }
   }
