@@ -1,12 +1,21 @@
-"""The backward kernel's work decomposition, restated in numpy and checked
-against the oracle's backward in float64 (no rounding): one work item per
-(sequence, 128-key tile, KV head); each item visits the packed query tiles
-(tq = 128 / G tokens x G heads) from floor(k0 / tq) (causal) or 0 to the
-sequence's last; a key row j sees packed column r iff r >= (k0 + j - t0) * G
-(causal) and k0 + j < L; rows past the sequence and padding rows carry
-lse = +inf and Delta = 0; dV and dK' accumulate per item, dQ' accumulates
-across items. This pins the index arithmetic of csrc/bwd_kernel.cuh on the
-CPU (the products themselves run on tensor cores there). CPU only."""
+"""The backward kernels' work decomposition, restated in numpy and checked
+against the oracle's backward in float64 (no rounding).
+
+dK' and dV (csrc/bwd_kernel.cuh): one work item per (sequence, 128-key tile,
+KV head); each item visits the packed query tiles (tq = 128 / G tokens x G
+heads) from floor(k0 / tq) (causal) or 0 to the sequence's last; a key row j
+sees packed column r iff r >= (k0 + j - t0) * G (causal) and k0 + j < L;
+rows past the sequence and padding rows carry lse = +inf and Delta = 0; dV
+and dK' accumulate per item.
+
+dQ' (csrc/bwd_q_kernel.cuh): one work item per (sequence, query tile, KV
+head); each item visits the key tiles below ceil(t_end / 128), t_end =
+min(t0 + tq, L) (causal) or L; packed row r sees key c of tile j iff
+j * 128 + c <= t0 + r / G (causal) or < L; dQ' is summed over the item's
+key tiles and written once per valid row.
+
+This pins the index arithmetic on the CPU (the products themselves run on
+tensor cores there). CPU only."""
 import numpy as np
 import pytest
 
@@ -65,12 +74,42 @@ def decomposed_backward(q, k, v, dout, cu, nq, nkv, theta, causal):
                     dST = PT * ((Vt @ dOt.T) - st_d[None, :])
                     dVt += PT @ dOt
                     dKt += dST @ Qt
-                    dQt = dST.T @ Kt
-                    for r in np.nonzero(valid)[0]:
-                        dq_acc[seq_start + t0 + tt[r], heads[r]] += dQt[r]
                 ok = key_in_seq < L
                 dv[keys[ok], kvh] = dVt[ok]
                 dk[keys[ok], kvh] = dKt[ok] / np.sqrt(d)
+    # dQ': query-tile items, the forward's packing
+    written = np.zeros(q.shape[:2], dtype=int)
+    for s in range(len(cu) - 1):
+        seq_start, L = int(cu[s]), int(cu[s + 1] - cu[s])
+        for l in range((L + tq - 1) // tq):
+            t0 = l * tq
+            t_end = min(t0 + tq, L) if causal else L
+            nkt = (t_end + BN - 1) // BN
+            toks = seq_start + t0 + tt
+            loaded = (r_idx < rows) & (toks < N)
+            valid = (r_idx < rows) & (t0 + tt < L)
+            tc = np.minimum(toks, N - 1)
+            last_key = (t0 + tt) if causal else np.full(BM, L - 1)
+            for kvh in range(nkv):
+                heads = kvh * G + hin
+                Qt = np.where(loaded[:, None], qr[tc, heads], 0.0)
+                dOt = np.where(loaded[:, None], dout[tc, heads], 0.0)
+                st_l2 = np.where(valid, lse2[heads, tc], np.inf)
+                st_d = np.where(valid, delta[heads, tc], 0.0)
+                dQt = np.zeros((BM, d))
+                for j in range(nkt):
+                    keys = seq_start + j * BN + np.arange(BN)
+                    in_n = keys < N
+                    Kt = np.where(in_n[:, None], kr[np.minimum(keys, N - 1), kvh], 0.0)
+                    Vt = np.where(in_n[:, None], v[np.minimum(keys, N - 1), kvh], 0.0)
+                    visible = (j * BN + np.arange(BN))[None, :] <= last_key[:, None]
+                    P = np.where(visible, np.exp2((Qt @ Kt.T) * sl2 - st_l2[:, None]), 0.0)
+                    dS = P * ((dOt @ Vt.T) - st_d[:, None])
+                    dQt += dS @ Kt
+                for r in np.nonzero(valid)[0]:
+                    dq_acc[seq_start + t0 + tt[r], heads[r]] = dQt[r]
+                    written[seq_start + t0 + tt[r], heads[r]] += 1
+    assert np.all(written == 1)  # every (token, head) row written exactly once
     return (orc.rope_backward(dq_acc / np.sqrt(d), pos, theta), orc.rope_backward(dk, pos, theta), dv)
 
 

@@ -12,39 +12,38 @@
 // The rotated operands Q', K' are the forward's, rounded to bf16 exactly as
 // the forward rounds them; the rounding passes gradients straight through.
 //
-// Three launches:
-//  * gqa_bwd_prep_kernel: the (sequence, key-tile) schedule, longest first;
-//    each token's (cos, sin) row; K' head-major and Q' [N, n_q, d] in the
-//    workspace; Delta and lse * log2(e) per (head, token); dQ' accumulator
-//    zeroed.
-//  * gqa_attn_bwd_kernel: one CTA per (KV head, 128-key tile). It loops over
-//    the packed query tiles (tq tokens x G heads = 128 rows, the forward's
-//    packing) that the causal mask lets see its keys. Per query tile, five
-//    tensor-core products:
+// Four launches:
+//  * gqa_bwd_prep_kernel: the (sequence, key-tile) schedule and the
+//    (sequence, query-tile) schedule, longest first; each token's (cos, sin)
+//    row; K' head-major and Q' [N, n_q, d] in the workspace; Delta and
+//    lse * log2(e) per (head, token).
+//  * gqa_attn_bwd_kernel: dK' and dV, one CTA per (KV head, 128-key tile).
+//    It loops over the packed query tiles (tq tokens x G heads = 128 rows,
+//    the forward's packing) that the causal mask lets see its keys. Per
+//    query tile, four tensor-core products:
 //        S^T  = K' Q'^T   (M = keys, N = packed q rows, K = d)  SS
 //        dP^T = V dO^T    (M = keys, N = packed q rows, K = d)  SS
 //        dV  += P^T dO    (A = P^T from TMEM, bf16)             TS
 //        dK' += dS^T Q'   (A = dS^T from shared memory)         SS
-//        dQ'  = dS K'     (A = dS: the same shared bytes, read MN-major)  SS
 //    P^T and dS^T are formed by one thread per key row (a TMEM lane); dV
-//    and dK' stay in TMEM over the whole loop and are written once; the dQ'
-//    tile of each query tile is added into an fp32 accumulator with vector
-//    atomics (several key tiles contribute to one query tile).
+//    and dK' stay in TMEM over the whole loop and are written once.
+//  * gqa_attn_bwd_q_kernel (bwd_q_kernel.cuh): dQ' = dS K', one CTA per
+//    (query tile, KV head), summed over its key tiles in TMEM and written
+//    once (P and dP recomputed there).
 //  * gqa_bwd_dq_kernel: dq = rope^T(dQ' / sqrt(d)) -> bf16.
 //
-// Warp roles of the attention-backward kernel (512 threads):
+// Warp roles of the key-tile kernel (512 threads):
 //   warp 0      TMA: K', V once; Q', dO per query tile (two stages each);
 //               lse * log2(e) and Delta of the tile's 128 rows into shared
 //               memory (all 32 lanes)
 //   warp 1      TMEM allocator; one thread issues every MMA
 //   warps 4-11  P^T and dS^T, one key row per thread: warps 4-7 the packed
 //               query columns [0, 64), warps 8-11 [64, 128)
-//   warps 12-15 dQ' tile -> fp32 atomics; at the end dV and dK' -> bf16
+//   warps 12-15 at the end dV and dK' -> bf16
 // Tensor memory (512 columns): [0,128) S^T, then P^T (bf16 pairs: packed
 // columns [0, 64) over S columns [0, 32), [64, 128) over [64, 96), so each
-// warpgroup overwrites only S columns it has read); [128,256) dP^T, then the
-// dQ' tile; [256, 256+d) dV;
-// [256+d, 256+2d) dK'.
+// warpgroup overwrites only S columns it has read); [128,256) dP^T;
+// [256, 256+d) dV; [256+d, 256+2d) dK'.
 #pragma once
 
 #include "attn_kernel.cuh"
@@ -76,9 +75,12 @@ struct BwdWsLayout {
   size_t qws;      // bf16[N][n_q][d]: Q'
   size_t lse2;     // float[n_q][N]: lse * log2(e)
   size_t delta;    // float[n_q][N]: Delta
-  size_t dq_acc;   // float[N][n_q][d]: dQ' accumulator
+  size_t dq_acc;   // float[N][n_q][d]: dQ' (written once per row by the query-tile kernel)
+  size_t qheader;  // int[16]: [0] number of (sequence, query tile) pairs
+  size_t qseq_pfx; // int[num_seqs + 1]
+  size_t qpairs;   // int2[max_qpairs]: (sequence, query tile), decreasing cost
   size_t total;
-  long long max_pairs;
+  long long max_pairs, max_qpairs;
 };
 
 __host__ inline BwdWsLayout bwd_ws_layout(int num_seqs, int N, int nq, int nkv, int d) {
@@ -99,6 +101,11 @@ __host__ inline BwdWsLayout bwd_ws_layout(int num_seqs, int N, int nq, int nkv, 
   w.lse2 = take((size_t)nq * N * 4);
   w.delta = take((size_t)nq * N * 4);
   w.dq_acc = take((size_t)N * nq * d * 4);
+  const int tq = tokens_per_tile(nq / nkv);
+  w.max_qpairs = (long long)(N + tq - 1) / tq + num_seqs;
+  w.qheader = take(16 * sizeof(int));
+  w.qseq_pfx = take((size_t)(num_seqs + 1) * sizeof(int));
+  w.qpairs = take((size_t)w.max_qpairs * 8);
   w.total = off;
   return w;
 }
@@ -121,7 +128,9 @@ struct BwdPrepParams {
   __nv_bfloat16* qws;
   float* lse2;
   float* delta;
-  float* dq_acc;
+  int* qheader;
+  int* qseq_pfx;
+  int2* qpairs;
 };
 
 struct BwdParams {
@@ -131,7 +140,6 @@ struct BwdParams {
   const float2* table;
   const float* lse2;
   const float* delta;
-  float* dq_acc;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int N, nq, nkv, G, tq, causal;
@@ -311,13 +319,24 @@ __global__ void __launch_bounds__(PREP_THREADS) gqa_bwd_prep_kernel(const BwdPre
     build_kv_schedule(p);
     return;
   }
-  const int b = blockIdx.x - 1, nb = gridDim.x - 1;
+  if (blockIdx.x == 1) {
+    // the query-tile schedule of gqa_attn_bwd_q_kernel: the forward's (sequence,
+    // q-tile) pairs, longest first
+    PrepParams q{};
+    q.cu = p.cu;
+    q.N = p.N;
+    q.num_seqs = p.num_seqs;
+    q.tq = p.tq;
+    q.causal = p.causal;
+    q.header = p.qheader;
+    q.seq_pfx = p.qseq_pfx;
+    q.pairs = p.qpairs;
+    build_schedule(q);
+    return;
+  }
+  const int b = blockIdx.x - 2, nb = gridDim.x - 2;
   bwd_rope_rows<D>(p, b, nb);
   bwd_delta_rows<D>(p, b, nb);
-  const long long n4 = (long long)p.N * p.nq * (D / 4);
-  float4* z = reinterpret_cast<float4*>(p.dq_acc);
-  for (long long i = (long long)b * PREP_THREADS + threadIdx.x; i < n4; i += (long long)nb * PREP_THREADS)
-    z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // ------------------------------------------------------------------ main kernel
@@ -358,7 +377,6 @@ struct BwdCfg {
                                        ((uint32_t)(BM >> 4) << 24);  // N = 128, A and B K-major
   static constexpr uint32_t IDESC_D = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                                       ((uint32_t)(D >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);  // N = d, B MN-major
-  static constexpr uint32_t IDESC_DQ = IDESC_D | (1u << 15);  // A MN-major too
   __host__ __device__ static constexpr int ds_off(int stage) {
     return DS_IN_DO ? OFF_DO + stage * TILE_BYTES : OFF_DS;
   }
@@ -378,7 +396,7 @@ struct BwdBarriers {
   uint64_t kv_full;
   uint64_t q_full[2], do_full[2], st_full[2];
   uint64_t q_empty[2], do_empty[2], st_empty[2];
-  uint64_t s_full, dp_full, p_full, dv_done, ds_full, dq_full, dq_free, acc_done, drain;
+  uint64_t s_full, dp_full, p_full, dv_done, ds_full, acc_done, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -433,16 +451,6 @@ __device__ __forceinline__ void bwd_mma_dk(uint32_t d_tmem, uint64_t da, uint64_
   }
 }
 
-// dQ' = dS K': A = dS, the dS^T bytes read MN-major (16 keys = 16 rows of
-// 128 bytes per step), B = K' (MN-major).
-template <class C>
-__device__ __forceinline__ void bwd_mma_dq(uint32_t d_tmem, uint64_t da, uint64_t db) {
-#pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk)
-    ptx::mma_ss(d_tmem, da + (uint64_t)((kk * 16 * 128) >> 4), db + (uint64_t)((kk * 16 * C::ROWB) >> 4),
-                C::IDESC_DQ, kk > 0 ? 1u : 0u);
-}
-
 template <int D>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     gqa_attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -482,8 +490,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     ptx::mbar_init(B(bars->p_full), 256);
     ptx::mbar_init(B(bars->dv_done), 1);
     ptx::mbar_init(B(bars->ds_full), 256);
-    ptx::mbar_init(B(bars->dq_full), 1);
-    ptx::mbar_init(B(bars->dq_free), 128);
     ptx::mbar_init(B(bars->acc_done), 1);
     ptx::mbar_init(B(bars->drain), 1);
     bars->abort_flag = 0;
@@ -600,14 +606,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     if (lane == 0) {
       const uint64_t dK_a = umma_desc(sbase + C::OFF_K, 16, C::SBO, C::UMMA_LAYOUT);
       const uint64_t dV_a = umma_desc(sbase + C::OFF_V, 16, C::SBO, C::UMMA_LAYOUT);
-      const uint64_t dK_mn = umma_desc(sbase + C::OFF_K, C::TILE_BOX_BYTES, C::SBO, C::UMMA_LAYOUT);
       const uint64_t dQ_k0 = umma_desc(sbase + C::OFF_Q, 16, C::SBO, C::UMMA_LAYOUT);
       const uint64_t dQ_mn0 = umma_desc(sbase + C::OFF_Q, C::TILE_BOX_BYTES, C::SBO, C::UMMA_LAYOUT);
       const uint64_t dO_k0 = umma_desc(sbase + C::OFF_DO, 16, C::SBO, C::UMMA_LAYOUT);
       const uint64_t dO_mn0 = umma_desc(sbase + C::OFF_DO, C::TILE_BOX_BYTES, C::SBO, C::UMMA_LAYOUT);
       const uint64_t stage_step = (uint64_t)(C::TILE_BYTES >> 4);
       auto dS_k = [&](int s) { return umma_desc(sbase + C::ds_off(s), 16, 1024, 2); };
-      auto dS_mn = [&](int s) { return umma_desc(sbase + C::ds_off(s), C::DS_BOX_BYTES, 1024, 2); };
       bool ok = bwait(B(bars->kv_full), 0, abort_flag);
       if (ok && (ok = bwait(B(bars->q_full[0]), 0, abort_flag))) {
         ptx::tc_fence_after();
@@ -638,13 +642,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         if (!(ok = bwait(B(bars->ds_full), ph, abort_flag))) break;
         ptx::tc_fence_after();
         bwd_mma_dk<C>(tmem + C::DK_COL, dS_k(s), dQ_mn0 + s * stage_step, i > 0);
-        bwd_mma_dq<C>(tmem + C::DP_COL, dS_mn(s), dK_mn);
-        ptx::mma_commit(B(bars->dq_full));
         ptx::mma_commit(B(bars->q_empty[s]));
         ptx::mma_commit(B(bars->do_empty[s]));
         if (more) {
+          // dS(i) is formed: the softmax threads have read dP(i), its columns are free
           if (!(ok = bwait(B(bars->do_full[s ^ 1]), nph, abort_flag))) break;
-          if (!(ok = bwait(B(bars->dq_free), ph, abort_flag))) break;
           ptx::tc_fence_after();
           bwd_mma_rows<C>(tmem + C::DP_COL, dV_a, dO_k0 + (s ^ 1) * stage_step);
           ptx::mma_commit(B(bars->dp_full));
@@ -713,36 +715,41 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 
       ok = __all_sync(0xffffffffu, bwait(B(bars->dp_full), ph, abort_flag));
       if (!ok) break;
-      if (C::DS_IN_DO) {  // dS(i) overwrites dO(i): dV(i) must have read it
-        ok = __all_sync(0xffffffffu, bwait(B(bars->dv_done), ph, abort_flag));
-        if (!ok) break;
-      }
       ptx::tc_fence_after();
-      uint8_t* ds = smem + C::ds_off(s);
+      // dS^T of this half row into registers first (bf16 pairs), then, once
+      // its shared-memory destination is free, stored
+      uint32_t dw[HC / 2];
 #pragma unroll
       for (int cc = 0; cc < HC / 32; ++cc) {
         const int c = c_lo + cc;
         ptx::tmem_ld32(trow + C::DP_COL + c * 32, v);
         ptx::tmem_wait_ld();
         ptx::reg_fence32(v);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int col = c * 32 + e;
+          const uint32_t pp = pw[(cc * 32 + e) >> 1];
+          const float d0 = __uint_as_float(pp << 16) * (__uint_as_float(v[e]) - st[BM + col]);
+          const float d1 = __uint_as_float(pp & 0xFFFF0000u) * (__uint_as_float(v[e + 1]) - st[BM + col + 1]);
+          dw[(cc * 32 + e) >> 1] = pack_bf16x2(d0, d1);
+        }
+      }
+      if (C::DS_IN_DO) {  // dS(i) overwrites dO(i): dV(i) must have read it
+        ok = __all_sync(0xffffffffu, bwait(B(bars->dv_done), ph, abort_flag));
+        if (!ok) break;
+      }
+      uint8_t* ds = smem + C::ds_off(s);
+#pragma unroll
+      for (int cc = 0; cc < HC / 32; ++cc) {
+        const int c = c_lo + cc;
         // columns [32c, 32c + 32) of row j: box c / 2, 16-byte chunks 4 (c & 1) .. + 3
         uint8_t* box = ds + (c >> 1) * C::DS_BOX_BYTES;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t dw[4];
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            const int ce = q4 * 8 + e;  // column inside the chunk of 32
-            const int col = c * 32 + ce;
-            const uint32_t pp = pw[(cc * 32 + ce) >> 1];
-            const float p0 = __uint_as_float(pp << 16);
-            const float p1 = __uint_as_float(pp & 0xFFFF0000u);
-            const float d0 = p0 * (__uint_as_float(v[ce]) - st[BM + col]);
-            const float d1 = p1 * (__uint_as_float(v[ce + 1]) - st[BM + col + 1]);
-            dw[e >> 1] = pack_bf16x2(d0, d1);
-          }
+          const int w0 = (cc * 32 + q4 * 8) >> 1;
           const int ch = (c & 1) * 4 + q4;
-          *reinterpret_cast<uint4*>(box + swz(j * 128 + ch * 16, 7)) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+          *reinterpret_cast<uint4*>(box + swz(j * 128 + ch * 16, 7)) =
+              make_uint4(dw[w0], dw[w0 + 1], dw[w0 + 2], dw[w0 + 3]);
         }
       }
       ptx::fence_proxy_async_smem();
@@ -753,40 +760,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     }
   } else {
     ptx::setmaxnreg_inc<BWD_REG_READOUT>();
-    // ------------------------------------------------------------ dQ' tiles; dV, dK' at the end
+    // ------------------------------------------------------------ dV, dK' at the end
     const int quad = warp - 12;
-    const int r = quad * 32 + lane;  // packed q row (dQ' tile) or key row (dV, dK') == TMEM lane
+    const int r = quad * 32 + lane;  // key row (dV, dK') == TMEM lane
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    const int tt = r / G;
-    const int hin = r - tt * G;
     bool ok = true;
     uint32_t v[32];
-    for (int i = 0; i < it.nt; ++i) {
-      const int tok = (it.qi0 + i) * tq + tt;
-      const bool valid = r < rows && tok < it.L;
-      ok = __all_sync(0xffffffffu, bwait(B(bars->dq_full), i & 1, abort_flag));
-      if (!ok) break;
-      ptx::tc_fence_after();
-      float* dst = valid ? p.dq_acc + ((size_t)(it.seq_start + tok) * p.nq + it.kvh * G + hin) * D : nullptr;
-      // the whole dQ' row into registers first, so that the next dP may
-      // overwrite these columns before the atomics are issued
-      uint32_t dqr[D];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(trow + C::DP_COL + c * 32, dqr + c * 32);
-      ptx::tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) ptx::reg_fence32(dqr + c * 32);
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(B(bars->dq_free));
-      if (valid) {
-#pragma unroll
-        for (int e = 0; e < D / 4; ++e)
-          atomicAdd(reinterpret_cast<float4*>(dst) + e,
-                    make_float4(__uint_as_float(dqr[4 * e]), __uint_as_float(dqr[4 * e + 1]),
-                                __uint_as_float(dqr[4 * e + 2]), __uint_as_float(dqr[4 * e + 3])));
-      }
-    }
-    if (ok) ok = __all_sync(0xffffffffu, bwait(B(bars->acc_done), 0, abort_flag));
+    // (a sleeping wait: these warps idle for the whole loop and share their
+    // schedulers with the P^T/dS^T warps)
+    if (ok) ok = __all_sync(0xffffffffu, bwait_lazy(B(bars->acc_done), 0, abort_flag));
     if (ok) {
       ptx::tc_fence_after();
       const int key = it.k0 + r;

@@ -17,6 +17,7 @@
 #include "../../include/gqa_rope_attn.h"
 #include "attn_kernel.cuh"
 #include "bwd_kernel.cuh"
+#include "bwd_q_kernel.cuh"
 #include "common.cuh"
 #include "decode_kernel.cuh"
 #include "masked_kernel.cuh"
@@ -371,7 +372,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
     DeviceState& ds = g_dev[device];
     if (!ds.bwd_attr_set[dim_index(D)]) {
       if (cudaFuncSetAttribute(gqa_attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               C::SMEM_BYTES) != cudaSuccess)
+                               C::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(gqa_attn_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdQCfg<D>::SMEM_BYTES) != cudaSuccess)
         return GQA_ERR_CUDA;
       ds.bwd_attr_set[dim_index(D)] = true;
     }
@@ -399,7 +402,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   pp.qws = reinterpret_cast<__nv_bfloat16*>(ws + lay.qws);
   pp.lse2 = reinterpret_cast<float*>(ws + lay.lse2);
   pp.delta = reinterpret_cast<float*>(ws + lay.delta);
-  pp.dq_acc = reinterpret_cast<float*>(ws + lay.dq_acc);
+  pp.qheader = reinterpret_cast<int*>(ws + lay.qheader);
+  pp.qseq_pfx = reinterpret_cast<int*>(ws + lay.qseq_pfx);
+  pp.qpairs = reinterpret_cast<int2*>(ws + lay.qpairs);
+  float* const dq_acc = reinterpret_cast<float*>(ws + lay.dq_acc);
 
   // Q' and dO: [N][nq][d], box (BOXC, G heads, tq tokens); K': [nkv][N][d],
   // box (BOXC, BN keys, 1); V: [N][nkv][d], box (BOXC, 1, BN keys).
@@ -430,7 +436,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   if (nb > cap) nb = cap;
   if (nb < 1) nb = 1;
   if (t_prof_ev[0] && cudaEventRecord(t_prof_ev[0], stream) != cudaSuccess) return GQA_ERR_CUDA;
-  gqa_bwd_prep_kernel<D><<<(unsigned)(nb + 1), PREP_THREADS, 0, stream>>>(pp);
+  gqa_bwd_prep_kernel<D><<<(unsigned)(nb + 2), PREP_THREADS, 0, stream>>>(pp);
   if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   if (t_prof_ev[1] && cudaEventRecord(t_prof_ev[1], stream) != cudaSuccess) return GQA_ERR_CUDA;
 
@@ -441,7 +447,6 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   bp.table = pp.table;
   bp.lse2 = pp.lse2;
   bp.delta = pp.delta;
-  bp.dq_acc = pp.dq_acc;
   bp.dk = reinterpret_cast<__nv_bfloat16*>(dk);
   bp.dv = reinterpret_cast<__nv_bfloat16*>(dv);
   bp.N = N;
@@ -457,17 +462,35 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   const unsigned grid = (unsigned)(lay.max_pairs * (long long)nkv);
   gqa_attn_bwd_kernel<D><<<grid, BWD_THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmDO, bp);
   if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+  // dQ' per (query tile, KV head); CTAs past the query-tile pair count exit at once
+  BwdQParams qp{};
+  qp.cu = cu;
+  qp.header = pp.qheader;
+  qp.pairs = pp.qpairs;
+  qp.lse2 = pp.lse2;
+  qp.delta = pp.delta;
+  qp.dq_acc = dq_acc;
+  qp.N = N;
+  qp.nq = nq;
+  qp.nkv = nkv;
+  qp.G = G;
+  qp.tq = tq;
+  qp.causal = causal;
+  qp.scale_log2 = bp.scale_log2;
+  const unsigned qgrid = (unsigned)(lay.max_qpairs * (long long)nkv);
+  gqa_attn_bwd_q_kernel<D><<<qgrid, BQ_THREADS, BwdQCfg<D>::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmDO, qp);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;
 
   const long long rows4 = (long long)N * nq * (D / 8);
   long long nbq = (rows4 + PREP_THREADS - 1) / PREP_THREADS;
   if (nbq > cap) nbq = cap;
   if (nbq < 1) nbq = 1;
-  gqa_bwd_dq_kernel<D><<<(unsigned)nbq, PREP_THREADS, 0, stream>>>(pp.dq_acc, pp.table,
+  gqa_bwd_dq_kernel<D><<<(unsigned)nbq, PREP_THREADS, 0, stream>>>(dq_acc, pp.table,
                                                                  reinterpret_cast<__nv_bfloat16*>(dq), N, nq,
                                                                  bp.scale);
   if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
-  t_last_launches = 3;
+  t_last_launches = 4;
   return GQA_OK;
 }
 
