@@ -260,17 +260,35 @@ __device__ void bwd_rope_rows(const BwdPrepParams& p, int block, int nblocks) {
     }
     *reinterpret_cast<float4*>(p.table + (size_t)t * HALF + i) = make_float4(c[0], sn[0], c[1], sn[1]);
     const uint32_t c2 = bf16x2_rn(c[0], c[1]), s2 = bf16x2_rn(sn[0], sn[1]);
-    auto rotate = [&](const __nv_bfloat16* src, __nv_bfloat16* dst) {
-      uint32_t ol, oh;
-      rope_bf16x2(*reinterpret_cast<const uint32_t*>(src + i), *reinterpret_cast<const uint32_t*>(src + i + HALF), c2,
-                  s2, ol, oh);
-      *reinterpret_cast<uint32_t*>(dst + i) = ol;
-      *reinterpret_cast<uint32_t*>(dst + i + HALF) = oh;
+    // heads in groups of HB: the group's words are all loaded before any is
+    // stored, so one memory latency covers the group
+    constexpr int HB = 8;
+    auto rotate_heads = [&](const __nv_bfloat16* src, int src_stride, __nv_bfloat16* dst, size_t dst_stride,
+                            int nh) {
+      for (int h0 = 0; h0 < nh; h0 += HB) {
+        uint32_t wl[HB], wh[HB];
+#pragma unroll
+        for (int u = 0; u < HB; ++u) {
+          if (h0 + u < nh) {
+            const __nv_bfloat16* r = src + (size_t)(h0 + u) * src_stride;
+            wl[u] = __ldg(reinterpret_cast<const unsigned int*>(r + i));
+            wh[u] = __ldg(reinterpret_cast<const unsigned int*>(r + i + HALF));
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < HB; ++u) {
+          if (h0 + u < nh) {
+            uint32_t ol, oh;
+            rope_bf16x2(wl[u], wh[u], c2, s2, ol, oh);
+            __nv_bfloat16* w = dst + (size_t)(h0 + u) * dst_stride;
+            *reinterpret_cast<uint32_t*>(w + i) = ol;
+            *reinterpret_cast<uint32_t*>(w + i + HALF) = oh;
+          }
+        }
+      }
     };
-    for (int h = 0; h < p.nkv; ++h)
-      rotate(p.k + ((size_t)t * p.nkv + h) * D, p.kws + ((size_t)h * p.N + t) * D);
-    for (int h = 0; h < p.nq; ++h)
-      rotate(p.q + ((size_t)t * p.nq + h) * D, p.qws + ((size_t)t * p.nq + h) * D);
+    rotate_heads(p.k + (size_t)t * p.nkv * D, D, p.kws + (size_t)t * D, (size_t)p.N * D, p.nkv);
+    rotate_heads(p.q + (size_t)t * p.nq * D, D, p.qws + (size_t)t * p.nq * D, (size_t)D, p.nq);
   }
 }
 

@@ -25,8 +25,8 @@
 // there is no running max. Rows past the sequence or padding rows take
 // lse = +inf and Delta = 0: their P and dS are 0.
 //
-// Warp roles (384 threads): warp 0 TMA (Q' and dO once, K'/V through two
-// stages) and the rows' statistics; warp 1 tensor memory and every MMA;
+// Warp roles (384 threads): warp 0 TMA (Q' and dO once, K' through three
+// stages, V through two) and the rows' statistics; warp 1 tensor memory and every MMA;
 // warps 4-11 dS, one row per thread and half of the tile's keys per
 // warpgroup (warps 4-7 keys [0, 64), 8-11 [64, 128)), then dQ' out.
 // Tensor memory: S/dS buffers at columns 0 and 128, dP at 256, dQ' at 384.
@@ -56,9 +56,13 @@ struct BwdQCfg {
   using A = AttnCfg<D>;
   static constexpr int OFF_Q = 0;                          // Q' tile
   static constexpr int OFF_DO = A::Q_BYTES;                // dO tile (same layout)
-  static constexpr int OFF_K = OFF_DO + A::Q_BYTES;        // two stages
-  static constexpr int OFF_V = OFF_K + 2 * A::KV_BYTES;    // two stages
-  static constexpr int OFF_ST = OFF_V + 2 * A::KV_BYTES;   // float [lse2, Delta][BM]
+  // K'_j is read by S(j) and dQ'(j), V_j by dP(j) only: K' has a deeper ring,
+  // so that K'_{j+3} loads once dQ'(j) is done and V_{j+2} once dP(j) is
+  static constexpr int KST = 3;
+  static constexpr int VST = 2;
+  static constexpr int OFF_K = OFF_DO + A::Q_BYTES;        // KST stages
+  static constexpr int OFF_V = OFF_K + KST * A::KV_BYTES;  // VST stages
+  static constexpr int OFF_ST = OFF_V + VST * A::KV_BYTES;  // float [lse2, Delta][BM]
   static constexpr int OFF_BAR = OFF_ST + 2 * BM * 4;
   static constexpr int SMEM_USED = OFF_BAR + 256 + 1024;  // + barriers + alignment slack
   // at least 120 KB, so that one CTA (which takes all 512 TMEM columns) runs per SM
@@ -72,7 +76,7 @@ struct BwdQCfg {
 
 struct BwdQBarriers {
   uint64_t q_full, st_full;
-  uint64_t k_full[2], v_full[2], kv_empty[2];
+  uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
   uint64_t s_full[2], dp_full, ds_full[2], dq_done[2];
   uint64_t o_full, drain;
   uint32_t tmem_base;
@@ -114,10 +118,15 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
   if (threadIdx.x == 0) {
     ptx::mbar_init(B(bars->q_full), 1);
     ptx::mbar_init(B(bars->st_full), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < C::KST; ++s) {
       ptx::mbar_init(B(bars->k_full[s]), 1);
+      ptx::mbar_init(B(bars->k_empty[s]), 1);
+    }
+    for (int s = 0; s < C::VST; ++s) {
       ptx::mbar_init(B(bars->v_full[s]), 1);
-      ptx::mbar_init(B(bars->kv_empty[s]), 1);
+      ptx::mbar_init(B(bars->v_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(B(bars->s_full[s]), 1);
       ptx::mbar_init(B(bars->ds_full[s]), 256);
       ptx::mbar_init(B(bars->dq_done[s]), 1);
@@ -192,25 +201,29 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
     if (lane == 0) {
       ptx::mbar_arrive(B(bars->st_full));
       for (int j = 0; j < nkt; ++j) {
-        const int s = j & 1;
-        const uint32_t par = ((j >> 1) & 1) ^ 1;  // previous use of stage s released
-        if (!(ok = bwait_lazy(B(bars->kv_empty[s]), par, abort_flag))) break;
-        ptx::mbar_arrive_expect_tx(B(bars->k_full[s]), (uint32_t)A::KV_BYTES);
+        const int ks = j % C::KST, vs = j % C::VST;
+        // previous use of each stage released
+        if (!(ok = bwait_lazy(B(bars->k_empty[ks]), ((j / C::KST) & 1) ^ 1, abort_flag))) break;
+        ptx::mbar_arrive_expect_tx(B(bars->k_full[ks]), (uint32_t)A::KV_BYTES);
         for (int b = 0; b < A::NBOX; ++b)
-          ptx::tma_load_3d(sbase + C::OFF_K + s * A::KV_BYTES + b * A::KV_BOX_BYTES, &tmK, B(bars->k_full[s]),
+          ptx::tma_load_3d(sbase + C::OFF_K + ks * A::KV_BYTES + b * A::KV_BOX_BYTES, &tmK, B(bars->k_full[ks]),
                            b * A::BOXC, seq_start + j * BN, kvh);
         ++nk;
-        ptx::mbar_arrive_expect_tx(B(bars->v_full[s]), (uint32_t)A::KV_BYTES);
+        if (!(ok = bwait_lazy(B(bars->v_empty[vs]), ((j / C::VST) & 1) ^ 1, abort_flag))) break;
+        ptx::mbar_arrive_expect_tx(B(bars->v_full[vs]), (uint32_t)A::KV_BYTES);
         for (int b = 0; b < A::NBOX; ++b)
-          ptx::tma_load_3d(sbase + C::OFF_V + s * A::KV_BYTES + b * A::KV_BOX_BYTES, &tmV, B(bars->v_full[s]),
+          ptx::tma_load_3d(sbase + C::OFF_V + vs * A::KV_BYTES + b * A::KV_BOX_BYTES, &tmV, B(bars->v_full[vs]),
                            b * A::BOXC, kvh, seq_start + j * BN);
         ++nv;
       }
       if (!ok) {  // every copy issued lands before the CTA exits
         drain_wait(B(bars->q_full), 0);
-        for (int s = 0; s < 2; ++s) {
-          const int uk = (nk - s + 1) / 2, uv = (nv - s + 1) / 2;
+        for (int s = 0; s < C::KST; ++s) {
+          const int uk = (nk - s + C::KST - 1) / C::KST;  // loads issued into stage s
           if (uk > 0) drain_wait(B(bars->k_full[s]), (uk - 1) & 1);
+        }
+        for (int s = 0; s < C::VST; ++s) {
+          const int uv = (nv - s + C::VST - 1) / C::VST;
           if (uv > 0) drain_wait(B(bars->v_full[s]), (uv - 1) & 1);
         }
       }
@@ -227,20 +240,21 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
       const uint64_t dkmn0 = umma_desc(sbase + C::OFF_K, A::KV_BOX_BYTES, A::SBO, A::UMMA_LAYOUT);
       const uint64_t stage = (uint64_t)(A::KV_BYTES >> 4);
       auto issue_s = [&](int j) -> bool {
-        const int s = j & 1;
+        const int s = j & 1, ks = j % C::KST;
         if (j >= 2 && !bwait(B(bars->dq_done[s]), ((j - 2) >> 1) & 1, abort_flag)) return false;
-        if (!bwait(B(bars->k_full[s]), (j >> 1) & 1, abort_flag)) return false;
+        if (!bwait(B(bars->k_full[ks]), (j / C::KST) & 1, abort_flag)) return false;
         ptx::tc_fence_after();
-        issue_s_mmas<A>(tmem + s * 128, dq, dk0 + s * stage);
+        issue_s_mmas<A>(tmem + s * 128, dq, dk0 + ks * stage);
         ptx::mma_commit(B(bars->s_full[s]));
         return true;
       };
       auto issue_dp = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!bwait(B(bars->v_full[s]), (j >> 1) & 1, abort_flag)) return false;
+        const int vs = j % C::VST;
+        if (!bwait(B(bars->v_full[vs]), (j / C::VST) & 1, abort_flag)) return false;
         ptx::tc_fence_after();
-        issue_s_mmas<A>(tmem + C::DP_COL, ddo, dv0 + s * stage);
+        issue_s_mmas<A>(tmem + C::DP_COL, ddo, dv0 + vs * stage);
         ptx::mma_commit(B(bars->dp_full));
+        ptx::mma_commit(B(bars->v_empty[vs]));  // dP(j) is V_j's only reader
         return true;
       };
       bool ok = bwait(B(bars->q_full), 0, abort_flag) && issue_s(0) && issue_dp(0);
@@ -249,9 +263,9 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
         if (j + 1 < nkt && !(ok = issue_s(j + 1))) break;
         if (!(ok = bwait(B(bars->ds_full[s]), (j >> 1) & 1, abort_flag))) break;
         ptx::tc_fence_after();
-        issue_pv_mmas<A>(tmem + C::DQ_COL, tmem + s * 128, dkmn0 + s * stage, j > 0);
+        issue_pv_mmas<A>(tmem + C::DQ_COL, tmem + s * 128, dkmn0 + (j % C::KST) * stage, j > 0);
         ptx::mma_commit(B(bars->dq_done[s]));
-        ptx::mma_commit(B(bars->kv_empty[s]));  // S(j), dP(j) and dQ'(j) have read K'_j and V_j
+        ptx::mma_commit(B(bars->k_empty[j % C::KST]));  // S(j) and dQ'(j) have read K'_j
         if (j + 1 < nkt && !(ok = issue_dp(j + 1))) break;
       }
       if (ok) ptx::mma_commit(B(bars->o_full));
