@@ -286,8 +286,8 @@ int gqa_rope_attn_decode(const void* q, const void* k_new, const void* v_new, vo
  * rotated q and k are computed exactly as the forward computes them; the
  * gradient passes the rotation's roundings unchanged (rope^T uses the fp32
  * cos/sin). P and dS enter their products as
- * bf16; every product accumulates in fp32; dq accumulates over key tiles in
- * fp32 in the workspace.
+ * bf16; every product accumulates in fp32; dq is summed over the key tiles
+ * of each query tile in fp32 (once per row, no atomics) and rotated back.
  *
  * All of q, k, v, out, dout, dq, dk, dv are bf16 in the forward's layout
  * (q, out, dout, dq: [total_tokens, n_q_heads, head_dim]; k, v, dk, dv:
@@ -298,8 +298,9 @@ int gqa_rope_attn_decode(const void* q, const void* k_new, const void* v_new, vo
  * GQA_ERR_BAD_SEQLENS in the status word; dk and dv are then not written).
  * dq, dk and dv are overwritten (not accumulated into). workspace: at least
  * gqa_rope_attn_bwd_workspace_size() bytes, 256-byte aligned, contents need
- * not be initialised, not shared by calls that may overlap. Three kernels
- * are queued on `stream`; the call does not wait. Returns GQA_OK or an
+ * not be initialised, not shared by calls that may overlap. Four kernels
+ * are queued on `stream` (prologue, dk/dv per key tile, dq per query tile,
+ * dq's rotation); the call does not wait. Returns GQA_OK or an
  * error code; on an error nothing has been queued.
  */
 size_t gqa_rope_attn_bwd_workspace_size(int num_seqs, int total_tokens, int n_q_heads, int n_kv_heads,

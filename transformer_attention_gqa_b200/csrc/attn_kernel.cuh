@@ -291,9 +291,10 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 // Of every emu_period(d) groups of 4 exponentials of a row, one is evaluated
 // on the FMA pipe, the rest on the special-function unit (0: all on the
-// SFU). With two softmax warps per sub-partition the SFU is the limit; at
-// d = 128, 1 in 8 measured fastest (1 in 4 and more run out of issue slots).
-__host__ __device__ constexpr int emu_period(int d) { return d == 128 ? 8 : (d == 64 ? 8 : 8); }
+// SFU). Measured: at d = 128, 1 in 16 (1 in 8 while the Q rotation's fp64
+// conversions also used the special-function unit); 1 in 4 and more run out
+// of issue slots; at d = 64, 1 in 8.
+__host__ __device__ constexpr int emu_period(int d) { return d == 128 ? 16 : 8; }
 
 __device__ __forceinline__ uint32_t swz(uint32_t lin, int mask) { return lin ^ (((lin >> 7) & mask) << 4); }
 
