@@ -22,8 +22,12 @@
 //   warp 3      one thread issues the O += P V MMAs
 //   warps 4-11  softmax: a row (TMEM lane) is shared by two threads, warps
 //               4-7 take its columns [0, 64) and warps 8-11 columns
-//               [64, 128); S -> P, running max (exchanged once per tile)
-//               and partial sums, O rescale of their half of O's columns
+//               [64, 128); S -> P, running max and partial sums, O
+//               rescale. At d <= 64 each half keeps its own running max
+//               and sum and accumulates into its own partial output (O_a
+//               or O_b), so the two never wait for each other; at d = 128
+//               they share one O and exchange their tile maxima once per
+//               tile (two outputs would not leave room for three S buffers)
 //   warps 12-15 Q tiles: TMA load, RoPE applied in shared memory before the
 //               first S MMA reads it; epilogue: O / l from TMEM, LSE
 // Two softmax warps per SM sub-partition keep the special-function unit
@@ -32,11 +36,15 @@
 // Tensor memory (512 columns x 128 lanes of 32 bit):
 //   [0,128) [128,256) [256,384): three S buffers; the bf16 P of each column
 //   half overwrites the first 32 columns of that half's S columns (keys
-//   [0, 64) at +0, keys [64, 128) at +64); [384, 384+d): O.
-// MMAs: S = Q K^T   kind::f16, A = Q (smem, K-major), B = K (smem, K-major),
-//                   M = 128, N = 128, fp32 accumulate, d/16 steps;
-//       O += P V    A = P (tmem), B = V (smem, MN-major), M = 128, N = d,
-//                   8 steps of 16 keys.
+//   [0, 64) at +0, keys [64, 128) at +64); from 384: O (d = 128), or O_a and
+//   O_b (d <= 64, d columns each), which the epilogue combines as the two
+//   partial sums of a split softmax: O = (a_a O_a + a_b O_b) / (a_a l_a +
+//   a_b l_b) with a_h = 2^(m_h - max(m_a, m_b)).
+// MMAs: S = Q K^T     kind::f16, A = Q (smem, K-major), B = K (smem,
+//                     K-major), M = 128, N = 128, fp32 accumulate, d/16 steps;
+//       O += P V        A = P (tmem), B = V (smem, MN-major), M = 128,
+//                     N = d, 8 steps of 16 keys; at d <= 64 as
+//                     O_h += P_h V_h, 4 steps over the keys of half h.
 #pragma once
 
 #include "common.cuh"
@@ -53,6 +61,7 @@ namespace gqa {
 // once.
 constexpr int ITEM_SLOTS = 8;
 constexpr int ITEM_READERS = 3 + 8 + 4;
+constexpr int KSTEPS_PV_HALF = BN / 2 / 16;  // P V K-steps of one column half
 
 // Register split (launch: 512 threads x 128): producers/MMA 56, softmax 160
 // (8 warps), Q rotation/epilogue 128 (the launch value).
@@ -69,10 +78,10 @@ struct WorkItem {
 struct Barriers {
   uint64_t q_loaded[2], q_ready[2], q_empty[2];
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[NUM_S_BUF], p_full[NUM_S_BUF], pv_done[NUM_S_BUF];
+  uint64_t s_full[NUM_S_BUF], p_full[NUM_S_BUF][2], pv_done[NUM_S_BUF];  // p_full: [buffer][column half]
   uint64_t o_free, drain;
   uint64_t stats_full, stats_empty;
-  uint64_t xchg[2][4];  // row-max exchange of the two softmax halves: [tile parity][lane quadrant]
+  uint64_t xchg[2][4];  // (d = 128) row-max exchange of the two softmax halves: [tile parity][lane quadrant]
   uint64_t item_full[ITEM_SLOTS], item_empty[ITEM_SLOTS];
   int item[ITEM_SLOTS];  // work-item index, -1 = no more items
   WorkItem witem[ITEM_SLOTS];  // the item decoded (sequence, tile, KV head), by the publisher
@@ -103,7 +112,15 @@ struct AttnCfg {
   static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t O_COL = 384;
+  // d <= 64 (SPLIT): the two softmax column halves keep their own running
+  // max and sum and their own partial output, O_a (keys [0, 64) of every
+  // tile) at O_COL and O_b (keys [64, 128)) at O_COL + D, and never wait
+  // for each other. d = 128: one O and a running max that the halves
+  // exchange once per tile (two outputs would cost the third S buffer, and
+  // measured slower there).
+  static constexpr bool SPLIT = D <= 64;
+  static constexpr int NSB = NUM_S_BUF;
+  static constexpr uint32_t O_COL = NSB * 128;
   static constexpr int KSTEPS_S = D / 16;
   static constexpr int KSTEPS_PV = BN / 16;
   static constexpr int STEPS_PER_BOX = BOXC / 16;
@@ -114,7 +131,7 @@ struct AttnCfg {
                                       ((uint32_t)(D >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(sizeof(Barriers) <= BAR_BYTES, "barrier area");
-  static_assert(O_COL + D <= TMEM_COLS, "tensor memory budget");
+  static_assert(O_COL + (SPLIT ? 2 : 1) * D <= TMEM_COLS, "tensor memory budget");
 };
 
 // Shared-memory matrix descriptor (tcgen05): start, leading/stride byte
@@ -422,73 +439,62 @@ __device__ __forceinline__ void scale_o_cols(uint32_t taddr, float alpha, uint32
   }
 }
 
-// Takes the CTA's it-th work item from the hand-off ring and rotates its Q
-// tile in shared memory (buffer it & 1) once the TMA load has landed, then
-// releases it to the S issuer. Run by the 128 threads of the
-// Q-rotation/epilogue warpgroup; thread 0 takes the item and loads Q, and
-// the item index reaches the others with the load's barrier. Returns false
-// on abort; w_out = the item's index, or -1 when no items are left.
-// Q tile of work item `it` into Q buffer it & 1, rotated in shared memory by
-// the Q warpgroup (128 threads). Every warp takes the item from the hand-off
-// ring; thread 0 loads the tile once the buffer's previous item has finished
-// its S MMAs; each thread's first cos/sin words are loaded before the tile
-// lands and the next ones while it rotates the current ones.
+// One Q tile (tokens [t_first, t_first + tq) of item wi, the G heads of its
+// KV head) into the shared-memory buffer qbuf, rotated there by the Q
+// warpgroup (128 threads): thread 0 loads the tile once the buffer's
+// previous tile has finished its S MMAs (bar_empty, phase ph ^ 1); each
+// thread's first cos/sin words are loaded before the tile lands and the next
+// ones while it rotates the current ones; then bar_ready. With have = false
+// nothing is loaded but every barrier still completes its phase. Returns
+// false on abort.
 template <class C>
-__device__ __forceinline__ bool rope_q_tile(const AttnParams& p, uint8_t* smem, Barriers* bars,
-                                            const CUtensorMap* tmQ, int it, int tid, volatile int* abort_flag,
-                                            int& w_out, WorkItem& wi_out) {
+__device__ __forceinline__ bool load_rope_q(const AttnParams& p, uint8_t* qbuf, uint32_t bar_empty,
+                                            uint32_t bar_loaded, uint32_t bar_ready, uint32_t ph, bool have,
+                                            const WorkItem& wi, int t_first, const CUtensorMap* tmQ, int tid,
+                                            volatile int* abort_flag) {
   constexpr int D = C::D;
   constexpr int NCH = D / 16;  // 16-byte chunks in the first half of a row
   constexpr int HALF = D / 2;
-  const int qb = it & 1;
   const int G = p.G;
-  int w;
-  WorkItem wi;
-  if (!take_item_warp(bars, it, w, wi, abort_flag)) return false;
   bool issued = false;
-  if (tid == 0 && bwait(ptx::smem_u32(&bars->q_empty[qb]), ((it >> 1) & 1) ^ 1, abort_flag)) {
-    // the buffer's previous tile has finished its S MMAs: load this tile's Q
-    const uint32_t bar = ptx::smem_u32(&bars->q_loaded[qb]);
-    if (w >= 0) {
+  if (tid == 0 && bwait(bar_empty, ph ^ 1, abort_flag)) {
+    if (have) {
       issued = true;
-      ptx::mbar_arrive_expect_tx(bar, (uint32_t)(D * 2 * G * p.tq));
+      ptx::mbar_arrive_expect_tx(bar_loaded, (uint32_t)(D * 2 * G * p.tq));
 #pragma unroll
       for (int b = 0; b < C::NBOX; ++b)
-        ptx::tma_load_3d(ptx::smem_u32(smem + qb * C::Q_BYTES + b * C::Q_BOX_BYTES), tmQ, bar, b * C::BOXC,
-                         wi.kvh * G, wi.seq_start + wi.t0);
+        ptx::tma_load_3d(ptx::smem_u32(qbuf + b * C::Q_BOX_BYTES), tmQ, bar_loaded, b * C::BOXC, wi.kvh * G,
+                         wi.seq_start + t_first);
     } else {
-      ptx::mbar_arrive(bar);
+      ptx::mbar_arrive(bar_loaded);
     }
   }
   // this thread's work: (token, 8-column chunk) pairs item = tid, tid + 128, ...
-  const int items = (w < 0 || p.q_rotated) ? 0 : p.tq * NCH;  // rotated Q tiles are used as loaded
+  const int items = (!have || p.q_rotated) ? 0 : p.tq * NCH;  // rotated Q tiles are used as loaded
   auto load_tab = [&](int item, float4& cf, float4& sf) {
     const int tt = item / NCH;
     const int ch = item - tt * NCH;
-    if (wi.t0 + tt < wi.L) {
+    if (t_first + tt < wi.L) {
       // bf16 cos and sin of frequencies ch*8 .. ch*8+7 (table_word layout)
-      const float4* tab = reinterpret_cast<const float4*>(p.table + table_word(wi.seq_start + wi.t0 + tt, HALF, ch * 8));
+      const float4* tab = reinterpret_cast<const float4*>(p.table + table_word(wi.seq_start + t_first + tt, HALF, ch * 8));
       cf = ptx::ld_cg_v4f32(tab);
       sf = ptx::ld_cg_v4f32(tab + 1);
     }
   };
   float4 cf = make_float4(0.f, 0.f, 0.f, 0.f), sf = cf;
   if (tid < items) load_tab(tid, cf, sf);
-  const bool ok = __all_sync(0xffffffffu, bwait_lazy(ptx::smem_u32(&bars->q_loaded[qb]), (it >> 1) & 1, abort_flag));
+  const bool ok = __all_sync(0xffffffffu, bwait_lazy(bar_loaded, ph, abort_flag));
   if (!ok) {  // a load issued above lands before the CTA may exit
-    if (issued) drain_wait(ptx::smem_u32(&bars->q_loaded[qb]), (it >> 1) & 1);
+    if (issued) drain_wait(bar_loaded, ph);
     return false;
   }
-  w_out = w;
-  wi_out = wi;
-  if (w < 0) return true;
-  uint8_t* qbuf = smem + qb * C::Q_BYTES;
+  if (!have) return true;
   for (int item = tid; item < items; item += 128) {
     float4 cfn = cf, sfn = sf;
     if (item + 128 < items) load_tab(item + 128, cfn, sfn);
     const int tt = item / NCH;
     const int ch = item - tt * NCH;
-    if (wi.t0 + tt < wi.L) {
+    if (t_first + tt < wi.L) {
       const uint32_t cw[4] = {__float_as_uint(cf.x), __float_as_uint(cf.y), __float_as_uint(cf.z),
                               __float_as_uint(cf.w)};
       const uint32_t sw[4] = {__float_as_uint(sf.x), __float_as_uint(sf.y), __float_as_uint(sf.z),
@@ -514,8 +520,26 @@ __device__ __forceinline__ bool rope_q_tile(const AttnParams& p, uint8_t* smem, 
     sf = sfn;
   }
   ptx::fence_proxy_async_smem();
-  ptx::mbar_arrive(ptx::smem_u32(&bars->q_ready[qb]));
+  ptx::mbar_arrive(bar_ready);
   return true;
+}
+
+// Q tile of the CTA's work item `it` into Q buffer it & 1: every warp of the
+// Q warpgroup takes the item from the hand-off ring (w_out = its index, -1
+// when no items are left), then load_rope_q. Returns false on abort.
+template <class C>
+__device__ __forceinline__ bool rope_q_tile(const AttnParams& p, uint8_t* smem, Barriers* bars,
+                                            const CUtensorMap* tmQ, int it, int tid, volatile int* abort_flag,
+                                            int& w_out, WorkItem& wi_out) {
+  const int qb = it & 1;
+  int w;
+  WorkItem wi;
+  if (!take_item_warp(bars, it, w, wi, abort_flag)) return false;
+  w_out = w;
+  wi_out = wi;
+  return load_rope_q<C>(p, smem + qb * C::Q_BYTES, ptx::smem_u32(&bars->q_empty[qb]),
+                        ptx::smem_u32(&bars->q_loaded[qb]), ptx::smem_u32(&bars->q_ready[qb]), (it >> 1) & 1,
+                        w >= 0, wi, wi.t0, tmQ, tid, abort_flag);
 }
 
 template <class C, bool OUT_FP32>
@@ -533,54 +557,71 @@ __device__ __forceinline__ bool epilogue_tile(const AttnParams& p, const WorkIte
   const bool row_valid = r < p.tq * G && tok < wi.L;
   bool ok = __all_sync(0xffffffffu, bwait(ptx::smem_u32(&bars->stats_full), it & 1, abort_flag));
   if (!ok) return false;
+  // (running max, sum) of the two column halves, each against its own max
   const float2 ml0 = reinterpret_cast<const float2*>(smem + C::OFF_STATS)[r];
   const float2 ml1 = reinterpret_cast<const float2*>(smem + C::OFF_STATS)[BM + r];
-  const float2 ml = make_float2(ml0.x, ml0.y + ml1.y);  // both halves hold the same running max
   ptx::mbar_arrive(ptx::smem_u32(&bars->stats_empty));
   const uint32_t gl = g + wi.nkv - 1;
   ok = __all_sync(0xffffffffu,
-                  bwait(ptx::smem_u32(&bars->pv_done[gl % NUM_S_BUF]), (gl / NUM_S_BUF) & 1, abort_flag));
+                  bwait(ptx::smem_u32(&bars->pv_done[gl % C::NSB]), (gl / C::NSB) & 1, abort_flag));
   if (!ok) return false;
   ptx::tc_fence_after();
 
-  const float inv_l = 1.f / ml.y;
+  float mrow, lrow, w0, w1;
+  if constexpr (C::SPLIT) {
+    // O = (a0 O_a + a1 O_b) / (a0 l_a + a1 l_b), a_h = 2^((m_h - m) scale) for
+    // the row max m; a half that saw no unmasked key (m_h = -inf) weighs 0
+    mrow = fmaxf(ml0.x, ml1.x);
+    const float a0 = ml0.x == -INFINITY ? 0.f : ptx::ex2((ml0.x - mrow) * p.scale_log2);
+    const float a1 = ml1.x == -INFINITY ? 0.f : ptx::ex2((ml1.x - mrow) * p.scale_log2);
+    lrow = a0 * ml0.y + a1 * ml1.y;
+    const float inv_l = 1.f / lrow;
+    w0 = a0 * inv_l;
+    w1 = a1 * inv_l;
+  } else {
+    mrow = ml0.x;  // both halves hold the same running max
+    lrow = ml0.y + ml1.y;
+    w0 = 1.f / lrow;
+    w1 = 0.f;
+  }
   const int h = wi.kvh * G + hin;
   const size_t orow = (size_t)(wi.seq_start + tok) * p.nq + h;
-  uint32_t o[32];
+  // 16 columns of O (of O_a and O_b) at a time
+  uint32_t oa[16], ob[16];
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
-    ptx::tmem_ld32(trow + C::O_COL + c * 32, o);
+  for (int c = 0; c < D / 16; ++c) {
+    ptx::tmem_ld16(trow + C::O_COL + c * 16, oa);
+    if constexpr (C::SPLIT) ptx::tmem_ld16(trow + C::O_COL + D + c * 16, ob);
     ptx::tmem_wait_ld();
-    ptx::reg_fence32(o);
-    if (c == D / 32 - 1) {  // O fully read: the next tile's first P.V may overwrite it
+    ptx::reg_fence16(oa);
+    if constexpr (C::SPLIT) ptx::reg_fence16(ob);
+    if (c == D / 16 - 1) {  // O fully read: the next tile's first P.V may overwrite it
       ptx::tc_fence_before();
       ptx::mbar_arrive(ptx::smem_u32(&bars->o_free));
     }
+    auto o = [&](int e) {
+      if constexpr (C::SPLIT) return fmaf(__uint_as_float(oa[e]), w0, __uint_as_float(ob[e]) * w1);
+      else return __uint_as_float(oa[e]) * w0;
+    };
     if constexpr (OUT_FP32) {
       if (row_valid) {
-        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + orow * D + c * 32);
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + orow * D + c * 16);
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
-                               __uint_as_float(o[4 * e + 2]) * inv_l, __uint_as_float(o[4 * e + 3]) * inv_l);
+        for (int e = 0; e < 4; ++e) dst[e] = make_float4(o(4 * e), o(4 * e + 1), o(4 * e + 2), o(4 * e + 3));
       }
     } else {
-      uint32_t pk[16];
+      uint32_t pk[8];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv_l,
-                                                        __uint_as_float(o[2 * e + 1]) * inv_l);
-        pk[e] = *reinterpret_cast<const uint32_t*>(&v2);
-      }
+      for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(o(2 * e), o(2 * e + 1));
       if (row_valid) {
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + orow * D + c * 32);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + orow * D + c * 16);
+        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
     }
   }
   if (row_valid && p.lse)
-    p.lse[(size_t)h * p.N + wi.seq_start + tok] = (ml.x * p.scale_log2 + __log2f(ml.y)) * 0.69314718055994531f;
+    p.lse[(size_t)h * p.N + wi.seq_start + tok] = (mrow * p.scale_log2 + __log2f(lrow)) * 0.69314718055994531f;
   return true;
 }
 
@@ -603,6 +644,17 @@ __device__ __forceinline__ void issue_pv_mmas(uint32_t o_tmem, uint32_t p_tmem, 
   for (int kk = 0; kk < C::KSTEPS_PV; ++kk)
     ptx::mma_ts(o_tmem, p_tmem + (kk >> 2) * 64 + (kk & 3) * 8, dv + (uint64_t)((kk * 16 * C::ROWB) >> 4),
                 C::IDESC_O, (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// O_h (+)= P_h V_h for one column half h of a KV tile: 4 K-steps of 16 keys;
+// p_tmem = the half's packed P columns, dv = V's descriptor at the half's
+// first key.
+template <class C>
+__device__ __forceinline__ void issue_pv_half(uint32_t o_tmem, uint32_t p_tmem, uint64_t dv, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < KSTEPS_PV_HALF; ++kk)
+    ptx::mma_ts(o_tmem, p_tmem + kk * 8, dv + (uint64_t)((kk * 16 * C::ROWB) >> 4), C::IDESC_O,
+                (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D, bool OUT_FP32>
@@ -638,15 +690,16 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     }
     for (int i = 0; i < NUM_S_BUF; ++i) {
       ptx::mbar_init(B(bars->s_full[i]), 1);
-      ptx::mbar_init(B(bars->p_full[i]), 256);
+      ptx::mbar_init(B(bars->p_full[i][0]), C::SPLIT ? 128 : 256);
+      ptx::mbar_init(B(bars->p_full[i][1]), 128);  // (SPLIT only)
       ptx::mbar_init(B(bars->pv_done[i]), 1);
     }
     ptx::mbar_init(B(bars->o_free), 128);
     ptx::mbar_init(B(bars->stats_full), 256);
     ptx::mbar_init(B(bars->stats_empty), 128);
-    ptx::mbar_init(B(bars->drain), 2);  // one commit per MMA-issuing thread
     for (int i = 0; i < 2; ++i)
       for (int qd = 0; qd < 4; ++qd) ptx::mbar_init(B(bars->xchg[i][qd]), 64);
+    ptx::mbar_init(B(bars->drain), 2);  // one commit per MMA-issuing thread
     for (int i = 0; i < ITEM_SLOTS; ++i) {
       ptx::mbar_init(B(bars->item_full[i]), 1);
       ptx::mbar_init(B(bars->item_empty[i]), ITEM_READERS);
@@ -668,10 +721,11 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  // Everything below reads what the prologue kernel wrote. The attention
-  // kernel is launched in plain stream order (a programmatic dependent
-  // launch measured slower), so this wait returns at once; it would order
-  // the reads if the launch were made programmatic.
+  // Everything below reads what the prologue kernel wrote. The forward
+  // launches this kernel as a programmatic dependent of the prologue, so the
+  // setup above overlaps the prologue's tail; this wait returns once the
+  // prologue grid has completed and its stores are visible (at once for a
+  // launch in plain stream order).
   ptx::griddep_wait();
   const int n_items = ptx::ld_cg_s32(p.header) * p.nkv;
 
@@ -766,8 +820,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         if (!(ok = bwait(bar_qr0 + 8 * qb, (it >> 1) & 1, abort_flag))) break;
         const uint64_t dq = dq_base + (uint64_t)((qb * C::Q_BYTES) >> 4);
         for (int j = 0; j < wi.nkv; ++j, ++gs) {
-          const int bs = gs % NUM_S_BUF, ks = gs % C::KST;
-          if (gs >= NUM_S_BUF && !(ok = bwait(bar_pv0 + 8 * bs, ((gs / NUM_S_BUF) - 1) & 1, abort_flag))) break;
+          const int bs = gs % C::NSB, ks = gs % C::KST;
+          if (gs >= C::NSB && !(ok = bwait(bar_pv0 + 8 * bs, ((gs / C::NSB) - 1) & 1, abort_flag))) break;
           if (!(ok = bwait(bar_kf0 + 8 * ks, (gs / C::KST) & 1, abort_flag))) break;
           ptx::tc_fence_after();
           issue_s_mmas<C>(tmem + bs * 128, dq, dk_base + (uint64_t)((ks * C::KV_BYTES) >> 4));
@@ -785,7 +839,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     // O += P(x) V(x) once the softmax has written P(x) into S buffer x % 3.
     if (lane == 0) {
       const uint64_t dv_base = umma_desc(sbase + C::OFF_V, C::KV_BOX_BYTES, C::SBO, C::UMMA_LAYOUT);
-      const uint32_t bar_pv0 = B(bars->pv_done[0]), bar_p0 = B(bars->p_full[0]);
+      const uint32_t bar_pv0 = B(bars->pv_done[0]), bar_p0 = B(bars->p_full[0][0]);
       const uint32_t bar_vf0 = B(bars->v_full[0]), bar_ve0 = B(bars->v_empty[0]), bar_of = B(bars->o_free);
       uint32_t g = 0;
       int it = 0;
@@ -795,12 +849,25 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         WorkItem wi;
         if (!(ok = take_item(bars, it, w, wi, abort_flag)) || w < 0) break;
         for (int j = 0; j < wi.nkv; ++j, ++g) {
-          const int b = g % NUM_S_BUF, vs = g % C::VST;
+          const int b = g % C::NSB, vs = g % C::VST;
           if (!(ok = bwait(bar_vf0 + 8 * vs, (g / C::VST) & 1, abort_flag))) break;
           if (j == 0 && !(ok = bwait(bar_of, (it & 1) ^ 1, abort_flag))) break;
-          if (!(ok = bwait(bar_p0 + 8 * b, (g / NUM_S_BUF) & 1, abort_flag))) break;
-          ptx::tc_fence_after();
-          issue_pv_mmas<C>(tmem + C::O_COL, tmem + b * 128, dv_base + (uint64_t)((vs * C::KV_BYTES) >> 4), j > 0);
+          const uint64_t dv = dv_base + (uint64_t)((vs * C::KV_BYTES) >> 4);
+          if constexpr (C::SPLIT) {
+            // each column half's P V as soon as that half has written its P
+            for (int h = 0; h < 2; ++h) {
+              if (!(ok = bwait(bar_p0 + 16 * b + 8 * h, (g / C::NSB) & 1, abort_flag))) break;
+              ptx::tc_fence_after();
+              issue_pv_half<C>(tmem + C::O_COL + h * D, tmem + b * 128 + h * (BN / 2),
+                               dv + (uint64_t)((h * (BN / 2) * C::ROWB) >> 4), j > 0);
+            }
+          } else {
+            if ((ok = bwait(bar_p0 + 16 * b, (g / C::NSB) & 1, abort_flag))) {
+              ptx::tc_fence_after();
+              issue_pv_mmas<C>(tmem + C::O_COL, tmem + b * 128, dv, j > 0);
+            }
+          }
+          if (!ok) break;
           ptx::mma_commit(bar_pv0 + 8 * b);
           ptx::mma_commit(bar_ve0 + 8 * vs);
         }
@@ -821,7 +888,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     const int tok_off = r / G;
     const float sl2 = p.scale_log2;
     float2* stats = reinterpret_cast<float2*>(smem + C::OFF_STATS) + half * BM;
-    float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);  // [parity][half][BM]
+    float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);  // [parity][half][BM] (d = 128)
     uint32_t g = 0;
     int it = 0;
     bool ok = true;
@@ -836,69 +903,103 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       float l = 0.f;
       for (int j = 0; j < wi.nkv; ++j) {
         const uint32_t gg = g + j;
-        const int b = gg % NUM_S_BUF;
+        const int b = gg % C::NSB;
         const uint32_t tS = trow + b * 128;
-        ok = __all_sync(0xffffffffu, bwait(B(bars->s_full[b]), (gg / NUM_S_BUF) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, bwait(B(bars->s_full[b]), (gg / C::NSB) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
         load_s_cols<NC>(tS, sr);
         const int lim = last_key - j * BN - half * NC;  // this half's columns > lim are masked
         if (lim < NC - 1) mask_cols<NC>(sr, lim);
-        // Both halves publish their max, then read the other's (mbarrier of
-        // 64 arrivals per lane quadrant, alternating by tile parity).
-        const int xp = gg & 1;
-        float* xm_mine = xmax + (xp * 2 + half) * BM + r;
-        const float* xm_other = xmax + (xp * 2 + (half ^ 1)) * BM + r;
-        const uint32_t xbar = B(bars->xchg[xp][quad]);
-        const uint32_t xpar = (gg >> 1) & 1;
         float alpha = 1.f;
         float lsum;
-        if (j == 0) {
-          const float mh = cols_max<NC>(sr);
-          *xm_mine = mh;
-          ptx::mbar_arrive(xbar);
-          ok = __all_sync(0xffffffffu, bwait(xbar, xpar, abort_flag));
-          if (!ok) break;
-          m = fmaxf(mh, *xm_other);
-          lsum = exp_pack<NC, emu_period(D)>(sr, -m * sl2, sl2, nullptr);
-        } else {
-          // Exponentials with the running max m, the tile's max alongside;
-          // if the row's max exceeds m by more than the threshold (2^8 in p)
-          // the tile is redone below with the new max.
-          float mh;
-          lsum = exp_pack<NC, emu_period(D)>(sr, -m * sl2, sl2, &mh);
-          *xm_mine = mh;
-          ptx::mbar_arrive(xbar);
-          ok = __all_sync(0xffffffffu, bwait(xbar, xpar, abort_flag));
-          if (!ok) break;
-          const float mx = fmaxf(mh, *xm_other);
-          bool need = false;
-          if (mx > m + p.rescale_thr) {
-            alpha = ptx::ex2((m - mx) * sl2);
-            m = mx;
-            need = true;
+        if constexpr (C::SPLIT) {
+          // The halves keep their own running max and sum (and their own O),
+          // so neither waits for the other. A half whose keys were all masked
+          // so far keeps m = -inf; its p are 0 (bias 0 on -inf scores).
+          if (j == 0) {
+            m = cols_max<NC>(sr);
+            lsum = exp_pack<NC, emu_period(D)>(sr, m == -INFINITY ? 0.f : -m * sl2, sl2, nullptr);
+          } else {
+            // Exponentials with the running max m, the tile's max alongside;
+            // if the tile's max exceeds m by more than the threshold (2^8 in
+            // p) the tile is redone below with the new max.
+            float mh;
+            lsum = exp_pack<NC, emu_period(D)>(sr, m == -INFINITY ? 0.f : -m * sl2, sl2, &mh);
+            const bool need = mh > m + p.rescale_thr;
+            if (__any_sync(0xffffffffu, need)) {
+              if (need) {
+                alpha = ptx::ex2((m - mh) * sl2);
+                m = mh;
+              }
+              load_s_cols<NC>(tS, sr);  // S is intact: P has not been stored yet
+              if (lim < NC - 1) mask_cols<NC>(sr, lim);
+              lsum = exp_pack<NC, emu_period(D)>(sr, m == -INFINITY ? 0.f : -m * sl2, sl2, nullptr);
+              // O_h holds this half's sum up to the previous tile: wait for
+              // PV(gg-1), then scale it (alpha = 1 on rows that kept their max)
+              const uint32_t gp = gg - 1;
+              ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[gp % C::NSB]), (gp / C::NSB) & 1, abort_flag));
+              if (!ok) break;
+              ptx::tc_fence_after();
+              // (sr[0, NC/2) holds the packed P; the upper half is free scratch)
+              scale_o_cols<D>(tmem + ((uint32_t)(quad * 32) << 16) + C::O_COL + half * D, alpha, sr + NC / 2);
+            }
           }
-          // Both halves see the same maxima, so they take this branch together.
-          if (__any_sync(0xffffffffu, need)) {
-            load_s_cols<NC>(tS, sr);  // S is intact: P has not been stored yet
-            if (lim < NC - 1) mask_cols<NC>(sr, lim);
-            lsum = exp_pack<NC, emu_period(D)>(sr, -m * sl2, sl2, nullptr);
-            // O holds the sum up to the previous tile: wait for PV(gg-1), then
-            // scale this half's share of O's columns.
-            const uint32_t gp = gg - 1;
-            ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[gp % NUM_S_BUF]), (gp / NUM_S_BUF) & 1, abort_flag));
+        } else {
+          // Both halves publish their max, then read the other's (mbarrier of
+          // 64 arrivals per lane quadrant, alternating by tile parity).
+          const int xp = gg & 1;
+          float* xm_mine = xmax + (xp * 2 + half) * BM + r;
+          const float* xm_other = xmax + (xp * 2 + (half ^ 1)) * BM + r;
+          const uint32_t xbar = B(bars->xchg[xp][quad]);
+          const uint32_t xpar = (gg >> 1) & 1;
+          if (j == 0) {
+            const float mh = cols_max<NC>(sr);
+            *xm_mine = mh;
+            ptx::mbar_arrive(xbar);
+            ok = __all_sync(0xffffffffu, bwait(xbar, xpar, abort_flag));
             if (!ok) break;
-            ptx::tc_fence_after();
-            // (sr[0, NC/2) holds the packed P; the upper half is free scratch)
-            scale_o_cols<D / 2>(tmem + ((uint32_t)(quad * 32) << 16) + C::O_COL + half * (D / 2), alpha,
-                                sr + NC / 2);
+            m = fmaxf(mh, *xm_other);
+            lsum = exp_pack<NC, emu_period(D)>(sr, -m * sl2, sl2, nullptr);
+          } else {
+            // Exponentials with the running max m, the tile's max alongside;
+            // if the row's max exceeds m by more than the threshold (2^8 in p)
+            // the tile is redone below with the new max.
+            float mh;
+            lsum = exp_pack<NC, emu_period(D)>(sr, -m * sl2, sl2, &mh);
+            *xm_mine = mh;
+            ptx::mbar_arrive(xbar);
+            ok = __all_sync(0xffffffffu, bwait(xbar, xpar, abort_flag));
+            if (!ok) break;
+            const float mx = fmaxf(mh, *xm_other);
+            bool need = false;
+            if (mx > m + p.rescale_thr) {
+              alpha = ptx::ex2((m - mx) * sl2);
+              m = mx;
+              need = true;
+            }
+            // Both halves see the same maxima, so they take this branch together.
+            if (__any_sync(0xffffffffu, need)) {
+              load_s_cols<NC>(tS, sr);  // S is intact: P has not been stored yet
+              if (lim < NC - 1) mask_cols<NC>(sr, lim);
+              lsum = exp_pack<NC, emu_period(D)>(sr, -m * sl2, sl2, nullptr);
+              // O holds the sum up to the previous tile: wait for PV(gg-1), then
+              // scale this half's share of O's columns.
+              const uint32_t gp = gg - 1;
+              ok = __all_sync(0xffffffffu, bwait(B(bars->pv_done[gp % C::NSB]), (gp / C::NSB) & 1, abort_flag));
+              if (!ok) break;
+              ptx::tc_fence_after();
+              // (sr[0, NC/2) holds the packed P; the upper half is free scratch)
+              scale_o_cols<D / 2>(tmem + ((uint32_t)(quad * 32) << 16) + C::O_COL + half * (D / 2), alpha,
+                                  sr + NC / 2);
+            }
           }
         }
         l = l * alpha + lsum;
         store_p<NC>(tS, sr);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(B(bars->p_full[b]));
+        ptx::mbar_arrive(B(bars->p_full[b][C::SPLIT ? half : 0]));
       }
       if (!ok) break;
       // ---- hand (m, this half's l) of every row to the epilogue warps

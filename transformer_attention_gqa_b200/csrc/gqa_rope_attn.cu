@@ -253,8 +253,15 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
   cfg.blockDim = dim3(ATTN_THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;  // plain stream order after the prologue kernel
+  // Programmatic dependent launch: the attention grid may be scheduled as
+  // soon as every prologue block has finished its stores (each block
+  // triggers at its end), so its launch and setup overlap the prologue's
+  // tail; it reads the prologue's results only after griddepcontrol.wait.
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, gqa_attn_fwd_kernel<D, FP32>, tmQ, tmK, tmV, ap) != cudaSuccess)
     return GQA_ERR_CUDA;
   if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;

@@ -264,14 +264,16 @@ __device__ void rope_k_and_table(const PrepParams& p, int block, int nblocks) {
 
 template <int D, bool FP32_IN>
 __global__ void __launch_bounds__(PREP_THREADS) gqa_prep_kernel(const PrepParams p) {
-  // Let the attention grid start its prologue; it reads nothing written
-  // here before its griddepcontrol.wait.
-  ptx::griddep_launch_dependents();
   if (blockIdx.x == 0) {
     build_schedule(p);
   } else {
     rope_k_and_table<D, FP32_IN>(p, blockIdx.x - 1, gridDim.x - 1);
   }
+  // This block's stores are issued: the attention grid (a programmatic
+  // dependent launch) may be scheduled once every block got here; it reads
+  // nothing written here before its griddepcontrol.wait, which returns once
+  // this grid has completed and its stores are visible.
+  ptx::griddep_launch_dependents();
 }
 
 }  // namespace gqa
