@@ -793,7 +793,7 @@ def run_masked(args, rank, world, local_rank, inp, mask_np):
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": None,
-                     "peak_source": f"{src} bf16_tflops (burst)", "kernel": "gqa_attn_fwd_masked_kernel",
+                     "peak_source": f"{src} bf16_tflops (burst)", "kernel": "gqa_attn_fwd_kernel (masked form)",
                      "kernel_ms": round(attn_ms, 4), "prologue_ms": round(prep_ms, 4)},
         "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},

@@ -215,11 +215,14 @@ int gqa_rope_attn_fwd_noalloc(const void* q, const void* k, const void* v, const
  * and lse = -inf. Arguments as for gqa_rope_attn_fwd (bf16 only), plus:
  *   mask      bf16 [mask_len, mask_ld] device array, 16-byte aligned
  *   mask_len  >= the longest sequence (checked on the device: a longer one
- *             gets no output and sets GQA_ERR_BAD_SEQLENS)
+ *             is attended without the mask, so its output has no meaning,
+ *             and sets GQA_ERR_BAD_SEQLENS; no mask element past mask_len
+ *             is read)
  *   mask_ld   elements between mask rows, >= mask_len, a multiple of 8
  * workspace: gqa_rope_attn_workspace_size(..., GQA_DTYPE_BF16) bytes. Two
- * kernels are queued (the forward's prologue, then the masked attention
- * kernel); the call does not wait.
+ * kernels are queued (the forward's prologue, then the attention kernel in
+ * its masked form: each softmax thread adds its mask values, loaded from
+ * global memory a tile ahead, to the raw scores); the call does not wait.
  */
 int gqa_rope_attn_fwd_masked(const void* q, const void* k, const void* v, const int32_t* positions,
                              double rope_theta, const int32_t* cu_seqlens, int num_seqs, int total_tokens,

@@ -21,6 +21,12 @@ float64, exact rotation) on the CPU:
   lse = (m s + log2(a_a l_a + a_b l_b)) ln 2, with s = log2(e) / sqrt(d)
   (with a shared max: a_a = a_b = 1).
 
+The masked form of the kernel adds mask[query, key] * sqrt(d) to every raw
+score of a visible key before the causal / length bound; a row that sees no
+key at all then gets out = 0 and lse = -inf. It is checked against
+``gqa_rope_attention_masked`` with masks that have holes, fully masked rows
+and fully masked first tiles.
+
 Planted mistakes in the model (the halves combined without their weights, a
 redo without the rescale) are shown to fail the comparison. CPU only."""
 import math
@@ -34,7 +40,7 @@ BM = BN = 128
 HALF = BN // 2
 
 
-def kernel_model(q, k, v, cu, nq, nkv, theta, causal, plant=None, stats=None, shared=False):
+def kernel_model(q, k, v, cu, nq, nkv, theta, causal, plant=None, stats=None, shared=False, mask=None):
     N, _, d = q.shape
     G = nq // nkv
     tq = BM // G
@@ -67,6 +73,9 @@ def kernel_model(q, k, v, cu, nq, nkv, theta, causal, plant=None, stats=None, sh
                         keys = j * BN + hf * HALF + np.arange(HALF)
                         kc = np.minimum(keys, L - 1)         # keys past L: any finite row (masked below)
                         t = qrow @ kr[a + kc, kvh].T         # [R, 64]
+                        if mask is not None:                 # keys past L read 0 (hidden below)
+                            mv = np.where(keys[None, :] < L, mask[np.minimum(tokc, mask.shape[0] - 1)][:, kc], 0.0)
+                            t = t + mv * math.sqrt(d)
                         sc.append(np.where(keys[None, :] > last_key[:, None], -np.inf, t))
                         vt.append(v[a + kc, kvh])            # [64, d]
                     mh = [x.max(axis=1) for x in sc]
@@ -79,7 +88,8 @@ def kernel_model(q, k, v, cu, nq, nkv, theta, causal, plant=None, stats=None, sh
                             need = mh[hf] > m[hf] + thr
                             if stats is not None:
                                 stats["redo"] += int(need.sum())
-                            alpha = np.where(need, np.exp2((m[hf] - mh[hf]) * s), 1.0)
+                            with np.errstate(invalid="ignore"):
+                                alpha = np.where(need, np.exp2((m[hf] - mh[hf]) * s), 1.0)
                             if plant != "redo without rescale":
                                 o[hf] *= alpha[:, None]
                                 l[hf] *= alpha
@@ -99,10 +109,12 @@ def kernel_model(q, k, v, cu, nq, nkv, theta, causal, plant=None, stats=None, sh
                     with np.errstate(invalid="ignore"):
                         wgt = np.where(m == -np.inf, 0.0, np.exp2((m - mrow[None, :]) * s))
                 lrow = (wgt * l).sum(axis=0)
-                orow = (wgt[:, :, None] * o).sum(axis=0) / lrow[:, None]
+                seen = lrow > 0                              # a row that saw no key: out 0, lse -inf
+                with np.errstate(invalid="ignore", divide="ignore"):
+                    orow = np.where(seen[:, None], (wgt[:, :, None] * o).sum(axis=0) / lrow[:, None], 0.0)
                 for r in np.nonzero(valid)[0]:
                     out[a + tok[r], h[r]] = orow[r]
-                    lse[h[r], a + tok[r]] = (mrow[r] * s + math.log2(lrow[r])) * math.log(2.0)
+                    lse[h[r], a + tok[r]] = (mrow[r] * s + math.log2(lrow[r])) * math.log(2.0) if seen[r] else -np.inf
     return out, lse
 
 
@@ -163,3 +175,42 @@ def test_planted_mistakes_fail(plant, k_ramp):
     ref_out, ref_lse = orc.gqa_rope_attention(q, k, v, cu, 8, 2, 1e4, operand_rounding=False)
     err = max(np.nanmax(np.abs(out - ref_out)), np.nanmax(np.abs(lse - ref_lse)))
     assert not err < 1e-3
+
+
+def _masked_case(seed, lens, nq, nkv, d, causal, holes, dead_rows=(), dead_prefix=0):
+    rng = np.random.default_rng(seed)
+    N = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    q, k, v = (rng.standard_normal((N, h, d)) for h in (nq, nkv, nkv))
+    Lm = max(lens)
+    mask = rng.standard_normal((Lm, Lm)) * 2.0
+    mask[rng.random((Lm, Lm)) < holes] = -np.inf
+    for i in dead_rows:
+        mask[i, :] = -np.inf
+    if dead_prefix:
+        mask[:, :dead_prefix] = -np.inf  # every row's first keys hidden
+    return q, k, v, cu, mask
+
+
+MASKED_CASES = {
+    "holes_causal_g4": dict(seed=1, lens=(300,), nq=8, nkv=2, d=32, causal=True, holes=0.3),
+    "holes_full_varlen_g3": dict(seed=2, lens=(150, 1, 40), nq=6, nkv=2, d=32, causal=False, holes=0.5),
+    "dead_rows": dict(seed=3, lens=(140,), nq=4, nkv=4, d=32, causal=True, holes=0.2, dead_rows=(0, 5, 139)),
+    "dead_first_tile": dict(seed=4, lens=(260,), nq=2, nkv=1, d=64, causal=False, holes=0.1, dead_prefix=200),
+}
+
+
+@pytest.mark.parametrize("shared", [False, True])
+@pytest.mark.parametrize("name", sorted(MASKED_CASES))
+def test_masked_form_matches_oracle(name, shared):
+    c = dict(MASKED_CASES[name])
+    q, k, v, cu, mask = _masked_case(**c)
+    ref_o, ref_l = orc.gqa_rope_attention_masked(q, k, v, cu, c["nq"], c["nkv"], 1e4, mask, causal=c["causal"],
+                                                 operand_rounding=False)
+    got_o, got_l = kernel_model(q, k, v, cu, c["nq"], c["nkv"], 1e4, c["causal"], shared=shared, mask=mask)
+    assert np.max(np.abs(got_o - ref_o)) < 1e-10
+    fin = np.isfinite(ref_l)
+    assert np.array_equal(fin, np.isfinite(got_l))
+    assert np.max(np.abs(got_l[fin] - ref_l[fin])) < 1e-10
+    if c.get("dead_rows"):
+        assert (~fin).any()

@@ -55,5 +55,5 @@ def test_setmaxnreg_kernels_launch_with_the_split_register_count(ptxas_report):
                 seen[kern] += 1
                 assert regs == want, (name, regs)
                 assert st == 0 and ld == 0, (name, st, ld)
-    # forward: 3 head dims x 2 dtypes; backward: 3 head dims
-    assert seen == {"gqa_attn_fwd_kernel": 6, "gqa_attn_bwd_kernel": 3}, seen
+    # forward: 3 head dims x (bf16, fp32, masked bf16); backward: 3 head dims
+    assert seen == {"gqa_attn_fwd_kernel": 9, "gqa_attn_bwd_kernel": 3}, seen

@@ -11,7 +11,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "gqa_rope_attn.cu")
 DEPS = [os.path.join(PKG, "csrc", f) for f in ("gqa_rope_attn.cu", "attn_kernel.cuh", "prep_kernel.cuh",
-                                               "decode_kernel.cuh", "bwd_kernel.cuh", "bwd_q_kernel.cuh", "proj_kernel.cuh", "masked_kernel.cuh", "common.cuh", "ptx.cuh",
+                                               "decode_kernel.cuh", "bwd_kernel.cuh", "bwd_q_kernel.cuh", "proj_kernel.cuh", "common.cuh", "ptx.cuh",
                                                "exp2_poly.cuh", "rope_round.cuh")] + [
     os.path.join(ROOT, "include", "gqa_rope_attn.h")]
 LIB_DIR = os.path.join(PKG, "lib")

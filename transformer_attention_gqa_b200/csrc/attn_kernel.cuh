@@ -8,6 +8,12 @@
 // are produced in tensor memory, turned into probabilities by an online
 // (running max / running sum) softmax and consumed by the P.V product.
 //
+// Masked form (MASK): the additive mask of the same page's section "The
+// compute thread" (and the masks of the "Kohaku-TT" page): each softmax
+// thread adds mask[token, key] * sqrt(d) to its raw scores, the values of
+// the next KV tile loaded from global memory while the current one runs; a
+// row that sees no key gets out = 0 and lse = -inf.
+//
 // One persistent CTA per SM takes work items (sequence, q-tile, KV head)
 // from a longest-first list: its first item statically, every further one
 // from a global counter (greedy list scheduling, so that faster CTAs take
@@ -69,6 +75,12 @@ constexpr int REG_PRODUCER = 56;
 constexpr int REG_SOFTMAX = 160;
 constexpr int REG_ROPE = 128;
 static_assert(REG_PRODUCER * 128 + REG_SOFTMAX * 256 + REG_ROPE * 128 <= 65536 / ATTN_THREADS * ATTN_THREADS,
+              "register split exceeds the launch's register file share");
+// masked form: 8 more per softmax thread for the mask words, from the Q
+// warpgroup (56 x 128 + 168 x 256 + 112 x 128 = 64512)
+constexpr int REG_SOFTMAX_MASKED = 168;
+constexpr int REG_ROPE_MASKED = 112;
+static_assert(REG_PRODUCER * 128 + REG_SOFTMAX_MASKED * 256 + REG_ROPE_MASKED * 128 <= 65536,
               "register split exceeds the launch's register file share");
 
 struct WorkItem {
@@ -542,7 +554,7 @@ __device__ __forceinline__ bool rope_q_tile(const AttnParams& p, uint8_t* smem, 
                         w >= 0, wi, wi.t0, tmQ, tid, abort_flag);
 }
 
-template <class C, bool OUT_FP32>
+template <class C, bool OUT_FP32, bool MASK>
 __device__ __forceinline__ bool epilogue_tile(const AttnParams& p, const WorkItem& wi, uint8_t* smem, Barriers* bars,
                                               uint32_t tmem, int it, uint32_t g, int tid,
                                               volatile int* abort_flag) {
@@ -575,13 +587,14 @@ __device__ __forceinline__ bool epilogue_tile(const AttnParams& p, const WorkIte
     const float a0 = ml0.x == -INFINITY ? 0.f : ptx::ex2((ml0.x - mrow) * p.scale_log2);
     const float a1 = ml1.x == -INFINITY ? 0.f : ptx::ex2((ml1.x - mrow) * p.scale_log2);
     lrow = a0 * ml0.y + a1 * ml1.y;
-    const float inv_l = 1.f / lrow;
+    // (masked form: a row that saw no visible key has l = 0: out = 0)
+    const float inv_l = (MASK && !(lrow > 0.f)) ? 0.f : 1.f / lrow;
     w0 = a0 * inv_l;
     w1 = a1 * inv_l;
   } else {
     mrow = ml0.x;  // both halves hold the same running max
     lrow = ml0.y + ml1.y;
-    w0 = 1.f / lrow;
+    w0 = (MASK && !(lrow > 0.f)) ? 0.f : 1.f / lrow;
     w1 = 0.f;
   }
   const int h = wi.kvh * G + hin;
@@ -621,8 +634,47 @@ __device__ __forceinline__ bool epilogue_tile(const AttnParams& p, const WorkIte
     }
   }
   if (row_valid && p.lse)
-    p.lse[(size_t)h * p.N + wi.seq_start + tok] = (mrow * p.scale_log2 + __log2f(lrow)) * 0.69314718055994531f;
+    p.lse[(size_t)h * p.N + wi.seq_start + tok] =
+        (MASK && !(lrow > 0.f)) ? -INFINITY : (mrow * p.scale_log2 + __log2f(lrow)) * 0.69314718055994531f;
   return true;
+}
+
+// The 64 mask values of query row mrow for keys [key0, key0 + 64) as bf16
+// pairs (key0 + 2e in the low half of m[e]); keys at or past L, and every
+// key of a null row, read 0 (the length mask hides them).
+__device__ __forceinline__ void load_mask_half(const __nv_bfloat16* mrow, int key0, int L, uint32_t* m) {
+#pragma unroll
+  for (int q4 = 0; q4 < 8; ++q4) {
+    const int key = key0 + 8 * q4;
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (mrow) {
+      if (key + 8 <= L) {
+        w = __ldg(reinterpret_cast<const uint4*>(mrow + key));
+      } else if (key < L) {
+        uint32_t h[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) h[e] = key + e < L ? (uint32_t)__bfloat16_as_ushort(mrow[key + e]) : 0u;
+        w = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+      }
+    }
+    m[4 * q4] = w.x;
+    m[4 * q4 + 1] = w.y;
+    m[4 * q4 + 2] = w.z;
+    m[4 * q4 + 3] = w.w;
+  }
+}
+
+// s += mask * scale on 64 raw scores (the bf16 pairs of load_mask_half).
+__device__ __forceinline__ void add_mask_half(uint32_t* sr, const uint32_t* m, float scale) {
+  const float2 sc2 = make_float2(scale, scale);
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    const uint32_t w = m[c >> 1];
+    const float2 mv = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    const float2 r = ffma2(mv, sc2, make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])));
+    sr[c] = __float_as_uint(r.x);
+    sr[c + 1] = __float_as_uint(r.y);
+  }
 }
 
 // S = Q K^T for one KV tile: D/16 K-steps, K-major A and B (SW128/SW64).
@@ -657,7 +709,7 @@ __device__ __forceinline__ void issue_pv_half(uint32_t o_tmem, uint32_t p_tmem, 
                 (accumulate || kk > 0) ? 1u : 0u);
 }
 
-template <int D, bool OUT_FP32>
+template <int D, bool OUT_FP32, bool MASK>
 __global__ void __launch_bounds__(ATTN_THREADS, 1)
     gqa_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -877,7 +929,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     }
    }
   } else if (warp < 12) {
-    ptx::setmaxnreg_inc<REG_SOFTMAX>();
+    ptx::setmaxnreg_inc<MASK ? REG_SOFTMAX_MASKED : REG_SOFTMAX>();
     // ------------------------------------------------------------ softmax
     constexpr int NC = BN / 2;           // columns per thread
     const int quad = warp & 3;
@@ -899,6 +951,18 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       if (!(ok = take_item_warp(bars, it, w, wi, abort_flag)) || w < 0) break;
       const int tok = wi.t0 + tok_off;  // index inside the sequence
       const int last_key = p.causal ? tok : wi.L - 1;
+      // masked form: the row's mask values, a tile ahead (null row past the
+      // sequence; a sequence longer than the mask is reported and unmasked)
+      const __nv_bfloat16* mrow = nullptr;
+      uint32_t mk[MASK ? NC / 2 : 1];
+      if constexpr (MASK) {
+        if (wi.L > p.mask_len) {
+          if (warp == 4 && lane == 0) atomicCAS(&g_status, 0, kStatusBadSeqlens);
+        } else if (tok < wi.L) {
+          mrow = p.mask + (size_t)tok * p.mask_ld;
+        }
+        load_mask_half(mrow, half * NC, wi.L, mk);
+      }
       float m = -INFINITY;
       float l = 0.f;
       for (int j = 0; j < wi.nkv; ++j) {
@@ -909,6 +973,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         if (!ok) break;
         ptx::tc_fence_after();
         load_s_cols<NC>(tS, sr);
+        if constexpr (MASK) add_mask_half(sr, mk, p.mask_scale);
         const int lim = last_key - j * BN - half * NC;  // this half's columns > lim are masked
         if (lim < NC - 1) mask_cols<NC>(sr, lim);
         float alpha = 1.f;
@@ -933,6 +998,10 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
                 m = mh;
               }
               load_s_cols<NC>(tS, sr);  // S is intact: P has not been stored yet
+              if constexpr (MASK) {
+                load_mask_half(mrow, j * BN + half * NC, wi.L, mk);
+                add_mask_half(sr, mk, p.mask_scale);
+              }
               if (lim < NC - 1) mask_cols<NC>(sr, lim);
               lsum = exp_pack<NC, emu_period(D)>(sr, m == -INFINITY ? 0.f : -m * sl2, sl2, nullptr);
               // O_h holds this half's sum up to the previous tile: wait for
@@ -960,13 +1029,13 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             ok = __all_sync(0xffffffffu, bwait(xbar, xpar, abort_flag));
             if (!ok) break;
             m = fmaxf(mh, *xm_other);
-            lsum = exp_pack<NC, emu_period(D)>(sr, -m * sl2, sl2, nullptr);
+            lsum = exp_pack<NC, emu_period(D)>(sr, (MASK && m == -INFINITY) ? 0.f : -m * sl2, sl2, nullptr);
           } else {
             // Exponentials with the running max m, the tile's max alongside;
             // if the row's max exceeds m by more than the threshold (2^8 in p)
             // the tile is redone below with the new max.
             float mh;
-            lsum = exp_pack<NC, emu_period(D)>(sr, -m * sl2, sl2, &mh);
+            lsum = exp_pack<NC, emu_period(D)>(sr, (MASK && m == -INFINITY) ? 0.f : -m * sl2, sl2, &mh);
             *xm_mine = mh;
             ptx::mbar_arrive(xbar);
             ok = __all_sync(0xffffffffu, bwait(xbar, xpar, abort_flag));
@@ -981,8 +1050,12 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             // Both halves see the same maxima, so they take this branch together.
             if (__any_sync(0xffffffffu, need)) {
               load_s_cols<NC>(tS, sr);  // S is intact: P has not been stored yet
+              if constexpr (MASK) {
+                load_mask_half(mrow, j * BN + half * NC, wi.L, mk);
+                add_mask_half(sr, mk, p.mask_scale);
+              }
               if (lim < NC - 1) mask_cols<NC>(sr, lim);
-              lsum = exp_pack<NC, emu_period(D)>(sr, -m * sl2, sl2, nullptr);
+              lsum = exp_pack<NC, emu_period(D)>(sr, (MASK && m == -INFINITY) ? 0.f : -m * sl2, sl2, nullptr);
               // O holds the sum up to the previous tile: wait for PV(gg-1), then
               // scale this half's share of O's columns.
               const uint32_t gp = gg - 1;
@@ -1000,6 +1073,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(B(bars->p_full[b][C::SPLIT ? half : 0]));
+        if constexpr (MASK)
+          if (j + 1 < wi.nkv) load_mask_half(mrow, (j + 1) * BN + half * NC, wi.L, mk);
       }
       if (!ok) break;
       // ---- hand (m, this half's l) of every row to the epilogue warps
@@ -1010,7 +1085,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       g += wi.nkv;
     }
   } else {
-    // (runs with the launch's REG_ROPE registers)
+    // (runs with the launch's REG_ROPE registers; REG_ROPE_MASKED in the masked form)
+    if constexpr (MASK) ptx::setmaxnreg_dec<REG_ROPE_MASKED>();
     // ------------------------------------------------------------ Q rotation + epilogue
     const int tid = threadIdx.x - 384;
     const int rows = p.tq * p.G;
@@ -1039,7 +1115,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       int wn;
       WorkItem win{};
       if (!(ok = rope_q_tile<C>(p, smem, bars, &tmQ, it + 1, tid, abort_flag, wn, win))) break;
-      ok = epilogue_tile<C, OUT_FP32>(p, wi, smem, bars, tmem, it, g, tid, abort_flag);
+      ok = epilogue_tile<C, OUT_FP32, MASK>(p, wi, smem, bars, tmem, it, g, tid, abort_flag);
       g += wi.nkv;
       w = wn;
       wi = win;

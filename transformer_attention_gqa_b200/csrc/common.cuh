@@ -128,6 +128,11 @@ struct AttnParams {
   int q_rotated;        // 1: the Q tiles arrive rotated (the caller's, or the prologue's Q'); 0: rotate them
   int k_token_major;    // 1: K is the caller's rotated token-major [N][n_kv][d] tensor; 0: K' head-major
                         // from the prologue
+  // additive mask (masked form of the kernel only): bf16 [mask_len][mask_ld]
+  // over in-sequence (query, key) indices, raw score += mask * mask_scale
+  const __nv_bfloat16* mask;
+  int mask_len, mask_ld;
+  float mask_scale;
 };
 
 }  // namespace gqa

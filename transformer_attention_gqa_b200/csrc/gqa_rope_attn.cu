@@ -1,7 +1,7 @@
 // Host side of the C ABI (include/gqa_rope_attn.h): argument checks, TMA
 // descriptor cache, the two launches of the fused forward (prologue, then
 // the attention kernel, in stream order), the two of the masked forward (the
-// same prologue, then the masked attention kernel), the two of the decoding
+// same prologue, then the attention kernel in its masked form), the two of the decoding
 // step (key-range kernel, then the merge), the three of the backward
 // (prologue, attention backward, dq rotation) and the two of the QKV
 // projection with its RoPE epilogue (cos/sin table, projection).
@@ -20,7 +20,6 @@
 #include "bwd_q_kernel.cuh"
 #include "common.cuh"
 #include "decode_kernel.cuh"
-#include "masked_kernel.cuh"
 #include "prep_kernel.cuh"
 #include "proj_kernel.cuh"
 
@@ -132,12 +131,15 @@ int dim_index(int d) { return d == 32 ? 0 : (d == 64 ? 1 : 2); }
 
 // prerotated: q and k are already rotated (bf16 only); the prologue builds
 // the schedule alone and K is read from the caller's token-major tensor.
+// mask (bf16 only): the attention kernel's masked form adds mask[query,
+// key] * sqrt(d) to every raw score.
 template <int D, bool FP32>
 int launch(const void* q, const void* k, const void* v, const int32_t* positions, double theta,
            const int32_t* cu, int num_seqs, int N, int nq, int nkv, int causal, void* out, float* lse,
            uint8_t* ws, const WsLayout& lay, cudaStream_t stream, int device, int sm_count,
-           bool prerotated = false) {
-  if (FP32 && prerotated) return GQA_ERR_UNSUPPORTED;
+           bool prerotated = false, const void* mask = nullptr, int mask_len = 0, int mask_ld = 0) {
+  if (FP32 && (prerotated || mask)) return GQA_ERR_UNSUPPORTED;
+  if (prerotated && mask) return GQA_ERR_UNSUPPORTED;
   using C = AttnCfg<D>;
   const int G = nq / nkv;
   const int tq = tokens_per_tile(G);
@@ -145,10 +147,18 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
   {  // caller holds g_mu
     DeviceState& ds = g_dev[device];
     if (!ds.attr_set[dim_index(D)][FP32 ? 1 : 0]) {
-      if (cudaFuncSetAttribute(gqa_attn_fwd_kernel<D, FP32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(gqa_attn_fwd_kernel<D, FP32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_BYTES) != cudaSuccess)
         return GQA_ERR_CUDA;
       ds.attr_set[dim_index(D)][FP32 ? 1 : 0] = true;
+    }
+    if constexpr (!FP32) {
+      if (mask && !ds.masked_attr_set[dim_index(D)]) {
+        if (cudaFuncSetAttribute(gqa_attn_fwd_kernel<D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess)
+          return GQA_ERR_CUDA;
+        ds.masked_attr_set[dim_index(D)] = true;
+      }
     }
   }
 
@@ -239,6 +249,10 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
   ap.rescale_thr = (float)(8.0 / (1.4426950408889634 / std::sqrt((double)D)));
   ap.q_rotated = (prerotated || q_in_ws) ? 1 : 0;
   ap.k_token_major = prerotated ? 1 : 0;
+  ap.mask = reinterpret_cast<const __nv_bfloat16*>(mask);
+  ap.mask_len = mask_len;
+  ap.mask_ld = mask_ld;
+  ap.mask_scale = (float)std::sqrt((double)D);
 
   const long long max_items = lay.max_pairs * (long long)nkv;
   const unsigned grid = (unsigned)(max_items < sm_count ? max_items : sm_count);
@@ -262,8 +276,14 @@ int launch(const void* q, const void* k, const void* v, const int32_t* positions
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, gqa_attn_fwd_kernel<D, FP32>, tmQ, tmK, tmV, ap) != cudaSuccess)
-    return GQA_ERR_CUDA;
+  cudaError_t le;
+  if constexpr (!FP32) {
+    le = mask ? cudaLaunchKernelEx(&cfg, gqa_attn_fwd_kernel<D, false, true>, tmQ, tmK, tmV, ap)
+              : cudaLaunchKernelEx(&cfg, gqa_attn_fwd_kernel<D, false, false>, tmQ, tmK, tmV, ap);
+  } else {
+    le = cudaLaunchKernelEx(&cfg, gqa_attn_fwd_kernel<D, true, false>, tmQ, tmK, tmV, ap);
+  }
+  if (le != cudaSuccess) return GQA_ERR_CUDA;
   if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;
   t_last_launches = 2;
   return GQA_OK;
@@ -557,108 +577,6 @@ int launch_qkv_proj(const void* x, const void* w, const int32_t* positions, doub
   pp.nkv = nkv;
   const dim3 grid((unsigned)((F + PJ_BN - 1) / PJ_BN), (unsigned)((N + PJ_BM - 1) / PJ_BM), 1);
   gqa_qkv_proj_kernel<D><<<grid, PJ_THREADS, PJ_SMEM_BYTES, stream>>>(tmX, tmW, pp);
-  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
-  if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;
-  t_last_launches = 2;
-  return GQA_OK;
-}
-
-// ---------------------------------------------------------------- masked forward
-
-template <int D>
-int launch_masked(const void* q, const void* k, const void* v, const int32_t* positions, double theta,
-                  const int32_t* cu, int num_seqs, int N, int nq, int nkv, int causal, const void* mask,
-                  int mask_len, int mask_ld, void* out, float* lse, uint8_t* ws, const WsLayout& lay,
-                  cudaStream_t stream, int device, int sm_count) {
-  using A = AttnCfg<D>;
-  using C = MaskedCfg<D>;
-  const int G = nq / nkv;
-  const int tq = tokens_per_tile(G);
-  {  // caller holds g_mu
-    DeviceState& ds = g_dev[device];
-    if (!ds.masked_attr_set[dim_index(D)]) {
-      if (cudaFuncSetAttribute(gqa_attn_fwd_masked_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               C::SMEM_BYTES) != cudaSuccess)
-        return GQA_ERR_CUDA;
-      ds.masked_attr_set[dim_index(D)] = true;
-    }
-  }
-  // the forward's prologue: schedule, cos/sin table, K' head-major
-  PrepParams pp{};
-  pp.q = q;
-  pp.k = k;
-  pp.v = v;
-  pp.positions = positions;
-  pp.cu = cu;
-  pp.N = N;
-  pp.num_seqs = num_seqs;
-  pp.nq = nq;
-  pp.nkv = nkv;
-  pp.tq = tq;
-  pp.causal = causal;
-  pp.theta = theta;
-  for (int i = 0; i < D / 2; ++i) pp.inv_freq[i] = std::pow(theta, -(2.0 * i) / D);
-  pp.header = reinterpret_cast<int*>(ws + lay.header);
-  pp.seq_pfx = reinterpret_cast<int*>(ws + lay.seq_pfx);
-  pp.pairs = reinterpret_cast<int2*>(ws + lay.pairs);
-  pp.table = reinterpret_cast<uint32_t*>(ws + lay.table);
-  pp.kws = reinterpret_cast<__nv_bfloat16*>(ws + lay.kws);
-  pp.qws = nullptr;
-  pp.vws = nullptr;
-
-  CUtensorMap tmQ, tmK, tmV;
-  {
-    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)nq, (uint64_t)N};
-    const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)nq * D * 2};
-    const uint32_t box[3] = {(uint32_t)A::BOXC, (uint32_t)G, (uint32_t)tq};
-    if (!make_tmap(device, q, dims, str, box, A::ROWB, &tmQ)) return GQA_ERR_CUDA;
-  }
-  {
-    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)N, (uint64_t)nkv};
-    const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)N * D * 2};
-    const uint32_t box[3] = {(uint32_t)A::BOXC, (uint32_t)BN, 1u};
-    if (!make_tmap(device, ws + lay.kws, dims, str, box, A::ROWB, &tmK)) return GQA_ERR_CUDA;
-  }
-  {
-    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)nkv, (uint64_t)N};
-    const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)nkv * D * 2};
-    const uint32_t box[3] = {(uint32_t)A::BOXC, 1u, (uint32_t)BN};
-    if (!make_tmap(device, v, dims, str, box, A::ROWB, &tmV)) return GQA_ERR_CUDA;
-  }
-  long long nb = ((long long)N * (D / 4) + PREP_THREADS - 1) / PREP_THREADS;
-  if (nb > (long long)sm_count * 8) nb = (long long)sm_count * 8;
-  if (nb < 1) nb = 1;
-  if (t_prof_ev[0] && cudaEventRecord(t_prof_ev[0], stream) != cudaSuccess) return GQA_ERR_CUDA;
-  gqa_prep_kernel<D, false><<<(unsigned)(nb + 1), PREP_THREADS, 0, stream>>>(pp);
-  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
-  if (t_prof_ev[1] && cudaEventRecord(t_prof_ev[1], stream) != cudaSuccess) return GQA_ERR_CUDA;
-
-  MaskedParams mp{};
-  AttnParams& ap = mp.base;
-  ap.cu = cu;
-  ap.header = pp.header;
-  ap.item_counter = pp.header + 8;
-  ap.pairs = pp.pairs;
-  ap.table = pp.table;
-  ap.out = out;
-  ap.lse = lse;
-  ap.N = N;
-  ap.nq = nq;
-  ap.nkv = nkv;
-  ap.G = G;
-  ap.tq = tq;
-  ap.causal = causal;
-  ap.sched_dynamic = 0;
-  ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  ap.rescale_thr = 0.f;
-  mp.mask = reinterpret_cast<const __nv_bfloat16*>(mask);
-  mp.mask_len = mask_len;
-  mp.mask_ld = mask_ld;
-  mp.sqrt_d = (float)std::sqrt((double)D);
-  // one CTA per (sequence, q-tile, KV head) work item; CTAs past the
-  // prologue's item count exit at once
-  const unsigned grid = (unsigned)(lay.max_pairs * (long long)nkv);
-  gqa_attn_fwd_masked_kernel<D><<<grid, MK_THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, mp);
   if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;
   t_last_launches = 2;
@@ -1137,9 +1055,9 @@ extern "C" int gqa_rope_attn_fwd_masked(const void* q, const void* k, const void
   std::lock_guard<std::mutex> lk(g_mu);  // descriptor cache
 #define GQA_MASKED_CASE(DD)                                                                                   \
   if (head_dim == DD)                                                                                         \
-    return launch_masked<DD>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads,  \
-                             n_kv_heads, causal, mask, mask_len, mask_ld, out, lse, ws, lay, st, device,      \
-                             sm_count);
+    return launch<DD, false>(q, k, v, positions, rope_theta, cu_seqlens, num_seqs, total_tokens, n_q_heads,  \
+                             n_kv_heads, causal, out, lse, ws, lay, st, device, sm_count, false, mask,        \
+                             mask_len, mask_ld);
   GQA_MASKED_CASE(32) GQA_MASKED_CASE(64) GQA_MASKED_CASE(128)
 #undef GQA_MASKED_CASE
   return GQA_ERR_UNSUPPORTED;
