@@ -575,7 +575,13 @@ int launch_qkv_proj(const void* x, const void* w, const int32_t* positions, doub
   pp.C = C;
   pp.nq = nq;
   pp.nkv = nkv;
-  const dim3 grid((unsigned)((F + PJ_BN - 1) / PJ_BN), (unsigned)((N + PJ_BM - 1) / PJ_BM), 1);
+  pp.n_tiles_n = (F + PJ_BN - 1) / PJ_BN;
+  const long long n_tiles = (long long)pp.n_tiles_n * ((N + PJ_BM - 1) / PJ_BM);
+  if (n_tiles > 0x7fffffffll) return GQA_ERR_UNSUPPORTED;
+  pp.n_tiles = (int)n_tiles;
+  // one persistent CTA per SM (each walks tiles b, b + grid, ...); with
+  // fewer than two tiles per SM, one CTA per tile (measured faster there)
+  const unsigned grid = (unsigned)(n_tiles <= 2LL * sm_count ? n_tiles : sm_count);
   gqa_qkv_proj_kernel<D><<<grid, PJ_THREADS, PJ_SMEM_BYTES, stream>>>(tmX, tmW, pp);
   if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
   if (t_prof_ev[2] && cudaEventRecord(t_prof_ev[2], stream) != cudaSuccess) return GQA_ERR_CUDA;
