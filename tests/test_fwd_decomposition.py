@@ -109,7 +109,7 @@ def kernel_model(q, k, v, cu, nq, nkv, theta, causal, plant=None, stats=None, sh
                     with np.errstate(invalid="ignore"):
                         wgt = np.where(m == -np.inf, 0.0, np.exp2((m - mrow[None, :]) * s))
                 lrow = (wgt * l).sum(axis=0)
-                seen = lrow > 0                              # a row that saw no key: out 0, lse -inf
+                seen = mrow > -np.inf                        # a row that saw no key: out 0, lse -inf
                 with np.errstate(invalid="ignore", divide="ignore"):
                     orow = np.where(seen[:, None], (wgt[:, :, None] * o).sum(axis=0) / lrow[:, None], 0.0)
                 for r in np.nonzero(valid)[0]:

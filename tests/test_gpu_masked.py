@@ -18,6 +18,10 @@ CASES = {
     "causal_holes_g4_d128": ((300, 77), 32, 8, 128, True, 0.3, ()),
     "full_holes_varlen_g3_d64": ((150, 1, 40), 6, 2, 64, False, 0.5, (3,)),
     "dead_rows_g1_d32": ((140,), 4, 4, 32, True, 0.2, (0, 5, 139)),
+    # the nano shapes of the benchmark's masked_nano workload (16 x 512 tokens, G = 3, d = 64)
+    "nano_shapes_g3_d64": ((512,) * 16, 6, 2, 64, True, 0.0, ()),
+    # one long sequence at the Llama-3-8B head layout: 16 KV tiles per q-tile row, 512 work items
+    "long_2048_g4_d128": ((2048,), 32, 8, 128, True, 0.1, ()),
 }
 
 

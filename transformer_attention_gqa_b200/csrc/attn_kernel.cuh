@@ -580,6 +580,7 @@ __device__ __forceinline__ bool epilogue_tile(const AttnParams& p, const WorkIte
   ptx::tc_fence_after();
 
   float mrow, lrow, w0, w1;
+  bool dead = false;  // masked form: the row saw no visible key (its running max stayed -inf): out 0, lse -inf
   if constexpr (C::SPLIT) {
     // O = (a0 O_a + a1 O_b) / (a0 l_a + a1 l_b), a_h = 2^((m_h - m) scale) for
     // the row max m; a half that saw no unmasked key (m_h = -inf) weighs 0
@@ -587,14 +588,15 @@ __device__ __forceinline__ bool epilogue_tile(const AttnParams& p, const WorkIte
     const float a0 = ml0.x == -INFINITY ? 0.f : ptx::ex2((ml0.x - mrow) * p.scale_log2);
     const float a1 = ml1.x == -INFINITY ? 0.f : ptx::ex2((ml1.x - mrow) * p.scale_log2);
     lrow = a0 * ml0.y + a1 * ml1.y;
-    // (masked form: a row that saw no visible key has l = 0: out = 0)
-    const float inv_l = (MASK && !(lrow > 0.f)) ? 0.f : 1.f / lrow;
+    dead = MASK && mrow == -INFINITY;
+    const float inv_l = dead ? 0.f : 1.f / lrow;
     w0 = a0 * inv_l;
     w1 = a1 * inv_l;
   } else {
     mrow = ml0.x;  // both halves hold the same running max
     lrow = ml0.y + ml1.y;
-    w0 = (MASK && !(lrow > 0.f)) ? 0.f : 1.f / lrow;
+    dead = MASK && mrow == -INFINITY;
+    w0 = dead ? 0.f : 1.f / lrow;
     w1 = 0.f;
   }
   const int h = wi.kvh * G + hin;
@@ -635,7 +637,7 @@ __device__ __forceinline__ bool epilogue_tile(const AttnParams& p, const WorkIte
   }
   if (row_valid && p.lse)
     p.lse[(size_t)h * p.N + wi.seq_start + tok] =
-        (MASK && !(lrow > 0.f)) ? -INFINITY : (mrow * p.scale_log2 + __log2f(lrow)) * 0.69314718055994531f;
+        dead ? -INFINITY : (mrow * p.scale_log2 + __log2f(lrow)) * 0.69314718055994531f;
   return true;
 }
 
